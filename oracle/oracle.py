@@ -1,0 +1,155 @@
+"""Python access to the fp64 CPU oracle for gated retention (gret_oracle.c).
+
+TEST INFRASTRUCTURE ONLY: imported by tests/, by the smoke check and by the benchmark's
+CPU-baseline leg, never by the library.  The arithmetic lives in gret_oracle.c; this module only
+converts arrays to contiguous fp64 and passes pointers.  See gret_oracle.c for the passages each
+function follows ("YOCO 完全拆解", sections "路线二：Multi-Head Gated Retention",
+"Prefill 与 Decode 为什么使用两种计算形态" and "单 token Decode 的实现骨架").
+
+Layout: q, k [T, H, dk]; v [T, H, dv]; g [T, H]; cu_seqlens [n_seqs+1];
+state [n_seqs, H, dk, dv]; returns o [T, H, dv] and the final state.
+"""
+import ctypes
+import os
+
+import numpy as np
+
+from . import build as _build
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ctypes.CDLL(path)
+        dp = ctypes.POINTER(ctypes.c_double)
+        ip = ctypes.POINTER(ctypes.c_int64)
+        common = [dp, dp, dp, dp, ctypes.c_double, ctypes.c_double, ctypes.c_int64,
+                  ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ctypes.c_int, dp, dp, dp]
+        for name in ("oracle_gret_recurrent", "oracle_gret_parallel"):
+            f = getattr(L, name)
+            f.argtypes = common
+            f.restype = ctypes.c_int
+        L.oracle_gret_chunkwise.argtypes = common + [ctypes.c_int]
+        L.oracle_gret_chunkwise.restype = ctypes.c_int
+        L.oracle_gret_decode_step.argtypes = [dp, dp, dp, dp, ctypes.c_double, ctypes.c_double,
+                                              ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                              ctypes.c_int, dp, dp]
+        L.oracle_gret_decode_step.restype = ctypes.c_int
+        L.oracle_groupnorm_gate.argtypes = [dp, dp, dp, dp, dp, ctypes.c_double, ctypes.c_int64,
+                                            ctypes.c_int, ctypes.c_int, ctypes.c_int, ip,
+                                            ctypes.c_int64, dp]
+        L.oracle_groupnorm_gate.restype = ctypes.c_int
+        L.oracle_log_gamma.argtypes = [ctypes.c_double, ctypes.c_double]
+        L.oracle_log_gamma.restype = ctypes.c_double
+        _lib = L
+    return _lib
+
+
+def _d(a):
+    """Contiguous fp64 copy of an array-like (torch tensors are moved to the CPU first)."""
+    if a is None:
+        return None
+    if hasattr(a, "detach"):
+        a = a.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def _cu(cu_seqlens, T):
+    if cu_seqlens is None:
+        cu_seqlens = [0, T]
+    if hasattr(cu_seqlens, "detach"):
+        cu_seqlens = cu_seqlens.detach().cpu().numpy()
+    return np.ascontiguousarray(np.asarray(cu_seqlens, dtype=np.int64))
+
+
+def threads():
+    """OpenMP threads the oracle will use (OMP_NUM_THREADS, else the usable cores)."""
+    env = os.environ.get("OMP_NUM_THREADS")
+    if env:
+        return int(env)
+    return len(os.sched_getaffinity(0))
+
+
+def _run(fname, q, k, v, g, tau, k_scale, cu_seqlens, state_in, extra=()):
+    q, k, v, g = _d(q), _d(k), _d(v), _d(g)
+    T, H, dk = q.shape
+    dv = v.shape[2]
+    assert k.shape == (T, H, dk) and v.shape == (T, H, dv) and g.shape == (T, H)
+    cu = _cu(cu_seqlens, T)
+    n = len(cu) - 1
+    s_in = _d(state_in)
+    if s_in is not None:
+        assert s_in.shape == (n, H, dk, dv)
+    o = np.zeros((T, H, dv))
+    s_out = np.zeros((n, H, dk, dv))
+    rc = getattr(lib(), fname)(_p(q), _p(k), _p(v), _p(g), float(tau), float(k_scale), T, H,
+                              dk, dv, cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), n,
+                              _p(s_in), _p(s_out), _p(o), *extra)
+    if rc != 0:
+        raise ValueError("%s rejected its arguments (rc=%d)" % (fname, rc))
+    return o, s_out
+
+
+def gret_recurrent(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):
+    """Recurrent gRet (the definition).  Returns (o [T,H,dv], state [n_seqs,H,dk,dv])."""
+    return _run("oracle_gret_recurrent", q, k, v, g, tau, k_scale, cu_seqlens, state_in)
+
+
+def gret_parallel(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):
+    """Brute-force unrolled form with explicit decay products (tiny inputs only)."""
+    return _run("oracle_gret_parallel", q, k, v, g, tau, k_scale, cu_seqlens, state_in)
+
+
+def gret_chunkwise(q, k, v, g, chunk, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):
+    """Chunkwise re-association evaluated in fp64 (checks the decomposition, not the GPU)."""
+    return _run("oracle_gret_chunkwise", q, k, v, g, tau, k_scale, cu_seqlens, state_in,
+                extra=(int(chunk),))
+
+
+def gret_decode_step(q, k, v, g, state, tau=16.0, k_scale=1.0):
+    """One decode step on [B,H,d] inputs; returns (o [B,H,dv], new state [B,H,dk,dv])."""
+    q, k, v, g = _d(q), _d(k), _d(v), _d(g)
+    S = _d(state).copy()
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    assert S.shape == (B, H, dk, dv) and g.shape == (B, H)
+    o = np.zeros((B, H, dv))
+    rc = lib().oracle_gret_decode_step(_p(q), _p(k), _p(v), _p(g), float(tau), float(k_scale),
+                                       B, H, dk, dv, _p(S), _p(o))
+    if rc != 0:
+        raise ValueError("oracle_gret_decode_step rc=%d" % rc)
+    return o, S
+
+
+def groupnorm_gate(o, x, w_g, H, gn_weight=None, gn_bias=None, eps=1e-5, rows=None):
+    """Per-head GroupNorm(o) * swish(x @ w_g) for the listed rows (all rows if None).
+
+    o [T, H*dv], x [T, D], w_g [D, H*dv].  Returns y [len(rows) or T, H*dv]."""
+    o, x, w_g = _d(o), _d(x), _d(w_g)
+    T, F = o.shape
+    D = x.shape[1]
+    assert F % H == 0 and x.shape[0] == T and w_g.shape == (D, F)
+    dv = F // H
+    gw, gb = _d(gn_weight), _d(gn_bias)
+    if rows is not None:
+        r = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
+        rp, nr = r.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), len(r)
+    else:
+        r, rp, nr = None, None, T
+    y = np.zeros((nr, F))
+    rc = lib().oracle_groupnorm_gate(_p(o), _p(x), _p(w_g), _p(gw), _p(gb), float(eps), T, H,
+                                     dv, D, rp, nr, _p(y))
+    if rc != 0:
+        raise ValueError("oracle_groupnorm_gate rc=%d" % rc)
+    return y
+
+
+def log_gamma(g, tau=16.0):
+    return lib().oracle_log_gamma(float(g), float(tau))

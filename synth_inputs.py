@@ -1,0 +1,100 @@
+"""Seeded synthetic inputs for gated retention, shared by the tests, the benchmark and the oracle
+checks.
+
+This module draws random numbers and nothing else: it holds none of the method's arithmetic.
+Every tensor is drawn from a torch.Generator seeded from (seed, tensor tag), so one call with
+the same arguments always returns the same values.  Inputs are drawn in fp32 and then rounded
+to the requested dtype; the rounded values are what both the CUDA path and the oracle see.
+
+Recipes (the 3B shapes of the YOCO pages: 24 heads of width 128, hidden 3072):
+  * q, k, v ~ N(0, 1) / sqrt(d)         (the 1/sqrt(d_h) key scaling is folded into the draw,
+                                          so the library is called with k_scale = 1)
+  * gate logits g ~ N(mean, std), fp32  (N(2, 1) for the dense configs, N(0, 2) for varlen)
+  * packed varlen lengths ~ U[lo, hi] (torch.randint, inclusive bounds)
+  * epilogue: x ~ N(0, 1), w_g ~ N(0, 0.02), bf16
+"""
+import math
+
+import torch
+
+_TAGS = {"q": 1, "k": 2, "v": 3, "g": 4, "s": 5, "x": 6, "w": 7, "len": 8, "gnw": 9, "gnb": 10}
+
+
+def _gen(seed, tag, device):
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed) * 1000003 + _TAGS[tag] * 7919)
+    return g
+
+
+def _randn(shape, seed, tag, device, std=1.0, mean=0.0):
+    gen = _gen(seed, tag, device)
+    t = torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+    if std != 1.0:
+        t.mul_(std)
+    if mean != 0.0:
+        t.add_(mean)
+    return t
+
+
+def gret_inputs(B, N, H, dk, dv=None, dtype=torch.bfloat16, g_mean=2.0, g_std=1.0, seed=0,
+                device="cpu", layout="bnhd", with_state=False, state_std=1.0):
+    """q, k [B,N,H,dk] (or [B,H,N,dk] when layout == "bhnd"), v [..,dv], g [B,N,H] fp32.
+
+    Returns a dict with q, k, v, g and, if with_state, an fp32 entry state s [B,H,dk,dv]
+    ~ N(0, state_std)."""
+    dv = dk if dv is None else dv
+    if layout == "bnhd":
+        shq, shv = (B, N, H, dk), (B, N, H, dv)
+    elif layout == "bhnd":
+        shq, shv = (B, H, N, dk), (B, H, N, dv)
+    else:
+        raise ValueError(layout)
+    out = {
+        "q": _randn(shq, seed, "q", device, std=1.0 / math.sqrt(dk)).to(dtype),
+        "k": _randn(shq, seed, "k", device, std=1.0 / math.sqrt(dk)).to(dtype),
+        "v": _randn(shv, seed, "v", device, std=1.0 / math.sqrt(dv)).to(dtype),
+        "g": _randn((B, N, H), seed, "g", device, std=g_std, mean=g_mean),
+    }
+    if with_state:
+        out["s"] = _randn((B, H, dk, dv), seed, "s", device, std=state_std)
+    return out
+
+
+def varlen_lengths(n_seqs, lo, hi, seed):
+    """n_seqs lengths drawn uniformly from [lo, hi] (inclusive), on the CPU."""
+    gen = _gen(seed, "len", "cpu")
+    return [int(x) for x in torch.randint(lo, hi + 1, (n_seqs,), generator=gen)]
+
+
+def cu_seqlens_of(lengths):
+    """Offsets [0, l0, l0+l1, ...] as a Python list."""
+    cu = [0]
+    for n in lengths:
+        cu.append(cu[-1] + int(n))
+    return cu
+
+
+def epilogue_inputs(T, D, F, seed=0, device="cpu", w_std=0.02, affine=False):
+    """x [T,D] ~ N(0,1) and w_g [D,F] ~ N(0, w_std) in bf16; optional GroupNorm affine
+    parameters (fp32, weight ~ 1 + N(0, 0.1), bias ~ N(0, 0.1))."""
+    out = {
+        "x": _randn((T, D), seed, "x", device).to(torch.bfloat16),
+        "w_g": _randn((D, F), seed, "w", device, std=w_std).to(torch.bfloat16),
+    }
+    if affine:
+        out["gn_weight"] = _randn((F,), seed, "gnw", device, std=0.1, mean=1.0)
+        out["gn_bias"] = _randn((F,), seed, "gnb", device, std=0.1)
+    return out
+
+
+# The five workloads, by what they are.
+TINY = dict(B=1, N=512, H=2, dk=64, dtype=torch.float32, g_mean=2.0, g_std=1.0, seed=1,
+            layout="bhnd", chunk=64)
+PREFILL_32K = dict(B=1, N=32768, H=24, dk=128, dtype=torch.bfloat16, g_mean=2.0, g_std=1.0,
+                   seed=2)
+PREFILL_512K = dict(B=1, N=524288, H=24, dk=128, dtype=torch.bfloat16, g_mean=2.0, g_std=1.0,
+                    seed=3)
+DECODE_BS64 = dict(B=64, prefill_N=4096, steps=256, H=24, dk=128, dtype=torch.bfloat16,
+                   g_mean=2.0, g_std=1.0, seed=4)
+VARLEN_EPILOGUE = dict(n_seqs=8, lo=1024, hi=65536, H=24, dk=128, dtype=torch.bfloat16,
+                       g_mean=0.0, g_std=2.0, D=3072, eps=1e-5, seed=5)
