@@ -1,0 +1,178 @@
+"""gated_retention_linear_b200 -- gated retention (the YOCO Self-Decoder mixer) on B200.
+
+A thin Python binding over the C ABI in include/gret.h (libgret.so, built in-tree by
+`python -m gated_retention_linear_b200.build`).  The functions here only marshal arguments:
+they read shapes and strides off torch tensors, allocate outputs and workspaces with torch, pass
+raw device pointers and the current CUDA stream, and raise on a non-OK status.  Every step of
+the computation runs in the library's CUDA kernels; there is no fallback.  If libgret.so is
+missing this import fails.
+"""
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgret.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError("libgret.so not found at %s; build it with "
+                      "`python -m gated_retention_linear_b200.build`" % LIB_PATH)
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+GRET_F32, GRET_BF16 = 0, 1
+STATUS = {0: "GRET_OK", 1: "GRET_ERR_INVALID_ARG", 2: "GRET_ERR_UNSUPPORTED",
+          3: "GRET_ERR_ALIGNMENT", 4: "GRET_ERR_WORKSPACE", 5: "GRET_ERR_CUDA",
+          6: "GRET_ERR_TIMEOUT"}
+
+_vp, _i64, _i32, _f32 = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int, ctypes.c_float
+
+_lib.gret_status_string.argtypes = [_i32]
+_lib.gret_status_string.restype = ctypes.c_char_p
+_lib.gret_prefill_workspace_size.argtypes = [_i32, _i64, _i32, _i32, _i32, _i32, _i32]
+_lib.gret_prefill_workspace_size.restype = ctypes.c_size_t
+_lib.gret_prefill_chunkwise.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _f32, _f32, _i32,
+                                        _i32, _i64, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp,
+                                        _i64, _i64, _i64, _i32, _vp, ctypes.c_size_t, _vp]
+_lib.gret_prefill_chunkwise.restype = _i32
+_lib.gret_workspace_status.argtypes = [_vp, _vp]
+_lib.gret_workspace_status.restype = _i32
+_lib.gret_decode_step.argtypes = [_vp, _vp, _vp, _vp, _f32, _f32, _i32, _i32, _i32, _i32, _i32,
+                                  _vp, _vp, _vp]
+_lib.gret_decode_step.restype = _i32
+_lib.gret_groupnorm_gate.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp,
+                                     _vp]
+_lib.gret_groupnorm_gate.restype = _i32
+
+
+class GretError(RuntimeError):
+    def __init__(self, fn, code):
+        self.code = code
+        super().__init__("%s failed: %s" % (fn, _lib.gret_status_string(code).decode()))
+
+
+def _check(fn, code):
+    if code != 0:
+        raise GretError(fn, code)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return GRET_BF16
+    if t.dtype == torch.float32:
+        return GRET_F32
+    raise TypeError("q/k/v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def gret_status_string(code):
+    return _lib.gret_status_string(int(code)).decode()
+
+
+def gret_prefill_workspace_size(dtype, total_tokens, n_seqs, H, d_k, d_v, chunk=0):
+    code = dtype if isinstance(dtype, int) else _dtype_code(torch.empty(0, dtype=dtype))
+    return int(_lib.gret_prefill_workspace_size(code, total_tokens, n_seqs, H, d_k, d_v, chunk))
+
+
+def _layout(t, head_major):
+    """(stride_batch, stride_tok, stride_head) of a 4-D [B,N,H,d] or [B,H,N,d] tensor, or of a
+    3-D packed [T,H,d] tensor (stride_batch = 0)."""
+    if t.stride(-1) != 1:
+        raise ValueError("last dimension must be contiguous")
+    if t.dim() == 3:
+        return 0, t.stride(0), t.stride(1)
+    if head_major:
+        return t.stride(0), t.stride(2), t.stride(1)
+    return t.stride(0), t.stride(1), t.stride(2)
+
+
+def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None,
+                           state_out=None, o=None, chunk=0, head_major=False, workspace=None,
+                           stream=None):
+    """Chunkwise gated-retention prefill through the C ABI.
+
+    q, k [B,N,H,dk] (head_major=False) or [B,H,N,dk] (head_major=True); v likewise with dv;
+    packed varlen: q, k, v [T,H,d] with cu_seqlens int32 [n_seqs+1] on the device.
+    g fp32 [B,N,H] or [T,H].  state_in / state_out fp32 [units,H,dk,dv] (state_out=True
+    allocates one).  Returns (o, state_out)."""
+    if k.stride() != q.stride() or v.stride()[:-1] != q.stride()[:-1]:
+        raise ValueError("q, k and v must share strides")
+    if q.dim() == 3:
+        B, (N, H, dk) = 1, q.shape
+    elif head_major:
+        B, H, N, dk = q.shape
+    else:
+        B, N, H, dk = q.shape
+    dv = v.shape[-1]
+    sb, st, sh = _layout(q, head_major)
+    if o is None:
+        o = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
+    osb, ost, osh = _layout(o, head_major)
+    if not g.is_contiguous() or g.dtype != torch.float32:
+        raise ValueError("g must be contiguous fp32")
+    n_seqs = 0
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1:
+            raise ValueError("cu_seqlens must be 1-D int32")
+        n_seqs = cu_seqlens.numel() - 1
+    units = n_seqs if cu_seqlens is not None else B
+    if state_out is True:
+        state_out = torch.empty((units, H, dk, dv), dtype=torch.float32, device=q.device)
+    code = _dtype_code(q)
+    total = N if cu_seqlens is not None else B * N
+    need = int(_lib.gret_prefill_workspace_size(code, total, units, H, dk, dv, chunk))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
+    wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check("gret_prefill_chunkwise", _lib.gret_prefill_chunkwise(
+        _ptr(q), _ptr(k), _ptr(v), sb, st, sh, _ptr(g), tau, k_scale, code, B, N, H, dk, dv,
+        _ptr(cu_seqlens), n_seqs, _ptr(state_in), _ptr(state_out), _ptr(o), osb, ost, osh,
+        chunk, _ptr(workspace), wbytes, _stream(stream)))
+    return o, state_out
+
+
+def gret_workspace_status(workspace, stream=None):
+    """Synchronise and return the status word of a prefill workspace (0 = OK)."""
+    return int(_lib.gret_workspace_status(_ptr(workspace), _stream(stream)))
+
+
+def gret_decode_step(q, k, v, g, state, tau=16.0, k_scale=1.0, o=None, stream=None):
+    """One decode step: q, k [B,H,dk], v [B,H,dv], g fp32 [B,H], state fp32 [B,H,dk,dv]
+    updated in place.  Returns o [B,H,dv]."""
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    for t in (q, k, v, g, state):
+        if not t.is_contiguous():
+            raise ValueError("decode tensors must be contiguous")
+    if o is None:
+        o = torch.empty((B, H, dv), dtype=q.dtype, device=q.device)
+    _check("gret_decode_step", _lib.gret_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), tau, k_scale, _dtype_code(q), B, H, dk, dv,
+        _ptr(state), _ptr(o), _stream(stream)))
+    return o
+
+
+def gret_groupnorm_gate(o, x, w_g, H, gn_weight=None, gn_bias=None, eps=1e-5, y=None,
+                        stream=None):
+    """y = GroupNorm_per_head(o) * swish(x @ w_g); o [T,H*dv], x [T,D], w_g [D,H*dv], bf16."""
+    T, F = o.shape
+    D = x.shape[1]
+    for t in (o, x, w_g):
+        if not t.is_contiguous() or t.dtype != torch.bfloat16:
+            raise ValueError("o, x, w_g must be contiguous bf16")
+    if y is None:
+        y = torch.empty((T, F), dtype=torch.bfloat16, device=o.device)
+    _check("gret_groupnorm_gate", _lib.gret_groupnorm_gate(
+        _ptr(o), _ptr(x), _ptr(w_g), _ptr(gn_weight), _ptr(gn_bias), eps, T, H, F // H, D,
+        _ptr(y), _stream(stream)))
+    return y

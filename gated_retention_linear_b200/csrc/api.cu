@@ -1,0 +1,154 @@
+// api.cu -- the C ABI declared in include/gret.h: argument checks, path choice, launches.
+//
+// Every check runs on the host before anything is launched, so a rejected call has no effect
+// on the device.  No entry point allocates device memory.
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "prefill_tc.cuh"
+#include "gn_gate.cuh"
+
+using namespace gret;
+
+namespace {
+
+bool dim_ok(int d) { return d == 64 || d == 128; }
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Which prefill kernel serves a call.
+enum class Path { Simt, TensorCore };
+
+Path choose_path(gret_dtype_t dtype, int dk, int dv, int chunk) {
+    if (dtype == GRET_BF16 && dk == 128 && dv == 128 && chunk == TC_CHUNK)
+        return Path::TensorCore;
+    return Path::Simt;
+}
+
+int default_simt_chunk() { return 64; }
+
+}  // namespace
+
+extern "C" {
+
+const char* gret_status_string(gret_status_t s) {
+    switch (s) {
+        case GRET_OK: return "GRET_OK";
+        case GRET_ERR_INVALID_ARG: return "GRET_ERR_INVALID_ARG: argument out of range";
+        case GRET_ERR_UNSUPPORTED: return "GRET_ERR_UNSUPPORTED: no kernel for this combination";
+        case GRET_ERR_ALIGNMENT: return "GRET_ERR_ALIGNMENT: pointer or stride not 16-byte aligned";
+        case GRET_ERR_WORKSPACE: return "GRET_ERR_WORKSPACE: workspace missing or too small";
+        case GRET_ERR_CUDA: return "GRET_ERR_CUDA: a CUDA runtime call failed";
+        case GRET_ERR_TIMEOUT: return "GRET_ERR_TIMEOUT: a bounded inter-block wait gave up";
+    }
+    return "GRET_ERR_UNKNOWN";
+}
+
+size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int n_seqs, int H,
+                                   int d_k, int d_v, int chunk) {
+    if (total_tokens < 0 || n_seqs < 0 || H < 0 || !dim_ok(d_k) || !dim_ok(d_v)) return 0;
+    if (choose_path(dtype, d_k, d_v, chunk) == Path::TensorCore)
+        return tc_workspace_size(total_tokens, n_seqs, H);
+    return 0;
+}
+
+gret_status_t gret_prefill_chunkwise(const void* q, const void* k, const void* v,
+                                     int64_t stride_batch, int64_t stride_tok,
+                                     int64_t stride_head, const float* g, float tau,
+                                     float k_scale, gret_dtype_t dtype, int B, int64_t N, int H,
+                                     int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
+                                     const float* state_in, float* state_out, void* o,
+                                     int64_t o_stride_batch, int64_t o_stride_tok,
+                                     int64_t o_stride_head, int chunk, void* workspace,
+                                     size_t workspace_bytes, gret_stream_t stream) {
+    if (dtype != GRET_F32 && dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
+    if (!dim_ok(d_k) || !dim_ok(d_v) || H < 1 || B < 0 || N < 0) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
+    if (stride_batch < 0 || stride_tok < 0 || stride_head < 0 || o_stride_batch < 0 ||
+        o_stride_tok < 0 || o_stride_head < 0)
+        return GRET_ERR_INVALID_ARG;
+    int units;
+    if (cu_seqlens) {
+        if (B != 1 || n_seqs < 0) return GRET_ERR_INVALID_ARG;
+        units = n_seqs;
+    } else {
+        units = B;
+    }
+    if (units > 65535 && choose_path(dtype, d_k, d_v, chunk) == Path::Simt)
+        return GRET_ERR_UNSUPPORTED;
+    const int64_t tokens = cu_seqlens ? N : (int64_t)B * N;
+    if (units == 0) return GRET_OK;
+    if (tokens > 0 && (!q || !k || !v || !g || !o)) return GRET_ERR_INVALID_ARG;
+
+    PrefillArgs a;
+    a.q = q; a.k = k; a.v = v;
+    a.sb = stride_batch; a.st = stride_tok; a.sh = stride_head;
+    a.g = g; a.tau = tau; a.k_scale = k_scale;
+    a.B = cu_seqlens ? 1 : B; a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
+    a.cu_seqlens = cu_seqlens; a.n_seqs = units;
+    a.state_in = state_in; a.state_out = state_out;
+    a.o = o; a.osb = o_stride_batch; a.ost = o_stride_tok; a.osh = o_stride_head;
+    a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+    a.stream = (cudaStream_t)stream;
+
+    if (choose_path(dtype, d_k, d_v, chunk) == Path::TensorCore) {
+        a.chunk = TC_CHUNK;
+        const size_t need = tc_workspace_size(tokens, units, H);
+        if (!workspace || workspace_bytes < need) return GRET_ERR_WORKSPACE;
+        if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_ALIGNMENT;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
+            return GRET_ERR_ALIGNMENT;
+        if ((stride_batch % 8) || (stride_tok % 8) || (stride_head % 8) || (o_stride_batch % 8) ||
+            (o_stride_tok % 8) || (o_stride_head % 8))
+            return GRET_ERR_ALIGNMENT;
+        gret_status_t st = launch_prefill_tc(a);
+        return st;
+    }
+    a.chunk = chunk == 0 ? default_simt_chunk() : chunk;
+    if (a.chunk != 16 && a.chunk != 32 && a.chunk != 64) return GRET_ERR_UNSUPPORTED;
+    if (tokens == 0 && !state_out) return GRET_OK;
+    cudaError_t e = launch_prefill_simt(a, dtype == GRET_BF16);
+    if (e == cudaErrorInvalidValue) return GRET_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status_t gret_workspace_status(const void* workspace, gret_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GRET_ERR_CUDA;
+    if (!workspace) return GRET_OK;
+    uint32_t word = 0;
+    if (cudaMemcpy(&word, workspace, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+        return GRET_ERR_CUDA;
+    return word == WS_ERR_NONE ? GRET_OK : GRET_ERR_TIMEOUT;
+}
+
+gret_status_t gret_decode_step(const void* q, const void* k, const void* v, const float* g,
+                               float tau, float k_scale, gret_dtype_t dtype, int B, int H,
+                               int d_k, int d_v, float* state, void* o, gret_stream_t stream) {
+    if (dtype != GRET_F32 && dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
+    if (!dim_ok(d_k) || !dim_ok(d_v) || B < 0 || H < 0) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
+    if ((int64_t)B * H == 0) return GRET_OK;
+    if ((int64_t)B * H > 0x7fffffffLL) return GRET_ERR_INVALID_ARG;
+    if (!q || !k || !v || !g || !state || !o) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(state)) return GRET_ERR_ALIGNMENT;
+    cudaError_t e = launch_decode(q, k, v, g, tau, k_scale, dtype == GRET_BF16, B, H, d_k, d_v,
+                                  state, o, (cudaStream_t)stream);
+    if (e == cudaErrorInvalidValue) return GRET_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status_t gret_groupnorm_gate(const void* o, const void* x, const void* w_g,
+                                  const float* gn_weight, const float* gn_bias, float eps,
+                                  int64_t T, int H, int d_v, int D, void* y,
+                                  gret_stream_t stream) {
+    if (T < 0 || H < 1 || D < 1 || !(eps >= 0.f) || !isfinite(eps)) return GRET_ERR_INVALID_ARG;
+    if (d_v != 128 || D % 64 != 0) return GRET_ERR_UNSUPPORTED;
+    if (T == 0) return GRET_OK;
+    if (!o || !x || !w_g || !y) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(x) || !aligned16(w_g) || !aligned16(y))
+        return GRET_ERR_ALIGNMENT;
+    return launch_gn_gate(o, x, w_g, gn_weight, gn_bias, eps, T, H, d_v, D, y,
+                          (cudaStream_t)stream);
+}
+
+}  // extern "C"

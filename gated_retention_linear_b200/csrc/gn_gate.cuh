@@ -1,0 +1,11 @@
+// gn_gate.cuh -- host interface of the GroupNorm * swish(X W_G) epilogue kernel.
+#pragma once
+#include "common.cuh"
+
+namespace gret {
+
+gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g,
+                             const float* gn_weight, const float* gn_bias, float eps, int64_t T,
+                             int H, int d_v, int D, void* y, cudaStream_t stream);
+
+}  // namespace gret

@@ -1,0 +1,145 @@
+/*
+ * gret.h -- C ABI of the gated-retention (gRet) library for NVIDIA B200 (sm_100a).
+ *
+ * Gated retention is the Self-Decoder mixer of YOCO.  Definitions follow the page
+ * "YOCO 完全拆解：Decoder-Decoder 架构如何让 KV Cache 只存一次" (pinghaoyang.com.cn/aigc/posts/yoco/):
+ *   section "路线二：Multi-Head Gated Retention"         -- gate, recurrence, GroupNorm + swish gate
+ *   section "Prefill 与 Decode 为什么使用两种计算形态"   -- chunkwise prefill form
+ *   section "单 token Decode 的实现骨架"                  -- the decode state update
+ *
+ * Per sequence and head, with row vectors q_t, k_t [1 x d_k], v_t [1 x d_v] and state S [d_k x d_v]:
+ *   log(gamma_t) = logsigmoid(g_t) / tau          (gamma = sigmoid(g)^(1/tau); g is the gate logit)
+ *   S_t = gamma_t S_{t-1} + (k_scale k_t)^T v_t   (decay the old state, then add the current token)
+ *   o_t = q_t S_t                                 (the output reads the updated state)
+ *
+ * Conventions shared by every entry point
+ *   - All data pointers are DEVICE pointers owned by the caller.  The library keeps no pointer
+ *     after a call returns and allocates no device memory.
+ *   - Every call is asynchronous on `stream` (0 = legacy default stream).
+ *   - Argument errors are detected on the host and returned before anything is launched.
+ *     A launch failure returns GRET_ERR_CUDA.  Faults of earlier asynchronous work surface on a
+ *     later call or on stream synchronisation, as usual in CUDA.
+ *   - Strides are in ELEMENTS; the last dimension of every tensor is contiguous.
+ *   - Gate logits must be finite (|g| <= 1e30 is fine; +-inf and NaN give undefined results).
+ *   - State tensors are fp32, [units, H, d_k, d_v], row-major (d_v contiguous).
+ */
+#ifndef GRET_H
+#define GRET_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* gret_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+    GRET_OK = 0,
+    GRET_ERR_INVALID_ARG = 1,  /* a size, pointer or stride is out of the documented range   */
+    GRET_ERR_UNSUPPORTED = 2,  /* a valid combination this build has no kernel for          */
+    GRET_ERR_ALIGNMENT = 3,    /* a pointer or stride breaks the 16-byte alignment rule      */
+    GRET_ERR_WORKSPACE = 4,    /* workspace NULL or smaller than gret_prefill_workspace_size */
+    GRET_ERR_CUDA = 5,         /* a CUDA runtime call failed (launch or attribute setup)     */
+    GRET_ERR_TIMEOUT = 6       /* a bounded inter-block wait gave up; results are invalid    */
+} gret_status_t;
+
+typedef enum { GRET_F32 = 0, GRET_BF16 = 1 } gret_dtype_t;
+
+/* Static string naming a status code.  Never NULL. */
+const char* gret_status_string(gret_status_t status);
+
+/*
+ * Bytes of device workspace gret_prefill_chunkwise needs for these sizes (0 is a valid answer
+ * only when nothing is launched).  `total_tokens` is B*N in dense mode and the packed token
+ * count in varlen mode; `n_seqs` is B in dense mode.  `chunk` as passed to the prefill call.
+ * Returns 0 and sets nothing on invalid sizes; callers pass the result through unchanged.
+ */
+size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int n_seqs, int H,
+                                   int d_k, int d_v, int chunk);
+
+/*
+ * Chunkwise prefill ("Prefill 与 Decode 为什么使用两种计算形态").  Tokens are cut into chunks of
+ * `chunk` positions that never straddle a sequence; within a chunk [a, b], with the in-chunk
+ * cumulative log-decay c_t = sum_{k=a..t} log(gamma_k) and the entry state S_{a-1}:
+ *   o_t = sum_{m=a..t} exp(c_t - c_m) (q_t . k_m) v_m  +  exp(c_t) q_t S_{a-1}
+ *   S_b = exp(c_b) S_{a-1} + sum_{m=a..b} exp(c_b - c_m) k_m^T v_m
+ * which equals the recurrence above up to rounding.  The last chunk of a sequence may be
+ * shorter; nothing needs padding.
+ *
+ *   q, k     [.., token, head, d_k] in `dtype`; element (b, t, h, i) at
+ *            b*stride_batch + t*stride_tok + h*stride_head + i.  Read only.
+ *   v        same strides, last dim d_v.  Read only.
+ *   g        fp32 gate logits, contiguous [B, N, H] (dense) or [total_tokens, H] (varlen).
+ *   tau      temperature (> 0); k_scale multiplies every key (e.g. d_k^-1/2, or 1.0).
+ *   dtype    GRET_BF16 (tensor-core path when d_k == d_v == 128, else a CUDA-core path with
+ *            fp32 accumulation) or GRET_F32 (CUDA-core path, full fp32 arithmetic).
+ *   B, N     dense mode: B sequences of N tokens each.
+ *   cu_seqlens  NULL for dense mode.  Varlen mode: device int32 [n_seqs + 1], non-decreasing,
+ *            cu_seqlens[0] == 0, cu_seqlens[n_seqs] == N; requires B == 1, tokens packed.
+ *            Empty sequences are allowed (their state passes through).
+ *   H, d_k, d_v  heads and head widths; d_k, d_v in {64, 128}.
+ *   state_in   fp32 [units, H, d_k, d_v] entry states, units = B (dense) or n_seqs (varlen);
+ *              NULL means zero.  Read only.
+ *   state_out  fp32, same shape; the state after each sequence's last token.  NULL skips it.
+ *              May alias state_in exactly (then it is read before it is overwritten).
+ *   o        output, same dtype as q, [.., token, head, d_v] with its own strides
+ *            (o_stride_batch, o_stride_tok, o_stride_head).  Must not overlap the inputs.
+ *   chunk    0 picks the tuned default; otherwise 16, 32 or 64 (CUDA-core path) or 128
+ *            (tensor-core path).  Other values return GRET_ERR_UNSUPPORTED.
+ *   workspace  device scratch of at least gret_prefill_workspace_size() bytes, 256-byte
+ *            aligned, owned by the caller; its contents need no initialisation and are
+ *            garbage afterwards.  Concurrent calls need separate workspaces.
+ * Alignment: for the tensor-core path, q/k/v/o base pointers must be 16-byte aligned and every
+ * stride (times 2 bytes) a multiple of 16 bytes; otherwise GRET_ERR_ALIGNMENT.
+ * A bounded wait between thread blocks that gives up sets an error word in the workspace;
+ * read it with gret_workspace_status() after the stream has synchronised.
+ */
+gret_status_t gret_prefill_chunkwise(
+    const void* q, const void* k, const void* v, int64_t stride_batch, int64_t stride_tok,
+    int64_t stride_head, const float* g, float tau, float k_scale, gret_dtype_t dtype, int B,
+    int64_t N, int H, int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
+    const float* state_in, float* state_out, void* o, int64_t o_stride_batch,
+    int64_t o_stride_tok, int64_t o_stride_head, int chunk, void* workspace,
+    size_t workspace_bytes, gret_stream_t stream);
+
+/*
+ * Synchronises `stream`, then reads the error word that gret_prefill_chunkwise keeps at the
+ * start of `workspace`.  Returns GRET_OK, GRET_ERR_TIMEOUT, or GRET_ERR_CUDA if the copy or the
+ * synchronisation failed.  Blocking; not for use inside stream capture.
+ */
+gret_status_t gret_workspace_status(const void* workspace, gret_stream_t stream);
+
+/*
+ * One recurrent decode step for a batch ("单 token Decode 的实现骨架"): for every (b, h)
+ *   S <- gamma S + (k_scale k)^T v ;  o = q S
+ *   q, k   [B, H, d_k] contiguous, `dtype`;   v [B, H, d_v];   g fp32 [B, H] gate logits.
+ *   state  fp32 [B, H, d_k, d_v], updated IN PLACE; 16-byte aligned.
+ *   o      [B, H, d_v] in `dtype`; must not overlap state or inputs.
+ * d_k, d_v in {64, 128}.  Memory-bound: the state is read and written once.
+ */
+gret_status_t gret_decode_step(const void* q, const void* k, const void* v, const float* g,
+                               float tau, float k_scale, gret_dtype_t dtype, int B, int H,
+                               int d_k, int d_v, float* state, void* o, gret_stream_t stream);
+
+/*
+ * Output epilogue ("路线二：Multi-Head Gated Retention"): per-head GroupNorm of the retention
+ * output times swish(X W_G):
+ *   z = X_t W_G ;  y_t[h*d_v + j] = GN_h(o_t)[j] * z[h*d_v + j] * sigmoid(z[h*d_v + j])
+ *   GN_h: mean and biased variance of o_t[h*d_v .. h*d_v + d_v - 1], (x - mean)/sqrt(var + eps),
+ *         then * gn_weight + gn_bias per channel (each may be NULL = identity).
+ *   o    bf16 [T, H*d_v] row-major;  x bf16 [T, D] row-major;  w_g bf16 [D, H*d_v] row-major.
+ *   gn_weight, gn_bias  fp32 [H*d_v] or NULL.      y  bf16 [T, H*d_v], must not overlap inputs.
+ * Requires d_v == 128, D a positive multiple of 64, T >= 0; pointers 16-byte aligned.
+ */
+gret_status_t gret_groupnorm_gate(const void* o, const void* x, const void* w_g,
+                                  const float* gn_weight, const float* gn_bias, float eps,
+                                  int64_t T, int H, int d_v, int D, void* y,
+                                  gret_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GRET_H */
