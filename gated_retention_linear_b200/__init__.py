@@ -32,7 +32,8 @@ _lib.gret_status_string.argtypes = [_i32]
 _lib.gret_status_string.restype = ctypes.c_char_p
 _lib.gret_prefill_workspace_size.argtypes = [_i32, _i64, _i32, _i32, _i32, _i32, _i32]
 _lib.gret_prefill_workspace_size.restype = ctypes.c_size_t
-_lib.gret_prefill_chunkwise.argtypes = [_vp, _vp, _vp, _i64, _i64, _i64, _vp, _f32, _f32, _i32,
+_lib.gret_prefill_chunkwise.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64, _vp,
+                                        _f32, _f32, _i32,
                                         _i32, _i64, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp,
                                         _i64, _i64, _i64, _i32, _vp, ctypes.c_size_t, _vp]
 _lib.gret_prefill_chunkwise.restype = _i32
@@ -105,8 +106,8 @@ def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, s
     packed varlen: q, k, v [T,H,d] with cu_seqlens int32 [n_seqs+1] on the device.
     g fp32 [B,N,H] or [T,H].  state_in / state_out fp32 [units,H,dk,dv] (state_out=True
     allocates one).  Returns (o, state_out)."""
-    if k.stride() != q.stride() or v.stride()[:-1] != q.stride()[:-1]:
-        raise ValueError("q, k and v must share strides")
+    if k.stride() != q.stride():
+        raise ValueError("q and k must share strides")
     if q.dim() == 3:
         B, (N, H, dk) = 1, q.shape
     elif head_major:
@@ -115,6 +116,7 @@ def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, s
         B, N, H, dk = q.shape
     dv = v.shape[-1]
     sb, st, sh = _layout(q, head_major)
+    vsb, vst, vsh = _layout(v, head_major)
     if o is None:
         o = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
     osb, ost, osh = _layout(o, head_major)
@@ -135,7 +137,8 @@ def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, s
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("gret_prefill_chunkwise", _lib.gret_prefill_chunkwise(
-        _ptr(q), _ptr(k), _ptr(v), sb, st, sh, _ptr(g), tau, k_scale, code, B, N, H, dk, dv,
+        _ptr(q), _ptr(k), sb, st, sh, _ptr(v), vsb, vst, vsh, _ptr(g), tau, k_scale, code, B,
+        N, H, dk, dv,
         _ptr(cu_seqlens), n_seqs, _ptr(state_in), _ptr(state_out), _ptr(o), osb, ost, osh,
         chunk, _ptr(workspace), wbytes, _stream(stream)))
     return o, state_out

@@ -20,7 +20,7 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 enum class Path { Simt, TensorCore };
 
 Path choose_path(gret_dtype_t dtype, int dk, int dv, int chunk) {
-    if (dtype == GRET_BF16 && dk == 128 && dv == 128 && chunk == TC_CHUNK)
+    if (dtype == GRET_BF16 && dk == 128 && dv == 128 && (chunk == 0 || chunk == TC_CHUNK))
         return Path::TensorCore;
     return Path::Simt;
 }
@@ -52,9 +52,10 @@ size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int
     return 0;
 }
 
-gret_status_t gret_prefill_chunkwise(const void* q, const void* k, const void* v,
-                                     int64_t stride_batch, int64_t stride_tok,
-                                     int64_t stride_head, const float* g, float tau,
+gret_status_t gret_prefill_chunkwise(const void* q, const void* k, int64_t stride_batch,
+                                     int64_t stride_tok, int64_t stride_head, const void* v,
+                                     int64_t v_stride_batch, int64_t v_stride_tok,
+                                     int64_t v_stride_head, const float* g, float tau,
                                      float k_scale, gret_dtype_t dtype, int B, int64_t N, int H,
                                      int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
                                      const float* state_in, float* state_out, void* o,
@@ -64,8 +65,9 @@ gret_status_t gret_prefill_chunkwise(const void* q, const void* k, const void* v
     if (dtype != GRET_F32 && dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
     if (!dim_ok(d_k) || !dim_ok(d_v) || H < 1 || B < 0 || N < 0) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
-    if (stride_batch < 0 || stride_tok < 0 || stride_head < 0 || o_stride_batch < 0 ||
-        o_stride_tok < 0 || o_stride_head < 0)
+    if (stride_batch < 0 || stride_tok < 0 || stride_head < 0 || v_stride_batch < 0 ||
+        v_stride_tok < 0 || v_stride_head < 0 || o_stride_batch < 0 || o_stride_tok < 0 ||
+        o_stride_head < 0)
         return GRET_ERR_INVALID_ARG;
     int units;
     if (cu_seqlens) {
@@ -83,6 +85,7 @@ gret_status_t gret_prefill_chunkwise(const void* q, const void* k, const void* v
     PrefillArgs a;
     a.q = q; a.k = k; a.v = v;
     a.sb = stride_batch; a.st = stride_tok; a.sh = stride_head;
+    a.vsb = v_stride_batch; a.vst = v_stride_tok; a.vsh = v_stride_head;
     a.g = g; a.tau = tau; a.k_scale = k_scale;
     a.B = cu_seqlens ? 1 : B; a.N = N; a.H = H; a.dk = d_k; a.dv = d_v;
     a.cu_seqlens = cu_seqlens; a.n_seqs = units;
@@ -98,8 +101,9 @@ gret_status_t gret_prefill_chunkwise(const void* q, const void* k, const void* v
         if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return GRET_ERR_ALIGNMENT;
         if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o))
             return GRET_ERR_ALIGNMENT;
-        if ((stride_batch % 8) || (stride_tok % 8) || (stride_head % 8) || (o_stride_batch % 8) ||
-            (o_stride_tok % 8) || (o_stride_head % 8))
+        if ((stride_batch % 8) || (stride_tok % 8) || (stride_head % 8) ||
+            (v_stride_batch % 8) || (v_stride_tok % 8) || (v_stride_head % 8) ||
+            (o_stride_batch % 8) || (o_stride_tok % 8) || (o_stride_head % 8))
             return GRET_ERR_ALIGNMENT;
         gret_status_t st = launch_prefill_tc(a);
         return st;

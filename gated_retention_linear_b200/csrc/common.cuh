@@ -45,7 +45,8 @@ struct PrefillArgs {
     const void* q;
     const void* k;
     const void* v;
-    int64_t sb, st, sh;     // q/k/v strides (elements)
+    int64_t sb, st, sh;     // q/k strides (elements)
+    int64_t vsb, vst, vsh;  // v strides (elements)
     const float* g;
     float tau, k_scale;
     int B;

@@ -47,7 +47,7 @@ __global__ void __launch_bounds__(256) prefill_simt_kernel(PrefillArgs p) {
     }
     const T* Q = (const T*)p.q + b * p.sb + h * p.sh;
     const T* K = (const T*)p.k + b * p.sb + h * p.sh;
-    const T* V = (const T*)p.v + b * p.sb + h * p.sh;
+    const T* V = (const T*)p.v + b * p.vsb + h * p.vsh;
     T* O = (T*)p.o + b * p.osb + h * p.osh;
     const float* G = p.g + (b * p.N) * p.H + h;
     const int64_t sidx = ((int64_t)unit * p.H + h) * DK * DV;
@@ -72,7 +72,7 @@ __global__ void __launch_bounds__(256) prefill_simt_kernel(PrefillArgs p) {
         for (int e = tid; e < C * DV; e += 256) {
             int r = e / DV, j = e % DV;
             int64_t t = t0 + a0 + r;
-            sm.v[r][j] = (r < n) ? to_f32(V[t * p.st + j]) : 0.f;
+            sm.v[r][j] = (r < n) ? to_f32(V[t * p.vst + j]) : 0.f;
         }
         if (tid < C) sm.c[tid] = (tid < n) ? logsigmoidf_(G[(t0 + a0 + tid) * p.H]) / p.tau : 0.f;
         __syncthreads();

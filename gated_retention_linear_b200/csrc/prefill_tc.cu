@@ -1,9 +1,992 @@
-// prefill_tc.cu -- tensor-core chunkwise prefill (placeholder until the tcgen05 kernel lands).
+// prefill_tc.cu -- chunkwise gated-retention prefill on the sm_100a tensor cores.
+//
+// Method: page "YOCO 完全拆解：Decoder-Decoder 架构如何让 KV Cache 只存一次", section
+// "Prefill 与 Decode 为什么使用两种计算形态".  Each chunk of C = 128 tokens of one head is done
+// with four 128x128x128 bf16 tcgen05 MMAs accumulating in fp32 tensor memory:
+//     A   = Q K^T                       (intra-chunk scores)
+//     P   = k_scale * exp(c_t - c_m) * A for m <= t, else 0     (decay mask, CUDA cores, bf16)
+//     O   = P V                         (inner term)
+//     OX  = Q S_prev                    (cross-chunk term; added as exp(c_t) * OX)
+//     dS  = (w K)^T V,  w_m = k_scale * exp(c_b - c_m)     (chunk contribution to the state)
+//     S   = exp(c_b) S_prev + dS        (fp32 master state, in registers)
+// c_t is the in-chunk inclusive cumulative log-decay (a warp-shuffle scan of logsigmoid(g)/tau),
+// always used as a difference inside one chunk, so no exponent can overflow.
+//
+// Parallelism across a sequence.  The chunk chain of one (sequence, head) is sequential, and
+// one 3B-shaped layer has only 24 chains for 148 SMs.  Each chain is therefore cut into spans
+// of G chunks.  A persistent CTA takes spans from an atomic ticket in chain order and runs:
+//   pass A: read K, V, g of the span and fold them into the span's aggregate state
+//           Agg = sum over chunks (decay to the span end) of dS        (MMA dS only)
+//   look-back: wait for the inclusive state of span s-1 of the same chain (a bounded spin on a
+//           flag in the workspace), entry E = that state (or state_in for s = 0), and publish
+//           the inclusive state exp(L_span) E + Agg for span s+1;
+//   pass B: the full chunk pipeline above from E, writing O.
+// The K and V of a span are read from HBM by pass A and again by pass B shortly after, from L2.
+// Inclusive states live in a two-slot ring per chain: span s+2 can only overwrite the slot of
+// span s after span s+1 has consumed it, because it needs span s+1's own inclusive state first.
+// Tickets are taken by running CTAs in increasing order and every span depends only on a smaller
+// ticket, so the chain always progresses.
+//
+// Warp roles (384 threads = 3 warpgroups, one CTA per SM):
+//   warp 0      TMA producer: K, V (and Q in pass B) tiles, two pipeline stages
+//   warp 1      tcgen05 MMA issuer (one thread); owns the 512-column TMEM allocation
+//   warps 2-3   idle (they complete the first warpgroup, whose registers are given away)
+//   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16) and the output
+//               epilogue O + exp(c_t) OX -> bf16 -> global
+//   warps 8-11  "state group": row scaling of K, the fp32 state (one row per thread), the
+//               look-back, and the bf16 copy of the state that the next Q S_prev MMA reads
+// Registers: launched at 168 per thread; the first warpgroup drops to 56, the P group rises to
+// 184 and the state group (128 fp32 state values per thread) to 232: 128 x (56 + 184 + 232)
+// = 60416 <= 384 x 158, so the split fits any launch allocation of at least 158 per thread,
+// and each SM sub-partition (one warp of each group) needs 32 x 472 <= 16384 registers.
+// TMEM columns: [0,128) A / P, [128,256) O, [256,384) OX, [384,512) dS.
+// Every wait is bounded (see sm100::mbar_wait); a wait that gives up records GRET_ERR_TIMEOUT in
+// the workspace, and the kernel drains its copies, frees TMEM and exits.
 #include "prefill_tc.cuh"
+
+#include <stdlib.h>
+
+#include <algorithm>
+
+#include "sm100.cuh"
+#include "tma_host.cuh"
 
 namespace gret {
 
-size_t tc_workspace_size(int64_t, int, int) { return 256; }
-gret_status_t launch_prefill_tc(const PrefillArgs&) { return GRET_ERR_UNSUPPORTED; }
+using namespace sm100;
+
+namespace {
+
+constexpr int C = 128;                  // tokens per chunk
+constexpr int D = 128;                  // head width (d_k = d_v)
+constexpr int TILE = C * D * 2;         // one bf16 128x128 tile
+constexpr int SLAB = TILE / 2;          // one 64-column slab
+constexpr int NTHREADS = 384;
+constexpr int ITEM_DEPTH = 4;
+constexpr uint64_t WAIT_NS = 2000000000ull;   // a wait gives up after 2 s
+constexpr uint64_t DRAIN_NS = 200000000ull;   // exit-time drains give up after 0.2 s
+
+constexpr uint32_t TM_A = 0, TM_O = 128, TM_OX = 256, TM_DS = 384;
+
+struct Item {
+    int32_t valid;
+    int32_t u, h, s;
+    int32_t c_begin, c_end;   // chunk range of the span, in chunks of the unit
+    int32_t first, last;      // first / last span of the chain
+    int32_t b;                // batch coordinate (dense) or 0
+    int32_t pad;
+    int64_t len;              // tokens in the unit
+    int64_t tok_first;        // token coordinate of the unit's first token
+    int64_t grow0;            // row of the unit's first token in g
+};
+
+struct __align__(1024) Smem {
+    unsigned char q[2][TILE];
+    unsigned char k[2][TILE];
+    unsigned char v[2][TILE];
+    unsigned char sbf[TILE];   // bf16 copy of the entry state for the Q S_prev MMA
+    uint64_t kv_full[2], stage_empty[2];
+    uint64_t item_full[ITEM_DEPTH], item_empty[ITEM_DEPTH];
+    uint64_t a_full, q16_ready, p_ready, o_full, o_free, v16_ready, k_ready, ds_full, ds_free,
+        s_ready, drain;
+    Item items[ITEM_DEPTH];
+    float cP[C];               // P group: in-chunk cumulative log2-decay of each token
+    float wsum[2][4];          // warp totals of the two scans (P group, state group)
+    float red[2][4];           // warp maxima of the tile-scale reductions
+    float sig_v[2];            // power-of-two scale of the fp16 V tile, by job parity
+    float sig_s[2];            // power-of-two scale of the fp16 entry state, by pass-B chunk parity
+    uint32_t dec[2][2];        // group-uniform wait decisions (double-buffered)
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+
+struct TcParams {
+    const float* g;
+    float inv_tau_log2e;       // log2(e) / tau
+    float k_scale;
+    __nv_bfloat16* o;
+    int64_t osb, ost, osh;
+    const float* state_in;
+    float* state_out;
+    uint32_t* err;
+    uint32_t* ticket;
+    uint32_t* flags;           // [units][H][2]
+    int32_t* prefix;           // varlen: [units + 1] span prefix; nullptr in dense mode
+    float* slots;              // [units][H][2][128*128] inclusive states
+    const int32_t* cu_seqlens;
+    int64_t N;                 // dense: tokens per sequence
+    int H, units, G;
+    int spans_per_unit;        // dense
+    int qk_pos_tok, qk_pos_head, qk_pos_b;   // tensor-map dimension of each coordinate
+    int v_pos_tok, v_pos_head, v_pos_b;
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ float logsigmoid_(float x) {
+    return fminf(x, 0.f) - log1pf(expf(-fabsf(x)));
+}
+
+__device__ __forceinline__ void named_sync(int id) {
+    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+}
+
+__device__ __forceinline__ void set_error(uint32_t* err) { atomicExch(err, WS_ERR_TIMEOUT); }
+
+// Exit-time wait for this CTA's own asynchronous work; bounded, and not cut short by an abort.
+__device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    uint32_t never = 0;
+    mbar_wait(bar, parity, &never, limit_ns);
+}
+
+// A wait taken by one thread of a 128-thread group and shared with the whole group through a
+// named barrier, so that every thread of the group takes the same branch afterwards.
+struct GroupWait {
+    Smem* sm;
+    const TcParams* p;
+    int gid;      // 0 = P group, 1 = state group
+    int tid;      // thread index within the group
+    int flip = 0;
+
+    __device__ bool wait(uint64_t* bar, uint32_t parity) {
+        if (tid == 0) {
+            bool ok = mbar_wait(bar, parity, &sm->abort, WAIT_NS);
+            if (!ok) {
+                if (!sm->abort) set_error(p->err);
+                atomicExch(&sm->abort, 1u);
+            }
+            sm->dec[gid][flip] = ok ? 0u : 1u;
+        }
+        named_sync(1 + gid);
+        bool ok = *reinterpret_cast<volatile uint32_t*>(&sm->dec[gid][flip]) == 0;
+        flip ^= 1;
+        return ok;
+    }
+
+    // Spin on a flag in global memory written by another CTA.
+    __device__ bool wait_flag(const uint32_t* flag, uint32_t want) {
+        if (tid == 0) {
+            bool ok = false;
+            const uint64_t t0 = globaltimer_ns();
+            while (true) {
+                uint32_t v;
+                asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
+                if (v == want) { ok = true; break; }
+                if (*reinterpret_cast<volatile uint32_t*>(&sm->abort)) break;
+                if (globaltimer_ns() - t0 > WAIT_NS) break;
+                __nanosleep(64);
+            }
+            if (!ok) {
+                if (!sm->abort) set_error(p->err);
+                atomicExch(&sm->abort, 1u);
+            }
+            sm->dec[gid][flip] = ok ? 0u : 1u;
+        }
+        named_sync(1 + gid);
+        bool ok = *reinterpret_cast<volatile uint32_t*>(&sm->dec[gid][flip]) == 0;
+        flip ^= 1;
+        return ok;
+    }
+};
+
+__device__ void decode_ticket(const TcParams& p, uint32_t ticket, uint32_t total, Item& it) {
+    it = Item{};
+    if (ticket >= total) return;
+    const uint32_t i = ticket / (uint32_t)p.H;
+    it.h = (int)(ticket % (uint32_t)p.H);
+    int64_t nc;
+    int ns;
+    if (p.prefix == nullptr) {
+        ns = p.spans_per_unit;
+        it.u = (int)(i / (uint32_t)ns);
+        it.s = (int)(i % (uint32_t)ns);
+        it.len = p.N;
+        it.tok_first = 0;
+        it.b = it.u;
+        it.grow0 = (int64_t)it.u * p.N;
+    } else {
+        int lo = 0, hi = p.units;   // prefix[lo] <= i < prefix[hi]
+        while (hi - lo > 1) {
+            int mid = (lo + hi) >> 1;
+            if ((uint32_t)p.prefix[mid] <= i) lo = mid; else hi = mid;
+        }
+        it.u = lo;
+        it.s = (int)(i - (uint32_t)p.prefix[lo]);
+        ns = p.prefix[lo + 1] - p.prefix[lo];
+        const int64_t a = p.cu_seqlens[lo];
+        it.len = (int64_t)p.cu_seqlens[lo + 1] - a;
+        it.tok_first = a;
+        it.b = 0;
+        it.grow0 = a;
+    }
+    nc = (it.len + C - 1) / C;
+    it.c_begin = it.s * p.G;
+    it.c_end = (int)(nc < (int64_t)it.c_begin + p.G ? nc : (int64_t)it.c_begin + p.G);
+    if (it.c_end < it.c_begin) it.c_end = it.c_begin;
+    it.first = it.s == 0;
+    it.last = it.s == ns - 1;
+    it.valid = 1;
+}
+
+__device__ __forceinline__ void set_coord(int (&c)[4], int pos_tok, int pos_head, int pos_b,
+                                          int col, int tok, int h, int b) {
+    c[0] = col;
+    c[pos_tok] = tok;
+    c[pos_head] = h;
+    c[pos_b] = b;
+}
+
+// ----------------------------------------------------------------------------------------------
+// warp 0: TMA producer
+
+__device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
+                         const CUtensorMap* tv, uint32_t total) {
+    int j = 0, it_n = 0;
+    bool aborted = false;
+    while (!aborted) {
+        const int slot = it_n % ITEM_DEPTH;
+        if (it_n >= ITEM_DEPTH &&
+            !mbar_wait(&sm.item_empty[slot], ((it_n / ITEM_DEPTH) - 1) & 1, &sm.abort, WAIT_NS)) {
+            aborted = true;
+            break;
+        }
+        const uint32_t ticket = atomicAdd(p.ticket, 1u);
+        Item it;
+        decode_ticket(p, ticket, total, it);
+        sm.items[slot] = it;
+        mbar_arrive(&sm.item_full[slot]);
+        ++it_n;
+        if (!it.valid) break;
+        for (int pass = 0; pass < 2 && !aborted; ++pass) {
+            for (int c = it.c_begin; c < it.c_end; ++c) {
+                const int st = j & 1;
+                if (j >= 2 &&
+                    !mbar_wait(&sm.stage_empty[st], ((j >> 1) - 1) & 1, &sm.abort, WAIT_NS)) {
+                    aborted = true;
+                    break;
+                }
+                mbar_arrive_expect_tx(&sm.kv_full[st], pass ? 3 * TILE : 2 * TILE);
+                const int tok = (int)(it.tok_first + (int64_t)c * C);
+                int ck[4], cv[4];
+                for (int half = 0; half < 2; ++half) {
+                    set_coord(ck, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b, half * 64, tok, it.h,
+                              it.b);
+                    set_coord(cv, p.v_pos_tok, p.v_pos_head, p.v_pos_b, half * 64, tok, it.h,
+                              it.b);
+                    tma_load_4d(sm.k[st] + half * SLAB, tk, &sm.kv_full[st], ck[0], ck[1], ck[2],
+                                ck[3]);
+                    tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], cv[0], cv[1], cv[2],
+                                cv[3]);
+                    if (pass)
+                        tma_load_4d(sm.q[st] + half * SLAB, tq, &sm.kv_full[st], ck[0], ck[1],
+                                    ck[2], ck[3]);
+                }
+                ++j;
+            }
+        }
+    }
+    if (aborted) {
+        set_error(p.err);
+        atomicExch(&sm.abort, 1u);
+    }
+    // make sure no TMA write into this CTA's shared memory is still in flight at exit
+    for (int jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj)
+        mbar_wait_drain(&sm.kv_full[jj & 1], (jj >> 1) & 1, DRAIN_NS);
+}
+
+// ----------------------------------------------------------------------------------------------
+// warp 1: MMA issuer (one thread)
+
+// D (+)= A B over K = 128, eight K-steps of 16; operands in shared memory.
+__device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, uint32_t b_base,
+                                        bool b_mn, bool bf16) {
+    const uint32_t idesc = idesc_f16kind(128, 128, a_mn, b_mn, bf16);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t aoff = a_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
+        const uint32_t boff = b_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
+        const uint64_t ad = a_mn ? sdesc_sw128(a_base + aoff, SLAB, 1024)
+                                 : sdesc_sw128(a_base + aoff, 16, 1024);
+        const uint64_t bd = b_mn ? sdesc_sw128(b_base + boff, SLAB, 1024)
+                                 : sdesc_sw128(b_base + boff, 16, 1024);
+        mma_ss(d, ad, bd, idesc, kk > 0);
+    }
+}
+
+__device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
+    int j = 0, b = 0, it_n = 0;
+    bool ok = true;
+    auto W = [&](uint64_t* bar, uint32_t par) {
+        if (ok && !mbar_wait(bar, par, &sm.abort, WAIT_NS)) {
+            ok = false;
+            if (!sm.abort) set_error(p.err);
+            atomicExch(&sm.abort, 1u);
+        }
+        return ok;
+    };
+    const uint32_t sbf = smem_u32(sm.sbf);
+    while (ok) {
+        const int slot = it_n % ITEM_DEPTH;
+        if (!W(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
+        const Item it = sm.items[slot];
+        mbar_arrive(&sm.item_empty[slot]);
+        ++it_n;
+        if (!it.valid) break;
+        // pass A: dS only
+        for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j) {
+            const int st = j & 1;
+            if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
+            if (!W(&sm.v16_ready, j & 1)) break;
+            if (!W(&sm.k_ready, j & 1)) break;
+            if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
+            tc_fence_after();
+            mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, false);
+            mma_commit(&sm.ds_full);
+            mma_commit(&sm.stage_empty[st]);
+        }
+        // pass B: the full chunk
+        for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j, ++b) {
+            const int st = j & 1;
+            if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
+            if (b > 0 && !W(&sm.o_full, (b - 1) & 1)) break;     // A/P region consumed
+            tc_fence_after();
+            mma_128(tmem + TM_A, smem_u32(sm.q[st]), false, smem_u32(sm.k[st]), false, true);
+            mma_commit(&sm.a_full);
+            if (!W(&sm.q16_ready, b & 1)) break;
+            if (!W(&sm.s_ready, b & 1)) break;
+            if (b > 0 && !W(&sm.o_free, (b - 1) & 1)) break;     // O, OX read out
+            tc_fence_after();
+            mma_128(tmem + TM_OX, smem_u32(sm.q[st]), false, sbf, true, false);
+            if (!W(&sm.p_ready, b & 1)) break;
+            if (!W(&sm.v16_ready, j & 1)) break;
+            tc_fence_after();
+            {
+                const uint32_t idesc = idesc_f16(128, 128, 0, 1);
+                const uint32_t vb = smem_u32(sm.v[st]);
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk)
+                    mma_ts(tmem + TM_O, tmem + TM_A + kk * 8,
+                           sdesc_sw128(vb + kk * 2048u, SLAB, 1024), idesc, kk > 0);
+            }
+            mma_commit(&sm.o_full);
+            if (!W(&sm.k_ready, j & 1)) break;
+            if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
+            tc_fence_after();
+            mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, false);
+            mma_commit(&sm.ds_full);
+            mma_commit(&sm.stage_empty[st]);
+        }
+    }
+    // all issued MMAs complete before TMEM is released
+    mma_commit(&sm.drain);
+    mbar_wait_drain(&sm.drain, 0, DRAIN_NS);
+}
+
+// ----------------------------------------------------------------------------------------------
+// helpers shared by the two 128-thread groups
+
+// Power of two that maps a magnitude bound `mx` into [2^14, 2^15): operands are rounded to fp16
+// after this scaling (so nothing overflows fp16's 65504 and the largest values keep all 11
+// bits), and the exact reciprocal is applied to the fp32 results.
+__device__ __forceinline__ float pow2_scale(float mx) {
+    if (!(mx > 0.f) || !isfinite(mx)) return 1.f;
+    int e = (int)((__float_as_uint(mx) >> 23) & 0xffu) - 127;   // floor(log2(mx)), normal mx
+    int s = 14 - e;
+    s = s < -126 ? -126 : (s > 127 ? 127 : s);
+    return __uint_as_float((uint32_t)(s + 127) << 23);
+}
+
+__device__ __forceinline__ float group_max(Smem& sm, int gid, int q, int lane, float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
+    if (lane == 0) sm.red[gid][q] = x;
+    named_sync(1 + gid);
+    const float m = fmaxf(fmaxf(sm.red[gid][0], sm.red[gid][1]), fmaxf(sm.red[gid][2], sm.red[gid][3]));
+    return m;
+}
+
+// gate scan: thread r (row r = 32 * (warp % 4) + lane) gets the inclusive cumulative
+// log2-decay c_r of its token, and the chunk total.
+__device__ __forceinline__ float chunk_scan(Smem& sm, const TcParams& p, const Item& it, int c,
+                                            int r, int q, int lane, int gid, float& total) {
+    const int64_t t = (int64_t)c * C + r;
+    float lam = 0.f;
+    if (t < it.len) lam = logsigmoid_(p.g[(it.grow0 + t) * p.H + it.h]) * p.inv_tau_log2e;
+    float x = lam;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    if (lane == 31) sm.wsum[gid][q] = x;
+    named_sync(1 + gid);
+    float pre = 0.f;
+    total = 0.f;
+#pragma unroll
+    for (int w = 0; w < 4; ++w) {
+        const float s = sm.wsum[gid][w];
+        if (w < q) pre += s;
+        total += s;
+    }
+    return x + pre;
+}
+
+// Max |x| over one 128-element bf16 row of a swizzled tile (rows are 128-byte lines in each of
+// the two 64-column slabs; the in-line chunk order does not matter for row-wise work).
+__device__ __forceinline__ float row_absmax_bf16(const unsigned char* tile, int r) {
+    float m = 0.f;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        const uint4* line = reinterpret_cast<const uint4*>(tile + half * SLAB + r * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4 u = line[c];
+            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(h2[e]);
+                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
+            }
+        }
+    }
+    return m;
+}
+
+// In place: bf16 row -> fp16(row * scale).
+__device__ __forceinline__ void row_bf16_to_f16(unsigned char* tile, int r, float scale) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        uint4* line = reinterpret_cast<uint4*>(tile + half * SLAB + r * 128);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+            uint4 u = line[c];
+            uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
+                w[e] = pack_f16x2(f.x * scale, f.y * scale);
+            }
+            line[c] = u;
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------------------------
+// warps 4-7: Q to fp16, decay mask, output epilogue
+
+__device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
+    GroupWait gw{&sm, &p, 0, (warp - 4) * 32 + lane};
+    const int q = warp & 3, r = q * 32 + lane;
+    const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
+    int b = 0, j = 0, it_n = 0;
+    while (true) {
+        const int slot = it_n % ITEM_DEPTH;
+        if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
+        const Item it = sm.items[slot];
+        mbar_arrive(&sm.item_empty[slot]);
+        ++it_n;
+        if (!it.valid) break;
+        bool ok = true;
+        j += it.c_end - it.c_begin;     // the span's pass-A jobs
+        for (int c = it.c_begin; c < it.c_end; ++c, ++b, ++j) {
+            const int st = j & 1;
+            float tot;
+            const float cr = chunk_scan(sm, p, it, c, r, q, lane, 0, tot);
+            sm.cP[r] = cr;
+            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }   // also publishes cP
+            tc_fence_after();
+            // Q row r -> fp16 with its own power-of-two scale (Q K^T has consumed the bf16 Q)
+            const float sq = pow2_scale(row_absmax_bf16(sm.q[st], r));
+            row_bf16_to_f16(sm.q[st], r, sq);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.q16_ready);
+            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, in fp32, then fp16 with a
+            // per-row power-of-two scale
+            float pv[C];
+            float pmax = 0.f;
+#pragma unroll
+            for (int jc = 0; jc < 4; ++jc) {
+                if (jc <= q) {
+                    float a[32];
+                    tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
+                    tmem_ld_wait();
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int m = jc * 32 + i;
+                        const float v = (m <= r) ? ex2f(cr - sm.cP[m]) * p.k_scale * a[i] : 0.f;
+                        pv[m] = v;
+                        pmax = fmaxf(pmax, fabsf(v));
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) pv[jc * 32 + i] = 0.f;
+                }
+            }
+            const float rho = pow2_scale(pmax);
+#pragma unroll
+            for (int jc = 0; jc < 4; ++jc) {
+                uint32_t pk[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+                    pk[i] = pack_f16x2(pv[jc * 32 + 2 * i] * rho, pv[jc * 32 + 2 * i + 1] * rho);
+                tmem_st16(tmem + lane_base + TM_A + jc * 16, pk);
+            }
+            // scales of V and of the entry state for this chunk (both published before their
+            // barriers complete; waiting here, before p_ready, cannot miss a phase)
+            if (!gw.wait(&sm.v16_ready, j & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.s_ready, b & 1)) { ok = false; break; }
+            const float inv_pv = 1.f / (rho * sm.sig_v[j & 1]);
+            const float inv_qs = 1.f / (sq * sm.sig_s[b & 1]);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready);
+            // epilogue: O = O_inner + 2^(c_r) O_cross, each unscaled
+            if (!gw.wait(&sm.o_full, b & 1)) { ok = false; break; }
+            tc_fence_after();
+            const float ec = ex2f(cr) * inv_qs;
+            const int64_t t = (int64_t)c * C + r;
+            const bool valid = t < it.len;
+            __nv_bfloat16* orow = p.o + (int64_t)it.b * p.osb + (it.tok_first + t) * p.ost +
+                                  (int64_t)it.h * p.osh;
+#pragma unroll 1
+            for (int jc = 0; jc < 4; ++jc) {
+                float o[32], ox[32];
+                tmem_ld32(tmem + lane_base + TM_O + jc * 32, o);
+                tmem_ld32(tmem + lane_base + TM_OX + jc * 32, ox);
+                tmem_ld_wait();
+                if (valid) {
+                    uint4* dst = reinterpret_cast<uint4*>(orow + jc * 32);
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4) {
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            y[e] = fmaf(ec, ox[8 * v4 + e], o[8 * v4 + e] * inv_pv);
+                        uint4 u;
+                        u.x = pack_bf16x2(y[0], y[1]);
+                        u.y = pack_bf16x2(y[2], y[3]);
+                        u.z = pack_bf16x2(y[4], y[5]);
+                        u.w = pack_bf16x2(y[6], y[7]);
+                        dst[v4] = u;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(&sm.o_free);
+        }
+        if (!ok) break;
+    }
+}
+
+// ----------------------------------------------------------------------------------------------
+// warps 8-11: V and decayed K to fp16, fp32 state, look-back
+
+// V tile -> fp16 with one power-of-two scale for the tile; returns the scale.
+__device__ __forceinline__ float convert_v(Smem& sm, unsigned char* vtile, int r, int q, int lane) {
+    const float sv = pow2_scale(group_max(sm, 1, q, lane, row_absmax_bf16(vtile, r)));
+    row_bf16_to_f16(vtile, r, sv);
+    return sv;
+}
+
+// K tile -> fp16 rows w_r * K_r with one power-of-two scale for the tile; returns the scale.
+__device__ __forceinline__ float convert_k(Smem& sm, unsigned char* ktile, int r, int q, int lane,
+                                           float w) {
+    const float sk = pow2_scale(group_max(sm, 1, q, lane, w * row_absmax_bf16(ktile, r)));
+    row_bf16_to_f16(ktile, r, w * sk);
+    return sk;
+}
+
+// fp16 copy of state row r (times `scale`) into the MN-major swizzled tile read by Q S_prev.
+__device__ __forceinline__ void write_state_f16(unsigned char* tile, int r, const float (&S)[D],
+                                                float scale) {
+#pragma unroll
+    for (int cc = 0; cc < 16; ++cc) {
+        uint4 u;
+        u.x = pack_f16x2(S[8 * cc + 0] * scale, S[8 * cc + 1] * scale);
+        u.y = pack_f16x2(S[8 * cc + 2] * scale, S[8 * cc + 3] * scale);
+        u.z = pack_f16x2(S[8 * cc + 4] * scale, S[8 * cc + 5] * scale);
+        u.w = pack_f16x2(S[8 * cc + 6] * scale, S[8 * cc + 7] * scale);
+        const int half = cc >> 3, c = cc & 7;
+        *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) = u;
+    }
+}
+
+__device__ __forceinline__ void publish_state(Smem& sm, int r, int q, int lane, const float (&S)[D],
+                                              int bslot) {
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < D; ++i) m = fmaxf(m, fabsf(S[i]));
+    const float ss = pow2_scale(group_max(sm, 1, q, lane, m));
+    write_state_f16(sm.sbf, r, S, ss);
+    if (r == 0) sm.sig_s[bslot] = ss;
+    fence_proxy_async_smem();
+    mbar_arrive(&sm.s_ready);
+}
+
+// S = 2^tot * S + dS / (sk * sv), dS read from TMEM
+__device__ __forceinline__ void fold_ds(uint32_t taddr, float (&S)[D], float eb, float inv) {
+#pragma unroll
+    for (int jc = 0; jc < 8; ++jc) {
+        float ds[16];
+        tmem_ld16(taddr + jc * 16, ds);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 16; ++i) S[jc * 16 + i] = fmaf(eb, S[jc * 16 + i], ds[i] * inv);
+    }
+}
+
+__device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
+    GroupWait gw{&sm, &p, 1, (warp - 8) * 32 + lane};
+    const int q = warp & 3, r = q * 32 + lane;
+    const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
+    float S[D];
+    int j = 0, b = 0, it_n = 0;
+    bool ok = true;
+    while (ok) {
+        const int slot = it_n % ITEM_DEPTH;
+        if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
+        const Item& it = sm.items[slot];   // read in place; released at the end of the span
+        ++it_n;
+        if (!it.valid) {
+            mbar_arrive(&sm.item_empty[slot]);
+            break;
+        }
+        // ---- pass A: span aggregate from zero
+#pragma unroll
+        for (int i = 0; i < D; ++i) S[i] = 0.f;
+        float L = 0.f;   // span log2-decay
+        for (int c = it.c_begin; c < it.c_end; ++c, ++j) {
+            const int st = j & 1;
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
+            float tot;
+            const float cr = chunk_scan(sm, p, it, c, r, q, lane, 1, tot);
+            const bool valid = (int64_t)c * C + r < it.len;
+            const float sv = convert_v(sm, sm.v[st], r, q, lane);
+            if (r == 0) sm.sig_v[j & 1] = sv;
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.v16_ready);
+            const float sk = convert_k(sm, sm.k[st], r, q, lane, valid ? ex2f(tot - cr) * p.k_scale : 0.f);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.k_ready);
+            if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
+            tc_fence_after();
+            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot), 1.f / (sk * sv));
+            tc_fence_before();
+            mbar_arrive(&sm.ds_free);
+            L += tot;
+        }
+        if (!ok) break;
+        // ---- look-back: entry state E of the span; publish exp(L) E + Agg
+        const int64_t chain = (int64_t)it.u * p.H + it.h;
+        const float* esrc = nullptr;
+        bool from_slot = false;
+        if (it.first) {
+            if (p.state_in) esrc = p.state_in + (chain * D + r) * D;
+        } else {
+            if (!gw.wait_flag(p.flags + chain * 2 + ((it.s - 1) & 1), (uint32_t)it.s)) break;
+            esrc = p.slots + (chain * 2 + ((it.s - 1) & 1)) * (D * D);
+            from_slot = true;
+        }
+        const float eL = ex2f(L);
+        float4* dst = it.last ? nullptr
+                              : reinterpret_cast<float4*>(p.slots + (chain * 2 + (it.s & 1)) * (D * D));
+#pragma unroll
+        for (int j4 = 0; j4 < D / 4; ++j4) {
+            float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (from_slot)
+                e = __ldcg(reinterpret_cast<const float4*>(esrc) + j4 * D + r);
+            else if (esrc)
+                e = reinterpret_cast<const float4*>(esrc)[j4];
+            if (dst) {
+                float4 inc;
+                inc.x = fmaf(eL, e.x, S[4 * j4 + 0]);
+                inc.y = fmaf(eL, e.y, S[4 * j4 + 1]);
+                inc.z = fmaf(eL, e.z, S[4 * j4 + 2]);
+                inc.w = fmaf(eL, e.w, S[4 * j4 + 3]);
+                __stcg(dst + j4 * D + r, inc);
+            }
+            S[4 * j4 + 0] = e.x;
+            S[4 * j4 + 1] = e.y;
+            S[4 * j4 + 2] = e.z;
+            S[4 * j4 + 3] = e.w;
+        }
+        if (dst) {
+            __threadfence();
+            named_sync(2);
+            if (r == 0) {
+                uint32_t* f = p.flags + chain * 2 + (it.s & 1);
+                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"((uint32_t)it.s + 1)
+                             : "memory");
+            }
+        }
+        if (it.c_end > it.c_begin) publish_state(sm, r, q, lane, S, b & 1);  // for the first chunk
+        // ---- pass B: running state from E
+        for (int c = it.c_begin; c < it.c_end; ++c, ++j, ++b) {
+            const int st = j & 1;
+            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
+            float tot;
+            const float cr = chunk_scan(sm, p, it, c, r, q, lane, 1, tot);
+            const bool valid = (int64_t)c * C + r < it.len;
+            const float sv = convert_v(sm, sm.v[st], r, q, lane);
+            if (r == 0) sm.sig_v[j & 1] = sv;
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.v16_ready);
+            const float sk = convert_k(sm, sm.k[st], r, q, lane, valid ? ex2f(tot - cr) * p.k_scale : 0.f);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.k_ready);
+            if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
+            tc_fence_after();
+            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot), 1.f / (sk * sv));
+            tc_fence_before();
+            mbar_arrive(&sm.ds_free);
+            if (c + 1 < it.c_end) publish_state(sm, r, q, lane, S, (b + 1) & 1);
+        }
+        if (!ok) break;
+        if (it.last && p.state_out) {
+            float4* so = reinterpret_cast<float4*>(p.state_out + (chain * D + r) * D);
+#pragma unroll
+            for (int j4 = 0; j4 < D / 4; ++j4)
+                so[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
+        }
+        mbar_arrive(&sm.item_empty[slot]);
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                      const __grid_constant__ CUtensorMap tv, const TcParams p, uint32_t total_dense) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if ((smem_u32(smem_raw) & 1023u) != 0) {   // the swizzled tiles need 1 KB alignment
+        if (tid == 0) set_error(p.err);
+        return;
+    }
+    if (tid == 0) {
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.stage_empty[s], 1);
+        }
+        for (int s = 0; s < ITEM_DEPTH; ++s) {
+            mbar_init(&sm.item_full[s], 1);
+            mbar_init(&sm.item_empty[s], 1 + 128 + 128);
+        }
+        mbar_init(&sm.a_full, 1);
+        mbar_init(&sm.q16_ready, 128);
+        mbar_init(&sm.p_ready, 128);
+        mbar_init(&sm.o_full, 1);
+        mbar_init(&sm.o_free, 128);
+        mbar_init(&sm.v16_ready, 128);
+        mbar_init(&sm.k_ready, 128);
+        mbar_init(&sm.ds_full, 1);
+        mbar_init(&sm.ds_free, 128);
+        mbar_init(&sm.s_ready, 128);
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        if (warp == 0) {
+            if (lane == 0) {
+                tma_prefetch_desc(&tq);
+                tma_prefetch_desc(&tk);
+                tma_prefetch_desc(&tv);
+                const uint32_t total =
+                    p.prefix ? (uint32_t)p.prefix[p.units] * (uint32_t)p.H : total_dense;
+                producer(sm, p, &tq, &tk, &tv, total);
+            }
+        } else if (warp == 1) {
+            if (lane == 0) mma_issuer(sm, p, tmem);
+        }
+    } else if (warp < 8) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+        p_group(sm, p, tmem, warp, lane);
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+        state_group(sm, p, tmem, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// Varlen: spans per sequence and their exclusive prefix (one CTA).
+__global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int units, int G,
+                                                    int32_t* __restrict__ prefix) {
+    __shared__ int32_t warp_tot[32];
+    __shared__ int32_t carry;
+    const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+    if (tid == 0) carry = 0;
+    __syncthreads();
+    for (int base = 0; base < units; base += 1024) {
+        const int u = base + tid;
+        int ns = 0;
+        if (u < units) {
+            const int64_t len = (int64_t)cu[u + 1] - cu[u];
+            const int64_t nc = (len + C - 1) / C;
+            ns = (int)((nc + G - 1) / G > 1 ? (nc + G - 1) / G : 1);
+        }
+        int x = ns;
+        for (int o = 1; o < 32; o <<= 1) {
+            int y = __shfl_up_sync(0xffffffffu, x, o);
+            if (lane >= o) x += y;
+        }
+        if (lane == 31) warp_tot[w] = x;
+        __syncthreads();
+        if (w == 0) {
+            int t = warp_tot[lane];
+            for (int o = 1; o < 32; o <<= 1) {
+                int y = __shfl_up_sync(0xffffffffu, t, o);
+                if (lane >= o) t += y;
+            }
+            warp_tot[lane] = t;   // inclusive over warps
+        }
+        __syncthreads();
+        const int excl = carry + (w > 0 ? warp_tot[w - 1] : 0) + x - ns;
+        if (u < units) prefix[u] = excl;
+        __syncthreads();
+        if (tid == 1023) carry = excl + ns;
+        __syncthreads();
+    }
+    if (tid == 0) prefix[units] = carry;
+}
+
+struct WsLayout {
+    size_t flags, prefix, slots, total;
+};
+
+WsLayout ws_layout(int units, int H) {
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    WsLayout l;
+    l.flags = 256;
+    l.prefix = l.flags + up((size_t)units * H * 2 * sizeof(uint32_t));
+    l.slots = l.prefix + up(((size_t)units + 1) * sizeof(int32_t));
+    l.total = l.slots + (size_t)units * H * 2 * D * D * sizeof(float);
+    return l;
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+// Order the (token, head, batch) dims of a [.., token, head, d] tensor by stride for the TMA map;
+// returns false if the driver rejects it.
+bool make_map(CUtensorMap* map, const void* base, int64_t st, int64_t sh, int64_t sb, int64_t ntok,
+              int H, int B, int& pos_tok, int& pos_head, int& pos_b) {
+    struct Dim { int64_t stride, extent; int which; };
+    Dim d[3] = {{st, ntok, 0}, {sh, H, 1}, {sb, B, 2}};
+    // a size-1 batch dimension gets a stride past the end of the other two
+    if (B == 1) {
+        int64_t end = 1;
+        for (int i = 0; i < 2; ++i) end = d[i].stride * d[i].extent > end ? d[i].stride * d[i].extent : end;
+        d[2].stride = end;
+    }
+    for (int i = 0; i < 3; ++i)
+        for (int k = i + 1; k < 3; ++k)
+            if (d[k].stride < d[i].stride) { Dim t = d[i]; d[i] = d[k]; d[k] = t; }
+    uint64_t dims[4] = {D, 0, 0, 0}, strides[3];
+    uint32_t box[4] = {64, 1, 1, 1};
+    for (int i = 0; i < 3; ++i) {
+        dims[i + 1] = (uint64_t)d[i].extent;
+        strides[i] = (uint64_t)d[i].stride * 2;
+        if (d[i].which == 0) { pos_tok = i + 1; box[i + 1] = C; }
+        if (d[i].which == 1) pos_head = i + 1;
+        if (d[i].which == 2) pos_b = i + 1;
+    }
+    return make_bf16_map(map, base, 4, dims, strides, box);
+}
+
+int span_chunks() {
+    static int g = -1;
+    if (g < 0) {
+        const char* e = getenv("GRET_SPAN_CHUNKS");
+        g = e ? atoi(e) : 4;
+        if (g < 1) g = 4;
+    }
+    return g;
+}
+
+}  // namespace
+
+size_t tc_workspace_size(int64_t, int n_units, int H) { return ws_layout(n_units, H).total; }
+
+gret_status_t launch_prefill_tc(const PrefillArgs& a) {
+    const bool varlen = a.cu_seqlens != nullptr;
+    const int units = a.n_seqs;
+    const WsLayout L = ws_layout(units, a.H);
+    unsigned char* ws = (unsigned char*)a.workspace;
+    const int G = span_chunks();
+
+    TcParams p;
+    p.g = a.g;
+    p.inv_tau_log2e = 1.4426950408889634f / a.tau;
+    p.k_scale = a.k_scale;
+    p.o = (__nv_bfloat16*)a.o;
+    p.osb = a.osb; p.ost = a.ost; p.osh = a.osh;
+    p.state_in = a.state_in;
+    p.state_out = a.state_out;
+    p.err = (uint32_t*)ws;
+    p.ticket = (uint32_t*)(ws + 4);
+    p.flags = (uint32_t*)(ws + L.flags);
+    p.prefix = varlen ? (int32_t*)(ws + L.prefix) : nullptr;
+    p.slots = (float*)(ws + L.slots);
+    p.cu_seqlens = a.cu_seqlens;
+    p.N = a.N;
+    p.H = a.H;
+    p.units = units;
+    p.G = G;
+    const int64_t nc_dense = (a.N + C - 1) / C;
+    p.spans_per_unit = (int)std::max<int64_t>(1, (nc_dense + G - 1) / G);
+
+    const int64_t ntok = a.N;   // dense: tokens per sequence; varlen: packed total
+    const int B = varlen ? 1 : a.B;
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, a.q, a.st, a.sh, a.sb, ntok, a.H, B, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b) ||
+        !make_map(&tk, a.k, a.st, a.sh, a.sb, ntok, a.H, B, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b) ||
+        !make_map(&tv, a.v, a.vst, a.vsh, a.vsb, ntok, a.H, B, p.v_pos_tok, p.v_pos_head, p.v_pos_b))
+        return GRET_ERR_UNSUPPORTED;
+
+    uint64_t total_dense = varlen ? 0 : (uint64_t)units * p.spans_per_unit * a.H;
+    if (total_dense > 0xFFFFFFF0ull) return GRET_ERR_UNSUPPORTED;
+    if (cudaMemsetAsync(ws, 0, L.prefix, a.stream) != cudaSuccess) return GRET_ERR_CUDA;
+    if (varlen) {
+        plan_kernel<<<1, 1024, 0, a.stream>>>(a.cu_seqlens, units, G, p.prefix);
+        if (cudaGetLastError() != cudaSuccess) return GRET_ERR_CUDA;
+    }
+    const size_t smem = sizeof(Smem);
+    if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return GRET_ERR_CUDA;
+    int grid = sm_count();
+    if (!varlen && total_dense < (uint64_t)grid) grid = (int)total_dense;
+    if (grid < 1) grid = 1;
+    prefill_tc_kernel<<<grid, NTHREADS, smem, a.stream>>>(tq, tk, tv, p, (uint32_t)total_dense);
+    return cudaGetLastError() == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
 
 }  // namespace gret

@@ -68,9 +68,10 @@ size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int
  * which equals the recurrence above up to rounding.  The last chunk of a sequence may be
  * shorter; nothing needs padding.
  *
- *   q, k     [.., token, head, d_k] in `dtype`; element (b, t, h, i) at
+ *   q, k     [.., token, head, d_k] in `dtype`, sharing strides; element (b, t, h, i) at
  *            b*stride_batch + t*stride_tok + h*stride_head + i.  Read only.
- *   v        same strides, last dim d_v.  Read only.
+ *   v        [.., token, head, d_v] in `dtype` with its own strides (v_stride_batch,
+ *            v_stride_tok, v_stride_head).  Read only.
  *   g        fp32 gate logits, contiguous [B, N, H] (dense) or [total_tokens, H] (varlen).
  *   tau      temperature (> 0); k_scale multiplies every key (e.g. d_k^-1/2, or 1.0).
  *   dtype    GRET_BF16 (tensor-core path when d_k == d_v == 128, else a CUDA-core path with
@@ -97,8 +98,9 @@ size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int
  * read it with gret_workspace_status() after the stream has synchronised.
  */
 gret_status_t gret_prefill_chunkwise(
-    const void* q, const void* k, const void* v, int64_t stride_batch, int64_t stride_tok,
-    int64_t stride_head, const float* g, float tau, float k_scale, gret_dtype_t dtype, int B,
+    const void* q, const void* k, int64_t stride_batch, int64_t stride_tok, int64_t stride_head,
+    const void* v, int64_t v_stride_batch, int64_t v_stride_tok, int64_t v_stride_head,
+    const float* g, float tau, float k_scale, gret_dtype_t dtype, int B,
     int64_t N, int H, int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
     const float* state_in, float* state_out, void* o, int64_t o_stride_batch,
     int64_t o_stride_tok, int64_t o_stride_head, int chunk, void* workspace,

@@ -33,7 +33,8 @@ def test_status_strings():
 
 
 def _prefill(lib, **kw):
-    a = dict(q=1024, k=1024, v=1024, sb=0, st=128 * 24, sh=128, g=1024, tau=16.0, ks=1.0,
+    a = dict(q=1024, k=1024, sb=0, st=128 * 24, sh=128, v=1024, vsb=0, vst=128 * 24, vsh=128,
+             g=1024, tau=16.0, ks=1.0,
              dtype=1, B=1, N=64, H=24, dk=128, dv=128, cu=None, n=0, sin=None, sout=None,
              o=2048, osb=0, ost=128 * 24, osh=128, chunk=0, ws=None, wsb=0, stream=None)
     a.update(kw)
