@@ -1,0 +1,391 @@
+"""Benchmark of the gated-retention hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+    python -m torch.distributed.run --nproc-per-node N bench.py --gpus N ...   (N > 1)
+
+One step = one chunkwise prefill of one gated-retention layer of the 3B shape (batch 1,
+24 heads, 32768 tokens, d_k = d_v = 128, bf16 inputs, fp32 state, g ~ N(2, 1), tau = 16) through
+the C ABI, inputs resident in HBM.  The printed JSON line carries:
+  value     whole-job prefill throughput (Mtok/s; every rank runs its own sequence: weak scaling)
+  roofline  the prefill kernel against measured HBM bandwidth (1028 algorithmic bytes per
+            token and head: q, k, v, o in bf16 plus the fp32 gate logit)
+  decode    batched decode at batch 64 (state of 64 x 24 x 128 x 128 fp32 from a 4096-token
+            prefill, 256 steps), tok/s and its HBM roofline
+  e2e       the same prefill metric with host buffers: pinned host -> device copies of q, k, v, g
+            and device -> host copies of o and the final state inside the timed region
+  cpu_baseline  the fp64 CPU oracle on the same workload (rank 0 only)
+With --impl reference the oracle alone is timed, on host cores, as the reference arm.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "gRet prefill Mtok/s (H=24,d=128,N=32K); decode tok/s @bs64; % of roofline"
+B, N, H, D = 1, 32768, 24, 128
+BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 4          # q, k, v, o (bf16) + g (fp32)
+DEC_B, DEC_PREFILL, DEC_STEPS = 64, 4096, 256
+DEC_BYTES_PER_HEAD = 2 * D * D * 4 + 4 * D * 2 + 4   # state read + write, q k v o, g
+WORKLOAD = ("gRet chunkwise prefill, batch 1, H=24, N=32768, d_k=d_v=128, bf16 q/k/v "
+            "~N(0,1)/sqrt(128), g~N(2,1), tau=16, fp32 state")
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            pk = json.load(f)
+        return float(pk["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle sampling in the background during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def dist_setup(n_gpus):
+    import torch
+    rank, world = 0, 1
+    if n_gpus > 1 or "WORLD_SIZE" in os.environ:
+        import datetime
+        import torch.distributed as dist
+        rank = int(os.environ.get("RANK", "0"))
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        local = int(os.environ.get("LOCAL_RANK", str(rank)))
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return rank, world
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def prefill_traffic_from_profile():
+    """DRAM bytes per launch of the prefill kernel from the committed ncu summary, if that
+    summary was taken on the current kernel source (else None)."""
+    import hashlib
+    src = os.path.join(ROOT, "gated_retention_linear_b200", "csrc", "prefill_tc.cu")
+    summ = os.path.join(ROOT, "profiles", "prefill_tc_kernel_32k.txt")
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+        kv = {}
+        for line in open(summ):
+            if ":" in line:
+                k, v = line.split(":", 1)
+                kv[k.strip()] = v.strip()
+        if kv.get("kernel_source_sha256_16") == sha:
+            return int(float(kv["dram_bytes_per_launch"]))
+    except Exception:
+        pass
+    return None
+
+
+def run_gpu(args):
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+
+    rank, world = dist_setup(args.gpus)
+    dev = torch.cuda.current_device()
+    stream = torch.cuda.current_stream()
+    hbm_peak, peak_kind = measured_peaks()
+
+    # ---------------- prefill, inputs resident in HBM
+    inp = SI.gret_inputs(B, N, H, D, dtype=torch.bfloat16, g_mean=2.0, g_std=1.0,
+                         seed=2 + 1000 * rank, device="cuda")
+    q, k, v, g = inp["q"], inp["k"], inp["v"], inp["g"]
+    o = torch.empty_like(v)
+    s_out = torch.empty((B, H, D, D), dtype=torch.float32, device="cuda")
+    need = G.gret_prefill_workspace_size(torch.bfloat16, B * N, B, H, D, D, 0)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+
+    def step():
+        G.gret_prefill_chunkwise(q, k, v, g, state_out=s_out, o=o, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if G.gret_workspace_status(ws) != 0:
+        raise RuntimeError("prefill reported a timed-out wait during warm-up")
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    clocks = ClockSampler(dev)
+    clocks.start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    t0.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    t1.record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    ms_total = t0.elapsed_time(t1)
+    launch_ms = statistics.mean(e0.elapsed_time(e1) for e0, e1 in ev)
+    ms_total = max_over_ranks(ms_total, world)
+    if G.gret_workspace_status(ws) != 0:
+        raise RuntimeError("prefill reported a timed-out wait")
+    ms_per_step = ms_total / args.steps
+    tokens_all = B * N * world * args.steps
+    value = tokens_all / (ms_total * 1e-3) / 1e6
+    alg_bytes = B * N * H * BYTES_PER_TOKEN_HEAD
+    achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
+
+    # ---------------- decode at batch 64
+    dec = None
+    if not args.no_decode:
+        dinp = SI.gret_inputs(DEC_B, DEC_PREFILL, H, D, dtype=torch.bfloat16, seed=4 + 1000 * rank,
+                              device="cuda")
+        _, state = G.gret_prefill_chunkwise(dinp["q"], dinp["k"], dinp["v"], dinp["g"],
+                                            state_out=True)
+        del dinp
+        steps_in = SI.gret_inputs(DEC_B, DEC_STEPS, H, D, dtype=torch.bfloat16,
+                                  seed=40 + 1000 * rank, device="cuda")
+        qs = steps_in["q"].permute(1, 0, 2, 3).contiguous()    # [steps, B, H, d]
+        ks = steps_in["k"].permute(1, 0, 2, 3).contiguous()
+        vs = steps_in["v"].permute(1, 0, 2, 3).contiguous()
+        gs = steps_in["g"].permute(1, 0, 2).contiguous()
+        od = torch.empty((DEC_B, H, D), dtype=torch.bfloat16, device="cuda")
+        state0 = state.clone()
+        for w in range(args.warmup):
+            G.gret_decode_step(qs[w], ks[w], vs[w], gs[w], state, o=od)
+        state.copy_(state0)
+        torch.cuda.synchronize()
+        barrier(world)
+        d0 = torch.cuda.Event(enable_timing=True)
+        d1 = torch.cuda.Event(enable_timing=True)
+        d0.record(stream)
+        for s in range(DEC_STEPS):
+            G.gret_decode_step(qs[s], ks[s], vs[s], gs[s], state, o=od)
+        d1.record(stream)
+        torch.cuda.synchronize()
+        dms = max_over_ranks(d0.elapsed_time(d1), world)
+        dec_bytes = DEC_B * H * DEC_BYTES_PER_HEAD
+        dec_ach = dec_bytes / (dms / DEC_STEPS * 1e-3) / 1e9
+        dec = {"value": DEC_B * DEC_STEPS * world / (dms * 1e-3), "unit": "tok/s",
+               "ms_per_step": dms / DEC_STEPS, "steps": DEC_STEPS, "batch": DEC_B,
+               "gpu_launches": DEC_STEPS,
+               "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": hbm_peak,
+                            "unit": "GB/s", "frac": dec_ach / hbm_peak,
+                            "peak_kind": peak_kind, "traffic": None},
+               "l2": "state (201 MB) larger than L2 (126 MB); not flushed between steps"}
+        del qs, ks, vs, gs, state, state0
+
+    clk = clocks.stop()
+
+    # ---------------- end to end: host buffers through the C ABI
+    e2e = None
+    if not args.no_e2e:
+        hq = q.cpu().pin_memory()
+        hk = k.cpu().pin_memory()
+        hv = v.cpu().pin_memory()
+        hg = g.cpu().pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        hs = torch.empty(s_out.shape, dtype=s_out.dtype).pin_memory()
+        dq, dk, dv, dg = (torch.empty_like(x) for x in (q, k, v, g))
+
+        def e2e_step():
+            dq.copy_(hq, non_blocking=True)
+            dk.copy_(hk, non_blocking=True)
+            dv.copy_(hv, non_blocking=True)
+            dg.copy_(hg, non_blocking=True)
+            G.gret_prefill_chunkwise(dq, dk, dv, dg, state_out=s_out, o=o, workspace=ws)
+            ho.copy_(o, non_blocking=True)
+            hs.copy_(s_out, non_blocking=True)
+
+        for _ in range(max(1, args.warmup)):
+            e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ems = max_over_ranks(e0.elapsed_time(e1), world)
+        bi = sum(x.numel() * x.element_size() for x in (hq, hk, hv, hg))
+        bo = ho.numel() * ho.element_size() + hs.numel() * hs.element_size()
+        e2e = {"value": B * N * world * args.steps / (ems * 1e-3) / 1e6, "unit": "Mtok/s",
+               "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo,
+               "ms_per_step": ems / args.steps}
+
+    # ---------------- CPU oracle baseline (rank 0 only)
+    cpu = None
+    if rank == 0 and not args.no_cpu:
+        cpu = cpu_baseline(q, k, v, g, args.cpu_tokens)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": "Mtok/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD, "tokens_per_rank": B * N, "heads": H, "d": D,
+                   "parallelism": "independent sequence per GPU" if world > 1 else "1 GPU",
+                   "l2": "inputs and outputs (808 MB per step) larger than L2 (126 MB); "
+                         "L2 not flushed"},
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
+                     "frac": achieved / hbm_peak, "peak_kind": peak_kind,
+                     "traffic": prefill_traffic_from_profile(),
+                     "kernel": "prefill_tc_kernel", "launch_ms": launch_ms,
+                     "algorithmic_bytes_per_launch": alg_bytes},
+        "decode": dec, "e2e": e2e, "clocks": clk, "gpu_launches": args.steps,
+        "cpu_baseline": cpu,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+
+
+def cpu_baseline(q, k, v, g, n_tokens):
+    """The fp64 oracle, as it stands, on the first n_tokens tokens of all 24 heads."""
+    from oracle import oracle
+    n = min(n_tokens, N)
+    qc = q[0, :n].cpu()
+    kc = k[0, :n].cpu()
+    vc = v[0, :n].cpu()
+    gc = g[0, :n].cpu()
+    t0 = time.perf_counter()
+    oracle.gret_recurrent(qc, kc, vc, gc)
+    dt = time.perf_counter() - t0
+    return {"value": n / dt / 1e6, "unit": "Mtok/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": "first %d of 32768 tokens, all 24 heads, fp64 recurrent oracle (OpenMP over "
+                      "heads); %.1f s wall" % (n, dt)}
+
+
+def run_reference(args):
+    """Reference arm: the fp64 CPU oracle on host cores (rank 0 only under torchrun)."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import torch
+
+    import synth_inputs as SI
+    from oracle import oracle
+    n = min(args.cpu_tokens, N)
+    inp = SI.gret_inputs(1, n, H, D, dtype=torch.bfloat16, seed=2, device="cpu")
+    q, k, v, g = (inp[x][0] for x in ("q", "k", "v", "g"))
+    for _ in range(args.warmup):
+        oracle.gret_recurrent(q, k, v, g)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.gret_recurrent(q, k, v, g)
+    dt = time.perf_counter() - t0
+    value = n * args.steps / dt / 1e6
+    sample = ("first %d of 32768 tokens of the 3B-shaped prefill, all 24 heads, fp64 recurrent "
+              "oracle per step" % n)
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "Mtok/s",
+        "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD},
+        "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": oracle.threads(),
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-tokens", type=int, default=32768)
+    ap.add_argument("--no-cpu", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "native":
+        args.warmup = 3
+    if args.impl == "reference":
+        if args.cpu_tokens == 32768:
+            args.cpu_tokens = 4096
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

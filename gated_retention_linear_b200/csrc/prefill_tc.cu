@@ -28,17 +28,19 @@
 // ticket, so the chain always progresses.
 //
 // Warp roles (384 threads = 3 warpgroups, one CTA per SM):
-//   warp 0      TMA producer: K, V (and Q in pass B) tiles, two pipeline stages
+//   warp 0      TMA producer (lane 0): K, V (and Q in pass B) tiles, two pipeline stages;
+//               the whole warp scans the chunk's gate logits into the stage's gate slot
 //   warp 1      tcgen05 MMA issuer (one thread); owns the 512-column TMEM allocation
-//   warps 2-3   idle (they complete the first warpgroup, whose registers are given away)
+//   warps 2-3   "convert group": V tiles to fp16 as they land, Q tiles to fp16 after Q K^T
 //   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16) and the output
 //               epilogue O + exp(c_t) OX -> bf16 -> global
 //   warps 8-11  "state group": row scaling of K, the fp32 state (one row per thread), the
 //               look-back, and the bf16 copy of the state that the next Q S_prev MMA reads
-// Registers: launched at 168 per thread; the first warpgroup drops to 56, the P group rises to
-// 184 and the state group (128 fp32 state values per thread) to 232: 128 x (56 + 184 + 232)
-// = 60416 <= 384 x 158, so the split fits any launch allocation of at least 158 per thread,
-// and each SM sub-partition (one warp of each group) needs 32 x 472 <= 16384 registers.
+// Registers: launched at 168 per thread (384 x 168 = 64512); the first warpgroup drops to 88,
+// the P group moves to 160 and the state group (128 fp32 state values per thread) rises to 256:
+// 128 x (88 + 160 + 256) = 64512, exactly the launch allocation, and each SM sub-partition (one
+// warp of each group) needs 32 x 504 <= 16384.  The host refuses to launch a build whose
+// per-thread register count is not 168, since a larger request than the block holds would wait.
 // TMEM columns: [0,128) A / P, [128,256) O, [256,384) OX, [384,512) dS.
 // Every wait is bounded (see sm100::mbar_wait); a wait that gives up records GRET_ERR_TIMEOUT in
 // the workspace, and the kernel drains its copies, frees TMEM and exits.
@@ -87,15 +89,16 @@ struct __align__(1024) Smem {
     unsigned char sbf[TILE];   // bf16 copy of the entry state for the Q S_prev MMA
     uint64_t kv_full[2], stage_empty[2];
     uint64_t item_full[ITEM_DEPTH], item_empty[ITEM_DEPTH];
-    uint64_t a_full, q16_ready, p_ready, o_full, o_free, v16_ready, k_ready, ds_full, ds_free,
-        s_ready, drain;
+    uint64_t v16_ready[2];     // per stage: V tile converted to fp16 (convert group)
+    uint64_t a_full, q16_ready, p_ready, o_full, o_free, k_ready, ds_full, ds_free, s_ready, drain;
     Item items[ITEM_DEPTH];
-    float cP[C];               // P group: in-chunk cumulative log2-decay of each token
-    float wsum[2][4];          // warp totals of the two scans (P group, state group)
-    float red[2][4];           // warp maxima of the tile-scale reductions
-    float sig_v[2];            // power-of-two scale of the fp16 V tile, by job parity
+    float gc[2][C];            // per stage: in-chunk inclusive cumulative log2-decay of each token
+    float gtot[2];             // per stage: the chunk's total log2-decay
+    float red[3][4];           // warp maxima of the tile-scale reductions (per group)
+    float sig_v[2];            // per stage: power-of-two scale of the fp16 V tile
+    float sq[2][C];            // per pass-B chunk parity: power-of-two scale of each fp16 Q row
     float sig_s[2];            // power-of-two scale of the fp16 entry state, by pass-B chunk parity
-    uint32_t dec[2][2];        // group-uniform wait decisions (double-buffered)
+    uint32_t dec[3][2];        // group-uniform wait decisions (double-buffered)
     uint32_t tmem_base;
     uint32_t abort;
 };
@@ -131,8 +134,8 @@ __device__ __forceinline__ float logsigmoid_(float x) {
     return fminf(x, 0.f) - log1pf(expf(-fabsf(x)));
 }
 
-__device__ __forceinline__ void named_sync(int id) {
-    asm volatile("bar.sync %0, 128;" ::"r"(id) : "memory");
+__device__ __forceinline__ void named_sync(int id, int nthreads = 128) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 __device__ __forceinline__ void set_error(uint32_t* err) { atomicExch(err, WS_ERR_TIMEOUT); }
@@ -148,8 +151,9 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 struct GroupWait {
     Smem* sm;
     const TcParams* p;
-    int gid;      // 0 = P group, 1 = state group
+    int gid;      // 0 = P group, 1 = state group, 2 = convert group
     int tid;      // thread index within the group
+    int nthreads = 128;
     int flip = 0;
 
     __device__ bool wait(uint64_t* bar, uint32_t parity) {
@@ -161,7 +165,7 @@ struct GroupWait {
             }
             sm->dec[gid][flip] = ok ? 0u : 1u;
         }
-        named_sync(1 + gid);
+        named_sync(1 + gid, nthreads);
         bool ok = *reinterpret_cast<volatile uint32_t*>(&sm->dec[gid][flip]) == 0;
         flip ^= 1;
         return ok;
@@ -241,61 +245,106 @@ __device__ __forceinline__ void set_coord(int (&c)[4], int pos_tok, int pos_head
 }
 
 // ----------------------------------------------------------------------------------------------
-// warp 0: TMA producer
+// warp 0: TMA producer (lane 0) and gate scan (all lanes)
+
+// The whole warp computes, for the chunk's 128 tokens (4 consecutive per lane), the in-chunk
+// inclusive cumulative log2-decay c_t = sum of logsigmoid(g)/tau * log2(e) over the chunk up to
+// t (0 past the end of the sequence) and the chunk total, into the stage's gate slot.
+__device__ __forceinline__ void gate_scan(Smem& sm, const TcParams& p, const Item& it, int c, int st,
+                                          int lane) {
+    float lam[4];
+    const int64_t t0 = (int64_t)c * C + 4 * lane;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {   // all four loads in flight before any use
+        const int64_t t = (t0 + e < it.len) ? t0 + e : 0;
+        lam[e] = __ldg(p.g + (it.grow0 + t) * p.H + it.h);
+    }
+#pragma unroll
+    for (int e = 0; e < 4; ++e)
+        lam[e] = (t0 + e < it.len) ? logsigmoid_(lam[e]) * p.inv_tau_log2e : 0.f;
+    lam[1] += lam[0];
+    lam[2] += lam[1];
+    lam[3] += lam[2];
+    float x = lam[3];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const float y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+    }
+    const float excl = x - lam[3];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) sm.gc[st][4 * lane + e] = excl + lam[e];
+    if (lane == 31) sm.gtot[st] = x;
+}
 
 __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
-                         const CUtensorMap* tv, uint32_t total) {
+                         const CUtensorMap* tv, uint32_t total, int lane) {
     int j = 0, it_n = 0;
     bool aborted = false;
     while (!aborted) {
         const int slot = it_n % ITEM_DEPTH;
-        if (it_n >= ITEM_DEPTH &&
-            !mbar_wait(&sm.item_empty[slot], ((it_n / ITEM_DEPTH) - 1) & 1, &sm.abort, WAIT_NS)) {
+        int ok = 1;
+        if (lane == 0 && it_n >= ITEM_DEPTH)
+            ok = mbar_wait(&sm.item_empty[slot], ((it_n / ITEM_DEPTH) - 1) & 1, &sm.abort, WAIT_NS);
+        if (!__shfl_sync(0xffffffffu, ok, 0)) {
             aborted = true;
             break;
         }
-        const uint32_t ticket = atomicAdd(p.ticket, 1u);
+        uint32_t ticket = 0;
+        if (lane == 0) ticket = atomicAdd(p.ticket, 1u);
+        ticket = __shfl_sync(0xffffffffu, ticket, 0);
         Item it;
         decode_ticket(p, ticket, total, it);
-        sm.items[slot] = it;
-        mbar_arrive(&sm.item_full[slot]);
+        if (lane == 0) {
+            sm.items[slot] = it;
+            mbar_arrive(&sm.item_full[slot]);
+        }
         ++it_n;
         if (!it.valid) break;
         for (int pass = 0; pass < 2 && !aborted; ++pass) {
             for (int c = it.c_begin; c < it.c_end; ++c) {
                 const int st = j & 1;
-                if (j >= 2 &&
-                    !mbar_wait(&sm.stage_empty[st], ((j >> 1) - 1) & 1, &sm.abort, WAIT_NS)) {
+                ok = 1;
+                if (lane == 0 && j >= 2)
+                    ok = mbar_wait(&sm.stage_empty[st], ((j >> 1) - 1) & 1, &sm.abort, WAIT_NS);
+                if (!__shfl_sync(0xffffffffu, ok, 0)) {
                     aborted = true;
                     break;
                 }
-                mbar_arrive_expect_tx(&sm.kv_full[st], pass ? 3 * TILE : 2 * TILE);
-                const int tok = (int)(it.tok_first + (int64_t)c * C);
-                int ck[4], cv[4];
-                for (int half = 0; half < 2; ++half) {
-                    set_coord(ck, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b, half * 64, tok, it.h,
-                              it.b);
-                    set_coord(cv, p.v_pos_tok, p.v_pos_head, p.v_pos_b, half * 64, tok, it.h,
-                              it.b);
-                    tma_load_4d(sm.k[st] + half * SLAB, tk, &sm.kv_full[st], ck[0], ck[1], ck[2],
-                                ck[3]);
-                    tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], cv[0], cv[1], cv[2],
-                                cv[3]);
-                    if (pass)
-                        tma_load_4d(sm.q[st] + half * SLAB, tq, &sm.kv_full[st], ck[0], ck[1],
+                if (lane == 0) {
+                    mbar_arrive_expect_tx(&sm.kv_full[st], pass ? 3 * TILE : 2 * TILE);
+                    const int tok = (int)(it.tok_first + (int64_t)c * C);
+                    int ck[4], cv[4];
+                    for (int half = 0; half < 2; ++half) {
+                        set_coord(ck, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b, half * 64, tok, it.h,
+                                  it.b);
+                        set_coord(cv, p.v_pos_tok, p.v_pos_head, p.v_pos_b, half * 64, tok, it.h,
+                                  it.b);
+                        tma_load_4d(sm.k[st] + half * SLAB, tk, &sm.kv_full[st], ck[0], ck[1],
                                     ck[2], ck[3]);
+                        tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], cv[0], cv[1],
+                                    cv[2], cv[3]);
+                        if (pass)
+                            tma_load_4d(sm.q[st] + half * SLAB, tq, &sm.kv_full[st], ck[0], ck[1],
+                                        ck[2], ck[3]);
+                    }
                 }
+                gate_scan(sm, p, it, c, st, lane);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.kv_full[st]);
                 ++j;
             }
         }
     }
-    if (aborted) {
-        set_error(p.err);
-        atomicExch(&sm.abort, 1u);
+    if (lane == 0) {
+        if (aborted) {
+            set_error(p.err);
+            atomicExch(&sm.abort, 1u);
+        }
+        // make sure no TMA write into this CTA's shared memory is still in flight at exit
+        for (int jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj)
+            mbar_wait_drain(&sm.kv_full[jj & 1], (jj >> 1) & 1, DRAIN_NS);
     }
-    // make sure no TMA write into this CTA's shared memory is still in flight at exit
-    for (int jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj)
-        mbar_wait_drain(&sm.kv_full[jj & 1], (jj >> 1) & 1, DRAIN_NS);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -340,7 +389,7 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
         for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j) {
             const int st = j & 1;
             if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
-            if (!W(&sm.v16_ready, j & 1)) break;
+            if (!W(&sm.v16_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.k_ready, j & 1)) break;
             if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
             tc_fence_after();
@@ -362,7 +411,7 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
             tc_fence_after();
             mma_128(tmem + TM_OX, smem_u32(sm.q[st]), false, sbf, true, false);
             if (!W(&sm.p_ready, b & 1)) break;
-            if (!W(&sm.v16_ready, j & 1)) break;
+            if (!W(&sm.v16_ready[st], (j >> 1) & 1)) break;
             tc_fence_after();
             {
                 const uint32_t idesc = idesc_f16(128, 128, 0, 1);
@@ -400,77 +449,54 @@ __device__ __forceinline__ float pow2_scale(float mx) {
     return __uint_as_float((uint32_t)(s + 127) << 23);
 }
 
-__device__ __forceinline__ float group_max(Smem& sm, int gid, int q, int lane, float x) {
+// Max over a 128-thread group (warp q = 0..3 of the group), or a 64-thread group (q = 0..1).
+__device__ __forceinline__ float group_max(Smem& sm, int gid, int q, int lane, float x,
+                                           int nwarps = 4) {
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
     if (lane == 0) sm.red[gid][q] = x;
-    named_sync(1 + gid);
-    const float m = fmaxf(fmaxf(sm.red[gid][0], sm.red[gid][1]), fmaxf(sm.red[gid][2], sm.red[gid][3]));
+    named_sync(1 + gid, 32 * nwarps);
+    float m = sm.red[gid][0];
+    for (int w = 1; w < nwarps; ++w) m = fmaxf(m, sm.red[gid][w]);
     return m;
 }
 
-// gate scan: thread r (row r = 32 * (warp % 4) + lane) gets the inclusive cumulative
-// log2-decay c_r of its token, and the chunk total.
-__device__ __forceinline__ float chunk_scan(Smem& sm, const TcParams& p, const Item& it, int c,
-                                            int r, int q, int lane, int gid, float& total) {
-    const int64_t t = (int64_t)c * C + r;
-    float lam = 0.f;
-    if (t < it.len) lam = logsigmoid_(p.g[(it.grow0 + t) * p.H + it.h]) * p.inv_tau_log2e;
-    float x = lam;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        float y = __shfl_up_sync(0xffffffffu, x, o);
-        if (lane >= o) x += y;
-    }
-    if (lane == 31) sm.wsum[gid][q] = x;
-    named_sync(1 + gid);
-    float pre = 0.f;
-    total = 0.f;
-#pragma unroll
-    for (int w = 0; w < 4; ++w) {
-        const float s = sm.wsum[gid][w];
-        if (w < q) pre += s;
-        total += s;
-    }
-    return x + pre;
-}
-
 // Max |x| over one 128-element bf16 row of a swizzled tile (rows are 128-byte lines in each of
-// the two 64-column slabs; the in-line chunk order does not matter for row-wise work).
+// the two 64-column slabs).  Row-wise work does not care about the order of the 16-byte chunks
+// in a line, so thread r visits chunk slot c ^ (r % 8): the 8 rows of a swizzle atom then hit 8
+// different bank groups on every step, instead of all 32 lanes hitting the same 4 banks.
 __device__ __forceinline__ float row_absmax_bf16(const unsigned char* tile, int r) {
-    float m = 0.f;
+    __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         const uint4* line = reinterpret_cast<const uint4*>(tile + half * SLAB + r * 128);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            uint4 u = line[c];
+            uint4 u = line[c ^ (r & 7)];
             const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(h2[e]);
-                m = fmaxf(m, fmaxf(fabsf(f.x), fabsf(f.y)));
-            }
+            for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h2[e]));
         }
     }
-    return m;
+    return fmaxf(__low2float(m2), __high2float(m2));
 }
 
-// In place: bf16 row -> fp16(row * scale).
+// In place: bf16 row -> fp16(row * scale) (same chunk order as row_absmax_bf16).
 __device__ __forceinline__ void row_bf16_to_f16(unsigned char* tile, int r, float scale) {
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         uint4* line = reinterpret_cast<uint4*>(tile + half * SLAB + r * 128);
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            uint4 u = line[c];
+            const int cs = c ^ (r & 7);
+            uint4 u = line[cs];
             uint32_t* w = reinterpret_cast<uint32_t*>(&u);
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
                 w[e] = pack_f16x2(f.x * scale, f.y * scale);
             }
-            line[c] = u;
+            line[cs] = u;
         }
     }
 }
@@ -494,53 +520,56 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
         j += it.c_end - it.c_begin;     // the span's pass-A jobs
         for (int c = it.c_begin; c < it.c_end; ++c, ++b, ++j) {
             const int st = j & 1;
-            float tot;
-            const float cr = chunk_scan(sm, p, it, c, r, q, lane, 0, tot);
-            sm.cP[r] = cr;
-            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }   // also publishes cP
+            // a_full first: this group waits only on pass-B chunks, and a parity wait on
+            // kv_full is exact only once Q K^T of this chunk (hence its load) has completed.
+            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }  // gate slot
+            const float cr = sm.gc[st][r];
             tc_fence_after();
-            // Q row r -> fp16 with its own power-of-two scale (Q K^T has consumed the bf16 Q)
-            const float sq = pow2_scale(row_absmax_bf16(sm.q[st], r));
-            row_bf16_to_f16(sm.q[st], r, sq);
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.q16_ready);
-            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, in fp32, then fp16 with a
-            // per-row power-of-two scale
-            float pv[C];
-            float pmax = 0.f;
+            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, rounded to fp16 after a per-row
+            // power-of-two scale.  The scale comes from the bound |P| <= k_scale |A| (decay <= 1):
+            // a first pass over the row of A finds max |A|, the second computes and packs P.
+            float amax = 0.f;
+#pragma unroll 1
+            for (int jc = 0; jc <= q; ++jc) {
+                float a[32];
+                tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
+                tmem_ld_wait();
 #pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (jc * 32 + i <= r) amax = fmaxf(amax, fabsf(a[i]));
+            }
+            const float rho = pow2_scale(amax * p.k_scale);
+            const float ksr = p.k_scale * rho;
+#pragma unroll 1
             for (int jc = 0; jc < 4; ++jc) {
+                uint32_t pk[16];
                 if (jc <= q) {
                     float a[32];
                     tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
                     tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int m = jc * 32 + i;
-                        const float v = (m <= r) ? ex2f(cr - sm.cP[m]) * p.k_scale * a[i] : 0.f;
-                        pv[m] = v;
-                        pmax = fmaxf(pmax, fabsf(v));
+                    for (int i = 0; i < 16; ++i) {
+                        const int m0 = jc * 32 + 2 * i;
+                        const float p0 = (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * ksr * a[2 * i] : 0.f;
+                        const float p1 =
+                            (m0 + 1 <= r) ? ex2f(cr - sm.gc[st][m0 + 1]) * ksr * a[2 * i + 1] : 0.f;
+                        pk[i] = pack_f16x2(p0, p1);
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 32; ++i) pv[jc * 32 + i] = 0.f;
+                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
                 }
-            }
-            const float rho = pow2_scale(pmax);
-#pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                uint32_t pk[16];
-#pragma unroll
-                for (int i = 0; i < 16; ++i)
-                    pk[i] = pack_f16x2(pv[jc * 32 + 2 * i] * rho, pv[jc * 32 + 2 * i + 1] * rho);
+                // columns [16 jc, 16 jc + 16) hold A values already read (chunks <= jc)
                 tmem_st16(tmem + lane_base + TM_A + jc * 16, pk);
             }
             // scales of V and of the entry state for this chunk (both published before their
             // barriers complete; waiting here, before p_ready, cannot miss a phase)
-            if (!gw.wait(&sm.v16_ready, j & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.v16_ready[st], (j >> 1) & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.q16_ready, b & 1)) { ok = false; break; }
             if (!gw.wait(&sm.s_ready, b & 1)) { ok = false; break; }
-            const float inv_pv = 1.f / (rho * sm.sig_v[j & 1]);
-            const float inv_qs = 1.f / (sq * sm.sig_s[b & 1]);
+            const float inv_pv = 1.f / (rho * sm.sig_v[st]);
+            const float inv_qs = 1.f / (sm.sq[b & 1][r] * sm.sig_s[b & 1]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&sm.p_ready);
@@ -585,12 +614,6 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
 // ----------------------------------------------------------------------------------------------
 // warps 8-11: V and decayed K to fp16, fp32 state, look-back
 
-// V tile -> fp16 with one power-of-two scale for the tile; returns the scale.
-__device__ __forceinline__ float convert_v(Smem& sm, unsigned char* vtile, int r, int q, int lane) {
-    const float sv = pow2_scale(group_max(sm, 1, q, lane, row_absmax_bf16(vtile, r)));
-    row_bf16_to_f16(vtile, r, sv);
-    return sv;
-}
 
 // K tile -> fp16 rows w_r * K_r with one power-of-two scale for the tile; returns the scale.
 __device__ __forceinline__ float convert_k(Smem& sm, unsigned char* ktile, int r, int q, int lane,
@@ -662,15 +685,12 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         for (int c = it.c_begin; c < it.c_end; ++c, ++j) {
             const int st = j & 1;
             if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
-            float tot;
-            const float cr = chunk_scan(sm, p, it, c, r, q, lane, 1, tot);
+            const float cr = sm.gc[st][r], tot = sm.gtot[st];
             const bool valid = (int64_t)c * C + r < it.len;
-            const float sv = convert_v(sm, sm.v[st], r, q, lane);
-            if (r == 0) sm.sig_v[j & 1] = sv;
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.v16_ready);
             const float sk = convert_k(sm, sm.k[st], r, q, lane, valid ? ex2f(tot - cr) * p.k_scale : 0.f);
             fence_proxy_async_smem();
+            if (!gw.wait(&sm.v16_ready[st], (j >> 1) & 1)) { ok = false; break; }
+            const float sv = sm.sig_v[st];
             mbar_arrive(&sm.k_ready);
             if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
             tc_fence_after();
@@ -694,25 +714,35 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         const float eL = ex2f(L);
         float4* dst = it.last ? nullptr
                               : reinterpret_cast<float4*>(p.slots + (chain * 2 + (it.s & 1)) * (D * D));
+        // two batches of 16 independent loads each, then the inclusive state and the swap
 #pragma unroll
-        for (int j4 = 0; j4 < D / 4; ++j4) {
-            float4 e = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (from_slot)
-                e = __ldcg(reinterpret_cast<const float4*>(esrc) + j4 * D + r);
-            else if (esrc)
-                e = reinterpret_cast<const float4*>(esrc)[j4];
-            if (dst) {
-                float4 inc;
-                inc.x = fmaf(eL, e.x, S[4 * j4 + 0]);
-                inc.y = fmaf(eL, e.y, S[4 * j4 + 1]);
-                inc.z = fmaf(eL, e.z, S[4 * j4 + 2]);
-                inc.w = fmaf(eL, e.w, S[4 * j4 + 3]);
-                __stcg(dst + j4 * D + r, inc);
+        for (int half = 0; half < 2; ++half) {
+            float4 e[16];
+#pragma unroll
+            for (int k4 = 0; k4 < 16; ++k4) {
+                const int j4 = half * 16 + k4;
+                e[k4] = make_float4(0.f, 0.f, 0.f, 0.f);
+                if (from_slot)
+                    e[k4] = __ldcg(reinterpret_cast<const float4*>(esrc) + j4 * D + r);
+                else if (esrc)
+                    e[k4] = __ldg(reinterpret_cast<const float4*>(esrc) + j4);
             }
-            S[4 * j4 + 0] = e.x;
-            S[4 * j4 + 1] = e.y;
-            S[4 * j4 + 2] = e.z;
-            S[4 * j4 + 3] = e.w;
+#pragma unroll
+            for (int k4 = 0; k4 < 16; ++k4) {
+                const int j4 = half * 16 + k4;
+                if (dst) {
+                    float4 inc;
+                    inc.x = fmaf(eL, e[k4].x, S[4 * j4 + 0]);
+                    inc.y = fmaf(eL, e[k4].y, S[4 * j4 + 1]);
+                    inc.z = fmaf(eL, e[k4].z, S[4 * j4 + 2]);
+                    inc.w = fmaf(eL, e[k4].w, S[4 * j4 + 3]);
+                    __stcg(dst + j4 * D + r, inc);
+                }
+                S[4 * j4 + 0] = e[k4].x;
+                S[4 * j4 + 1] = e[k4].y;
+                S[4 * j4 + 2] = e[k4].z;
+                S[4 * j4 + 3] = e[k4].w;
+            }
         }
         if (dst) {
             __threadfence();
@@ -727,16 +757,14 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         // ---- pass B: running state from E
         for (int c = it.c_begin; c < it.c_end; ++c, ++j, ++b) {
             const int st = j & 1;
-            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
-            float tot;
-            const float cr = chunk_scan(sm, p, it, c, r, q, lane, 1, tot);
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
+            const float cr = sm.gc[st][r], tot = sm.gtot[st];
             const bool valid = (int64_t)c * C + r < it.len;
-            const float sv = convert_v(sm, sm.v[st], r, q, lane);
-            if (r == 0) sm.sig_v[j & 1] = sv;
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.v16_ready);
+            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }  // Q K^T done with K
             const float sk = convert_k(sm, sm.k[st], r, q, lane, valid ? ex2f(tot - cr) * p.k_scale : 0.f);
             fence_proxy_async_smem();
+            if (!gw.wait(&sm.v16_ready[st], (j >> 1) & 1)) { ok = false; break; }
+            const float sv = sm.sig_v[st];
             mbar_arrive(&sm.k_ready);
             if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
             tc_fence_after();
@@ -756,6 +784,53 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
     }
 }
 
+// ----------------------------------------------------------------------------------------------
+// warps 2-3: V tile to fp16 as soon as it lands (every chunk), Q tile to fp16 after Q K^T
+// (pass-B chunks).  64 threads, two rows each.
+
+__device__ void convert_group(Smem& sm, const TcParams& p, int warp, int lane) {
+    GroupWait gw{&sm, &p, 2, (warp - 2) * 32 + lane, 64};
+    const int w = warp - 2, t = w * 32 + lane;     // rows t and t + 64
+    int j = 0, b = 0, it_n = 0;
+    bool ok = true;
+    while (ok) {
+        const int slot = it_n % ITEM_DEPTH;
+        if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
+        const Item it = sm.items[slot];
+        mbar_arrive(&sm.item_empty[slot]);
+        ++it_n;
+        if (!it.valid) break;
+        const int n_ch = it.c_end - it.c_begin;
+        for (int jj = 0; jj < 2 * n_ch; ++jj, ++j) {
+            const int st = j & 1;
+            const bool passb = jj >= n_ch;
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
+            // V: one power-of-two scale for the tile
+            const float m = fmaxf(row_absmax_bf16(sm.v[st], t), row_absmax_bf16(sm.v[st], t + 64));
+            const float sv = pow2_scale(group_max(sm, 2, w, lane, m, 2));
+            row_bf16_to_f16(sm.v[st], t, sv);
+            row_bf16_to_f16(sm.v[st], t + 64, sv);
+            if (t == 0) sm.sig_v[st] = sv;
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.v16_ready[st]);
+            if (passb) {
+                // Q: a power-of-two scale per row, once Q K^T has read the bf16 Q
+                if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
+#pragma unroll
+                for (int h2 = 0; h2 < 2; ++h2) {
+                    const int row = t + 64 * h2;
+                    const float sq = pow2_scale(row_absmax_bf16(sm.q[st], row));
+                    row_bf16_to_f16(sm.q[st], row, sq);
+                    sm.sq[b & 1][row] = sq;
+                }
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.q16_ready);
+                ++b;
+            }
+        }
+    }
+}
+
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, const TcParams p, uint32_t total_dense) {
@@ -768,19 +843,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_full[s], 2);   // TMA bytes + expect_tx arrival, gate arrival
             mbar_init(&sm.stage_empty[s], 1);
         }
         for (int s = 0; s < ITEM_DEPTH; ++s) {
             mbar_init(&sm.item_full[s], 1);
-            mbar_init(&sm.item_empty[s], 1 + 128 + 128);
+            mbar_init(&sm.item_empty[s], 1 + 128 + 128 + 64);
         }
         mbar_init(&sm.a_full, 1);
-        mbar_init(&sm.q16_ready, 128);
+        mbar_init(&sm.q16_ready, 64);
+        mbar_init(&sm.v16_ready[0], 64);
+        mbar_init(&sm.v16_ready[1], 64);
         mbar_init(&sm.p_ready, 128);
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.o_free, 128);
-        mbar_init(&sm.v16_ready, 128);
         mbar_init(&sm.k_ready, 128);
         mbar_init(&sm.ds_full, 1);
         mbar_init(&sm.ds_free, 128);
@@ -798,24 +874,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
         if (warp == 0) {
             if (lane == 0) {
                 tma_prefetch_desc(&tq);
                 tma_prefetch_desc(&tk);
                 tma_prefetch_desc(&tv);
-                const uint32_t total =
-                    p.prefix ? (uint32_t)p.prefix[p.units] * (uint32_t)p.H : total_dense;
-                producer(sm, p, &tq, &tk, &tv, total);
             }
+            const uint32_t total =
+                p.prefix ? (uint32_t)p.prefix[p.units] * (uint32_t)p.H : total_dense;
+            producer(sm, p, &tq, &tk, &tv, total, lane);
         } else if (warp == 1) {
             if (lane == 0) mma_issuer(sm, p, tmem);
+        } else {
+            convert_group(sm, p, warp, lane);
         }
     } else if (warp < 8) {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 200;" ::: "memory");
+        // 168 -> 160 is a decrease: setmaxnreg.inc must never ask for fewer registers than the
+        // warp holds, and .dec never for more.
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 160;" ::: "memory");
         p_group(sm, p, tmem, warp, lane);
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 256;" ::: "memory");
         state_group(sm, p, tmem, warp, lane);
     }
     tc_fence_before();
@@ -925,8 +1005,8 @@ int span_chunks() {
     static int g = -1;
     if (g < 0) {
         const char* e = getenv("GRET_SPAN_CHUNKS");
-        g = e ? atoi(e) : 4;
-        if (g < 1) g = 4;
+        g = e ? atoi(e) : 8;
+        if (g < 1) g = 8;
     }
     return g;
 }
@@ -982,6 +1062,16 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
     if (cudaFuncSetAttribute(prefill_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return GRET_ERR_CUDA;
+    {
+        // the in-kernel register split (setmaxnreg) assumes exactly 168 registers per thread
+        static int regs = -1;
+        if (regs < 0) {
+            cudaFuncAttributes fa;
+            if (cudaFuncGetAttributes(&fa, prefill_tc_kernel) != cudaSuccess) return GRET_ERR_CUDA;
+            regs = fa.numRegs;
+        }
+        if (regs != 168) return GRET_ERR_UNSUPPORTED;
+    }
     int grid = sm_count();
     if (!varlen && total_dense < (uint64_t)grid) grid = (int)total_dense;
     if (grid < 1) grid = 1;
