@@ -2,21 +2,28 @@
 //
 // Method: page "YOCO 完全拆解：Decoder-Decoder 架构如何让 KV Cache 只存一次", section
 // "Prefill 与 Decode 为什么使用两种计算形态".  Each chunk of C = 128 tokens of one head is done
-// with four 128x128x128 bf16 tcgen05 MMAs accumulating in fp32 tensor memory:
-//     A   = Q K^T                       (intra-chunk scores)
-//     P   = k_scale * exp(c_t - c_m) * A for m <= t, else 0     (decay mask, CUDA cores, bf16)
+// with 128x128x128 tcgen05 MMAs accumulating in fp32 tensor memory:
+//     A   = Q K^T                       (intra-chunk scores, exact from the bf16 inputs)
+//     P   = k_scale * exp(c_t - c_m) * A for m <= t, else 0     (decay mask, CUDA cores)
 //     O   = P V                         (inner term)
 //     OX  = Q S_prev                    (cross-chunk term; added as exp(c_t) * OX)
 //     dS  = (w K)^T V,  w_m = k_scale * exp(c_b - c_m)     (chunk contribution to the state)
 //     S   = exp(c_b) S_prev + dS        (fp32 master state, in registers)
-// c_t is the in-chunk inclusive cumulative log-decay (a warp-shuffle scan of logsigmoid(g)/tau),
-// always used as a difference inside one chunk, so no exponent can overflow.
+// c_t is the in-chunk inclusive cumulative log-decay (a warp scan of logsigmoid(g)/tau), always
+// used as a difference inside one chunk, so no exponent can overflow.
+//
+// Precision.  P, the state copy and w K are fp32 values that an MMA needs as bf16.  Rounding
+// each to bf16 once costs up to 2^-8 relative per element and, measured against an fp64
+// reference, left errors of 1-3% of rms on large outputs.  Each is therefore split into a bf16
+// high half and a bf16 low half (x - hi), and both halves go through the MMA: P V and Q S_prev
+// and (w K)^T V are each two MMAs, which keeps them within a few 1e-6 of fp32.  V and Q are used
+// exactly as loaded.
 //
 // Parallelism across a sequence.  The chunk chain of one (sequence, head) is sequential, and
 // one 3B-shaped layer has only 24 chains for 148 SMs.  Each chain is therefore cut into spans
 // of G chunks.  A persistent CTA takes spans from an atomic ticket in chain order and runs:
 //   pass A: read K, V, g of the span and fold them into the span's aggregate state
-//           Agg = sum over chunks (decay to the span end) of dS        (MMA dS only)
+//           Agg = sum over chunks (decay to the span end) of dS        (dS MMAs only)
 //   look-back: wait for the inclusive state of span s-1 of the same chain (a bounded spin on a
 //           flag in the workspace), entry E = that state (or state_in for s = 0), and publish
 //           the inclusive state exp(L_span) E + Agg for span s+1;
@@ -31,17 +38,18 @@
 //   warp 0      TMA producer (lane 0): K, V (and Q in pass B) tiles, two pipeline stages;
 //               the whole warp scans the chunk's gate logits into the stage's gate slot
 //   warp 1      tcgen05 MMA issuer (one thread); owns the 512-column TMEM allocation
-//   warps 2-3   "convert group": V tiles to fp16 as they land, Q tiles to fp16 after Q K^T
-//   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16) and the output
-//               epilogue O + exp(c_t) OX -> bf16 -> global
-//   warps 8-11  "state group": row scaling of K, the fp32 state (one row per thread), the
-//               look-back, and the bf16 copy of the state that the next Q S_prev MMA reads
+//   warps 2-3   their share of the w K split (5 of the 16 chunks of every row)
+//   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16 halves) and the
+//               output epilogue O + exp(c_t) OX -> bf16 -> global
+//   warps 8-11  "state group": w K split into halves, the fp32 state (one row per thread), the
+//               look-back, and the bf16 halves of the state that Q S_prev reads
 // Registers: launched at 168 per thread (384 x 168 = 64512); the first warpgroup drops to 88,
-// the P group moves to 160 and the state group (128 fp32 state values per thread) rises to 256:
-// 128 x (88 + 160 + 256) = 64512, exactly the launch allocation, and each SM sub-partition (one
-// warp of each group) needs 32 x 504 <= 16384.  The host refuses to launch a build whose
-// per-thread register count is not 168, since a larger request than the block holds would wait.
-// TMEM columns: [0,128) A / P, [128,256) O, [256,384) OX, [384,512) dS.
+// the P group to 136 and the state group (128 fp32 state values per thread) rises to 256:
+// 128 x (88 + 136 + 256) = 61440 <= 64512, and each SM sub-partition (one warp of each group)
+// needs 32 x 480 <= 16384.  The host refuses to launch a build whose per-thread register count
+// is not 168, since a request for more registers than the block holds would wait forever.
+// TMEM columns: [0,128) A, then P (bf16 halves, see mma_pv); [128,256) O; [256,384) OX;
+// [384,512) dS.
 // Every wait is bounded (see sm100::mbar_wait); a wait that gives up records GRET_ERR_TIMEOUT in
 // the workspace, and the kernel drains its copies, frees TMEM and exits.
 #include "prefill_tc.cuh"
@@ -83,21 +91,22 @@ struct Item {
 };
 
 struct __align__(1024) Smem {
-    unsigned char q[2][TILE];
-    unsigned char k[2][TILE];
+    unsigned char q[2][TILE];  // Q tile; in pass A, and after Q S in pass B, the low half of w K
+    unsigned char k[2][TILE];  // K tile; rewritten in place as the high half of w K
     unsigned char v[2][TILE];
-    unsigned char sbf[TILE];   // bf16 copy of the entry state for the Q S_prev MMA
+    unsigned char sbf[TILE];   // bf16 high half, then low half, of the entry state (Q S_prev)
     uint64_t kv_full[2], stage_empty[2];
     uint64_t item_full[ITEM_DEPTH], item_empty[ITEM_DEPTH];
-    uint64_t v16_ready[2];     // per stage: V tile converted to fp16 (convert group)
-    uint64_t a_full, q16_ready, p_ready, o_full, o_free, k_ready, ds_full, ds_free, s_ready, drain;
+    // k_ready / kh_ready (per stage): the state group's / the helpers' share of the w K split
+    // is written.  Each has one producing group, so arrivals of different groups never mix, and
+    // being per stage, a group can reach the next phase of a stage's barrier only after the MMA
+    // has released that stage -- so no waiter can be left two phases behind.
+    uint64_t k_ready[2], kh_ready[2];
+    uint64_t a_full, s3a_done, q_free, p_ready, s_lo_ready, o_full, o_free, ds_full, ds_free,
+        s_ready, drain;
     Item items[ITEM_DEPTH];
     float gc[2][C];            // per stage: in-chunk inclusive cumulative log2-decay of each token
     float gtot[2];             // per stage: the chunk's total log2-decay
-    float red[3][4];           // warp maxima of the tile-scale reductions (per group)
-    float sig_v[2];            // per stage: power-of-two scale of the fp16 V tile
-    float sq[2][C];            // per pass-B chunk parity: power-of-two scale of each fp16 Q row
-    float sig_s[2];            // power-of-two scale of the fp16 entry state, by pass-B chunk parity
     uint32_t dec[3][2];        // group-uniform wait decisions (double-buffered)
     uint32_t tmem_base;
     uint32_t abort;
@@ -151,7 +160,7 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 struct GroupWait {
     Smem* sm;
     const TcParams* p;
-    int gid;      // 0 = P group, 1 = state group, 2 = convert group
+    int gid;      // 0 = P group, 1 = state group, 2 = split helpers
     int tid;      // thread index within the group
     int nthreads = 128;
     int flip = 0;
@@ -350,10 +359,10 @@ __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, con
 // ----------------------------------------------------------------------------------------------
 // warp 1: MMA issuer (one thread)
 
-// D (+)= A B over K = 128, eight K-steps of 16; operands in shared memory.
+// D (+)= A B over K = 128, eight K-steps of 16; bf16 operands in shared memory.
 __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, uint32_t b_base,
-                                        bool b_mn, bool bf16) {
-    const uint32_t idesc = idesc_f16kind(128, 128, a_mn, b_mn, bf16);
+                                        bool b_mn, bool accumulate) {
+    const uint32_t idesc = idesc_bf16(128, 128, a_mn, b_mn);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         const uint32_t aoff = a_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
@@ -362,8 +371,27 @@ __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, 
                                  : sdesc_sw128(a_base + aoff, 16, 1024);
         const uint64_t bd = b_mn ? sdesc_sw128(b_base + boff, SLAB, 1024)
                                  : sdesc_sw128(b_base + boff, 16, 1024);
-        mma_ss(d, ad, bd, idesc, kk > 0);
+        mma_ss(d, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
     }
+}
+
+// D (+)= P V with P (bf16, K-major) in TMEM.  P is stored per 32-token group g = 0..3 as
+// [16 columns of high halves | 16 columns of low halves] at columns 32 g; the K-step of tokens
+// [16 kk, 16 kk + 16) of one half starts at column 32 (kk / 2) + 8 (kk % 2) + 16 * half.
+__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
+                                       bool accumulate) {
+    const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
+               sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
+}
+
+// dS = (w K)^T V as the sum of its bf16 high half (K slot) and low half (Q slot).
+__device__ __forceinline__ void mma_ds(uint32_t tmem, Smem& sm, int st) {
+    mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, false);
+    mma_128(tmem + TM_DS, smem_u32(sm.q[st]), true, smem_u32(sm.v[st]), true, true);
 }
 
 __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
@@ -389,43 +417,50 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
         for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j) {
             const int st = j & 1;
             if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
-            if (!W(&sm.v16_ready[st], (j >> 1) & 1)) break;
-            if (!W(&sm.k_ready, j & 1)) break;
+            if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
+            if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
             if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
             tc_fence_after();
-            mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, false);
+            mma_ds(tmem, sm, st);
             mma_commit(&sm.ds_full);
             mma_commit(&sm.stage_empty[st]);
         }
-        // pass B: the full chunk
+        // pass B: the full chunk.  Order per chunk: Q K^T (issued one chunk ahead), Q S_hi,
+        // Q S_lo (after which the Q slot is free for the low half of w K), P V, then Q K^T of the
+        // next chunk, then dS -- so the decay mask of chunk c + 1 overlaps the state update of c.
+        auto issue_qk = [&](int jj, int bb) {
+            const int st = jj & 1;
+            if (!W(&sm.kv_full[st], (jj >> 1) & 1)) return false;
+            if (bb > 0 && !W(&sm.o_full, (bb - 1) & 1)) return false;   // P of chunk bb-1 used
+            tc_fence_after();
+            mma_128(tmem + TM_A, smem_u32(sm.q[st]), false, smem_u32(sm.k[st]), false, false);
+            mma_commit(&sm.a_full);
+            return true;
+        };
+        if (it.c_end > it.c_begin && !issue_qk(j, b)) break;
         for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j, ++b) {
             const int st = j & 1;
-            if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
-            if (b > 0 && !W(&sm.o_full, (b - 1) & 1)) break;     // A/P region consumed
-            tc_fence_after();
-            mma_128(tmem + TM_A, smem_u32(sm.q[st]), false, smem_u32(sm.k[st]), false, true);
-            mma_commit(&sm.a_full);
-            if (!W(&sm.q16_ready, b & 1)) break;
+            const uint32_t qb = smem_u32(sm.q[st]), vb = smem_u32(sm.v[st]);
             if (!W(&sm.s_ready, b & 1)) break;
             if (b > 0 && !W(&sm.o_free, (b - 1) & 1)) break;     // O, OX read out
             tc_fence_after();
-            mma_128(tmem + TM_OX, smem_u32(sm.q[st]), false, sbf, true, false);
-            if (!W(&sm.p_ready, b & 1)) break;
-            if (!W(&sm.v16_ready[st], (j >> 1) & 1)) break;
+            mma_128(tmem + TM_OX, qb, false, sbf, true, false);   // OX = Q S_hi
+            mma_commit(&sm.s3a_done);
+            if (!W(&sm.s_lo_ready, b & 1)) break;
             tc_fence_after();
-            {
-                const uint32_t idesc = idesc_f16(128, 128, 0, 1);
-                const uint32_t vb = smem_u32(sm.v[st]);
-#pragma unroll
-                for (int kk = 0; kk < 8; ++kk)
-                    mma_ts(tmem + TM_O, tmem + TM_A + kk * 8,
-                           sdesc_sw128(vb + kk * 2048u, SLAB, 1024), idesc, kk > 0);
-            }
+            mma_128(tmem + TM_OX, qb, false, sbf, true, true);    // OX += Q S_lo
+            mma_commit(&sm.q_free);
+            if (!W(&sm.p_ready, b & 1)) break;
+            tc_fence_after();
+            mma_pv(tmem + TM_O, tmem + TM_A, 0, vb, false);        // O  = P_hi V
+            mma_pv(tmem + TM_O, tmem + TM_A, 1, vb, true);         // O += P_lo V
             mma_commit(&sm.o_full);
-            if (!W(&sm.k_ready, j & 1)) break;
+            if (c + 1 < it.c_end && !issue_qk(j + 1, b + 1)) break;
+            if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
+            if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
             if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
             tc_fence_after();
-            mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, false);
+            mma_ds(tmem, sm, st);
             mma_commit(&sm.ds_full);
             mma_commit(&sm.stage_empty[st]);
         }
@@ -436,73 +471,90 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
 }
 
 // ----------------------------------------------------------------------------------------------
-// helpers shared by the two 128-thread groups
+// bf16 splitting: x = hi + lo with hi = bf16(x) and lo = bf16(x - hi).  The pair carries about
+// 16 significant bits, so products with bf16 operands accumulated in fp32 keep the P V, Q S and
+// K^T V contractions within a few 1e-6 of fp32.
 
-// Power of two that maps a magnitude bound `mx` into [2^14, 2^15): operands are rounded to fp16
-// after this scaling (so nothing overflows fp16's 65504 and the largest values keep all 11
-// bits), and the exact reciprocal is applied to the fp32 results.
-__device__ __forceinline__ float pow2_scale(float mx) {
-    if (!(mx > 0.f) || !isfinite(mx)) return 1.f;
-    int e = (int)((__float_as_uint(mx) >> 23) & 0xffu) - 127;   // floor(log2(mx)), normal mx
-    int s = 14 - e;
-    s = s < -126 ? -126 : (s > 127 ? 127 : s);
-    return __uint_as_float((uint32_t)(s + 127) << 23);
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Max over a 128-thread group (warp q = 0..3 of the group), or a 64-thread group (q = 0..1).
-__device__ __forceinline__ float group_max(Smem& sm, int gid, int q, int lane, float x,
-                                           int nwarps = 4) {
+// Chunks [I0, I0 + N) of row r of a swizzled K tile (16 chunks of 8 elements per row; chunk i
+// sits in slab i / 8 at slot (i % 8) ^ (r % 8)): w * K split into a high half written back in
+// place and a low half written to the same position of `lotile`.  All loads are issued before
+// the first store (loads cannot move past stores to the same array).
+template <int I0, int N>
+__device__ __forceinline__ void split_k_chunks(unsigned char* ktile, unsigned char* lotile, int r,
+                                               float w) {
+    uint4 row[N];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) x = fmaxf(x, __shfl_xor_sync(0xffffffffu, x, o));
-    if (lane == 0) sm.red[gid][q] = x;
-    named_sync(1 + gid, 32 * nwarps);
-    float m = sm.red[gid][0];
-    for (int w = 1; w < nwarps; ++w) m = fmaxf(m, sm.red[gid][w]);
-    return m;
-}
-
-// Max |x| over one 128-element bf16 row of a swizzled tile (rows are 128-byte lines in each of
-// the two 64-column slabs).  Row-wise work does not care about the order of the 16-byte chunks
-// in a line, so thread r visits chunk slot c ^ (r % 8): the 8 rows of a swizzle atom then hit 8
-// different bank groups on every step, instead of all 32 lanes hitting the same 4 banks.
-__device__ __forceinline__ float row_absmax_bf16(const unsigned char* tile, int r) {
-    __nv_bfloat162 m2 = __float2bfloat162_rn(0.f);
-#pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        const uint4* line = reinterpret_cast<const uint4*>(tile + half * SLAB + r * 128);
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            uint4 u = line[c ^ (r & 7)];
-            const __nv_bfloat162* h2 = reinterpret_cast<const __nv_bfloat162*>(&u);
-#pragma unroll
-            for (int e = 0; e < 4; ++e) m2 = __hmax2(m2, __habs2(h2[e]));
-        }
+    for (int n = 0; n < N; ++n) {
+        const int i = I0 + n;
+        row[n] = *reinterpret_cast<const uint4*>(ktile + (i >> 3) * SLAB + r * 128 +
+                                                 (((i & 7) ^ (r & 7)) << 4));
     }
-    return fmaxf(__low2float(m2), __high2float(m2));
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        const int i = I0 + n;
+        const int off = (i >> 3) * SLAB + r * 128 + (((i & 7) ^ (r & 7)) << 4);
+        uint32_t* x = reinterpret_cast<uint32_t*>(&row[n]);
+        uint4 lo;
+        uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[e]));
+            split2(f.x * w, f.y * w, x[e], l[e]);
+        }
+        *reinterpret_cast<uint4*>(ktile + off) = row[n];
+        *reinterpret_cast<uint4*>(lotile + off) = lo;
+    }
 }
 
-// In place: bf16 row -> fp16(row * scale) (same chunk order as row_absmax_bf16).
-__device__ __forceinline__ void row_bf16_to_f16(unsigned char* tile, int r, float scale) {
+// The split of w K is shared: the state group takes chunks 0-10 of its own row, warps 2-3 take
+// chunks 11-15 of two rows each.
+constexpr int SPLIT_OWN = 11;
+
+// weight of token r of chunk c: k_scale * exp(c_b - c_r), zero past the end of the sequence
+__device__ __forceinline__ float k_weight(const Smem& sm, const TcParams& p, const Item& it, int c,
+                                          int st, int r) {
+    const bool valid = (int64_t)c * C + r < it.len;
+    return valid ? ex2f(sm.gtot[st] - sm.gc[st][r]) * p.k_scale : 0.f;
+}
+
+// Row r of the state into the MN-major swizzled tile read by Q S: its bf16 high half (LOW ==
+// false) or its low half (LOW == true).
+template <bool LOW>
+__device__ __forceinline__ void write_state_half(unsigned char* tile, int r, const float (&S)[D]) {
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-        uint4* line = reinterpret_cast<uint4*>(tile + half * SLAB + r * 128);
+    for (int cc = 0; cc < 16; ++cc) {
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const int cs = c ^ (r & 7);
-            uint4 u = line[cs];
-            uint32_t* w = reinterpret_cast<uint32_t*>(&u);
+        for (int e = 0; e < 4; ++e) split2(S[8 * cc + 2 * e], S[8 * cc + 2 * e + 1], hi[e], lo[e]);
+        const uint32_t* w = LOW ? lo : hi;
+        const int half = cc >> 3, c = cc & 7;
+        *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+// S = 2^tot * S + dS, dS read from TMEM 32 columns at a time
+__device__ __forceinline__ void fold_ds(uint32_t taddr, float (&S)[D], float eb) {
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const float2 f = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&w[e]));
-                w[e] = pack_f16x2(f.x * scale, f.y * scale);
-            }
-            line[cs] = u;
-        }
+    for (int jc = 0; jc < 4; ++jc) {
+        float d[32];
+        tmem_ld32(taddr + jc * 32, d);
+        tmem_ld_wait();
+#pragma unroll
+        for (int i = 0; i < 32; ++i) S[jc * 32 + i] = fmaf(eb, S[jc * 32 + i], d[i]);
     }
 }
 
 // ----------------------------------------------------------------------------------------------
-// warps 4-7: Q to fp16, decay mask, output epilogue
+// warps 4-7: decay mask (P split into bf16 halves in TMEM) and output epilogue
 
 __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
     GroupWait gw{&sm, &p, 0, (warp - 4) * 32 + lane};
@@ -526,24 +578,11 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
             if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }  // gate slot
             const float cr = sm.gc[st][r];
             tc_fence_after();
-            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, rounded to fp16 after a per-row
-            // power-of-two scale.  The scale comes from the bound |P| <= k_scale |A| (decay <= 1):
-            // a first pass over the row of A finds max |A|, the second computes and packs P.
-            float amax = 0.f;
-#pragma unroll 1
-            for (int jc = 0; jc <= q; ++jc) {
-                float a[32];
-                tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
-                tmem_ld_wait();
+            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, split into bf16 halves; each
+            // 32-column group of A is replaced in place by [16 high | 16 low] columns of P.
 #pragma unroll
-                for (int i = 0; i < 32; ++i)
-                    if (jc * 32 + i <= r) amax = fmaxf(amax, fabsf(a[i]));
-            }
-            const float rho = pow2_scale(amax * p.k_scale);
-            const float ksr = p.k_scale * rho;
-#pragma unroll 1
             for (int jc = 0; jc < 4; ++jc) {
-                uint32_t pk[16];
+                uint32_t ph[32];
                 if (jc <= q) {
                     float a[32];
                     tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
@@ -551,32 +590,24 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         const int m0 = jc * 32 + 2 * i;
-                        const float p0 = (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * ksr * a[2 * i] : 0.f;
+                        const float p0 = (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * p.k_scale * a[2 * i] : 0.f;
                         const float p1 =
-                            (m0 + 1 <= r) ? ex2f(cr - sm.gc[st][m0 + 1]) * ksr * a[2 * i + 1] : 0.f;
-                        pk[i] = pack_f16x2(p0, p1);
+                            (m0 + 1 <= r) ? ex2f(cr - sm.gc[st][m0 + 1]) * p.k_scale * a[2 * i + 1] : 0.f;
+                        split2(p0, p1, ph[i], ph[16 + i]);
                     }
                 } else {
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) pk[i] = 0u;
+                    for (int i = 0; i < 32; ++i) ph[i] = 0u;
                 }
-                // columns [16 jc, 16 jc + 16) hold A values already read (chunks <= jc)
-                tmem_st16(tmem + lane_base + TM_A + jc * 16, pk);
+                tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
             }
-            // scales of V and of the entry state for this chunk (both published before their
-            // barriers complete; waiting here, before p_ready, cannot miss a phase)
-            if (!gw.wait(&sm.v16_ready[st], (j >> 1) & 1)) { ok = false; break; }
-            if (!gw.wait(&sm.q16_ready, b & 1)) { ok = false; break; }
-            if (!gw.wait(&sm.s_ready, b & 1)) { ok = false; break; }
-            const float inv_pv = 1.f / (rho * sm.sig_v[st]);
-            const float inv_qs = 1.f / (sm.sq[b & 1][r] * sm.sig_s[b & 1]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&sm.p_ready);
-            // epilogue: O = O_inner + 2^(c_r) O_cross, each unscaled
+            // epilogue: O = O_inner + 2^(c_r) O_cross
             if (!gw.wait(&sm.o_full, b & 1)) { ok = false; break; }
             tc_fence_after();
-            const float ec = ex2f(cr) * inv_qs;
+            const float ec = ex2f(cr);
             const int64_t t = (int64_t)c * C + r;
             const bool valid = t < it.len;
             __nv_bfloat16* orow = p.o + (int64_t)it.b * p.osb + (it.tok_first + t) * p.ost +
@@ -591,15 +622,15 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
                     uint4* dst = reinterpret_cast<uint4*>(orow + jc * 32);
 #pragma unroll
                     for (int v4 = 0; v4 < 4; ++v4) {
-                        float y[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            y[e] = fmaf(ec, ox[8 * v4 + e], o[8 * v4 + e] * inv_pv);
                         uint4 u;
-                        u.x = pack_bf16x2(y[0], y[1]);
-                        u.y = pack_bf16x2(y[2], y[3]);
-                        u.z = pack_bf16x2(y[4], y[5]);
-                        u.w = pack_bf16x2(y[6], y[7]);
+                        u.x = pack_bf16x2(fmaf(ec, ox[8 * v4 + 0], o[8 * v4 + 0]),
+                                          fmaf(ec, ox[8 * v4 + 1], o[8 * v4 + 1]));
+                        u.y = pack_bf16x2(fmaf(ec, ox[8 * v4 + 2], o[8 * v4 + 2]),
+                                          fmaf(ec, ox[8 * v4 + 3], o[8 * v4 + 3]));
+                        u.z = pack_bf16x2(fmaf(ec, ox[8 * v4 + 4], o[8 * v4 + 4]),
+                                          fmaf(ec, ox[8 * v4 + 5], o[8 * v4 + 5]));
+                        u.w = pack_bf16x2(fmaf(ec, ox[8 * v4 + 6], o[8 * v4 + 6]),
+                                          fmaf(ec, ox[8 * v4 + 7], o[8 * v4 + 7]));
                         dst[v4] = u;
                     }
                 }
@@ -612,55 +643,7 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
 }
 
 // ----------------------------------------------------------------------------------------------
-// warps 8-11: V and decayed K to fp16, fp32 state, look-back
-
-
-// K tile -> fp16 rows w_r * K_r with one power-of-two scale for the tile; returns the scale.
-__device__ __forceinline__ float convert_k(Smem& sm, unsigned char* ktile, int r, int q, int lane,
-                                           float w) {
-    const float sk = pow2_scale(group_max(sm, 1, q, lane, w * row_absmax_bf16(ktile, r)));
-    row_bf16_to_f16(ktile, r, w * sk);
-    return sk;
-}
-
-// fp16 copy of state row r (times `scale`) into the MN-major swizzled tile read by Q S_prev.
-__device__ __forceinline__ void write_state_f16(unsigned char* tile, int r, const float (&S)[D],
-                                                float scale) {
-#pragma unroll
-    for (int cc = 0; cc < 16; ++cc) {
-        uint4 u;
-        u.x = pack_f16x2(S[8 * cc + 0] * scale, S[8 * cc + 1] * scale);
-        u.y = pack_f16x2(S[8 * cc + 2] * scale, S[8 * cc + 3] * scale);
-        u.z = pack_f16x2(S[8 * cc + 4] * scale, S[8 * cc + 5] * scale);
-        u.w = pack_f16x2(S[8 * cc + 6] * scale, S[8 * cc + 7] * scale);
-        const int half = cc >> 3, c = cc & 7;
-        *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) = u;
-    }
-}
-
-__device__ __forceinline__ void publish_state(Smem& sm, int r, int q, int lane, const float (&S)[D],
-                                              int bslot) {
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < D; ++i) m = fmaxf(m, fabsf(S[i]));
-    const float ss = pow2_scale(group_max(sm, 1, q, lane, m));
-    write_state_f16(sm.sbf, r, S, ss);
-    if (r == 0) sm.sig_s[bslot] = ss;
-    fence_proxy_async_smem();
-    mbar_arrive(&sm.s_ready);
-}
-
-// S = 2^tot * S + dS / (sk * sv), dS read from TMEM
-__device__ __forceinline__ void fold_ds(uint32_t taddr, float (&S)[D], float eb, float inv) {
-#pragma unroll
-    for (int jc = 0; jc < 8; ++jc) {
-        float ds[16];
-        tmem_ld16(taddr + jc * 16, ds);
-        tmem_ld_wait();
-#pragma unroll
-        for (int i = 0; i < 16; ++i) S[jc * 16 + i] = fmaf(eb, S[jc * 16 + i], ds[i] * inv);
-    }
-}
+// warps 8-11: decayed K split, fp32 state, look-back
 
 __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
     GroupWait gw{&sm, &p, 1, (warp - 8) * 32 + lane};
@@ -678,26 +661,38 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
             mbar_arrive(&sm.item_empty[slot]);
             break;
         }
-        // ---- pass A: span aggregate from zero
+        // ---- pass A: span aggregate from zero.  The split of chunk c + 1 is done while the
+        // dS MMA of chunk c runs (its tile is already resident: the producer runs two stages
+        // ahead, and that stage was released by the MMA of chunk c - 1).
 #pragma unroll
         for (int i = 0; i < D; ++i) S[i] = 0.f;
         float L = 0.f;   // span log2-decay
-        for (int c = it.c_begin; c < it.c_end; ++c, ++j) {
+        float tot = 0.f;
+        if (it.c_end > it.c_begin) {
             const int st = j & 1;
-            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
-            const float cr = sm.gc[st][r], tot = sm.gtot[st];
-            const bool valid = (int64_t)c * C + r < it.len;
-            const float sk = convert_k(sm, sm.k[st], r, q, lane, valid ? ex2f(tot - cr) * p.k_scale : 0.f);
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) break;
+            tot = sm.gtot[st];
+            split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r, k_weight(sm, p, it, it.c_begin, st, r));
             fence_proxy_async_smem();
-            if (!gw.wait(&sm.v16_ready[st], (j >> 1) & 1)) { ok = false; break; }
-            const float sv = sm.sig_v[st];
-            mbar_arrive(&sm.k_ready);
+            mbar_arrive(&sm.k_ready[st]);
+        }
+        for (int c = it.c_begin; c < it.c_end; ++c, ++j) {
+            float tot_next = 0.f;
+            if (c + 1 < it.c_end) {
+                const int st = (j + 1) & 1;
+                if (!gw.wait(&sm.kv_full[st], ((j + 1) >> 1) & 1)) { ok = false; break; }
+                tot_next = sm.gtot[st];
+                split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r, k_weight(sm, p, it, c + 1, st, r));
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.k_ready[st]);
+            }
             if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
             tc_fence_after();
-            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot), 1.f / (sk * sv));
+            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
             L += tot;
+            tot = tot_next;
         }
         if (!ok) break;
         // ---- look-back: entry state E of the span; publish exp(L) E + Agg
@@ -714,13 +709,13 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         const float eL = ex2f(L);
         float4* dst = it.last ? nullptr
                               : reinterpret_cast<float4*>(p.slots + (chain * 2 + (it.s & 1)) * (D * D));
-        // two batches of 16 independent loads each, then the inclusive state and the swap
+        // four batches of 8 independent loads each, then the inclusive state and the swap
 #pragma unroll
-        for (int half = 0; half < 2; ++half) {
-            float4 e[16];
+        for (int quarter = 0; quarter < 4; ++quarter) {
+            float4 e[8];
 #pragma unroll
-            for (int k4 = 0; k4 < 16; ++k4) {
-                const int j4 = half * 16 + k4;
+            for (int k4 = 0; k4 < 8; ++k4) {
+                const int j4 = quarter * 8 + k4;
                 e[k4] = make_float4(0.f, 0.f, 0.f, 0.f);
                 if (from_slot)
                     e[k4] = __ldcg(reinterpret_cast<const float4*>(esrc) + j4 * D + r);
@@ -728,8 +723,8 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
                     e[k4] = __ldg(reinterpret_cast<const float4*>(esrc) + j4);
             }
 #pragma unroll
-            for (int k4 = 0; k4 < 16; ++k4) {
-                const int j4 = half * 16 + k4;
+            for (int k4 = 0; k4 < 8; ++k4) {
+                const int j4 = quarter * 8 + k4;
                 if (dst) {
                     float4 inc;
                     inc.x = fmaf(eL, e[k4].x, S[4 * j4 + 0]);
@@ -753,25 +748,36 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
                              : "memory");
             }
         }
-        if (it.c_end > it.c_begin) publish_state(sm, r, q, lane, S, b & 1);  // for the first chunk
+        if (it.c_end > it.c_begin) {   // high half of E for the first chunk's Q S
+            write_state_half<false>(sm.sbf, r, S);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.s_ready);
+        }
         // ---- pass B: running state from E
         for (int c = it.c_begin; c < it.c_end; ++c, ++j, ++b) {
             const int st = j & 1;
             if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
-            const float cr = sm.gc[st][r], tot = sm.gtot[st];
-            const bool valid = (int64_t)c * C + r < it.len;
-            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }  // Q K^T done with K
-            const float sk = convert_k(sm, sm.k[st], r, q, lane, valid ? ex2f(tot - cr) * p.k_scale : 0.f);
+            const float tot = sm.gtot[st];
+            // Q S_hi done (hence Q K^T too): the state buffer takes the low half, K is free
+            if (!gw.wait(&sm.s3a_done, b & 1)) { ok = false; break; }
+            write_state_half<true>(sm.sbf, r, S);
             fence_proxy_async_smem();
-            if (!gw.wait(&sm.v16_ready[st], (j >> 1) & 1)) { ok = false; break; }
-            const float sv = sm.sig_v[st];
-            mbar_arrive(&sm.k_ready);
+            mbar_arrive(&sm.s_lo_ready);
+            // every MMA reading Q has completed: its slot takes the low half of w K
+            if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
+            split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r, k_weight(sm, p, it, c, st, r));
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.k_ready[st]);
             if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
             tc_fence_after();
-            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot), 1.f / (sk * sv));
+            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
-            if (c + 1 < it.c_end) publish_state(sm, r, q, lane, S, (b + 1) & 1);
+            if (c + 1 < it.c_end) {
+                write_state_half<false>(sm.sbf, r, S);
+                fence_proxy_async_smem();
+                mbar_arrive(&sm.s_ready);
+            }
         }
         if (!ok) break;
         if (it.last && p.state_out) {
@@ -785,12 +791,11 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
 }
 
 // ----------------------------------------------------------------------------------------------
-// warps 2-3: V tile to fp16 as soon as it lands (every chunk), Q tile to fp16 after Q K^T
-// (pass-B chunks).  64 threads, two rows each.
+// warps 2-3: their share of the w K split (chunks 11-15 of rows 2t and 2t + 1), every chunk
 
-__device__ void convert_group(Smem& sm, const TcParams& p, int warp, int lane) {
+__device__ void split_helper(Smem& sm, const TcParams& p, int warp, int lane) {
     GroupWait gw{&sm, &p, 2, (warp - 2) * 32 + lane, 64};
-    const int w = warp - 2, t = w * 32 + lane;     // rows t and t + 64
+    const int t = (warp - 2) * 32 + lane;
     int j = 0, b = 0, it_n = 0;
     bool ok = true;
     while (ok) {
@@ -803,30 +808,20 @@ __device__ void convert_group(Smem& sm, const TcParams& p, int warp, int lane) {
         const int n_ch = it.c_end - it.c_begin;
         for (int jj = 0; jj < 2 * n_ch; ++jj, ++j) {
             const int st = j & 1;
-            const bool passb = jj >= n_ch;
+            const int c = it.c_begin + (jj < n_ch ? jj : jj - n_ch);
             if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
-            // V: one power-of-two scale for the tile
-            const float m = fmaxf(row_absmax_bf16(sm.v[st], t), row_absmax_bf16(sm.v[st], t + 64));
-            const float sv = pow2_scale(group_max(sm, 2, w, lane, m, 2));
-            row_bf16_to_f16(sm.v[st], t, sv);
-            row_bf16_to_f16(sm.v[st], t + 64, sv);
-            if (t == 0) sm.sig_v[st] = sv;
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.v16_ready[st]);
-            if (passb) {
-                // Q: a power-of-two scale per row, once Q K^T has read the bf16 Q
-                if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
-#pragma unroll
-                for (int h2 = 0; h2 < 2; ++h2) {
-                    const int row = t + 64 * h2;
-                    const float sq = pow2_scale(row_absmax_bf16(sm.q[st], row));
-                    row_bf16_to_f16(sm.q[st], row, sq);
-                    sm.sq[b & 1][row] = sq;
-                }
-                fence_proxy_async_smem();
-                mbar_arrive(&sm.q16_ready);
+            if (jj >= n_ch) {   // pass B: the Q slot is free once both Q S MMAs are done
+                if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
                 ++b;
             }
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+                const int r = 2 * t + h;
+                split_k_chunks<SPLIT_OWN, 16 - SPLIT_OWN>(sm.k[st], sm.q[st], r,
+                                                          k_weight(sm, p, it, c, st, r));
+            }
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.kh_ready[st]);
         }
     }
 }
@@ -851,13 +846,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(&sm.item_empty[s], 1 + 128 + 128 + 64);
         }
         mbar_init(&sm.a_full, 1);
-        mbar_init(&sm.q16_ready, 64);
-        mbar_init(&sm.v16_ready[0], 64);
-        mbar_init(&sm.v16_ready[1], 64);
+        mbar_init(&sm.s3a_done, 1);
+        mbar_init(&sm.q_free, 1);
         mbar_init(&sm.p_ready, 128);
+        mbar_init(&sm.s_lo_ready, 128);
         mbar_init(&sm.o_full, 1);
         mbar_init(&sm.o_free, 128);
-        mbar_init(&sm.k_ready, 128);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.k_ready[s], 128);
+            mbar_init(&sm.kh_ready[s], 64);
+        }
         mbar_init(&sm.ds_full, 1);
         mbar_init(&sm.ds_free, 128);
         mbar_init(&sm.s_ready, 128);
@@ -887,12 +885,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         } else if (warp == 1) {
             if (lane == 0) mma_issuer(sm, p, tmem);
         } else {
-            convert_group(sm, p, warp, lane);
+            split_helper(sm, p, warp, lane);
         }
     } else if (warp < 8) {
-        // 168 -> 160 is a decrease: setmaxnreg.inc must never ask for fewer registers than the
+        // 168 -> 136 is a decrease: setmaxnreg.inc must never ask for fewer registers than the
         // warp holds, and .dec never for more.
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 160;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 136;" ::: "memory");
         p_group(sm, p, tmem, warp, lane);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 256;" ::: "memory");
