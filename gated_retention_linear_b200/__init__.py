@@ -1,7 +1,7 @@
 """gated_retention_linear_b200 -- gated retention (the YOCO Self-Decoder mixer) on B200.
 
 A thin Python binding over the C ABI in include/gret.h (libgret.so, built in-tree by
-`python -m gated_retention_linear_b200.build`).  The functions here only marshal arguments:
+`python gated_retention_linear_b200/build.py`).  The functions here only marshal arguments:
 they read shapes and strides off torch tensors, allocate outputs and workspaces with torch, pass
 raw device pointers and the current CUDA stream, and raise on a non-OK status.  Every step of
 the computation runs in the library's CUDA kernels; there is no fallback.  If libgret.so is
@@ -17,7 +17,7 @@ LIB_PATH = os.path.join(_HERE, "libgret.so")
 
 if not os.path.exists(LIB_PATH):
     raise ImportError("libgret.so not found at %s; build it with "
-                      "`python -m gated_retention_linear_b200.build`" % LIB_PATH)
+                      "`python gated_retention_linear_b200/build.py`" % LIB_PATH)
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -37,6 +37,11 @@ _lib.gret_prefill_chunkwise.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _
                                         _i32, _i64, _i32, _i32, _i32, _vp, _i32, _vp, _vp, _vp,
                                         _i64, _i64, _i64, _i32, _vp, ctypes.c_size_t, _vp]
 _lib.gret_prefill_chunkwise.restype = _i32
+_lib.gret_prefill_chunkwise_noalloc.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp, _i64, _i64, _i64,
+                                                _vp, _f32, _f32, _i32, _i32, _i64, _i32, _i32,
+                                                _i32, _vp, _i32, _vp, _vp, _vp, _i64, _i64, _i64,
+                                                _i32, _vp]
+_lib.gret_prefill_chunkwise_noalloc.restype = _i32
 _lib.gret_workspace_status.argtypes = [_vp, _vp]
 _lib.gret_workspace_status.restype = _i32
 _lib.gret_decode_step.argtypes = [_vp, _vp, _vp, _vp, _f32, _f32, _i32, _i32, _i32, _i32, _i32,
@@ -141,6 +146,39 @@ def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, s
         N, H, dk, dv,
         _ptr(cu_seqlens), n_seqs, _ptr(state_in), _ptr(state_out), _ptr(o), osb, ost, osh,
         chunk, _ptr(workspace), wbytes, _stream(stream)))
+    return o, state_out
+
+
+def gret_prefill_chunkwise_noalloc(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None,
+                                   state_in=None, state_out=None, o=None, chunk=0,
+                                   head_major=False, stream=None):
+    """gret_prefill_chunkwise through the entry point that needs no workspace and allocates no
+    device memory (its scratch is a fixed 8 MiB array inside the library; calls that overlap
+    on the GPU race).  Same arguments and results as gret_prefill_chunkwise; `o` and
+    `state_out=True` are allocated here by torch for convenience, so pass them in to allocate
+    nothing at call time."""
+    if k.stride() != q.stride():
+        raise ValueError("q and k must share strides")
+    if q.dim() == 3:
+        B, (N, H, dk) = 1, q.shape
+    elif head_major:
+        B, H, N, dk = q.shape
+    else:
+        B, N, H, dk = q.shape
+    dv = v.shape[-1]
+    sb, st, sh = _layout(q, head_major)
+    vsb, vst, vsh = _layout(v, head_major)
+    if o is None:
+        o = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
+    osb, ost, osh = _layout(o, head_major)
+    n_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    units = n_seqs if cu_seqlens is not None else B
+    if state_out is True:
+        state_out = torch.empty((units, H, dk, dv), dtype=torch.float32, device=q.device)
+    _check("gret_prefill_chunkwise_noalloc", _lib.gret_prefill_chunkwise_noalloc(
+        _ptr(q), _ptr(k), sb, st, sh, _ptr(v), vsb, vst, vsh, _ptr(g), tau, k_scale,
+        _dtype_code(q), B, N, H, dk, dv, _ptr(cu_seqlens), n_seqs, _ptr(state_in),
+        _ptr(state_out), _ptr(o), osb, ost, osh, chunk, _stream(stream)))
     return o, state_out
 
 

@@ -1,6 +1,8 @@
 """Build libgret.so (the C-ABI CUDA library) in-tree for sm_100a with nvcc.
 
-    python -m gated_retention_linear_b200.build [--force] [--verbose]
+    python gated_retention_linear_b200/build.py [--force] [--verbose]
+
+(run by path: importing the package first would load the library being rebuilt)
 
 Each csrc/*.cu compiles to an object under _build/ (in parallel, rebuilt when it or any header
 is newer), then the objects link into gated_retention_linear_b200/libgret.so with the CUDA

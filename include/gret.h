@@ -107,6 +107,32 @@ gret_status_t gret_prefill_chunkwise(
     size_t workspace_bytes, gret_stream_t stream);
 
 /*
+ * gret_prefill_chunkwise without a workspace argument and without allocating.  The paper has no
+ * counterpart: this entry point exists for callers that cannot allocate device memory when they
+ * call, for example a serving process that gives all device memory to its own pool at start-up,
+ * or a latency-critical loop in which a cudaMalloc would synchronize the device.
+ *   - Arguments, results and errors are those of gret_prefill_chunkwise, minus the workspace.
+ *   - Its scratch is one static device array of 8 MiB inside this library, present on every GPU
+ *     that loads the library until the process exits.  A call whose workspace need
+ *     (gret_prefill_workspace_size) exceeds 8 MiB returns GRET_ERR_WORKSPACE before doing
+ *     anything; with d_k = d_v = 128 and bf16 that allows about 63 (sequence, head) chains.
+ *   - The first call on a device looks up the scratch's device address (once per device); make
+ *     that first call before any stream capture.
+ *   - Every call shares the one scratch array: calls that overlap on the GPU (other streams, or
+ *     other host threads using the same device) race and give wrong results.  The call clears
+ *     what must start at zero itself; the array keeps the previous call's contents otherwise.
+ *   - The bounded-wait error word lives in the private scratch, so a timed-out wait is not
+ *     reported to the caller of this variant.
+ */
+gret_status_t gret_prefill_chunkwise_noalloc(
+    const void* q, const void* k, int64_t stride_batch, int64_t stride_tok, int64_t stride_head,
+    const void* v, int64_t v_stride_batch, int64_t v_stride_tok, int64_t v_stride_head,
+    const float* g, float tau, float k_scale, gret_dtype_t dtype, int B,
+    int64_t N, int H, int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
+    const float* state_in, float* state_out, void* o, int64_t o_stride_batch,
+    int64_t o_stride_tok, int64_t o_stride_head, int chunk, gret_stream_t stream);
+
+/*
  * Synchronises `stream`, then reads the error word that gret_prefill_chunkwise keeps at the
  * start of `workspace`.  Returns GRET_OK, GRET_ERR_TIMEOUT, or GRET_ERR_CUDA if the copy or the
  * synchronisation failed.  Blocking; not for use inside stream capture.
