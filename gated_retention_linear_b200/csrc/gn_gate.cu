@@ -1,11 +1,315 @@
-// gn_gate.cu -- GroupNorm * swish(X W_G) epilogue (placeholder until the tcgen05 GEMM lands).
+// gn_gate.cu -- the gated-retention output epilogue: per-head GroupNorm of O times swish(X W_G).
+//
+// Page "YOCO 完全拆解：Decoder-Decoder 架构如何让 KV Cache 只存一次", section
+// "路线二：Multi-Head Gated Retention": the retention output of each head is group-normalised (one
+// group per head, so heads cannot drift in scale) and multiplied element-wise by swish(X W_G),
+// which chooses the channels written back to the residual stream.  For token t and head h:
+//     z   = X_t W_G                                          (GEMM, [T, D] x [D, H*d_v])
+//     n_j = (o_j - mean) / sqrt(var + eps) * gn_w + gn_b     (o = O_t[h*d_v .. h*d_v + d_v))
+//     y_j = n_j * z_j * sigmoid(z_j)
+//
+// The GEMM dominates (2 D H d_v FLOP per token): a persistent tcgen05 kernel, one CTA per SM,
+// output tiles of 128 tokens x 256 columns (two heads), K in blocks of 64 through a 4-stage
+// TMA ring, fp32 accumulators in TMEM, two accumulator buffers so the epilogue of one tile runs
+// under the MMAs of the next.  The epilogue is fused: GroupNorm statistics of the O row, swish
+// of the accumulator, the product, bf16 out; z never goes to memory.
+//
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (owns TMEM), warps 2-3 idle,
+// warps 4-7 epilogue for the first head of a tile, warps 8-11 for the second.  Tiles are
+// assigned round-robin (tile = blockIdx.x + i * gridDim.x), M-block major, so the CTAs working
+// at one time share a few X row-blocks and all of W_G (9.4 MB at D = 3072) through L2.
+// Every wait is bounded; a wait that gives up makes every role exit.
 #include "gn_gate.cuh"
+
+#include "sm100.cuh"
+#include "tma_host.cuh"
 
 namespace gret {
 
-gret_status_t launch_gn_gate(const void*, const void*, const void*, const float*, const float*,
-                             float, int64_t, int, int, int, void*, cudaStream_t) {
-    return GRET_ERR_UNSUPPORTED;
+using namespace sm100;
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;            // 16 KB
+constexpr int B_BYTES = BN * BK * 2;            // 32 KB
+constexpr int NTHREADS = 384;
+constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_NS = 200000000ull;
+
+struct __align__(1024) GSmem {
+    unsigned char a[STAGES][A_BYTES];
+    unsigned char b[STAGES][B_BYTES];
+    uint64_t full[STAGES], empty[STAGES];
+    uint64_t acc_full[2], acc_empty[2], drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+
+struct GParams {
+    const __nv_bfloat16* o;
+    const float* gn_w;
+    const float* gn_b;
+    __nv_bfloat16* y;
+    float eps;
+    int64_t T;
+    int F, D;          // F = H * 128
+    int m_blocks, n_blocks, n_tiles;
+};
+
+__device__ __forceinline__ bool wait_bar(GSmem& sm, uint64_t* bar, uint32_t parity) {
+    if (mbar_wait(bar, parity, &sm.abort, WAIT_NS)) return true;
+    atomicExch(&sm.abort, 1u);
+    return false;
+}
+
+__device__ void producer(GSmem& sm, const GParams& p, const CUtensorMap* tx, const CUtensorMap* tw) {
+    const int kblocks = p.D / BK;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+        const int mb = tile / p.n_blocks, nb = tile % p.n_blocks;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+            const int s = it % STAGES;
+            if (it >= STAGES && !wait_bar(sm, &sm.empty[s], ((it / STAGES) - 1) & 1)) {
+                ok = false;
+                break;
+            }
+            mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
+            tma_load_2d(sm.a[s], tx, &sm.full[s], kb * BK, mb * BM);
+#pragma unroll
+            for (int j = 0; j < BN / 64; ++j)
+                tma_load_2d(sm.b[s] + j * (BK * 128), tw, &sm.full[s], nb * BN + j * 64, kb * BK);
+        }
+    }
+    // no TMA write may be in flight when the CTA exits
+    uint32_t never = 0;
+    for (int jj = (it >= STAGES ? it - STAGES : 0); jj < it; ++jj)
+        mbar_wait(&sm.full[jj % STAGES], (jj / STAGES) & 1, &never, DRAIN_NS);
+}
+
+__device__ void mma_issuer(GSmem& sm, const GParams& p, uint32_t tmem) {
+    const int kblocks = p.D / BK;
+    const uint32_t idesc = idesc_bf16(BM, BN, 0, 1);
+    int it = 0, t_local = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++t_local) {
+        const int buf = t_local & 1;
+        if (t_local >= 2 && !wait_bar(sm, &sm.acc_empty[buf], ((t_local >> 1) - 1) & 1)) break;
+        tc_fence_after();
+        const uint32_t d = tmem + buf * BN;
+        for (int kb = 0; kb < kblocks; ++kb, ++it) {
+            const int s = it % STAGES;
+            if (!wait_bar(sm, &sm.full[s], (it / STAGES) & 1)) { ok = false; break; }
+            tc_fence_after();
+            const uint32_t ab = smem_u32(sm.a[s]), bb = smem_u32(sm.b[s]);
+#pragma unroll
+            for (int kk = 0; kk < BK / 16; ++kk)
+                mma_ss(d, sdesc_sw128(ab + kk * 32, 16, 1024),
+                       sdesc_sw128(bb + kk * 2048, BK * 128, 1024), idesc,
+                       (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit(&sm.empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&sm.acc_full[buf]);
+    }
+    uint32_t never = 0;
+    mma_commit(&sm.drain);
+    mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
+}
+
+// One epilogue thread: token row r of the tile, one head (128 columns) of it.
+__device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, int lane) {
+    const int q = warp & 3, r = q * 32 + lane;
+    const int half = (warp - 4) >> 2;                    // which head of the 256-column tile
+    const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
+    int t_local = 0;
+    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++t_local) {
+        const int buf = t_local & 1;
+        const int mb = tile / p.n_blocks, nb = tile % p.n_blocks;
+        const int64_t t = (int64_t)mb * BM + r;
+        const int col0 = nb * BN + half * 128;
+        // GroupNorm statistics of this head's slice of O, computed while the MMAs run; the row
+        // (256 bytes) is read again per 32 columns below, from L1
+        float mean = 0.f, inv = 0.f;
+        const bool valid = t < p.T;
+        const uint4* src = reinterpret_cast<const uint4*>(p.o + t * p.F + col0);
+        if (valid) {
+            float s = 0.f, s2 = 0.f;
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint4 u = __ldg(src + i);
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                    s += f.x + f.y;
+                }
+            }
+            mean = s * (1.f / 128.f);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                const uint4 u = __ldg(src + i);
+                const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&w4[e]));
+                    s2 += (f.x - mean) * (f.x - mean) + (f.y - mean) * (f.y - mean);
+                }
+            }
+            inv = rsqrtf(s2 * (1.f / 128.f) + p.eps);
+        }
+        if (!mbar_wait(&sm.acc_full[buf], (t_local >> 1) & 1, &sm.abort, WAIT_NS)) {
+            atomicExch(&sm.abort, 1u);
+            return;
+        }
+        tc_fence_after();
+        __nv_bfloat16* dst = p.y + t * p.F + col0;
+#pragma unroll 1
+        for (int jc = 0; jc < 4; ++jc) {
+            float z[32];
+            tmem_ld32(tmem + lane_base + buf * BN + half * 128 + jc * 32, z);
+            tmem_ld_wait();
+            if (valid) {
+                uint32_t ow[16];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint4 u = __ldg(src + jc * 4 + i);
+                    ow[4 * i + 0] = u.x;
+                    ow[4 * i + 1] = u.y;
+                    ow[4 * i + 2] = u.z;
+                    ow[4 * i + 3] = u.w;
+                }
+                uint32_t out[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int c = jc * 32 + 2 * i;
+                    const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[i]));
+                    float n0 = (f.x - mean) * inv, n1 = (f.y - mean) * inv;
+                    if (p.gn_w) {
+                        n0 *= __ldg(p.gn_w + col0 + c);
+                        n1 *= __ldg(p.gn_w + col0 + c + 1);
+                    }
+                    if (p.gn_b) {
+                        n0 += __ldg(p.gn_b + col0 + c);
+                        n1 += __ldg(p.gn_b + col0 + c + 1);
+                    }
+                    const float z0 = z[2 * i], z1 = z[2 * i + 1];
+                    const float s0 = z0 / (1.f + __expf(-z0)), s1 = z1 / (1.f + __expf(-z1));
+                    out[i] = pack_bf16x2(n0 * s0, n1 * s1);
+                }
+                uint4* d4 = reinterpret_cast<uint4*>(dst + jc * 32);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    d4[v4] = make_uint4(out[4 * v4], out[4 * v4 + 1], out[4 * v4 + 2], out[4 * v4 + 3]);
+            }
+        }
+        tc_fence_before();
+        mbar_arrive(&sm.acc_empty[buf]);
+    }
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    gn_gate_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
+                   const GParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    GSmem& sm = *reinterpret_cast<GSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if ((smem_u32(smem_raw) & 1023u) != 0) return;   // the swizzled tiles need 1 KB alignment
+    if (tid == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], 1);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], 256);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    if (warp == 0) {
+        if (lane == 0) {
+            tma_prefetch_desc(&tx);
+            tma_prefetch_desc(&tw);
+            producer(sm, p, &tx, &tw);
+        }
+    } else if (warp == 1) {
+        if (lane == 0) mma_issuer(sm, p, tmem);
+    } else if (warp >= 4) {
+        epilogue(sm, p, tmem, warp, lane);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+int sm_count() {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+}  // namespace
+
+gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g, const float* gn_weight,
+                             const float* gn_bias, float eps, int64_t T, int H, int d_v, int D,
+                             void* y, cudaStream_t stream) {
+    const int F = H * d_v;
+    if (d_v != 128 || F % BN != 0 || D % BK != 0) return GRET_ERR_UNSUPPORTED;
+    if (T > ((int64_t)1 << 31) - BM) return GRET_ERR_UNSUPPORTED;
+    CUtensorMap tx, tw;
+    {
+        uint64_t dims[2] = {(uint64_t)D, (uint64_t)T};
+        uint64_t strides[1] = {(uint64_t)D * 2};
+        uint32_t box[2] = {BK, BM};
+        if (!make_bf16_map(&tx, x, 2, dims, strides, box)) return GRET_ERR_UNSUPPORTED;
+    }
+    {
+        uint64_t dims[2] = {(uint64_t)F, (uint64_t)D};
+        uint64_t strides[1] = {(uint64_t)F * 2};
+        uint32_t box[2] = {64, BK};
+        if (!make_bf16_map(&tw, w_g, 2, dims, strides, box)) return GRET_ERR_UNSUPPORTED;
+    }
+    GParams p;
+    p.o = (const __nv_bfloat16*)o;
+    p.gn_w = gn_weight;
+    p.gn_b = gn_bias;
+    p.y = (__nv_bfloat16*)y;
+    p.eps = eps;
+    p.T = T;
+    p.F = F;
+    p.D = D;
+    p.m_blocks = (int)((T + BM - 1) / BM);
+    p.n_blocks = F / BN;
+    p.n_tiles = p.m_blocks * p.n_blocks;
+    const size_t smem = sizeof(GSmem);
+    if (cudaFuncSetAttribute(gn_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return GRET_ERR_CUDA;
+    int grid = sm_count();
+    if (p.n_tiles < grid) grid = p.n_tiles;
+    gn_gate_kernel<<<grid, NTHREADS, smem, stream>>>(tx, tw, p);
+    return cudaGetLastError() == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
 }  // namespace gret
