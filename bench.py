@@ -13,6 +13,10 @@ the C ABI, inputs resident in HBM.  The printed JSON line carries:
             prefill, 256 steps), tok/s and its HBM roofline
   e2e       the same prefill metric with host buffers: pinned host -> device copies of q, k, v, g
             and device -> host copies of o and the final state inside the timed region
+  varlen_epilogue  8 packed sequences of seeded lengths in [1024, 65536] with harsher gates
+            (g ~ N(0, 2)): varlen prefill, then the per-head GroupNorm * swish(X W_G) epilogue
+            (X [T, 3072], W_G [3072, 3072]); Mtok/s of the pair, and the epilogue GEMM against
+            the measured bf16 tensor peak
   cpu_baseline  the fp64 CPU oracle on the same workload (rank 0 only)
 With --impl reference the oracle alone is timed, on host cores, as the reference arm.
 """
@@ -44,6 +48,15 @@ def measured_peaks():
         return float(pk["hbm_gbs"]), "measured"
     except Exception:
         return 6650.0, "fallback"
+
+
+def measured_tensor_peak():
+    """bf16 dense TFLOP/s: the burst figure (a kernel timed on its own)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
 
 
 class ClockSampler:
@@ -247,6 +260,11 @@ def run_gpu(args):
                "l2": "state (201 MB) larger than L2 (126 MB); not flushed between steps"}
         del qs, ks, vs, gs, state, state0
 
+    # ---------------- varlen prefill + GroupNorm * swish(X W_G) epilogue
+    epi = None
+    if not args.no_epilogue:
+        epi = run_varlen_epilogue(args, rank, world, stream, hbm_peak)
+
     clk = clocks.stop()
 
     # ---------------- end to end: host buffers through the C ABI
@@ -306,7 +324,8 @@ def run_gpu(args):
                      "traffic": prefill_traffic_from_profile(),
                      "kernel": "prefill_tc_kernel", "launch_ms": launch_ms,
                      "algorithmic_bytes_per_launch": alg_bytes},
-        "decode": dec, "e2e": e2e, "clocks": clk, "gpu_launches": args.steps,
+        "decode": dec, "varlen_epilogue": epi, "e2e": e2e, "clocks": clk,
+        "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }
     if rank == 0:
@@ -314,6 +333,63 @@ def run_gpu(args):
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+    lens = SI.varlen_lengths(8, 1024, 65536, seed=5)
+    cu = SI.cu_seqlens_of(lens)
+    T, Dm = cu[-1], 3072
+    inp = SI.gret_inputs(1, T, H, D, dtype=torch.bfloat16, g_mean=0.0, g_std=2.0,
+                         seed=5 + 1000 * rank, device="cuda")
+    q, k, v, g = (inp[x][0] for x in ("q", "k", "v", "g"))
+    del inp
+    ep = SI.epilogue_inputs(T, Dm, H * D, seed=5 + 1000 * rank, device="cuda")
+    cu_d = torch.tensor(cu, dtype=torch.int32, device="cuda")
+    o = torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, H * D), dtype=torch.bfloat16, device="cuda")
+    need = G.gret_prefill_workspace_size(torch.bfloat16, T, len(lens), H, D, D, 0)
+    ws = torch.empty(need, dtype=torch.uint8, device="cuda")
+
+    def step(ev=None):
+        G.gret_prefill_chunkwise(q, k, v, g, cu_seqlens=cu_d, o=o, workspace=ws)
+        if ev is not None:
+            ev.record(stream)
+        G.gret_groupnorm_gate(o.view(T, H * D), ep["x"], ep["w_g"], H, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 5))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n)]
+    barrier(world)
+    for i in range(n):
+        evs[i][0].record(stream)
+        step(evs[i][1])
+        evs[i][2].record(stream)
+    torch.cuda.synchronize()
+    tot_ms = statistics.mean(e[0].elapsed_time(e[2]) for e in evs)
+    pre_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    epi_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    tot_ms = max_over_ranks(tot_ms, world)
+    if G.gret_workspace_status(ws) != 0:
+        raise RuntimeError("varlen prefill reported a timed-out wait")
+    flops = 2.0 * T * Dm * H * D
+    tpeak, tkind = measured_tensor_peak()
+    ach = flops / (epi_ms * 1e-3) / 1e12
+    pre_bytes = T * H * BYTES_PER_TOKEN_HEAD
+    return {"value": T * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtok/s", "tokens": T,
+            "lengths": lens, "ms_per_step": tot_ms, "prefill_ms": pre_ms, "epilogue_ms": epi_ms,
+            "steps": n, "gpu_launches_per_step": 3,
+            "prefill_roofline": {"bound": "hbm", "achieved": pre_bytes / (pre_ms * 1e-3) / 1e9,
+                                 "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / hbm_peak},
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
+                         "frac": ach / tpeak, "peak_kind": tkind + " burst", "traffic": None,
+                         "kernel": "gn_gate_kernel", "algorithmic_flops_per_launch": flops}}
 
 
 def cpu_baseline(q, k, v, g, n_tokens):
@@ -376,6 +452,7 @@ def main():
     ap.add_argument("--no-cpu", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-epilogue", action="store_true")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3
