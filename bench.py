@@ -136,13 +136,20 @@ def barrier(world):
 
 
 def max_over_ranks(x, world):
+    """Max of a host float over all ranks (the slowest rank sets the job's time)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_seed(base, rank):
+    """Seed of a rank's own synthetic sequence: every rank processes different data."""
+    return base + 1000 * rank
 
 
 def prefill_traffic_from_profile():
@@ -178,7 +185,7 @@ def run_gpu(args):
 
     # ---------------- prefill, inputs resident in HBM
     inp = SI.gret_inputs(B, N, H, D, dtype=torch.bfloat16, g_mean=2.0, g_std=1.0,
-                         seed=2 + 1000 * rank, device="cuda")
+                         seed=rank_seed(2, rank), device="cuda")
     q, k, v, g = inp["q"], inp["k"], inp["v"], inp["g"]
     o = torch.empty_like(v)
     s_out = torch.empty((B, H, D, D), dtype=torch.float32, device="cuda")
@@ -223,13 +230,14 @@ def run_gpu(args):
     # ---------------- decode at batch 64
     dec = None
     if not args.no_decode:
-        dinp = SI.gret_inputs(DEC_B, DEC_PREFILL, H, D, dtype=torch.bfloat16, seed=4 + 1000 * rank,
+        dinp = SI.gret_inputs(DEC_B, DEC_PREFILL, H, D, dtype=torch.bfloat16,
+                              seed=rank_seed(4, rank),
                               device="cuda")
         _, state = G.gret_prefill_chunkwise(dinp["q"], dinp["k"], dinp["v"], dinp["g"],
                                             state_out=True)
         del dinp
         steps_in = SI.gret_inputs(DEC_B, DEC_STEPS, H, D, dtype=torch.bfloat16,
-                                  seed=40 + 1000 * rank, device="cuda")
+                                  seed=rank_seed(40, rank), device="cuda")
         qs = steps_in["q"].permute(1, 0, 2, 3).contiguous()    # [steps, B, H, d]
         ks = steps_in["k"].permute(1, 0, 2, 3).contiguous()
         vs = steps_in["v"].permute(1, 0, 2, 3).contiguous()
@@ -340,14 +348,14 @@ def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
 
     import gated_retention_linear_b200 as G
     import synth_inputs as SI
-    lens = SI.varlen_lengths(8, 1024, 65536, seed=5)
+    lens = SI.varlen_lengths(8, 1024, args.varlen_max_len, seed=5)
     cu = SI.cu_seqlens_of(lens)
     T, Dm = cu[-1], 3072
     inp = SI.gret_inputs(1, T, H, D, dtype=torch.bfloat16, g_mean=0.0, g_std=2.0,
-                         seed=5 + 1000 * rank, device="cuda")
+                         seed=rank_seed(5, rank), device="cuda")
     q, k, v, g = (inp[x][0] for x in ("q", "k", "v", "g"))
     del inp
-    ep = SI.epilogue_inputs(T, Dm, H * D, seed=5 + 1000 * rank, device="cuda")
+    ep = SI.epilogue_inputs(T, Dm, H * D, seed=rank_seed(5, rank), device="cuda")
     cu_d = torch.tensor(cu, dtype=torch.int32, device="cuda")
     o = torch.empty((T, H, D), dtype=torch.bfloat16, device="cuda")
     y = torch.empty((T, H * D), dtype=torch.bfloat16, device="cuda")
@@ -453,6 +461,9 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-epilogue", action="store_true")
+    ap.add_argument("--varlen-max-len", type=int, default=65536,
+                    help="longest sequence of the varlen + epilogue leg (a smaller value gives "
+                         "a small case for profiling)")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "native":
         args.warmup = 3

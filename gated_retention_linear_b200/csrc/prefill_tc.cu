@@ -363,7 +363,7 @@ __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, con
 __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, uint32_t b_base,
                                         bool b_mn, bool accumulate) {
     const uint32_t idesc = idesc_bf16(128, 128, a_mn, b_mn);
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 8; ++kk) {
         const uint32_t aoff = a_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
         const uint32_t boff = b_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
@@ -381,7 +381,7 @@ __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, 
 __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
                                        bool accumulate) {
     const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
-#pragma unroll
+#pragma unroll 1
     for (int kk = 0; kk < 8; ++kk)
         mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
                sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
@@ -525,19 +525,18 @@ __device__ __forceinline__ float k_weight(const Smem& sm, const TcParams& p, con
     return valid ? ex2f(sm.gtot[st] - sm.gc[st][r]) * p.k_scale : 0.f;
 }
 
-// Row r of the state into the MN-major swizzled tile read by Q S: its bf16 high half (LOW ==
-// false) or its low half (LOW == true).
-template <bool LOW>
-__device__ __forceinline__ void write_state_half(unsigned char* tile, int r, const float (&S)[D]) {
+// Row r of the state into the MN-major swizzled tile read by Q S: its bf16 high half (low ==
+// false) or its low half (low == true).
+__device__ __forceinline__ void write_state_half(unsigned char* tile, int r, const float (&S)[D],
+                                                 bool low) {
 #pragma unroll
     for (int cc = 0; cc < 16; ++cc) {
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) split2(S[8 * cc + 2 * e], S[8 * cc + 2 * e + 1], hi[e], lo[e]);
-        const uint32_t* w = LOW ? lo : hi;
         const int half = cc >> 3, c = cc & 7;
         *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(w[0], w[1], w[2], w[3]);
+            low ? make_uint4(lo[0], lo[1], lo[2], lo[3]) : make_uint4(hi[0], hi[1], hi[2], hi[3]);
     }
 }
 
@@ -580,7 +579,7 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
             tc_fence_after();
             // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, split into bf16 halves; each
             // 32-column group of A is replaced in place by [16 high | 16 low] columns of P.
-#pragma unroll
+#pragma unroll 1
             for (int jc = 0; jc < 4; ++jc) {
                 uint32_t ph[32];
                 if (jc <= q) {
@@ -663,37 +662,37 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         }
         // ---- pass A: span aggregate from zero.  The split of chunk c + 1 is done while the
         // dS MMA of chunk c runs (its tile is already resident: the producer runs two stages
-        // ahead, and that stage was released by the MMA of chunk c - 1).
+        // ahead, and that stage was released by the MMA of chunk c - 1).  One split and one
+        // fold site each, so that the group's code stays small for the instruction cache.
 #pragma unroll
         for (int i = 0; i < D; ++i) S[i] = 0.f;
-        float L = 0.f;   // span log2-decay
-        float tot = 0.f;
-        if (it.c_end > it.c_begin) {
-            const int st = j & 1;
-            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) break;
-            tot = sm.gtot[st];
-            split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r, k_weight(sm, p, it, it.c_begin, st, r));
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.k_ready[st]);
-        }
-        for (int c = it.c_begin; c < it.c_end; ++c, ++j) {
-            float tot_next = 0.f;
-            if (c + 1 < it.c_end) {
-                const int st = (j + 1) & 1;
-                if (!gw.wait(&sm.kv_full[st], ((j + 1) >> 1) & 1)) { ok = false; break; }
-                tot_next = sm.gtot[st];
-                split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r, k_weight(sm, p, it, c + 1, st, r));
+        float L = 0.f;                  // span log2-decay
+        float tot0 = 0.f, tot1 = 0.f;   // chunk log2-decay by stage parity, read at the split
+        const int n = it.c_end - it.c_begin;
+#pragma unroll 1
+        for (int i = 0; i <= n; ++i) {
+            if (i < n) {   // split of chunk i
+                const int st = (j + i) & 1;
+                if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
+                const float t = sm.gtot[st];
+                if (st) tot1 = t; else tot0 = t;
+                split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r,
+                                             k_weight(sm, p, it, it.c_begin + i, st, r));
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.k_ready[st]);
             }
-            if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
-            tc_fence_after();
-            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
-            tc_fence_before();
-            mbar_arrive(&sm.ds_free);
-            L += tot;
-            tot = tot_next;
+            if (i > 0) {   // fold of chunk i - 1
+                const int jf = j + i - 1;
+                if (!gw.wait(&sm.ds_full, jf & 1)) { ok = false; break; }
+                const float tot = (jf & 1) ? tot1 : tot0;
+                tc_fence_after();
+                fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
+                tc_fence_before();
+                mbar_arrive(&sm.ds_free);
+                L += tot;
+            }
         }
+        j += n;
         if (!ok) break;
         // ---- look-back: entry state E of the span; publish exp(L) E + Agg
         const int64_t chain = (int64_t)it.u * p.H + it.h;
@@ -748,37 +747,40 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
                              : "memory");
             }
         }
-        if (it.c_end > it.c_begin) {   // high half of E for the first chunk's Q S
-            write_state_half<false>(sm.sbf, r, S);
+        // ---- pass B: running state from E.  The state buffer takes, in turn, the high half of
+        // E, then per chunk the low half of the state before it (once Q S_hi is done) and, but
+        // after the last chunk, the high half of the state after it.  Writes w = 0 .. 2n-1:
+        // even w high halves, odd w low halves of chunk (w - 1) / 2, each low half followed by
+        // the chunk's split and fold.
+#pragma unroll 1
+        for (int w = 0; w < 2 * n; ++w) {
+            const bool low = w & 1;
+            const int i = w >> 1;           // chunk of a low half
+            const int st = (j + i) & 1;
+            if (low) {
+                if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
+                if (!gw.wait(&sm.s3a_done, (b + i) & 1)) { ok = false; break; }
+            }
+            write_state_half(sm.sbf, r, S, low);
             fence_proxy_async_smem();
-            mbar_arrive(&sm.s_ready);
-        }
-        // ---- pass B: running state from E
-        for (int c = it.c_begin; c < it.c_end; ++c, ++j, ++b) {
-            const int st = j & 1;
-            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
+            mbar_arrive(low ? &sm.s_lo_ready : &sm.s_ready);
+            if (!low) continue;
             const float tot = sm.gtot[st];
-            // Q S_hi done (hence Q K^T too): the state buffer takes the low half, K is free
-            if (!gw.wait(&sm.s3a_done, b & 1)) { ok = false; break; }
-            write_state_half<true>(sm.sbf, r, S);
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.s_lo_ready);
             // every MMA reading Q has completed: its slot takes the low half of w K
-            if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
-            split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r, k_weight(sm, p, it, c, st, r));
+            if (!gw.wait(&sm.q_free, (b + i) & 1)) { ok = false; break; }
+            split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r,
+                                         k_weight(sm, p, it, it.c_begin + i, st, r));
             fence_proxy_async_smem();
             mbar_arrive(&sm.k_ready[st]);
-            if (!gw.wait(&sm.ds_full, j & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.ds_full, (j + i) & 1)) { ok = false; break; }
             tc_fence_after();
             fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
-            if (c + 1 < it.c_end) {
-                write_state_half<false>(sm.sbf, r, S);
-                fence_proxy_async_smem();
-                mbar_arrive(&sm.s_ready);
-            }
+            if (i + 1 == n) break;          // no high half after the last chunk
         }
+        j += n;
+        b += n;
         if (!ok) break;
         if (it.last && p.state_out) {
             float4* so = reinterpret_cast<float4*>(p.state_out + (chain * D + r) * D);
@@ -999,14 +1001,30 @@ bool make_map(CUtensorMap* map, const void* base, int64_t st, int64_t sh, int64_
     return make_bf16_map(map, base, 4, dims, strides, box);
 }
 
-int span_chunks() {
-    static int g = -1;
-    if (g < 0) {
+// Chunks per span.  A span costs about G chunk-times plus one for its look-back; spans run in
+// waves of `grid` CTAs, and the look-backs of one chain run one after the other.  G minimises
+// the larger of the two; it stays at most 8 so that the K and V tiles read by pass A (G x 64 KB
+// per CTA) are still in L2 when pass B reads them again.  GRET_SPAN_CHUNKS overrides the choice.
+int span_chunks(int64_t chunks_per_unit, int64_t chains, int grid) {
+    static int forced = -2;
+    if (forced == -2) {
         const char* e = getenv("GRET_SPAN_CHUNKS");
-        g = e ? atoi(e) : 8;
-        if (g < 1) g = 8;
+        forced = e ? atoi(e) : -1;
+        if (forced < 1) forced = -1;
     }
-    return g;
+    if (forced > 0) return forced;
+    int best = 8;
+    int64_t best_cost = -1;
+    for (int g = 8; g >= 2; --g) {
+        const int64_t spans = (chunks_per_unit + g - 1) / g;
+        const int64_t waves = (chains * std::max<int64_t>(spans, 1) + grid - 1) / grid;
+        const int64_t cost = std::max(waves * (g + 1), spans + g);
+        if (best_cost < 0 || cost < best_cost) {
+            best = g;
+            best_cost = cost;
+        }
+    }
+    return best;
 }
 
 }  // namespace
@@ -1018,7 +1036,9 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
     const int units = a.n_seqs;
     const WsLayout L = ws_layout(units, a.H);
     unsigned char* ws = (unsigned char*)a.workspace;
-    const int G = span_chunks();
+    const int64_t chunks_per_unit =
+        units > 0 ? ((varlen ? a.N / units : a.N) + C - 1) / C : 0;   // varlen: the mean
+    const int G = span_chunks(chunks_per_unit, (int64_t)units * a.H, sm_count());
 
     TcParams p;
     p.g = a.g;
