@@ -94,16 +94,18 @@ struct __align__(1024) Smem {
     unsigned char q[2][TILE];  // Q tile; in pass A, and after Q S in pass B, the low half of w K
     unsigned char k[2][TILE];  // K tile; rewritten in place as the high half of w K
     unsigned char v[2][TILE];
-    unsigned char sbf[TILE];   // bf16 high half, then low half, of the entry state (Q S_prev)
+    // bf16 high half, then low half, of the state that Q S_prev reads; between a chunk's Q S_lo
+    // and the next high half, the chunk's bf16 output tile on its way out by TMA store
+    unsigned char sbf[TILE];
     uint64_t kv_full[2], stage_empty[2];
     uint64_t item_full[ITEM_DEPTH], item_empty[ITEM_DEPTH];
-    // k_ready / kh_ready (per stage): the state group's / the helpers' share of the w K split
-    // is written.  Each has one producing group, so arrivals of different groups never mix, and
+    // k_ready / kp_ready / kh_ready (per stage): the state group's / the P group's / the helpers'
+    // share of the w K split is written.  Each has one producing group, so arrivals of different groups never mix, and
     // being per stage, a group can reach the next phase of a stage's barrier only after the MMA
     // has released that stage -- so no waiter can be left two phases behind.
-    uint64_t k_ready[2], kh_ready[2];
+    uint64_t k_ready[2], kh_ready[2], kp_ready[2];
     uint64_t a_full, s3a_done, q_free, p_ready, s_lo_ready, o_full, o_free, ds_full, ds_free,
-        s_ready, drain;
+        s_ready, sbf_free, drain;
     Item items[ITEM_DEPTH];
     float gc[2][C];            // per stage: in-chunk inclusive cumulative log2-decay of each token
     float gtot[2];             // per stage: the chunk's total log2-decay
@@ -131,6 +133,7 @@ struct TcParams {
     int spans_per_unit;        // dense
     int qk_pos_tok, qk_pos_head, qk_pos_b;   // tensor-map dimension of each coordinate
     int v_pos_tok, v_pos_head, v_pos_b;
+    int o_pos_tok, o_pos_head, o_pos_b;
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -139,8 +142,10 @@ __device__ __forceinline__ float ex2f(float x) {
     return y;
 }
 
+// log(sigmoid(x)) = min(x, 0) - log(1 + exp(-|x|)) with the fast exponential and logarithm:
+// the absolute error stays near 1e-7, which is what the cumulative decay (a sum of these) sees.
 __device__ __forceinline__ float logsigmoid_(float x) {
-    return fminf(x, 0.f) - log1pf(expf(-fabsf(x)));
+    return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
 }
 
 __device__ __forceinline__ void named_sync(int id, int nthreads = 128) {
@@ -418,6 +423,7 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
             const int st = j & 1;
             if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
             if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
+            if (!W(&sm.kp_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
             if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
             tc_fence_after();
@@ -426,8 +432,9 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
             mma_commit(&sm.stage_empty[st]);
         }
         // pass B: the full chunk.  Order per chunk: Q K^T (issued one chunk ahead), Q S_hi,
-        // Q S_lo (after which the Q slot is free for the low half of w K), P V, then Q K^T of the
-        // next chunk, then dS -- so the decay mask of chunk c + 1 overlaps the state update of c.
+        // Q S_lo (after which the Q slot is free for the low half of w K), P V (which runs while
+        // w K is split), dS (on the state chain, so as soon as the split is done), then Q K^T of
+        // the next chunk once P V has read P out of the tensor memory it overwrites.
         auto issue_qk = [&](int jj, int bb) {
             const int st = jj & 1;
             if (!W(&sm.kv_full[st], (jj >> 1) & 1)) return false;
@@ -455,14 +462,15 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
             mma_pv(tmem + TM_O, tmem + TM_A, 0, vb, false);        // O  = P_hi V
             mma_pv(tmem + TM_O, tmem + TM_A, 1, vb, true);         // O += P_lo V
             mma_commit(&sm.o_full);
-            if (c + 1 < it.c_end && !issue_qk(j + 1, b + 1)) break;
             if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
+            if (!W(&sm.kp_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
             if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
             tc_fence_after();
             mma_ds(tmem, sm, st);
             mma_commit(&sm.ds_full);
             mma_commit(&sm.stage_empty[st]);
+            if (c + 1 < it.c_end && !issue_qk(j + 1, b + 1)) break;
         }
     }
     // all issued MMAs complete before TMEM is released
@@ -514,9 +522,11 @@ __device__ __forceinline__ void split_k_chunks(unsigned char* ktile, unsigned ch
     }
 }
 
-// The split of w K is shared: the state group takes chunks 0-10 of its own row, warps 2-3 take
-// chunks 11-15 of two rows each.
-constexpr int SPLIT_OWN = 11;
+// The split of w K is shared by three groups, by 16-byte chunks of each 128-element row: the state
+// group takes chunks 0-6 of its own row, the P group chunks 7-12 of its own row, and warps 2-3
+// chunks 13-15 of two rows each.
+constexpr int SPLIT_STATE = 7, SPLIT_P = 6;
+constexpr int SPLIT_HELP0 = SPLIT_STATE + SPLIT_P, SPLIT_HELP = 16 - SPLIT_HELP0;
 
 // weight of token r of chunk c: k_scale * exp(c_b - c_r), zero past the end of the sequence
 __device__ __forceinline__ float k_weight(const Smem& sm, const TcParams& p, const Item& it, int c,
@@ -525,18 +535,29 @@ __device__ __forceinline__ float k_weight(const Smem& sm, const TcParams& p, con
     return valid ? ex2f(sm.gtot[st] - sm.gc[st][r]) * p.k_scale : 0.f;
 }
 
-// Row r of the state into the MN-major swizzled tile read by Q S: its bf16 high half (low ==
-// false) or its low half (low == true).
-__device__ __forceinline__ void write_state_half(unsigned char* tile, int r, const float (&S)[D],
-                                                 bool low) {
+// Row r of the state into the MN-major swizzled tile read by Q S: the bf16 high half is
+// written and the low half kept in registers for write_state_lo.
+__device__ __forceinline__ void write_state_hi(unsigned char* tile, int r, const float (&S)[D],
+                                               uint32_t (&lo)[D / 2]) {
 #pragma unroll
     for (int cc = 0; cc < 16; ++cc) {
-        uint32_t hi[4], lo[4];
+        uint32_t hi[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) split2(S[8 * cc + 2 * e], S[8 * cc + 2 * e + 1], hi[e], lo[e]);
+        for (int e = 0; e < 4; ++e)
+            split2(S[8 * cc + 2 * e], S[8 * cc + 2 * e + 1], hi[e], lo[4 * cc + e]);
         const int half = cc >> 3, c = cc & 7;
         *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) =
-            low ? make_uint4(lo[0], lo[1], lo[2], lo[3]) : make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    }
+}
+
+__device__ __forceinline__ void write_state_lo(unsigned char* tile, int r,
+                                               const uint32_t (&lo)[D / 2]) {
+#pragma unroll
+    for (int cc = 0; cc < 16; ++cc) {
+        const int half = cc >> 3, c = cc & 7;
+        *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) =
+            make_uint4(lo[4 * cc], lo[4 * cc + 1], lo[4 * cc + 2], lo[4 * cc + 3]);
     }
 }
 
@@ -555,7 +576,8 @@ __device__ __forceinline__ void fold_ds(uint32_t taddr, float (&S)[D], float eb)
 // ----------------------------------------------------------------------------------------------
 // warps 4-7: decay mask (P split into bf16 halves in TMEM) and output epilogue
 
-__device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
+__device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint32_t tmem, int warp,
+                        int lane) {
     GroupWait gw{&sm, &p, 0, (warp - 4) * 32 + lane};
     const int q = warp & 3, r = q * 32 + lane;
     const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
@@ -568,46 +590,68 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
         ++it_n;
         if (!it.valid) break;
         bool ok = true;
-        j += it.c_end - it.c_begin;     // the span's pass-A jobs
-        for (int c = it.c_begin; c < it.c_end; ++c, ++b, ++j) {
+        const int n = it.c_end - it.c_begin;
+        // every job of the span: pass A (its share of the w K split only), then pass B
+        for (int jj = 0; jj < 2 * n; ++jj, ++j) {
             const int st = j & 1;
-            // a_full first: this group waits only on pass-B chunks, and a parity wait on
-            // kv_full is exact only once Q K^T of this chunk (hence its load) has completed.
-            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
-            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }  // gate slot
-            const float cr = sm.gc[st][r];
-            tc_fence_after();
-            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, split into bf16 halves; each
-            // 32-column group of A is replaced in place by [16 high | 16 low] columns of P.
+            const bool pass_b = jj >= n;
+            const int c = it.c_begin + (pass_b ? jj - n : jj);
+            // the stage's gate slot is read before this group's split share is released: after
+            // that the stage may be refilled
+            float cr = 0.f;
+            if (!pass_b) {
+                if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
+            } else {
+                if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
+                if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }  // gate slot
+                cr = sm.gc[st][r];
+                tc_fence_after();
+                // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, split into bf16 halves; each
+                // 32-column group of A is replaced in place by [16 high | 16 low] columns of P.
 #pragma unroll 1
-            for (int jc = 0; jc < 4; ++jc) {
-                uint32_t ph[32];
-                if (jc <= q) {
-                    float a[32];
-                    tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
-                    tmem_ld_wait();
+                for (int jc = 0; jc < 4; ++jc) {
+                    uint32_t ph[32];
+                    if (jc <= q) {
+                        float a[32];
+                        tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
+                        tmem_ld_wait();
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int m0 = jc * 32 + 2 * i;
-                        const float p0 = (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * p.k_scale * a[2 * i] : 0.f;
-                        const float p1 =
-                            (m0 + 1 <= r) ? ex2f(cr - sm.gc[st][m0 + 1]) * p.k_scale * a[2 * i + 1] : 0.f;
-                        split2(p0, p1, ph[i], ph[16 + i]);
+                        for (int i = 0; i < 16; ++i) {
+                            const int m0 = jc * 32 + 2 * i;
+                            const float p0 =
+                                (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * p.k_scale * a[2 * i] : 0.f;
+                            const float p1 = (m0 + 1 <= r)
+                                                 ? ex2f(cr - sm.gc[st][m0 + 1]) * p.k_scale * a[2 * i + 1]
+                                                 : 0.f;
+                            split2(p0, p1, ph[i], ph[16 + i]);
+                        }
+                    } else {
+#pragma unroll
+                        for (int i = 0; i < 32; ++i) ph[i] = 0u;
                     }
-                } else {
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) ph[i] = 0u;
+                    tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
                 }
-                tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.p_ready);
+                // both Q S MMAs are done: the Q slot takes the low half of w K
+                if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
             }
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&sm.p_ready);
-            // epilogue: O = O_inner + 2^(c_r) O_cross
+            split_k_chunks<SPLIT_STATE, SPLIT_P>(sm.k[st], sm.q[st], r,
+                                                 k_weight(sm, p, it, c, st, r));
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.kp_ready[st]);
+            if (!pass_b) continue;
+            // epilogue: O = O_inner + 2^(c_r) O_cross, rounded to bf16.  A chunk that lies wholly
+            // inside its sequence goes out as one tile: rows into the state buffer (free between
+            // Q S_lo and the next state write) in the swizzled layout, then two TMA stores.  The
+            // rows of a partial chunk are stored one by one, so that nothing past the end of the
+            // sequence (the next packed sequence) is written.
             if (!gw.wait(&sm.o_full, b & 1)) { ok = false; break; }
             tc_fence_after();
             const float ec = ex2f(cr);
             const int64_t t = (int64_t)c * C + r;
+            const bool full = (int64_t)(c + 1) * C <= it.len;
             const bool valid = t < it.len;
             __nv_bfloat16* orow = p.o + (int64_t)it.b * p.osb + (it.tok_first + t) * p.ost +
                                   (int64_t)it.h * p.osh;
@@ -617,28 +661,55 @@ __device__ void p_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, in
                 tmem_ld32(tmem + lane_base + TM_O + jc * 32, o);
                 tmem_ld32(tmem + lane_base + TM_OX + jc * 32, ox);
                 tmem_ld_wait();
-                if (valid) {
+                uint4 u[4];
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    u[v4].x = pack_bf16x2(fmaf(ec, ox[8 * v4 + 0], o[8 * v4 + 0]),
+                                          fmaf(ec, ox[8 * v4 + 1], o[8 * v4 + 1]));
+                    u[v4].y = pack_bf16x2(fmaf(ec, ox[8 * v4 + 2], o[8 * v4 + 2]),
+                                          fmaf(ec, ox[8 * v4 + 3], o[8 * v4 + 3]));
+                    u[v4].z = pack_bf16x2(fmaf(ec, ox[8 * v4 + 4], o[8 * v4 + 4]),
+                                          fmaf(ec, ox[8 * v4 + 5], o[8 * v4 + 5]));
+                    u[v4].w = pack_bf16x2(fmaf(ec, ox[8 * v4 + 6], o[8 * v4 + 6]),
+                                          fmaf(ec, ox[8 * v4 + 7], o[8 * v4 + 7]));
+                }
+                if (full) {
+                    // columns 32 jc .. 32 jc + 31: 16-byte chunks 4 (jc % 2) + v4 of slab jc / 2
+                    unsigned char* rowp = sm.sbf + (jc >> 1) * SLAB + r * 128;
+#pragma unroll
+                    for (int v4 = 0; v4 < 4; ++v4)
+                        *reinterpret_cast<uint4*>(rowp + (((4 * (jc & 1) + v4) ^ (r & 7)) << 4)) =
+                            u[v4];
+                } else if (valid) {
                     uint4* dst = reinterpret_cast<uint4*>(orow + jc * 32);
 #pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) {
-                        uint4 u;
-                        u.x = pack_bf16x2(fmaf(ec, ox[8 * v4 + 0], o[8 * v4 + 0]),
-                                          fmaf(ec, ox[8 * v4 + 1], o[8 * v4 + 1]));
-                        u.y = pack_bf16x2(fmaf(ec, ox[8 * v4 + 2], o[8 * v4 + 2]),
-                                          fmaf(ec, ox[8 * v4 + 3], o[8 * v4 + 3]));
-                        u.z = pack_bf16x2(fmaf(ec, ox[8 * v4 + 4], o[8 * v4 + 4]),
-                                          fmaf(ec, ox[8 * v4 + 5], o[8 * v4 + 5]));
-                        u.w = pack_bf16x2(fmaf(ec, ox[8 * v4 + 6], o[8 * v4 + 6]),
-                                          fmaf(ec, ox[8 * v4 + 7], o[8 * v4 + 7]));
-                        dst[v4] = u;
-                    }
+                    for (int v4 = 0; v4 < 4; ++v4) dst[v4] = u[v4];
                 }
             }
             tc_fence_before();
             mbar_arrive(&sm.o_free);
+            if (full) {
+                fence_proxy_async_smem();
+                named_sync(1);   // every row of the tile is written
+                if (gw.tid == 0) {
+                    const int tok = (int)(it.tok_first + (int64_t)c * C);
+                    int co[4];
+#pragma unroll 1
+                    for (int half = 0; half < 2; ++half) {
+                        set_coord(co, p.o_pos_tok, p.o_pos_head, p.o_pos_b, half * 64, tok, it.h,
+                                  it.b);
+                        tma_store_4d(to, sm.sbf + half * SLAB, co[0], co[1], co[2], co[3]);
+                    }
+                    bulk_commit_group();
+                    bulk_wait_group_read0();
+                }
+            }
+            if (gw.tid == 0) mbar_arrive(&sm.sbf_free);   // the state buffer can be rewritten
+            ++b;
         }
         if (!ok) break;
     }
+    if (gw.tid == 0) bulk_wait_group0();   // the last output tiles are written before exit
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -676,7 +747,7 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
                 if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
                 const float t = sm.gtot[st];
                 if (st) tot1 = t; else tot0 = t;
-                split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r,
+                split_k_chunks<0, SPLIT_STATE>(sm.k[st], sm.q[st], r,
                                              k_weight(sm, p, it, it.c_begin + i, st, r));
                 fence_proxy_async_smem();
                 mbar_arrive(&sm.k_ready[st]);
@@ -708,67 +779,73 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         const float eL = ex2f(L);
         float4* dst = it.last ? nullptr
                               : reinterpret_cast<float4*>(p.slots + (chain * 2 + (it.s & 1)) * (D * D));
-        // four batches of 8 independent loads each, then the inclusive state and the swap
+        // E comes in through the state buffer, free once the previous chunk's output tile has
+        // left it: two rounds of 16 float4 per thread, each thread copying and reading back only
+        // its own elements (no barrier between the rounds), with all 16 copies of a round in
+        // flight.
+        if (b > 0 && !gw.wait(&sm.sbf_free, (b - 1) & 1)) break;
+        float4* ebuf = reinterpret_cast<float4*>(sm.sbf) + r;
+        // float4 j4 of the row: slot layout [j4][row], state_in layout [row][j4]
+        const float4* esrc4 =
+            reinterpret_cast<const float4*>(esrc) + (from_slot ? r : 0);
+        const int estep = from_slot ? D : 1;
 #pragma unroll
-        for (int quarter = 0; quarter < 4; ++quarter) {
-            float4 e[8];
-#pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-                const int j4 = quarter * 8 + k4;
-                e[k4] = make_float4(0.f, 0.f, 0.f, 0.f);
-                if (from_slot)
-                    e[k4] = __ldcg(reinterpret_cast<const float4*>(esrc) + j4 * D + r);
-                else if (esrc)
-                    e[k4] = __ldg(reinterpret_cast<const float4*>(esrc) + j4);
+        for (int half = 0; half < 2; ++half) {
+            if (esrc) {
+#pragma unroll 1
+                for (int k = 0; k < 16; ++k)
+                    cp_async_16(ebuf + k * D, esrc4 + (half * 16 + k) * estep);
+                cp_async_wait_all();
             }
 #pragma unroll
-            for (int k4 = 0; k4 < 8; ++k4) {
-                const int j4 = quarter * 8 + k4;
+            for (int k = 0; k < 16; ++k) {
+                const int j4 = half * 16 + k;
+                const float4 x = esrc ? ebuf[k * D] : make_float4(0.f, 0.f, 0.f, 0.f);
                 if (dst) {
                     float4 inc;
-                    inc.x = fmaf(eL, e[k4].x, S[4 * j4 + 0]);
-                    inc.y = fmaf(eL, e[k4].y, S[4 * j4 + 1]);
-                    inc.z = fmaf(eL, e[k4].z, S[4 * j4 + 2]);
-                    inc.w = fmaf(eL, e[k4].w, S[4 * j4 + 3]);
+                    inc.x = fmaf(eL, x.x, S[4 * j4 + 0]);
+                    inc.y = fmaf(eL, x.y, S[4 * j4 + 1]);
+                    inc.z = fmaf(eL, x.z, S[4 * j4 + 2]);
+                    inc.w = fmaf(eL, x.w, S[4 * j4 + 3]);
                     __stcg(dst + j4 * D + r, inc);
                 }
-                S[4 * j4 + 0] = e[k4].x;
-                S[4 * j4 + 1] = e[k4].y;
-                S[4 * j4 + 2] = e[k4].z;
-                S[4 * j4 + 3] = e[k4].w;
+                S[4 * j4 + 0] = x.x;
+                S[4 * j4 + 1] = x.y;
+                S[4 * j4 + 2] = x.z;
+                S[4 * j4 + 3] = x.w;
             }
         }
-        if (dst) {
-            __threadfence();
-            named_sync(2);
-            if (r == 0) {
-                uint32_t* f = p.flags + chain * 2 + (it.s & 1);
-                asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"((uint32_t)it.s + 1)
-                             : "memory");
-            }
+        // One barrier for two orders: every thread has read its part of E out of the state
+        // buffer before any thread writes its row of the state into it (the two layouts differ),
+        // and every published row is stored and fenced before the flag is raised.
+        if (dst) __threadfence();
+        named_sync(2);
+        if (dst && r == 0) {
+            uint32_t* f = p.flags + chain * 2 + (it.s & 1);
+            asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"((uint32_t)it.s + 1)
+                         : "memory");
         }
-        // ---- pass B: running state from E.  The state buffer takes, in turn, the high half of
-        // E, then per chunk the low half of the state before it (once Q S_hi is done) and, but
-        // after the last chunk, the high half of the state after it.  Writes w = 0 .. 2n-1:
-        // even w high halves, odd w low halves of chunk (w - 1) / 2, each low half followed by
-        // the chunk's split and fold.
+        // ---- pass B: running state from E.  Per chunk: the bf16 high half of the state before
+        // it goes into the state buffer (once the previous chunk's output tile has left it) for
+        // Q S_hi, then its low half (kept in registers) once Q S_hi is done, then the chunk's
+        // split of w K (into the Q slot, free after Q S_lo) and the fold of its dS.
 #pragma unroll 1
-        for (int w = 0; w < 2 * n; ++w) {
-            const bool low = w & 1;
-            const int i = w >> 1;           // chunk of a low half
+        for (int i = 0; i < n; ++i) {
             const int st = (j + i) & 1;
-            if (low) {
-                if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
-                if (!gw.wait(&sm.s3a_done, (b + i) & 1)) { ok = false; break; }
-            }
-            write_state_half(sm.sbf, r, S, low);
+            uint32_t slo[D / 2];   // bf16 low half of the state row, between its two writes
+            if (b + i > 0 && !gw.wait(&sm.sbf_free, (b + i - 1) & 1)) { ok = false; break; }
+            write_state_hi(sm.sbf, r, S, slo);
             fence_proxy_async_smem();
-            mbar_arrive(low ? &sm.s_lo_ready : &sm.s_ready);
-            if (!low) continue;
+            mbar_arrive(&sm.s_ready);
+            if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.s3a_done, (b + i) & 1)) { ok = false; break; }
+            write_state_lo(sm.sbf, r, slo);
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.s_lo_ready);
             const float tot = sm.gtot[st];
             // every MMA reading Q has completed: its slot takes the low half of w K
             if (!gw.wait(&sm.q_free, (b + i) & 1)) { ok = false; break; }
-            split_k_chunks<0, SPLIT_OWN>(sm.k[st], sm.q[st], r,
+            split_k_chunks<0, SPLIT_STATE>(sm.k[st], sm.q[st], r,
                                          k_weight(sm, p, it, it.c_begin + i, st, r));
             fence_proxy_async_smem();
             mbar_arrive(&sm.k_ready[st]);
@@ -777,7 +854,6 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
             fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
-            if (i + 1 == n) break;          // no high half after the last chunk
         }
         j += n;
         b += n;
@@ -816,11 +892,11 @@ __device__ void split_helper(Smem& sm, const TcParams& p, int warp, int lane) {
                 if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
                 ++b;
             }
-#pragma unroll
+#pragma unroll 1
             for (int h = 0; h < 2; ++h) {
                 const int r = 2 * t + h;
-                split_k_chunks<SPLIT_OWN, 16 - SPLIT_OWN>(sm.k[st], sm.q[st], r,
-                                                          k_weight(sm, p, it, c, st, r));
+                split_k_chunks<SPLIT_HELP0, SPLIT_HELP>(sm.k[st], sm.q[st], r,
+                                                        k_weight(sm, p, it, c, st, r));
             }
             fence_proxy_async_smem();
             mbar_arrive(&sm.kh_ready[st]);
@@ -830,7 +906,8 @@ __device__ void split_helper(Smem& sm, const TcParams& p, int warp, int lane) {
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                      const __grid_constant__ CUtensorMap tv, const TcParams p, uint32_t total_dense) {
+                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                      const TcParams p, uint32_t total_dense) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -856,11 +933,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         mbar_init(&sm.o_free, 128);
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.k_ready[s], 128);
+            mbar_init(&sm.kp_ready[s], 128);
             mbar_init(&sm.kh_ready[s], 64);
         }
         mbar_init(&sm.ds_full, 1);
         mbar_init(&sm.ds_free, 128);
         mbar_init(&sm.s_ready, 128);
+        mbar_init(&sm.sbf_free, 1);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -880,6 +959,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tma_prefetch_desc(&tq);
                 tma_prefetch_desc(&tk);
                 tma_prefetch_desc(&tv);
+                tma_prefetch_desc(&to);
             }
             const uint32_t total =
                 p.prefix ? (uint32_t)p.prefix[p.units] * (uint32_t)p.H : total_dense;
@@ -893,7 +973,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         // 168 -> 136 is a decrease: setmaxnreg.inc must never ask for fewer registers than the
         // warp holds, and .dec never for more.
         asm volatile("setmaxnreg.dec.sync.aligned.u32 136;" ::: "memory");
-        p_group(sm, p, tmem, warp, lane);
+        p_group(sm, p, &to, tmem, warp, lane);
     } else {
         asm volatile("setmaxnreg.inc.sync.aligned.u32 256;" ::: "memory");
         state_group(sm, p, tmem, warp, lane);
@@ -1063,10 +1143,11 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
 
     const int64_t ntok = a.N;   // dense: tokens per sequence; varlen: packed total
     const int B = varlen ? 1 : a.B;
-    CUtensorMap tq, tk, tv;
+    CUtensorMap tq, tk, tv, to;
     if (!make_map(&tq, a.q, a.st, a.sh, a.sb, ntok, a.H, B, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b) ||
         !make_map(&tk, a.k, a.st, a.sh, a.sb, ntok, a.H, B, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b) ||
-        !make_map(&tv, a.v, a.vst, a.vsh, a.vsb, ntok, a.H, B, p.v_pos_tok, p.v_pos_head, p.v_pos_b))
+        !make_map(&tv, a.v, a.vst, a.vsh, a.vsb, ntok, a.H, B, p.v_pos_tok, p.v_pos_head, p.v_pos_b) ||
+        !make_map(&to, a.o, a.ost, a.osh, a.osb, ntok, a.H, B, p.o_pos_tok, p.o_pos_head, p.o_pos_b))
         return GRET_ERR_UNSUPPORTED;
 
     uint64_t total_dense = varlen ? 0 : (uint64_t)units * p.spans_per_unit * a.H;
@@ -1093,7 +1174,7 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
     int grid = sm_count();
     if (!varlen && total_dense < (uint64_t)grid) grid = (int)total_dense;
     if (grid < 1) grid = 1;
-    prefill_tc_kernel<<<grid, NTHREADS, smem, a.stream>>>(tq, tk, tv, p, (uint32_t)total_dense);
+    prefill_tc_kernel<<<grid, NTHREADS, smem, a.stream>>>(tq, tk, tv, to, p, (uint32_t)total_dense);
     return cudaGetLastError() == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 

@@ -95,6 +95,26 @@ def test_repeated_calls_reuse_workspace():
     assert G.gret_workspace_status(ws) == 0
 
 
+@pytest.mark.parametrize("N", [1553, 4096])
+def test_repeated_multi_span_calls_into_poisoned_output(N):
+    """Chains of several spans, called again and again into an output pre-filled with NaN: a
+    row that a call fails to write, or an entry state read while another warp overwrites it,
+    shows up in one of the repetitions even when it is rare."""
+    G = lib()
+    H = 3
+    inp = SI.gret_inputs(1, N, H, 128, dtype=BF, seed=N + 7, with_state=True)
+    o_ref, s_ref = oracle.gret_recurrent(inp["q"][0], inp["k"][0], inp["v"][0], inp["g"][0],
+                                         state_in=inp["s"])
+    d = {k: v.cuda() for k, v in inp.items()}
+    for _ in range(8):
+        o = torch.full((1, N, H, 128), float("nan"), dtype=BF, device="cuda")
+        _, s = G.gret_prefill_chunkwise(d["q"], d["k"], d["v"], d["g"], state_in=d["s"],
+                                        state_out=True, o=o)
+        torch.cuda.synchronize()
+        assert_parity("o", o[0], o_ref, 1e-2, stored_bf16=True)
+        assert_parity("state", s, s_ref, 1e-2, stored_bf16=False)
+
+
 def _sampled_heads(B, N, H, seed, heads, g_mean=2.0, g_std=1.0):
     """Full-size run on the GPU; oracle on a subset of heads (heads are independent)."""
     G = lib()
