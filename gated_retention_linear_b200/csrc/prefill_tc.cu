@@ -109,6 +109,9 @@ struct __align__(1024) Smem {
     Item items[ITEM_DEPTH];
     float gc[2][C];            // per stage: in-chunk inclusive cumulative log2-decay of each token
     float gtot[2];             // per stage: the chunk's total log2-decay
+    // per stage: exponent base of the key weights w_m = k_scale * 2^(gbase - c_m): the chunk
+    // total in pass B, the chunk total plus that of the span's later chunks in pass A
+    float gbase[2];
     uint32_t dec[3][2];        // group-uniform wait decisions (double-buffered)
     uint32_t tmem_base;
     uint32_t abort;
@@ -261,21 +264,29 @@ __device__ __forceinline__ void set_coord(int (&c)[4], int pos_tok, int pos_head
 // ----------------------------------------------------------------------------------------------
 // warp 0: TMA producer (lane 0) and gate scan (all lanes)
 
-// The whole warp computes, for the chunk's 128 tokens (4 consecutive per lane), the in-chunk
-// inclusive cumulative log2-decay c_t = sum of logsigmoid(g)/tau * log2(e) over the chunk up to
-// t (0 past the end of the sequence) and the chunk total, into the stage's gate slot.
-__device__ __forceinline__ void gate_scan(Smem& sm, const TcParams& p, const Item& it, int c, int st,
-                                          int lane) {
+// The chunk's gate logits, 4 consecutive tokens per lane (token 0's logit past the end of the
+// sequence, masked by the scan).
+__device__ __forceinline__ void gate_load(const TcParams& p, const Item& it, int c, int lane,
+                                          float (&g4)[4]) {
+    const int64_t t0 = (int64_t)c * C + 4 * lane;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        const int64_t t = (t0 + e < it.len) ? t0 + e : 0;
+        g4[e] = __ldg(p.g + (it.grow0 + t) * p.H + it.h);
+    }
+}
+
+// The whole warp computes, for the chunk's 128 tokens, the in-chunk inclusive cumulative
+// log2-decay c_t = sum of logsigmoid(g)/tau * log2(e) over the chunk up to t (0 past the end of
+// the sequence), the chunk total and the weight base `after` + total into the stage's gate slot;
+// returns the chunk total on every lane.
+__device__ __forceinline__ float gate_scan(Smem& sm, const TcParams& p, const Item& it, int c,
+                                           int st, int lane, const float (&g4)[4], float after) {
     float lam[4];
     const int64_t t0 = (int64_t)c * C + 4 * lane;
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {   // all four loads in flight before any use
-        const int64_t t = (t0 + e < it.len) ? t0 + e : 0;
-        lam[e] = __ldg(p.g + (it.grow0 + t) * p.H + it.h);
-    }
-#pragma unroll
     for (int e = 0; e < 4; ++e)
-        lam[e] = (t0 + e < it.len) ? logsigmoid_(lam[e]) * p.inv_tau_log2e : 0.f;
+        lam[e] = (t0 + e < it.len) ? logsigmoid_(g4[e]) * p.inv_tau_log2e : 0.f;
     lam[1] += lam[0];
     lam[2] += lam[1];
     lam[3] += lam[2];
@@ -288,7 +299,12 @@ __device__ __forceinline__ void gate_scan(Smem& sm, const TcParams& p, const Ite
     const float excl = x - lam[3];
 #pragma unroll
     for (int e = 0; e < 4; ++e) sm.gc[st][4 * lane + e] = excl + lam[e];
-    if (lane == 31) sm.gtot[st] = x;
+    const float tot = __shfl_sync(0xffffffffu, x, 31);
+    if (lane == 31) {
+        sm.gtot[st] = tot;
+        sm.gbase[st] = after + tot;
+    }
+    return tot;
 }
 
 __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
@@ -315,39 +331,45 @@ __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, con
         }
         ++it_n;
         if (!it.valid) break;
-        for (int pass = 0; pass < 2 && !aborted; ++pass) {
-            for (int c = it.c_begin; c < it.c_end; ++c) {
-                const int st = j & 1;
-                ok = 1;
-                if (lane == 0 && j >= 2)
-                    ok = mbar_wait(&sm.stage_empty[st], ((j >> 1) - 1) & 1, &sm.abort, WAIT_NS);
-                if (!__shfl_sync(0xffffffffu, ok, 0)) {
-                    aborted = true;
-                    break;
-                }
-                if (lane == 0) {
-                    mbar_arrive_expect_tx(&sm.kv_full[st], pass ? 3 * TILE : 2 * TILE);
-                    const int tok = (int)(it.tok_first + (int64_t)c * C);
-                    int ck[4], cv[4];
-                    for (int half = 0; half < 2; ++half) {
-                        set_coord(ck, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b, half * 64, tok, it.h,
-                                  it.b);
-                        set_coord(cv, p.v_pos_tok, p.v_pos_head, p.v_pos_b, half * 64, tok, it.h,
-                                  it.b);
-                        tma_load_4d(sm.k[st] + half * SLAB, tk, &sm.kv_full[st], ck[0], ck[1],
-                                    ck[2], ck[3]);
-                        tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], cv[0], cv[1],
-                                    cv[2], cv[3]);
-                        if (pass)
-                            tma_load_4d(sm.q[st] + half * SLAB, tq, &sm.kv_full[st], ck[0], ck[1],
-                                        ck[2], ck[3]);
-                    }
-                }
-                gate_scan(sm, p, it, c, st, lane);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.kv_full[st]);
-                ++j;
+        // pass A visits the span's chunks last to first (its aggregate is accumulated by the
+        // MMAs with each key weighted by its decay to the end of the span); pass B first to last
+        const int n = it.c_end - it.c_begin;
+        float after = 0.f;   // pass A: log2-decay of the chunks after the current one
+        for (int jj = 0; jj < 2 * n; ++jj) {
+            const bool pass_b = jj >= n;
+            const int c = pass_b ? it.c_begin + (jj - n) : it.c_end - 1 - jj;
+            const int st = j & 1;
+            float g4[4];
+            gate_load(p, it, c, lane, g4);   // in flight while the stage is awaited
+            ok = 1;
+            if (lane == 0 && j >= 2)
+                ok = mbar_wait(&sm.stage_empty[st], ((j >> 1) - 1) & 1, &sm.abort, WAIT_NS);
+            if (!__shfl_sync(0xffffffffu, ok, 0)) {
+                aborted = true;
+                break;
             }
+            if (lane == 0) {
+                mbar_arrive_expect_tx(&sm.kv_full[st], pass_b ? 3 * TILE : 2 * TILE);
+                const int tok = (int)(it.tok_first + (int64_t)c * C);
+                int ck[4], cv[4];
+                for (int half = 0; half < 2; ++half) {
+                    set_coord(ck, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b, half * 64, tok, it.h,
+                              it.b);
+                    set_coord(cv, p.v_pos_tok, p.v_pos_head, p.v_pos_b, half * 64, tok, it.h, it.b);
+                    tma_load_4d(sm.k[st] + half * SLAB, tk, &sm.kv_full[st], ck[0], ck[1], ck[2],
+                                ck[3]);
+                    tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], cv[0], cv[1], cv[2],
+                                cv[3]);
+                    if (pass_b)
+                        tma_load_4d(sm.q[st] + half * SLAB, tq, &sm.kv_full[st], ck[0], ck[1],
+                                    ck[2], ck[3]);
+                }
+            }
+            const float tot = gate_scan(sm, p, it, c, st, lane, g4, pass_b ? 0.f : after);
+            if (!pass_b) after += tot;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.kv_full[st]);
+            ++j;
         }
     }
     if (lane == 0) {
@@ -393,14 +415,15 @@ __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, ui
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// dS = (w K)^T V as the sum of its bf16 high half (K slot) and low half (Q slot).
-__device__ __forceinline__ void mma_ds(uint32_t tmem, Smem& sm, int st) {
-    mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, false);
+// dS (+)= (w K)^T V as the sum of its bf16 high half (K slot) and low half (Q slot).
+__device__ __forceinline__ void mma_ds(uint32_t tmem, Smem& sm, int st, bool accumulate) {
+    mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, accumulate);
     mma_128(tmem + TM_DS, smem_u32(sm.q[st]), true, smem_u32(sm.v[st]), true, true);
 }
 
 __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
     int j = 0, b = 0, it_n = 0;
+    int dsn = 0;   // dS results handed to the state group so far (phases of ds_full)
     bool ok = true;
     auto W = [&](uint64_t* bar, uint32_t par) {
         if (ok && !mbar_wait(bar, par, &sm.abort, WAIT_NS)) {
@@ -418,18 +441,24 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
         mbar_arrive(&sm.item_empty[slot]);
         ++it_n;
         if (!it.valid) break;
-        // pass A: dS only
-        for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j) {
+        // pass A: the span's aggregate, one dS result accumulated over its chunks (which the
+        // producer delivers last to first, each key weighted by its decay to the span's end)
+        const int n = it.c_end - it.c_begin;
+        for (int i = 0; i < n && ok; ++i, ++j) {
             const int st = j & 1;
             if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
             if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.kp_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
-            if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
+            if (i == 0 && dsn > 0 && !W(&sm.ds_free, (dsn - 1) & 1)) break;
             tc_fence_after();
-            mma_ds(tmem, sm, st);
-            mma_commit(&sm.ds_full);
+            mma_ds(tmem, sm, st, i > 0);
             mma_commit(&sm.stage_empty[st]);
+        }
+        if (!ok) break;
+        if (n > 0) {
+            mma_commit(&sm.ds_full);
+            ++dsn;
         }
         // pass B: the full chunk.  Order per chunk: Q K^T (issued one chunk ahead), Q S_hi,
         // Q S_lo (after which the Q slot is free for the low half of w K), P V (which runs while
@@ -465,11 +494,12 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
             if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.kp_ready[st], (j >> 1) & 1)) break;
             if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
-            if (j > 0 && !W(&sm.ds_free, (j - 1) & 1)) break;
+            if (dsn > 0 && !W(&sm.ds_free, (dsn - 1) & 1)) break;
             tc_fence_after();
-            mma_ds(tmem, sm, st);
+            mma_ds(tmem, sm, st, false);
             mma_commit(&sm.ds_full);
             mma_commit(&sm.stage_empty[st]);
+            ++dsn;
             if (c + 1 < it.c_end && !issue_qk(j + 1, b + 1)) break;
         }
     }
@@ -532,7 +562,7 @@ constexpr int SPLIT_HELP0 = SPLIT_STATE + SPLIT_P, SPLIT_HELP = 16 - SPLIT_HELP0
 __device__ __forceinline__ float k_weight(const Smem& sm, const TcParams& p, const Item& it, int c,
                                           int st, int r) {
     const bool valid = (int64_t)c * C + r < it.len;
-    return valid ? ex2f(sm.gtot[st] - sm.gc[st][r]) * p.k_scale : 0.f;
+    return valid ? ex2f(sm.gbase[st] - sm.gc[st][r]) * p.k_scale : 0.f;
 }
 
 // Row r of the state into the MN-major swizzled tile read by Q S: the bf16 high half is
@@ -595,7 +625,7 @@ __device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint
         for (int jj = 0; jj < 2 * n; ++jj, ++j) {
             const int st = j & 1;
             const bool pass_b = jj >= n;
-            const int c = it.c_begin + (pass_b ? jj - n : jj);
+            const int c = pass_b ? it.c_begin + (jj - n) : it.c_end - 1 - jj;
             // the stage's gate slot is read before this group's split share is released: after
             // that the stage may be refilled
             float cr = 0.f;
@@ -721,6 +751,7 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
     const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
     float S[D];
     int j = 0, b = 0, it_n = 0;
+    int dsn = 0;   // dS results taken from the MMA so far (phases of ds_full)
     bool ok = true;
     while (ok) {
         const int slot = it_n % ITEM_DEPTH;
@@ -731,40 +762,34 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
             mbar_arrive(&sm.item_empty[slot]);
             break;
         }
-        // ---- pass A: span aggregate from zero.  The split of chunk c + 1 is done while the
-        // dS MMA of chunk c runs (its tile is already resident: the producer runs two stages
-        // ahead, and that stage was released by the MMA of chunk c - 1).  One split and one
-        // fold site each, so that the group's code stays small for the instruction cache.
+        // ---- pass A: the span's aggregate Agg = sum over its keys of (decay to the span's end)
+        // k^T v is accumulated by the dS MMAs over the span's chunks, which arrive last to
+        // first; this group splits its share of w K and sums the span's log2-decay L, then
+        // reads Agg once.
+        const int n = it.c_end - it.c_begin;
 #pragma unroll
         for (int i = 0; i < D; ++i) S[i] = 0.f;
-        float L = 0.f;                  // span log2-decay
-        float tot0 = 0.f, tot1 = 0.f;   // chunk log2-decay by stage parity, read at the split
-        const int n = it.c_end - it.c_begin;
+        float L = 0.f;
 #pragma unroll 1
-        for (int i = 0; i <= n; ++i) {
-            if (i < n) {   // split of chunk i
-                const int st = (j + i) & 1;
-                if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
-                const float t = sm.gtot[st];
-                if (st) tot1 = t; else tot0 = t;
-                split_k_chunks<0, SPLIT_STATE>(sm.k[st], sm.q[st], r,
-                                             k_weight(sm, p, it, it.c_begin + i, st, r));
-                fence_proxy_async_smem();
-                mbar_arrive(&sm.k_ready[st]);
-            }
-            if (i > 0) {   // fold of chunk i - 1
-                const int jf = j + i - 1;
-                if (!gw.wait(&sm.ds_full, jf & 1)) { ok = false; break; }
-                const float tot = (jf & 1) ? tot1 : tot0;
-                tc_fence_after();
-                fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
-                tc_fence_before();
-                mbar_arrive(&sm.ds_free);
-                L += tot;
-            }
+        for (int i = 0; i < n; ++i) {
+            const int st = (j + i) & 1;
+            if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
+            L += sm.gtot[st];
+            split_k_chunks<0, SPLIT_STATE>(sm.k[st], sm.q[st], r,
+                                           k_weight(sm, p, it, it.c_end - 1 - i, st, r));
+            fence_proxy_async_smem();
+            mbar_arrive(&sm.k_ready[st]);
         }
         j += n;
         if (!ok) break;
+        if (n > 0) {
+            if (!gw.wait(&sm.ds_full, dsn & 1)) break;
+            tc_fence_after();
+            fold_ds(tmem + lane_base + TM_DS, S, 0.f);   // S = Agg
+            tc_fence_before();
+            mbar_arrive(&sm.ds_free);
+            ++dsn;
+        }
         // ---- look-back: entry state E of the span; publish exp(L) E + Agg
         const int64_t chain = (int64_t)it.u * p.H + it.h;
         const float* esrc = nullptr;
@@ -849,11 +874,12 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
                                          k_weight(sm, p, it, it.c_begin + i, st, r));
             fence_proxy_async_smem();
             mbar_arrive(&sm.k_ready[st]);
-            if (!gw.wait(&sm.ds_full, (j + i) & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.ds_full, dsn & 1)) { ok = false; break; }
             tc_fence_after();
             fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
+            ++dsn;
         }
         j += n;
         b += n;
@@ -886,7 +912,7 @@ __device__ void split_helper(Smem& sm, const TcParams& p, int warp, int lane) {
         const int n_ch = it.c_end - it.c_begin;
         for (int jj = 0; jj < 2 * n_ch; ++jj, ++j) {
             const int st = j & 1;
-            const int c = it.c_begin + (jj < n_ch ? jj : jj - n_ch);
+            const int c = jj < n_ch ? it.c_end - 1 - jj : it.c_begin + (jj - n_ch);
             if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
             if (jj >= n_ch) {   // pass B: the Q slot is free once both Q S MMAs are done
                 if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
