@@ -25,6 +25,12 @@ def test_several_spans_per_chain(N):
     run_dense(1, N, 4, 128, 128, BF, seed=N + 1, state=True)
 
 
+def test_single_long_chain():
+    # one head of 40000 tokens (313 chunks): the span-size model cuts a lone chain into many
+    # short spans, so the look-back runs as a long serial chain of flags
+    run_dense(1, 40000, 1, 128, 128, BF, seed=41, state=True)
+
+
 def test_batch_of_sequences():
     run_dense(3, 700, 2, 128, 128, BF, seed=31, state=True)
 
