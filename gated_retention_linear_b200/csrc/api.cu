@@ -132,7 +132,7 @@ gret_status_t gret_decode_step(const void* q, const void* k, const void* v, cons
     if (!dim_ok(d_k) || !dim_ok(d_v) || B < 0 || H < 0) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
     if ((int64_t)B * H == 0) return GRET_OK;
-    if ((int64_t)B * H > 0x7fffffffLL) return GRET_ERR_INVALID_ARG;
+    if ((int64_t)B * H > 0x3fffffffLL) return GRET_ERR_INVALID_ARG;   // 2 CTAs per (b, h)
     if (!q || !k || !v || !g || !state || !o) return GRET_ERR_INVALID_ARG;
     if (!aligned16(state)) return GRET_ERR_ALIGNMENT;
     cudaError_t e = launch_decode(q, k, v, g, tau, k_scale, dtype == GRET_BF16, B, H, d_k, d_v,

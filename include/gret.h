@@ -145,7 +145,8 @@ gret_status_t gret_workspace_status(const void* workspace, gret_stream_t stream)
  *   q, k   [B, H, d_k] contiguous, `dtype`;   v [B, H, d_v];   g fp32 [B, H] gate logits.
  *   state  fp32 [B, H, d_k, d_v], updated IN PLACE; 16-byte aligned.
  *   o      [B, H, d_v] in `dtype`; must not overlap state or inputs.
- * d_k, d_v in {64, 128}.  Memory-bound: the state is read and written once.
+ * d_k, d_v in {64, 128}; B * H at most 2^30 - 1 (GRET_ERR_INVALID_ARG beyond).  Memory-bound:
+ * the state is read and written once.
  */
 gret_status_t gret_decode_step(const void* q, const void* k, const void* v, const float* g,
                                float tau, float k_scale, gret_dtype_t dtype, int B, int H,
