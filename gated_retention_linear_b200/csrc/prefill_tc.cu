@@ -1179,8 +1179,17 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
         !make_map(&to, a.o, a.ost, a.osh, a.osb, ntok, a.H, B, p.o_pos_tok, p.o_pos_head, p.o_pos_b))
         return GRET_ERR_UNSUPPORTED;
 
+    // TMA coordinates are 32-bit: token coordinates (and the tile past the last one) must fit
+    if (a.N > (int64_t)0x7FFFFF00) return GRET_ERR_UNSUPPORTED;
     uint64_t total_dense = varlen ? 0 : (uint64_t)units * p.spans_per_unit * a.H;
     if (total_dense > 0xFFFFFFF0ull) return GRET_ERR_UNSUPPORTED;
+    if (varlen) {
+        // tickets are counted in 32 bits on the device: a sequence of len tokens has at most
+        // len / (C G) + 1 spans, so N / (C G) + n_seqs + 1 bounds the total without reading
+        // cu_seqlens
+        const uint64_t span_bound = (uint64_t)(a.N / ((int64_t)C * G)) + (uint64_t)units + 1;
+        if (span_bound * (uint64_t)a.H > 0xFFFFFFF0ull) return GRET_ERR_UNSUPPORTED;
+    }
     if (cudaMemsetAsync(ws, 0, L.prefix, a.stream) != cudaSuccess) return GRET_ERR_CUDA;
     if (varlen) {
         plan_kernel<<<1, 1024, 0, a.stream>>>(a.cu_seqlens, units, G, p.prefix);

@@ -93,7 +93,9 @@ size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int
  *            aligned, owned by the caller; its contents need no initialisation and are
  *            garbage afterwards.  Concurrent calls need separate workspaces.
  * Alignment: for the tensor-core path, q/k/v/o base pointers must be 16-byte aligned and every
- * stride (times 2 bytes) a multiple of 16 bytes; otherwise GRET_ERR_ALIGNMENT.
+ * stride (times 2 bytes) a multiple of 16 bytes; otherwise GRET_ERR_ALIGNMENT.  Its tile
+ * copies take 32-bit token coordinates: N (tokens per sequence, or the packed total) above
+ * 2^31 - 256 returns GRET_ERR_UNSUPPORTED.
  * A bounded wait between thread blocks that gives up sets an error word in the workspace;
  * read it with gret_workspace_status() after the stream has synchronised.
  */
