@@ -152,20 +152,30 @@ def rank_seed(base, rank):
     return base + 1000 * rank
 
 
+def kernel_code_digest(path):
+    """sha256 (16 hex digits) of a CUDA source with its comments and whitespace removed, so that
+    a measurement taken on the code stays valid across comment-only edits."""
+    import hashlib
+    import re
+    src = open(path).read()
+    src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", " ", src)
+    src = re.sub(r"\s+", " ", src).strip()
+    return hashlib.sha256(src.encode()).hexdigest()[:16]
+
+
 def prefill_traffic_from_profile():
     """DRAM bytes per launch of the prefill kernel from the committed ncu summary, if that
-    summary was taken on the current kernel source (else None)."""
-    import hashlib
+    summary was taken on the current kernel code (else None)."""
     src = os.path.join(ROOT, "gated_retention_linear_b200", "csrc", "prefill_tc.cu")
     summ = os.path.join(ROOT, "profiles", "prefill_tc_kernel_32k.txt")
     try:
-        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
         kv = {}
         for line in open(summ):
             if ":" in line:
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-        if kv.get("kernel_source_sha256_16") == sha:
+        if kv.get("kernel_code_sha256_16") == kernel_code_digest(src):
             return int(float(kv["dram_bytes_per_launch"]))
     except Exception:
         pass

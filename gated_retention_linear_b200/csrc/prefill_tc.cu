@@ -21,14 +21,18 @@
 //
 // Parallelism across a sequence.  The chunk chain of one (sequence, head) is sequential, and
 // one 3B-shaped layer has only 24 chains for 148 SMs.  Each chain is therefore cut into spans
-// of G chunks.  A persistent CTA takes spans from an atomic ticket in chain order and runs:
-//   pass A: read K, V, g of the span and fold them into the span's aggregate state
-//           Agg = sum over chunks (decay to the span end) of dS        (dS MMAs only)
+// of G chunks (G chosen on the host from a wave model, see span_chunks).  A persistent CTA
+// takes spans from an atomic ticket in chain order and runs:
+//   pass A: read K, V, g of the span's chunks, last to first, each key weighted by its decay
+//           to the end of the span, so that every dS MMA of the span accumulates into one
+//           tensor-memory result: the span's aggregate Agg = sum over its keys of
+//           (decay to the span end) k^T v;
 //   look-back: wait for the inclusive state of span s-1 of the same chain (a bounded spin on a
 //           flag in the workspace), entry E = that state (or state_in for s = 0), and publish
 //           the inclusive state exp(L_span) E + Agg for span s+1;
 //   pass B: the full chunk pipeline above from E, writing O.
-// The K and V of a span are read from HBM by pass A and again by pass B shortly after, from L2.
+// Pass B reads the span's K and V a second time: from L2 when spans are short, from DRAM when
+// the CTAs' spans together outgrow L2 (longer spans still win: fewer look-backs, fuller waves).
 // Inclusive states live in a two-slot ring per chain: span s+2 can only overwrite the slot of
 // span s after span s+1 has consumed it, because it needs span s+1's own inclusive state first.
 // Tickets are taken by running CTAs in increasing order and every span depends only on a smaller
@@ -38,11 +42,13 @@
 //   warp 0      TMA producer (lane 0): K, V (and Q in pass B) tiles, two pipeline stages;
 //               the whole warp scans the chunk's gate logits into the stage's gate slot
 //   warp 1      tcgen05 MMA issuer (one thread); owns the 512-column TMEM allocation
-//   warps 2-3   their share of the w K split (5 of the 16 chunks of every row)
-//   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16 halves) and the
-//               output epilogue O + exp(c_t) OX -> bf16 -> global
-//   warps 8-11  "state group": w K split into halves, the fp32 state (one row per thread), the
-//               look-back, and the bf16 halves of the state that Q S_prev reads
+//   warps 2-3   their share of the w K split (3 of the 16 chunks of two rows each)
+//   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16 halves), its share
+//               of the w K split (6 chunks of its row), and the output epilogue
+//               O + exp(c_t) OX -> bf16 -> TMA store through the state buffer
+//   warps 8-11  "state group": its share of the w K split (7 chunks of its row), the fp32
+//               state (one row per thread), the look-back, and the bf16 halves of the state
+//               that Q S_prev reads
 // Registers: launched at 168 per thread (384 x 168 = 64512); the first warpgroup drops to 88,
 // the P group to 136 and the state group (128 fp32 state values per thread) rises to 256:
 // 128 x (88 + 136 + 256) = 61440 <= 64512, and each SM sub-partition (one warp of each group)
