@@ -41,6 +41,14 @@ WORKLOAD = ("gRet chunkwise prefill, batch 1, H=24, N=32768, d_k=d_v=128, bf16 q
             "~N(0,1)/sqrt(128), g~N(2,1), tau=16, fp32 state")
 
 
+def bench_config(world):
+    """The workload description printed by both arms."""
+    return {"workload": WORKLOAD, "tokens_per_rank": B * N, "heads": H, "d": D,
+            "parallelism": "independent sequence per GPU" if world > 1 else "1 GPU",
+            "l2": "inputs and outputs (808 MB per step) larger than L2 (126 MB); "
+                  "L2 not flushed"}
+
+
 def measured_peaks():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -360,10 +368,7 @@ def run_gpu(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_per_step,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD, "tokens_per_rank": B * N, "heads": H, "d": D,
-                   "parallelism": "independent sequence per GPU" if world > 1 else "1 GPU",
-                   "l2": "inputs and outputs (808 MB per step) larger than L2 (126 MB); "
-                         "L2 not flushed"},
+        "config": bench_config(world),
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "traffic": prefill_traffic_from_profile(),
@@ -484,7 +489,7 @@ def run_reference(args):
         "n_gpus": int(os.environ.get("WORLD_SIZE", "1")), "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD},
+        "config": bench_config(int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": value, "unit": "Mtok/s", "cores": oracle.threads(),
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "Mtok/s", "h2d_bytes_per_step": 0,
