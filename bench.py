@@ -291,6 +291,11 @@ def run_gpu(args):
     if not args.no_epilogue:
         epi = run_varlen_epilogue(args, rank, world, stream, hbm_peak)
 
+    # ---------------- one mixer layer: projection GEMM -> prefill -> GroupNorm * gate
+    lay = None
+    if not args.no_layer:
+        lay = run_layer(args, rank, world, stream, hbm_peak)
+
     clk = clocks.stop()
 
     # ---------------- end to end: host buffers through the C ABI.  Every step uploads its
@@ -374,7 +379,7 @@ def run_gpu(args):
                      "traffic": prefill_traffic_from_profile(),
                      "kernel": "prefill_tc_kernel", "launch_ms": launch_ms,
                      "algorithmic_bytes_per_launch": alg_bytes},
-        "decode": dec, "varlen_epilogue": epi, "e2e": e2e, "clocks": clk,
+        "decode": dec, "varlen_epilogue": epi, "layer": lay, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }
@@ -440,6 +445,76 @@ def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
             "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
                          "frac": ach / tpeak, "peak_kind": tkind + " burst", "traffic": None,
                          "kernel": "gn_gate_kernel", "algorithmic_flops_per_launch": flops}}
+
+
+def run_layer(args, rank, world, stream, hbm_peak):
+    """One gated-retention mixer layer at the 3B shapes (32768 tokens of one sequence, hidden
+    3072, 24 heads of 128): the [q | k | v | g] = x W projection (one tcgen05 GEMM), the
+    chunkwise prefill (k scaled by d^-1/2) and the GroupNorm * swish(x W_G) output gate, with
+    events between the three launches on the launching stream."""
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+    c = SI.LAYER_32K
+    T, Dm, Hh, d = c["T"], c["D"], c["H"], c["dk"]
+    F = 3 * Hh * d + Hh
+    li = SI.layer_inputs(T, Dm, Hh, d, seed=rank_seed(c["seed"], rank), device="cuda",
+                         pad=(-F) % 8, pad_value=0.0)
+    x, w, w_g = li["x"], li["w_qkvg"], li["w_g"]
+    cu_d = torch.tensor([0, T], dtype=torch.int32, device="cuda")
+    o = torch.empty((T, Hh, d), dtype=torch.bfloat16, device="cuda")
+    y = torch.empty((T, Hh * d), dtype=torch.bfloat16, device="cuda")
+    ws = torch.empty(G.gret_prefill_workspace_size(torch.bfloat16, T, 1, Hh, d, d, 0),
+                     dtype=torch.uint8, device="cuda")
+
+    def step(ev=None):
+        q, k, v, g = G.gret_qkvg_projection(x, w, Hh, d)
+        if ev is not None:
+            ev[1].record(stream)
+        G.gret_prefill_chunkwise(q, k, v, g, k_scale=d ** -0.5, cu_seqlens=cu_d, o=o,
+                                 workspace=ws)
+        if ev is not None:
+            ev[2].record(stream)
+        G.gret_groupnorm_gate(o.view(T, Hh * d), x, w_g, Hh, y=y)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 5))
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(n)]
+    barrier(world)
+    for i in range(n):
+        evs[i][0].record(stream)
+        step(evs[i])
+        evs[i][3].record(stream)
+    torch.cuda.synchronize()
+    tot_ms = max_over_ranks(statistics.mean(e[0].elapsed_time(e[3]) for e in evs), world)
+    proj_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    pre_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in evs)
+    gn_ms = statistics.mean(e[2].elapsed_time(e[3]) for e in evs)
+    if G.gret_workspace_status(ws) != 0:
+        raise RuntimeError("layer prefill reported a timed-out wait")
+    tpeak, tkind = measured_tensor_peak()
+    proj_flops = 2.0 * T * Dm * F
+    gn_flops = 2.0 * T * Dm * Hh * d
+    pre_bytes = T * Hh * BYTES_PER_TOKEN_HEAD
+    ach = proj_flops / (proj_ms * 1e-3) / 1e12
+    return {"value": T * world / (tot_ms * 1e-3) / 1e6, "unit": "Mtok/s", "tokens": T,
+            "hidden": Dm, "heads": Hh, "ms_per_step": tot_ms, "projection_ms": proj_ms,
+            "prefill_ms": pre_ms, "gate_ms": gn_ms, "steps": n, "gpu_launches_per_step": 4,
+            "l2": "x (201 MB) and q, k, v (604 MB) larger than L2 (126 MB); not flushed",
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
+                         "frac": ach / tpeak, "peak_kind": tkind + " burst", "traffic": None,
+                         "kernel": "qkvg_projection (gn_gate_kernel<EPI_PROJECTION>)",
+                         "algorithmic_flops_per_launch": proj_flops},
+            "prefill_roofline": {"bound": "hbm", "achieved": pre_bytes / (pre_ms * 1e-3) / 1e9,
+                                 "peak": hbm_peak, "unit": "GB/s",
+                                 "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / hbm_peak},
+            "gate_roofline": {"bound": "tensor",
+                              "achieved": gn_flops / (gn_ms * 1e-3) / 1e12, "peak": tpeak,
+                              "unit": "TFLOP/s",
+                              "frac": gn_flops / (gn_ms * 1e-3) / 1e12 / tpeak}}
 
 
 def cpu_baseline(q, k, v, g, n_tokens, min_seconds=8.0, max_reps=8):
@@ -508,6 +583,7 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-epilogue", action="store_true")
+    ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--varlen-max-len", type=int, default=65536,
                     help="longest sequence of the varlen + epilogue leg (a smaller value gives "
                          "a small case for profiling)")

@@ -50,6 +50,9 @@ _lib.gret_decode_step.restype = _i32
 _lib.gret_groupnorm_gate.argtypes = [_vp, _vp, _vp, _vp, _vp, _f32, _i64, _i32, _i32, _i32, _vp,
                                      _vp]
 _lib.gret_groupnorm_gate.restype = _i32
+_lib.gret_qkvg_projection.argtypes = [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
+                                      _vp]
+_lib.gret_qkvg_projection.restype = _i32
 
 
 class GretError(RuntimeError):
@@ -217,3 +220,43 @@ def gret_groupnorm_gate(o, x, w_g, H, gn_weight=None, gn_bias=None, eps=1e-5, y=
         _ptr(o), _ptr(x), _ptr(w_g), _ptr(gn_weight), _ptr(gn_bias), eps, T, H, F // H, D,
         _ptr(y), _stream(stream)))
     return y
+
+
+def gret_qkvg_projection(x, w, H, d=128, stream=None):
+    """[q | k | v | g] = x @ w in one GEMM: x [T, D] bf16, w [D, >= 3*H*d + H] bf16 (W_Q, W_K,
+    W_V, W_gamma side by side; extra columns, if any, are padding).  Returns q, k, v bf16
+    [T, H, d] and the gate logits g fp32 [T, H]."""
+    T, D = x.shape
+    for t in (x, w):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("x and w must be bfloat16 with contiguous rows")
+    if x.stride(0) != D:
+        raise ValueError("x must be contiguous")
+    q = torch.empty((T, H, d), dtype=torch.bfloat16, device=x.device)
+    k = torch.empty_like(q)
+    v = torch.empty_like(q)
+    g = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    _check("gret_qkvg_projection", _lib.gret_qkvg_projection(
+        _ptr(x), _ptr(w), w.stride(0), T, H, d, D, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+        _stream(stream)))
+    return q, k, v, g
+
+
+def gret_layer_forward(x, w_qkvg, w_g, H, d=128, cu_seqlens=None, state_in=None, tau=16.0,
+                       k_scale=None, gn_weight=None, gn_bias=None, eps=1e-5, stream=None):
+    """One gated-retention mixer layer through the library's kernels: the q / k / v / gate-logit
+    projection of x, the chunkwise prefill (k scaled by d^-1/2 unless k_scale is given), and the
+    per-head GroupNorm * swish(x @ w_g) output gate.  x [T, D] bf16 is one packed batch
+    (cu_seqlens marks its sequences; None means one sequence).  Returns y [T, H*d] bf16 and the
+    final fp32 states [n_seqs, H, d, d]."""
+    T = x.shape[0]
+    q, k, v, g = gret_qkvg_projection(x, w_qkvg, H, d, stream=stream)
+    if cu_seqlens is None:
+        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=x.device)
+    o, state = gret_prefill_chunkwise(q, k, v, g, tau=tau,
+                                      k_scale=d ** -0.5 if k_scale is None else k_scale,
+                                      cu_seqlens=cu_seqlens, state_in=state_in, state_out=True,
+                                      stream=stream)
+    y = gret_groupnorm_gate(o.view(T, H * d), x, w_g, H, gn_weight=gn_weight, gn_bias=gn_bias,
+                            eps=eps, stream=stream)
+    return y, state

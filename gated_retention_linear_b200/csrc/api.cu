@@ -155,4 +155,19 @@ gret_status_t gret_groupnorm_gate(const void* o, const void* x, const void* w_g,
                           (cudaStream_t)stream);
 }
 
+gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, int64_t T, int H,
+                                   int d, int D, void* q, void* k, void* v, float* g,
+                                   gret_stream_t stream) {
+    if (T < 0 || H < 1 || D < 1 || d < 1) return GRET_ERR_INVALID_ARG;
+    const int64_t F = 3 * (int64_t)H * d + H;
+    if (ldw < F) return GRET_ERR_INVALID_ARG;
+    if (d != 128 || H > 128 || D % 64 != 0) return GRET_ERR_UNSUPPORTED;
+    if (T == 0) return GRET_OK;
+    if (!x || !w || !q || !k || !v || !g) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(x) || !aligned16(w) || !aligned16(q) || !aligned16(k) || !aligned16(v) ||
+        (reinterpret_cast<uintptr_t>(g) & 3u) != 0 || ldw % 8 != 0)
+        return GRET_ERR_ALIGNMENT;
+    return launch_qkvg_projection(x, w, ldw, T, H, D, q, k, v, g, (cudaStream_t)stream);
+}
+
 }  // extern "C"

@@ -14,6 +14,10 @@
 // under the MMAs of the next.  The epilogue is fused: GroupNorm statistics of the O row, swish
 // of the accumulator, the product, bf16 out; z never goes to memory.
 //
+// The same GEMM, with a plain epilogue, is the layer's input projection: X W_qkvg with
+// W_qkvg = [W_Q | W_K | W_V | W_gamma] gives q, k, v (bf16, [T, H, d] each) and the gate logits
+// g (fp32, [T, H]) in one pass over X (qkvg_projection below).
+//
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (owns TMEM), warps 2-3 idle,
 // warps 4-7 epilogue for the first head of a tile, warps 8-11 for the second.  Tiles are
 // assigned round-robin (tile = blockIdx.x + i * gridDim.x), M-block major, so the CTAs working
@@ -53,9 +57,15 @@ struct GParams {
     __nv_bfloat16* y;
     float eps;
     int64_t T;
-    int F, D;          // F = H * 128
+    int F, D;          // F: output columns (GroupNorm gate: H * 128; projection: 3 H 128 + H)
     int m_blocks, n_blocks, n_tiles;
+    // projection outputs
+    __nv_bfloat16* qkv[3];   // q, k, v: [T, H, 128] bf16
+    float* g;                // [T, H] fp32
+    int H;
 };
+
+enum EpilogueMode { EPI_GN_GATE = 0, EPI_PROJECTION = 1 };
 
 __device__ __forceinline__ bool wait_bar(GSmem& sm, uint64_t* bar, uint32_t parity) {
     if (mbar_wait(bar, parity, &sm.abort, WAIT_NS)) return true;
@@ -118,7 +128,47 @@ __device__ void mma_issuer(GSmem& sm, const GParams& p, uint32_t tmem) {
     mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
 }
 
+// Projection epilogue of one thread: token row t, the 128 accumulator columns starting at
+// col0 (one head of q, k or v, or the gate logits and padding).
+__device__ __forceinline__ void store_projection(const GParams& p, uint32_t taddr, int64_t t,
+                                                 int col0, bool valid) {
+    const int hd = p.H * 128;
+    if (col0 < 3 * hd) {
+        const int which = col0 / hd;
+        __nv_bfloat16* base = which == 0 ? p.qkv[0] : (which == 1 ? p.qkv[1] : p.qkv[2]);
+        __nv_bfloat16* dst = base + t * hd + (col0 - which * hd);
+#pragma unroll 1
+        for (int jc = 0; jc < 4; ++jc) {
+            float z[32];
+            tmem_ld32(taddr + jc * 32, z);
+            tmem_ld_wait();
+            if (valid) {
+                uint4* d4 = reinterpret_cast<uint4*>(dst + jc * 32);
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4)
+                    d4[v4] = make_uint4(pack_bf16x2(z[8 * v4 + 0], z[8 * v4 + 1]),
+                                        pack_bf16x2(z[8 * v4 + 2], z[8 * v4 + 3]),
+                                        pack_bf16x2(z[8 * v4 + 4], z[8 * v4 + 5]),
+                                        pack_bf16x2(z[8 * v4 + 6], z[8 * v4 + 7]));
+            }
+        }
+    } else if (col0 == 3 * hd) {   // the H gate-logit columns (H <= 128), then padding
+#pragma unroll 1
+        for (int jc = 0; jc * 32 < p.H; ++jc) {
+            float z[32];
+            tmem_ld32(taddr + jc * 32, z);
+            tmem_ld_wait();
+            if (valid) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i)
+                    if (jc * 32 + i < p.H) p.g[t * p.H + jc * 32 + i] = z[i];
+            }
+        }
+    }
+}
+
 // One epilogue thread: token row r of the tile, one head (128 columns) of it.
+template <int MODE>
 __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, int lane) {
     const int q = warp & 3, r = q * 32 + lane;
     const int half = (warp - 4) >> 2;                    // which head of the 256-column tile
@@ -129,10 +179,21 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
         const int mb = tile / p.n_blocks, nb = tile % p.n_blocks;
         const int64_t t = (int64_t)mb * BM + r;
         const int col0 = nb * BN + half * 128;
+        const bool valid = t < p.T;
+        if (MODE == EPI_PROJECTION) {
+            if (!mbar_wait(&sm.acc_full[buf], (t_local >> 1) & 1, &sm.abort, WAIT_NS)) {
+                atomicExch(&sm.abort, 1u);
+                return;
+            }
+            tc_fence_after();
+            store_projection(p, tmem + lane_base + buf * BN + half * 128, t, col0, valid);
+            tc_fence_before();
+            mbar_arrive(&sm.acc_empty[buf]);
+            continue;
+        }
         // GroupNorm statistics of this head's slice of O, computed while the MMAs run; the row
         // (256 bytes) is read again per 32 columns below, from L1
         float mean = 0.f, inv = 0.f;
-        const bool valid = t < p.T;
         const uint4* src = reinterpret_cast<const uint4*>(p.o + t * p.F + col0);
         if (valid) {
             float s = 0.f, s2 = 0.f;
@@ -209,6 +270,7 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
     }
 }
 
+template <int MODE>
 __global__ void __launch_bounds__(NTHREADS, 1)
     gn_gate_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                    const GParams p) {
@@ -246,7 +308,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     } else if (warp == 1) {
         if (lane == 0) mma_issuer(sm, p, tmem);
     } else if (warp >= 4) {
-        epilogue(sm, p, tmem, warp, lane);
+        epilogue<MODE>(sm, p, tmem, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -267,6 +329,19 @@ int sm_count() {
         cached[dev] = n > 0 ? n : 148;
     }
     return cached[dev];
+}
+
+template <int MODE>
+gret_status_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const GParams& p,
+                          cudaStream_t stream) {
+    const size_t smem = sizeof(GSmem);
+    if (cudaFuncSetAttribute(gn_gate_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem) != cudaSuccess)
+        return GRET_ERR_CUDA;
+    int grid = sm_count();
+    if (p.n_tiles < grid) grid = p.n_tiles;
+    gn_gate_kernel<MODE><<<grid, NTHREADS, smem, stream>>>(tx, tw, p);
+    return cudaGetLastError() == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
 }  // namespace
@@ -290,7 +365,7 @@ gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g, cons
         uint32_t box[2] = {64, BK};
         if (!make_bf16_map(&tw, w_g, 2, dims, strides, box)) return GRET_ERR_UNSUPPORTED;
     }
-    GParams p;
+    GParams p = {};
     p.o = (const __nv_bfloat16*)o;
     p.gn_w = gn_weight;
     p.gn_b = gn_bias;
@@ -302,14 +377,42 @@ gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g, cons
     p.m_blocks = (int)((T + BM - 1) / BM);
     p.n_blocks = F / BN;
     p.n_tiles = p.m_blocks * p.n_blocks;
-    const size_t smem = sizeof(GSmem);
-    if (cudaFuncSetAttribute(gn_gate_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)smem) != cudaSuccess)
-        return GRET_ERR_CUDA;
-    int grid = sm_count();
-    if (p.n_tiles < grid) grid = p.n_tiles;
-    gn_gate_kernel<<<grid, NTHREADS, smem, stream>>>(tx, tw, p);
-    return cudaGetLastError() == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+    return launch_gemm<EPI_GN_GATE>(tx, tw, p, stream);
+}
+
+gret_status_t launch_qkvg_projection(const void* x, const void* w, int64_t ldw, int64_t T, int H,
+                                     int D, void* q, void* k, void* v, float* g,
+                                     cudaStream_t stream) {
+    const int F = 3 * H * 128 + H;
+    if (H < 1 || H > 128 || D % BK != 0) return GRET_ERR_UNSUPPORTED;
+    if (T > ((int64_t)1 << 31) - BM) return GRET_ERR_UNSUPPORTED;
+    CUtensorMap tx, tw;
+    {
+        uint64_t dims[2] = {(uint64_t)D, (uint64_t)T};
+        uint64_t strides[1] = {(uint64_t)D * 2};
+        uint32_t box[2] = {BK, BM};
+        if (!make_bf16_map(&tx, x, 2, dims, strides, box)) return GRET_ERR_UNSUPPORTED;
+    }
+    {
+        // columns past F (the last tile's padding) are read as zeros
+        uint64_t dims[2] = {(uint64_t)F, (uint64_t)D};
+        uint64_t strides[1] = {(uint64_t)ldw * 2};
+        uint32_t box[2] = {64, BK};
+        if (!make_bf16_map(&tw, w, 2, dims, strides, box)) return GRET_ERR_UNSUPPORTED;
+    }
+    GParams p = {};
+    p.T = T;
+    p.F = F;
+    p.D = D;
+    p.H = H;
+    p.qkv[0] = (__nv_bfloat16*)q;
+    p.qkv[1] = (__nv_bfloat16*)k;
+    p.qkv[2] = (__nv_bfloat16*)v;
+    p.g = g;
+    p.m_blocks = (int)((T + BM - 1) / BM);
+    p.n_blocks = (F + BN - 1) / BN;
+    p.n_tiles = p.m_blocks * p.n_blocks;
+    return launch_gemm<EPI_PROJECTION>(tx, tw, p, stream);
 }
 
 }  // namespace gret

@@ -169,6 +169,24 @@ gret_status_t gret_groupnorm_gate(const void* o, const void* x, const void* w_g,
                                   int64_t T, int H, int d_v, int D, void* y,
                                   gret_stream_t stream);
 
+/*
+ * The layer's input projection in one GEMM ("路线二：Multi-Head Gated Retention": the per-head
+ * gate comes from a learned projection of the layer input, next to the query, key and value
+ * projections):
+ *   [q | k | v | g]_t = X_t W_qkvg ,  W_qkvg = [W_Q | W_K | W_V | W_gamma]
+ *   x    bf16 [T, D] row-major.
+ *   w    bf16 [D, F] with F = 3 H d + H columns (H d each for W_Q, W_K, W_V, then H for
+ *        W_gamma), row stride ldw >= F elements (a multiple of 8: rows start 16-byte aligned).
+ *   q, k, v  bf16 [T, H, d] (token-major, contiguous), ready for gret_prefill_chunkwise.
+ *   g    fp32 [T, H] gate logits (gamma = sigmoid(g)^(1/tau) is taken by the prefill).
+ * fp32 accumulation; q, k, v rounded to bf16 once.  Requires d == 128, 1 <= H <= 128, D a
+ * positive multiple of 64; x, w, q, k, v 16-byte aligned, g 4-byte aligned
+ * (GRET_ERR_ALIGNMENT otherwise).  Outputs must not overlap the inputs or each other.
+ */
+gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, int64_t T, int H,
+                                   int d, int D, void* q, void* k, void* v, float* g,
+                                   gret_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -153,3 +153,43 @@ def groupnorm_gate(o, x, w_g, H, gn_weight=None, gn_bias=None, eps=1e-5, rows=No
 
 def log_gamma(g, tau=16.0):
     return lib().oracle_log_gamma(float(g), float(tau))
+
+
+def qkvg_projection(x, w, H, d=128):
+    """The layer's input projection, [q | k | v | g] = x @ w, in fp64 ("路线二：Multi-Head Gated
+    Retention": the gate is a learned projection of the layer input, beside the query, key and
+    value projections).  x [T, D]; w [D, >= 3 H d + H] (W_Q, W_K, W_V, W_gamma side by side).
+    A library matmul is the whole step; the blocks are then read off by column.
+    Returns q, k, v [T, H, d] and g [T, H]."""
+    x, w = _d(x), _d(w)
+    T = x.shape[0]
+    hd = H * d
+    z = x @ w[:, :3 * hd + H]
+    q = z[:, 0:hd].reshape(T, H, d)
+    k = z[:, hd:2 * hd].reshape(T, H, d)
+    v = z[:, 2 * hd:3 * hd].reshape(T, H, d)
+    g = z[:, 3 * hd:3 * hd + H]
+    return q, k, v, g
+
+
+def _round_bf16(a):
+    """Round fp64 values to bfloat16 (round to nearest even), back in fp64."""
+    import torch
+    return torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
+
+
+def layer_forward(x, w_qkvg, w_g, H, d=128, cu_seqlens=None, state_in=None, tau=16.0,
+                  k_scale=None, gn_weight=None, gn_bias=None, eps=1e-5, rows=None, with_o=False):
+    """One gated-retention mixer layer from the oracle's own steps: the projection (q, k, v
+    stored in bf16, the layer's dtype; g kept as computed), the recurrence, and the GroupNorm *
+    swish(x W_G) gate on the retention output rounded to bf16 (as the layer stores it).
+    Returns y [T or len(rows), H d] and the final states (and the bf16-rounded retention
+    output o [T, H d] when with_o is set)."""
+    q, k, v, g = qkvg_projection(x, w_qkvg, H, d)
+    q, k, v = _round_bf16(q), _round_bf16(k), _round_bf16(v)
+    o, s = gret_recurrent(q, k, v, g, tau=tau, k_scale=d ** -0.5 if k_scale is None else k_scale,
+                          cu_seqlens=cu_seqlens, state_in=state_in)
+    T = o.shape[0]
+    o = _round_bf16(o).reshape(T, H * d)
+    y = groupnorm_gate(o, x, w_g, H, gn_weight=gn_weight, gn_bias=gn_bias, eps=eps, rows=rows)
+    return (y, s, o) if with_o else (y, s)

@@ -12,12 +12,16 @@ Recipes (the 3B shapes of the YOCO pages: 24 heads of width 128, hidden 3072):
   * gate logits g ~ N(mean, std), fp32  (N(2, 1) for the dense configs, N(0, 2) for varlen)
   * packed varlen lengths ~ U[lo, hi] (torch.randint, inclusive bounds)
   * epilogue: x ~ N(0, 1), w_g ~ N(0, 0.02), bf16
+  * layer: x ~ N(0, 1) with a constant column x[:, 0] = 1; W_Q, W_K, W_V ~ N(0, 1/D);
+    W_gamma ~ N(0, 0.05^2 / D) plus a per-head bias ~ N(2, 1) on the constant row, so the
+    gate logits sit near N(2, 1) per head; w_g ~ N(0, 0.02); bf16
 """
 import math
 
 import torch
 
-_TAGS = {"q": 1, "k": 2, "v": 3, "g": 4, "s": 5, "x": 6, "w": 7, "len": 8, "gnw": 9, "gnb": 10}
+_TAGS = {"q": 1, "k": 2, "v": 3, "g": 4, "s": 5, "x": 6, "w": 7, "len": 8, "gnw": 9, "gnb": 10,
+         "wqkvg": 11, "gbias": 12}
 
 
 def _gen(seed, tag, device):
@@ -87,6 +91,23 @@ def epilogue_inputs(T, D, F, seed=0, device="cpu", w_std=0.02, affine=False):
     return out
 
 
+def layer_inputs(T, D, H, d=128, seed=0, device="cpu", pad=0, pad_value=float("nan")):
+    """One mixer layer's input and weights, bf16: x [T, D], w_qkvg [D, 3 H d + H + pad] (W_Q,
+    W_K, W_V and W_gamma side by side; the pad columns, if any, hold pad_value) and
+    w_g [D, H d]."""
+    F = 3 * H * d + H
+    x = _randn((T, D), seed, "x", device)
+    x[:, 0] = 1.0
+    w = _randn((D, F + pad), seed, "wqkvg", device, std=D ** -0.5)
+    w[:, 3 * H * d:F] *= 0.05
+    w[0, 3 * H * d:F] = _randn((H,), seed, "gbias", device, mean=2.0)
+    if pad:
+        w[:, F:] = pad_value
+    w_g = _randn((D, H * d), seed, "w", device, std=0.02)
+    return {"x": x.to(torch.bfloat16), "w_qkvg": w.to(torch.bfloat16),
+            "w_g": w_g.to(torch.bfloat16)}
+
+
 # The five workloads, by what they are.
 TINY = dict(B=1, N=512, H=2, dk=64, dtype=torch.float32, g_mean=2.0, g_std=1.0, seed=1,
             layout="bhnd", chunk=64)
@@ -96,5 +117,6 @@ PREFILL_512K = dict(B=1, N=524288, H=24, dk=128, dtype=torch.bfloat16, g_mean=2.
                     seed=3)
 DECODE_BS64 = dict(B=64, prefill_N=4096, steps=256, H=24, dk=128, dtype=torch.bfloat16,
                    g_mean=2.0, g_std=1.0, seed=4)
+LAYER_32K = dict(T=32768, D=3072, H=24, dk=128, seed=6)
 VARLEN_EPILOGUE = dict(n_seqs=8, lo=1024, hi=65536, H=24, dk=128, dtype=torch.bfloat16,
                        g_mean=0.0, g_std=2.0, D=3072, eps=1e-5, seed=5)

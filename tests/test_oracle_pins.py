@@ -266,3 +266,74 @@ def test_groupnorm_moments_and_gate(oracle_mod):
     # a row subset returns exactly those rows
     ys = oracle_mod.groupnorm_gate(o, x, w, H=H, eps=eps, rows=[4, 1])
     assert np.array_equal(ys, y[[4, 1]])
+
+
+# ---- the layer's input projection and the layer composition
+
+
+def test_projection_brute_force(oracle_mod):
+    """[q | k | v | g] = x W against explicit loops on a tiny case."""
+    rng = np.random.default_rng(11)
+    T, D, H, d = 3, 5, 2, 3
+    F = 3 * H * d + H
+    x = rng.standard_normal((T, D))
+    w = rng.standard_normal((D, F + 2))              # two padding columns, ignored
+    q, k, v, g = oracle_mod.qkvg_projection(x, w, H, d)
+    for t in range(T):
+        for c in range(F):
+            ref = sum(x[t, i] * w[i, c] for i in range(D))
+            blk, rem = divmod(c, H * d)
+            got = (q, k, v)[blk][t, rem // d, rem % d] if blk < 3 else g[t, c - 3 * H * d]
+            assert abs(got - ref) < 1e-12
+
+
+def test_projection_blocks_one_hot(oracle_mod):
+    """W with one 1 per column: each output reads one input column, so the block layout of q, k,
+    v (heads of d consecutive columns) and g shows directly."""
+    T, D, H, d = 2, 64, 2, 4
+    F = 3 * H * d + H
+    x = np.arange(T * D, dtype=np.float64).reshape(T, D)
+    w = np.zeros((D, F))
+    for c in range(F):
+        w[(7 * c + 3) % D, c] = 1.0
+    q, k, v, g = oracle_mod.qkvg_projection(x, w, H, d)
+    for t in range(T):
+        for h in range(H):
+            for j in range(d):
+                for blk, arr in enumerate((q, k, v)):
+                    c = blk * H * d + h * d + j
+                    assert arr[t, h, j] == x[t, (7 * c + 3) % D]
+            c = 3 * H * d + h
+            assert g[t, h] == x[t, (7 * c + 3) % D]
+
+
+def test_layer_with_closed_gates_is_per_token(oracle_mod):
+    """gamma == 0 (every gate logit -1e4 through a constant input column): each token attends
+    only to itself, o_t = k_scale (q_t . k_t) v_t per head with k_scale = d^-1/2, so the layer is
+    GroupNorm(bf16(o_t)) * swish(x_t W_G) token by token, with q, k, v rounded to bf16 first."""
+    rng = np.random.default_rng(12)
+    T, D, H, d = 6, 64, 2, 4
+    F = 3 * H * d + H
+    x = rng.standard_normal((T, D)) * 0.5
+    x[:, 0] = 1.0
+    w = rng.standard_normal((D, F)) * 0.3
+    w[:, 3 * H * d:] = 0.0
+    w[0, 3 * H * d:] = -1e4
+    w_g = rng.standard_normal((D, H * d)) * 0.3
+    y, _ = oracle_mod.layer_forward(x, w, w_g, H, d)
+    import torch
+    bf = lambda a: torch.from_numpy(np.ascontiguousarray(a)).to(torch.bfloat16).double().numpy()
+    z = x @ w
+    hd = H * d
+    q = bf(z[:, :hd]).reshape(T, H, d)
+    k = bf(z[:, hd:2 * hd]).reshape(T, H, d)
+    v = bf(z[:, 2 * hd:3 * hd]).reshape(T, H, d)
+    o = bf(np.einsum("thj,thj->th", q, k)[:, :, None] * d ** -0.5 * v)
+    zg = x @ w_g
+    for t in range(T):
+        for h in range(H):
+            row = o[t, h]
+            n = (row - row.mean()) / np.sqrt(row.var() + 1e-5)
+            zz = zg[t, h * d:(h + 1) * d]
+            ref = n * zz / (1.0 + np.exp(-zz))
+            assert np.allclose(y[t, h * d:(h + 1) * d], ref, rtol=1e-9, atol=1e-12)
