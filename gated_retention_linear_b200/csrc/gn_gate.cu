@@ -73,12 +73,26 @@ __device__ __forceinline__ bool wait_bar(GSmem& sm, uint64_t* bar, uint32_t pari
     return false;
 }
 
+// Tile order: runs of GROUP_M row blocks, and inside a run the row blocks fastest, so that one
+// wave of CTAs shares few rows of X and few column blocks of W and both stay in L2 while the
+// wave runs (a wide W, as in the projection, is otherwise streamed once per few row blocks).
+constexpr int GROUP_M = 16;
+
+__device__ __forceinline__ void tile_coords(const GParams& p, int tile, int& mb, int& nb) {
+    const int per_group = GROUP_M * p.n_blocks;
+    const int grp = tile / per_group, rem = tile - grp * per_group;
+    const int rows = min(GROUP_M, p.m_blocks - grp * GROUP_M);
+    nb = rem / rows;
+    mb = grp * GROUP_M + (rem - nb * rows);
+}
+
 __device__ void producer(GSmem& sm, const GParams& p, const CUtensorMap* tx, const CUtensorMap* tw) {
     const int kblocks = p.D / BK;
     int it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
-        const int mb = tile / p.n_blocks, nb = tile % p.n_blocks;
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
             const int s = it % STAGES;
             if (it >= STAGES && !wait_bar(sm, &sm.empty[s], ((it / STAGES) - 1) & 1)) {
@@ -176,7 +190,8 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
     int t_local = 0;
     for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++t_local) {
         const int buf = t_local & 1;
-        const int mb = tile / p.n_blocks, nb = tile % p.n_blocks;
+        int mb, nb;
+        tile_coords(p, tile, mb, nb);
         const int64_t t = (int64_t)mb * BM + r;
         const int col0 = nb * BN + half * 128;
         const bool valid = t < p.T;
