@@ -316,3 +316,51 @@ int oracle_groupnorm_gate(const double* o, const double* x, const double* wg,
     }
     return 0;
 }
+
+/*
+ * Element-wise (per key channel) gate, the alternative that [P1, "路线二"] weighs against the
+ * head-wise scalar gate: instead of one gamma per head and token, every key channel i of the
+ * state has its own decay alpha_t[i] = sigmoid(g_t[i])^(1/tau), so
+ *   S[i][:] <- alpha_t[i] * S[i][:] + (k_scale * K_t[i]) V_t      (decay first, then add)
+ *   O_t <- Q_t S
+ * Reading: "element-wise" is taken per state row (one gate per key channel, d_k gates per
+ * head and token); a separate gate for each of the d_k * d_v state entries would need a gate
+ * tensor the size of the state per token, which the page does not describe.
+ * Layout as above except g: [T][H][dk].  Returns 0, or -1 on inconsistent sequence offsets.
+ */
+int oracle_gret_recurrent_ew(const double* q, const double* k, const double* v, const double* g,
+                             double tau, double k_scale, int64_t T, int H, int dk, int dv,
+                             const int64_t* cu_seqlens, int n_seqs, const double* state_in,
+                             double* state_out, double* o) {
+    if (check_seqs(cu_seqlens, n_seqs, T)) return -1;
+    int64_t units = (int64_t)n_seqs * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < units; ++u) {
+        int s = (int)(u / H), h = (int)(u % H);
+        double* S = (double*)malloc(sizeof(double) * (size_t)dk * dv);
+        if (state_in)
+            memcpy(S, state_in + u * dk * dv, sizeof(double) * (size_t)dk * dv);
+        else
+            memset(S, 0, sizeof(double) * (size_t)dk * dv);
+        for (int64_t t = cu_seqlens[s]; t < cu_seqlens[s + 1]; ++t) {
+            const double* qt = q + (t * H + h) * dk;
+            const double* kt = k + (t * H + h) * dk;
+            const double* vt = v + (t * H + h) * dv;
+            const double* gt = g + (t * H + h) * dk;
+            for (int i = 0; i < dk; ++i) {
+                double alpha = exp(oracle_log_gamma(gt[i], tau));
+                for (int j = 0; j < dv; ++j)
+                    S[i * dv + j] = alpha * S[i * dv + j] + (k_scale * kt[i]) * vt[j];
+            }
+            double* ot = o + (t * H + h) * dv;
+            for (int j = 0; j < dv; ++j) {
+                double acc = 0.0;
+                for (int i = 0; i < dk; ++i) acc += qt[i] * S[i * dv + j];
+                ot[j] = acc;
+            }
+        }
+        if (state_out) memcpy(state_out + u * dk * dv, S, sizeof(double) * (size_t)dk * dv);
+        free(S);
+    }
+    return 0;
+}

@@ -32,6 +32,8 @@ def lib():
             f = getattr(L, name)
             f.argtypes = common
             f.restype = ctypes.c_int
+        L.oracle_gret_recurrent_ew.argtypes = common
+        L.oracle_gret_recurrent_ew.restype = ctypes.c_int
         L.oracle_gret_chunkwise.argtypes = common + [ctypes.c_int]
         L.oracle_gret_chunkwise.restype = ctypes.c_int
         L.oracle_gret_decode_step.argtypes = [dp, dp, dp, dp, ctypes.c_double, ctypes.c_double,
@@ -77,11 +79,12 @@ def threads():
     return len(os.sched_getaffinity(0))
 
 
-def _run(fname, q, k, v, g, tau, k_scale, cu_seqlens, state_in, extra=()):
+def _run(fname, q, k, v, g, tau, k_scale, cu_seqlens, state_in, extra=(), g_per_channel=False):
     q, k, v, g = _d(q), _d(k), _d(v), _d(g)
     T, H, dk = q.shape
     dv = v.shape[2]
-    assert k.shape == (T, H, dk) and v.shape == (T, H, dv) and g.shape == (T, H)
+    assert k.shape == (T, H, dk) and v.shape == (T, H, dv)
+    assert g.shape == ((T, H, dk) if g_per_channel else (T, H))
     cu = _cu(cu_seqlens, T)
     n = len(cu) - 1
     s_in = _d(state_in)
@@ -100,6 +103,13 @@ def _run(fname, q, k, v, g, tau, k_scale, cu_seqlens, state_in, extra=()):
 def gret_recurrent(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):
     """Recurrent gRet (the definition).  Returns (o [T,H,dv], state [n_seqs,H,dk,dv])."""
     return _run("oracle_gret_recurrent", q, k, v, g, tau, k_scale, cu_seqlens, state_in)
+
+
+def gret_recurrent_ew(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):
+    """Recurrent gated retention with one gate per key channel: g [T, H, dk], the state row i
+    decays by sigmoid(g[..., i])^(1/tau).  Returns (o [T,H,dv], state [n_seqs,H,dk,dv])."""
+    return _run("oracle_gret_recurrent_ew", q, k, v, g, tau, k_scale, cu_seqlens, state_in,
+                g_per_channel=True)
 
 
 def gret_parallel(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):

@@ -337,3 +337,72 @@ def test_layer_with_closed_gates_is_per_token(oracle_mod):
             zz = zg[t, h * d:(h + 1) * d]
             ref = n * zz / (1.0 + np.exp(-zz))
             assert np.allclose(y[t, h * d:(h + 1) * d], ref, rtol=1e-9, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------------
+# Element-wise (per key channel) gate: the alternative that "路线二：Multi-Head Gated Retention"
+# weighs against the head-wise gate.  State row i decays by alpha_t[i] = sigmoid(g_t[i])^(1/tau).
+
+def ew_case(seed, T, H, dk, dv, g_mean=2.0, g_std=1.0, state=False, n_seqs=1):
+    rng = np.random.default_rng(seed)
+    q, k, v, _, s0 = case(seed, T, H, dk, dv, state=state, n_seqs=n_seqs)
+    g = rnd(rng, (T, H, dk), g_std, g_mean)
+    return q, k, v, g, s0
+
+
+def test_ew_equal_channel_gates_is_headwise(oracle_mod):
+    """One gate shared by every channel of a head reduces to the head-wise recurrence (a
+    separate function of the oracle), across sequences with an entry state."""
+    q, k, v, g1, s0 = case(41, 23, 2, 6, 5, g_std=2.0, state=True, n_seqs=3)
+    g = np.repeat(g1[:, :, None], 6, axis=2)
+    cu = [0, 7, 7, 23]
+    o_ew, s_ew = oracle_mod.gret_recurrent_ew(q, k, v, g, k_scale=0.7, cu_seqlens=cu,
+                                              state_in=s0)
+    o_hw, s_hw = oracle_mod.gret_recurrent(q, k, v, g1, k_scale=0.7, cu_seqlens=cu,
+                                           state_in=s0)
+    assert close(o_ew, o_hw) and close(s_ew, s_hw)
+
+
+def test_ew_brute_force_products(oracle_mod):
+    """The unrolled per-channel form, with the survival products of each channel formed term by
+    term and the gate from its closed form sigmoid(g)^(1/tau):
+        O_n[j] = sum_i Q_n[i] ( sum_{m<=n} k_scale K_m[i] V_m[j] prod_{m<l<=n} alpha_l[i]
+                                + S_0[i][j] prod_{l<=n} alpha_l[i] )."""
+    T, H, dk, dv, tau, ks = 9, 2, 3, 4, 16.0, 0.8
+    q, k, v, g, s0 = ew_case(42, T, H, dk, dv, g_mean=0.0, g_std=3.0, state=True)
+    alpha = (1.0 / (1.0 + np.exp(-g))) ** (1.0 / tau)
+    o_ref = np.zeros((T, H, dv))
+    for h in range(H):
+        for n in range(T):
+            for i in range(dk):
+                for j in range(dv):
+                    acc = s0[0, h, i, j] * np.prod(alpha[:n + 1, h, i])
+                    for m in range(n + 1):
+                        acc += ks * k[m, h, i] * v[m, h, j] * np.prod(alpha[m + 1:n + 1, h, i])
+                    o_ref[n, h, j] += q[n, h, i] * acc
+    o, _ = oracle_mod.gret_recurrent_ew(q, k, v, g, tau=tau, k_scale=ks, state_in=s0)
+    assert close(o, o_ref, 1e-12)
+
+
+def test_ew_one_hot_query_reads_one_decayed_row(oracle_mod):
+    """With q = e_c, o_t is row c of the state, which must follow a scalar-gate recurrence with
+    channel c's gate and key (d_k != d_v, so a gate applied along the value axis fails)."""
+    T, H, dk, dv = 17, 1, 5, 3
+    _, k, v, g, s0 = ew_case(43, T, H, dk, dv, g_mean=0.0, g_std=2.0, state=True)
+    for c in (0, 3):
+        q = np.zeros((T, H, dk))
+        q[:, :, c] = 1.0
+        o, s = oracle_mod.gret_recurrent_ew(q, k, v, g, state_in=s0)
+        o1, s1 = oracle_mod.gret_recurrent(np.ones((T, H, 1)), k[:, :, c:c + 1], v, g[:, :, c],
+                                           state_in=s0[:, :, c:c + 1, :])
+        assert close(o, o1) and close(s[:, :, c:c + 1, :], s1)
+
+
+def test_ew_closed_gates_keep_current_token(oracle_mod):
+    """alpha == 0 on every channel (g = -1e4): O_n = k_scale (Q_n . K_n) V_n and S_N = K_N^T V_N."""
+    q, k, v, _, s0 = ew_case(44, 11, 2, 4, 6, state=True)
+    g = np.full((11, 2, 4), -1e4)
+    o, s = oracle_mod.gret_recurrent_ew(q, k, v, g, k_scale=0.5, state_in=s0)
+    o_ref = 0.5 * np.einsum("thi,thi->th", q, k)[:, :, None] * v
+    assert close(o, o_ref)
+    assert close(s[0], 0.5 * np.einsum("hi,hj->hij", k[-1], v[-1]))
