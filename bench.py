@@ -291,6 +291,11 @@ def run_gpu(args):
     if not args.no_epilogue:
         epi = run_varlen_epilogue(args, rank, world, stream, hbm_peak)
 
+    # ---------------- per-key-channel gate variant of the prefill, same 3B shapes
+    ew = None
+    if not args.no_elementwise:
+        ew = run_elementwise(args, rank, world, stream, ms_per_step)
+
     # ---------------- one mixer layer: projection GEMM -> prefill -> GroupNorm * gate
     lay = None
     if not args.no_layer:
@@ -379,7 +384,8 @@ def run_gpu(args):
                      "traffic": prefill_traffic_from_profile(),
                      "kernel": "prefill_tc_kernel", "launch_ms": launch_ms,
                      "algorithmic_bytes_per_launch": alg_bytes},
-        "decode": dec, "varlen_epilogue": epi, "layer": lay, "e2e": e2e, "clocks": clk,
+        "decode": dec, "varlen_epilogue": epi, "layer": lay,
+        "elementwise_gate": ew, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }
@@ -445,6 +451,71 @@ def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
             "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
                          "frac": ach / tpeak, "peak_kind": tkind + " burst", "traffic": None,
                          "kernel": "gn_gate_kernel", "algorithmic_flops_per_launch": flops}}
+
+
+# fp32 FMA peak of the CUDA-core path: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (the
+# maximum SM clock); FLOP per token and head of the per-channel-gate prefill at chunk 64:
+# chunk state 2 d^2, cross-chunk output 2 d^2, in-chunk scores and A V 2 d (C + 1) / 2 each,
+# scan 2 d^2 / C.
+FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
+EW_FLOP_PER_TOKEN_HEAD = 2 * D * D + 2 * D * D + 2 * (2 * D * (64 + 1) // 2) + 2 * D * D // 64
+
+
+def run_elementwise(args, rank, world, stream, headwise_ms):
+    """The per-key-channel-gate prefill (three CUDA-core launches: chunk states, scan over
+    chunks, chunk outputs) on the 3B shapes, 32768 tokens x 24 heads, bf16 q, k, v and one fp32
+    gate logit per key channel.  Also reports the head-wise kernel's time on the same shapes
+    over this variant's: the hardware-efficiency cost of a gate per channel."""
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+    c = SI.ELEMENTWISE_32K
+    Bq, Nq, Hq = c["B"], c["N"], c["H"]
+    inp = SI.gret_inputs(Bq, Nq, Hq, D, dtype=torch.bfloat16, seed=rank_seed(c["seed"], rank),
+                         device="cuda")
+    q, k, v = inp["q"], inp["k"], inp["v"]
+    del inp
+    g = SI.channel_gates(Bq, Nq, Hq, D, g_mean=c["g_mean"], g_std=c["g_std"],
+                         seed=rank_seed(c["seed"], rank), device="cuda")
+    o = torch.empty_like(q)
+    s_out = torch.empty((Bq, Hq, D, D), dtype=torch.float32, device="cuda")
+    ws = torch.empty(G.gret_prefill_elementwise_workspace_size(Bq, Nq, Hq, D),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        G.gret_prefill_elementwise(q, k, v, g, state_out=s_out, o=o, workspace=ws)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 10))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    tokens = Bq * Nq
+    flops = float(EW_FLOP_PER_TOKEN_HEAD) * tokens * Hq
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"value": tokens * world / (ms * 1e-3) / 1e6, "unit": "Mtok/s", "tokens": tokens,
+            "heads": Hq, "ms_per_step": ms, "steps": n, "gpu_launches_per_step": 3,
+            "gate": "one logit per key channel, g ~ N(2, 1)",
+            "headwise_ms_same_shapes": headwise_ms,
+            "slowdown_vs_headwise": ms / headwise_ms,
+            "workspace_bytes": ws.numel(),
+            "l2": "inputs (1.2 GB) and the 812 MB chunk-state workspace larger than L2; "
+                  "not flushed",
+            "roofline": {"bound": "alu", "achieved": ach, "peak": FP32_FMA_PEAK_TFLOPS,
+                         "unit": "TFLOP/s", "frac": ach / FP32_FMA_PEAK_TFLOPS,
+                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
+                         "traffic": None,
+                         "kernel": "ew_chunk_state + ew_state_scan + ew_chunk_output",
+                         "algorithmic_flops_per_launch": flops}}
 
 
 def run_layer(args, rank, world, stream, hbm_peak):
@@ -584,6 +655,7 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-epilogue", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
+    ap.add_argument("--no-elementwise", action="store_true")
     ap.add_argument("--varlen-max-len", type=int, default=65536,
                     help="longest sequence of the varlen + epilogue leg (a smaller value gives "
                          "a small case for profiling)")

@@ -53,6 +53,11 @@ _lib.gret_groupnorm_gate.restype = _i32
 _lib.gret_qkvg_projection.argtypes = [_vp, _vp, _i64, _i64, _i32, _i32, _i32, _vp, _vp, _vp, _vp,
                                       _vp]
 _lib.gret_qkvg_projection.restype = _i32
+_lib.gret_prefill_elementwise.argtypes = [_vp, _vp, _vp, _vp, _f32, _f32, _i32, _i64, _i32, _i32,
+                                          _vp, _vp, _vp, _vp, ctypes.c_size_t, _vp]
+_lib.gret_prefill_elementwise.restype = _i32
+_lib.gret_prefill_elementwise_workspace_size.argtypes = [_i32, _i64, _i32, _i32]
+_lib.gret_prefill_elementwise_workspace_size.restype = ctypes.c_size_t
 
 
 class GretError(RuntimeError):
@@ -240,6 +245,36 @@ def gret_qkvg_projection(x, w, H, d=128, stream=None):
         _ptr(x), _ptr(w), w.stride(0), T, H, d, D, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
         _stream(stream)))
     return q, k, v, g
+
+
+def gret_prefill_elementwise_workspace_size(B, N, H, d=128):
+    return int(_lib.gret_prefill_elementwise_workspace_size(B, N, H, d))
+
+
+def gret_prefill_elementwise(q, k, v, g, tau=16.0, k_scale=1.0, state_in=None, state_out=None,
+                             o=None, workspace=None, stream=None):
+    """Chunkwise prefill with one gate per key channel (state row i decays by
+    sigmoid(g[..., i])^(1/tau)).  q, k, v [B, N, H, 128] bf16 and g [B, N, H, 128] fp32, all
+    contiguous; state_in / state_out fp32 [B, H, 128, 128] (state_out=True allocates one).
+    Returns (o, state_out)."""
+    B, N, H, d = q.shape
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != (B, N, H, d):
+            raise ValueError("q, k, v must be contiguous bfloat16 [B, N, H, d]")
+    if g.dtype != torch.float32 or not g.is_contiguous() or g.shape != (B, N, H, d):
+        raise ValueError("g must be contiguous float32 [B, N, H, d]")
+    if o is None:
+        o = torch.empty_like(q)
+    if state_out is True:
+        state_out = torch.empty((B, H, d, d), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        need = gret_prefill_elementwise_workspace_size(B, N, H, d)
+        workspace = torch.empty(max(need, 16), dtype=torch.uint8, device=q.device)
+    _check("gret_prefill_elementwise", _lib.gret_prefill_elementwise(
+        _ptr(q), _ptr(k), _ptr(v), _ptr(g), tau, k_scale, B, N, H, d, _ptr(state_in),
+        _ptr(state_out), _ptr(o), _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream(stream)))
+    return o, state_out
 
 
 def gret_layer_forward(x, w_qkvg, w_g, H, d=128, cu_seqlens=None, state_in=None, tau=16.0,

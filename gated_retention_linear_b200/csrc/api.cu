@@ -8,6 +8,7 @@
 #include "common.cuh"
 #include "prefill_tc.cuh"
 #include "gn_gate.cuh"
+#include "prefill_ew.cuh"
 
 using namespace gret;
 
@@ -168,6 +169,51 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
         (reinterpret_cast<uintptr_t>(g) & 3u) != 0 || ldw % 8 != 0)
         return GRET_ERR_ALIGNMENT;
     return launch_qkvg_projection(x, w, ldw, T, H, D, q, k, v, g, (cudaStream_t)stream);
+}
+
+size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d) {
+    if (B < 0 || N < 0 || H < 1 || d != EW_DIM) return 0;
+    return ew_workspace_bytes(B, N, H);
+}
+
+gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void* v,
+                                       const float* g, float tau, float k_scale, int B,
+                                       int64_t N, int H, int d, const float* state_in,
+                                       float* state_out, void* o, void* workspace,
+                                       size_t workspace_bytes, gret_stream_t stream) {
+    if (B < 0 || N < 0 || H < 1 || d < 1) return GRET_ERR_INVALID_ARG;
+    if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
+    if (d != EW_DIM) return GRET_ERR_UNSUPPORTED;
+    const int64_t nch = (N + EW_CHUNK - 1) / EW_CHUNK;
+    if (B > 65535 || H > 65535 || nch > 0x7fffffff) return GRET_ERR_UNSUPPORTED;
+    if (B == 0) return GRET_OK;
+    if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
+        return GRET_ERR_ALIGNMENT;
+    const cudaStream_t s = (cudaStream_t)stream;
+    const size_t state_bytes = (size_t)B * H * EW_DIM * EW_DIM * sizeof(float);
+    if (N == 0) {   // no tokens: the final state is the entry state
+        if (!state_out || state_out == state_in) return GRET_OK;
+        const cudaError_t e = state_in ? cudaMemcpyAsync(state_out, state_in, state_bytes,
+                                                         cudaMemcpyDeviceToDevice, s)
+                                       : cudaMemsetAsync(state_out, 0, state_bytes, s);
+        return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+    }
+    if (!q || !k || !v || !g || !o) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(g) || !aligned16(o))
+        return GRET_ERR_ALIGNMENT;
+    if (!workspace || workspace_bytes < ew_workspace_bytes(B, N, H)) return GRET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GRET_ERR_ALIGNMENT;
+    EwArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.g = g; a.tau = tau; a.k_scale = k_scale;
+    a.B = B; a.N = N; a.H = H; a.nch = (int)nch;
+    a.state_in = state_in; a.state_out = state_out;
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.ws_S = static_cast<float*>(workspace);
+    a.ws_a = a.ws_S + (size_t)B * H * nch * EW_DIM * EW_DIM;
+    return launch_prefill_ew(a, s) == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -187,6 +187,37 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
                                    int d, int D, void* q, void* k, void* v, float* g,
                                    gret_stream_t stream);
 
+/*
+ * Chunkwise prefill with one gate per key channel: the element-wise alternative that
+ * "路线二：Multi-Head Gated Retention" weighs against the head-wise scalar gate (YOCO keeps the
+ * head-wise one because it keeps every contraction a plain matrix product).  Per sequence and
+ * head, with a gate logit per key channel i:
+ *   alpha_t[i] = sigmoid(g_t[i])^(1/tau)
+ *   S_t[i][:] = alpha_t[i] S_{t-1}[i][:] + (k_scale k_t[i]) v_t      (each state row decays
+ *                                                                     at its channel's rate)
+ *   o_t = q_t S_t
+ * A gate shared by all channels of a head gives gret_prefill_chunkwise's result.
+ *   q, k, v, o  bf16 [B, N, H, d] contiguous (token-major);  g  fp32 [B, N, H, d] contiguous.
+ *   state_in    fp32 [B, H, d, d] or NULL (zero entry state);  state_out likewise, or NULL;
+ *               state_out may alias state_in.
+ *   workspace   device memory of at least gret_prefill_elementwise_workspace_size(B, N, H, d)
+ *               bytes, 16-byte aligned, owned by the caller; its contents on entry do not
+ *               matter and are overwritten.
+ * Runs on CUDA cores in fp32 (three launches: chunk states, a scan over chunks, chunk
+ * outputs).  Requires d == 128, B <= 65535, H <= 65535; q, k, v, g, o and the states 16-byte
+ * aligned (GRET_ERR_ALIGNMENT otherwise).  N == 0 copies state_in (or zeros) to state_out.
+ * o must not overlap the inputs.
+ */
+gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void* v,
+                                       const float* g, float tau, float k_scale, int B,
+                                       int64_t N, int H, int d, const float* state_in,
+                                       float* state_out, void* o, void* workspace,
+                                       size_t workspace_bytes, gret_stream_t stream);
+
+/* Workspace bytes gret_prefill_elementwise needs: B * H * ceil(N / 64) * (d*d + d) * 4.
+ * Returns 0 on invalid sizes or d != 128. */
+size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d);
+
 #ifdef __cplusplus
 }
 #endif

@@ -9,7 +9,8 @@ to the requested dtype; the rounded values are what both the CUDA path and the o
 Recipes (the 3B shapes of the YOCO pages: 24 heads of width 128, hidden 3072):
   * q, k, v ~ N(0, 1) / sqrt(d)         (the 1/sqrt(d_h) key scaling is folded into the draw,
                                           so the library is called with k_scale = 1)
-  * gate logits g ~ N(mean, std), fp32  (N(2, 1) for the dense configs, N(0, 2) for varlen)
+  * gate logits g ~ N(mean, std), fp32  (N(2, 1) for the dense configs, N(0, 2) for varlen);
+    the per-key-channel gate variant draws one such logit per channel
   * packed varlen lengths ~ U[lo, hi] (torch.randint, inclusive bounds)
   * epilogue: x ~ N(0, 1), w_g ~ N(0, 0.02), bf16
   * layer: x ~ N(0, 1) with a constant column x[:, 0] = 1; W_Q, W_K, W_V ~ N(0, 1/D);
@@ -21,7 +22,7 @@ import math
 import torch
 
 _TAGS = {"q": 1, "k": 2, "v": 3, "g": 4, "s": 5, "x": 6, "w": 7, "len": 8, "gnw": 9, "gnb": 10,
-         "wqkvg": 11, "gbias": 12}
+         "wqkvg": 11, "gbias": 12, "gch": 13}
 
 
 def _gen(seed, tag, device):
@@ -91,6 +92,11 @@ def epilogue_inputs(T, D, F, seed=0, device="cpu", w_std=0.02, affine=False):
     return out
 
 
+def channel_gates(B, N, H, dk, g_mean=2.0, g_std=1.0, seed=0, device="cpu"):
+    """Gate logits with one value per key channel, g [B, N, H, dk] fp32 ~ N(g_mean, g_std)."""
+    return _randn((B, N, H, dk), seed, "gch", device, std=g_std, mean=g_mean)
+
+
 def layer_inputs(T, D, H, d=128, seed=0, device="cpu", pad=0, pad_value=float("nan")):
     """One mixer layer's input and weights, bf16: x [T, D], w_qkvg [D, 3 H d + H + pad] (W_Q,
     W_K, W_V and W_gamma side by side; the pad columns, if any, hold pad_value) and
@@ -117,6 +123,7 @@ PREFILL_512K = dict(B=1, N=524288, H=24, dk=128, dtype=torch.bfloat16, g_mean=2.
                     seed=3)
 DECODE_BS64 = dict(B=64, prefill_N=4096, steps=256, H=24, dk=128, dtype=torch.bfloat16,
                    g_mean=2.0, g_std=1.0, seed=4)
+ELEMENTWISE_32K = dict(B=1, N=32768, H=24, dk=128, g_mean=2.0, g_std=1.0, seed=7)
 LAYER_32K = dict(T=32768, D=3072, H=24, dk=128, seed=6)
 VARLEN_EPILOGUE = dict(n_seqs=8, lo=1024, hi=65536, H=24, dk=128, dtype=torch.bfloat16,
                        g_mean=0.0, g_std=2.0, D=3072, eps=1e-5, seed=5)
