@@ -62,15 +62,24 @@ __device__ __forceinline__ void load_tile(__nv_bfloat16* dst, const __nv_bfloat1
     }
 }
 
-// Thread `tid` < D: channel tid's inclusive cumulative log-decay over tokens [0, L) of the
-// chunk, written to c[t * stride + tid].  Returns the chunk total.
-__device__ __forceinline__ float channel_scan(const EwArgs& a, int64_t row0, int L, int tid,
-                                              float* c, int stride) {
-    float cum = 0.f;
+// Log-decays logsigmoid(g) / tau of tokens [0, L) of the chunk into c[t * stride + i], by all
+// threads of the block (no barrier inside).
+__device__ __forceinline__ void log_decays(const EwArgs& a, int64_t row0, int L, int tid,
+                                           float* c, int stride) {
     const float inv_tau = 1.f / a.tau;
-#pragma unroll 8
+    for (int e = tid; e < L * D; e += NT) {
+        const int t = e / D, i = e - t * D;
+        c[t * stride + i] = logsigmoidf_(a.g[(row0 + (int64_t)t * a.H) * D + i]) * inv_tau;
+    }
+}
+
+// Thread `tid` < D: turn channel tid's log-decays into the inclusive cumulative sum over the
+// chunk, in place.  Returns the chunk total.
+__device__ __forceinline__ float channel_cumsum(int L, int tid, float* c, int stride) {
+    float cum = 0.f;
+#pragma unroll 16
     for (int t = 0; t < L; ++t) {
-        cum += logsigmoidf_(a.g[(row0 + (int64_t)t * a.H) * D + tid]) * inv_tau;
+        cum += c[t * stride + tid];
         c[t * stride + tid] = cum;
     }
     return cum;
@@ -88,15 +97,15 @@ __global__ void __launch_bounds__(NT) ew_chunk_state(EwArgs a) {
     const int64_t row0 = ((int64_t)b * a.N + t0) * a.H + h;
     const int64_t slot = ((int64_t)b * a.H + h) * a.nch + c;
 
-    if (tid < D)
-        clast[tid] = channel_scan(a, row0, L, tid, kt, D);   // kt holds c_t for now
-    else
-        load_tile(vs, a.v, row0, a.H, L, tid, D, NT - D);
+    load_tile(vs, a.v, row0, a.H, L, tid, 0, NT);
+    log_decays(a, row0, L, tid, kt, D);                      // kt holds c_t for now
+    __syncthreads();
+    if (tid < D) clast[tid] = channel_cumsum(L, tid, kt, D);
     __syncthreads();
     for (int e = tid; e < L * D; e += NT) {
         const int t = e / D, i = e - t * D;
         const float kv = __bfloat162float(a.k[(row0 + (int64_t)t * a.H) * D + i]);
-        kt[e] = a.k_scale * kv * expf(clast[i] - kt[e]);
+        kt[e] = a.k_scale * kv * __expf(clast[i] - kt[e]);
     }
     if (tid < D) a.ws_a[slot * D + tid] = expf(clast[tid]);
     __syncthreads();
@@ -185,7 +194,9 @@ __global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
     load_tile(qs, a.q, row0, a.H, L, tid, 0, NT);
     load_tile(kv, a.k, row0, a.H, L, tid, 0, NT);
     for (int e = tid; e < C * C; e += NT) At[e] = 0.f;
-    if (tid < D) channel_scan(a, row0, L, tid, cq, CQS);
+    log_decays(a, row0, L, tid, cq, CQS);
+    __syncthreads();
+    if (tid < D) channel_cumsum(L, tid, cq, CQS);
     __syncthreads();
 
     // A inside each sub-chunk: one warp per (t, m) pair, lanes over the channels.
@@ -198,7 +209,7 @@ __global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
         for (int u = 0; u < D / 32; ++u) {
             const int i = lane + 32 * u;
             acc += __bfloat162float(qs[t * D + i]) * __bfloat162float(kv[m * D + i]) *
-                   expf(cq[t * CQS + i] - cq[m * CQS + i]);
+                   __expf(cq[t * CQS + i] - cq[m * CQS + i]);
         }
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
@@ -218,10 +229,11 @@ __global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
                     const int t = ts * SC + r;
                     if (t < L)
                         val = __bfloat162float(qs[t * D + i]) *
-                              expf(cq[t * CQS + i] - cq[p * CQS + i]);
+                              __expf(cq[t * CQS + i] - cq[p * CQS + i]);
                 } else {
                     const int m = ms * SC + (r - SC);
-                    val = __bfloat162float(kv[m * D + i]) * expf(cq[p * CQS + i] - cq[m * CQS + i]);
+                    val = __bfloat162float(kv[m * D + i]) *
+                          __expf(cq[p * CQS + i] - cq[m * CQS + i]);
                 }
                 scr[r * SS + i] = val;
             }
@@ -241,11 +253,19 @@ __global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
     }
     __syncthreads();   // all of A written; k and the log-decays no longer needed as such
 
+    // The entry state of the chunk is read in slices of SR rows, each fetched into registers
+    // one slice ahead of its use; the first fetch overlaps the work below.
+    constexpr int SR = 2 * SC, PF = SR * D / 4 / NT;
+    const float4* Sp = reinterpret_cast<const float4*>(a.ws_S + slot * (int64_t)(D * D));
+    float4 pf[PF];
+#pragma unroll
+    for (int u = 0; u < PF; ++u) pf[u] = Sp[tid + u * NT];
+
     // q * e^{c} in place (zero rows past L), and v into the k tile.
     for (int e = tid; e < C * D; e += NT) {
         const int t = e / D, i = e - t * D;
         float val = 0.f;
-        if (t < L) val = __bfloat162float(qs[t * D + i]) * expf(cq[t * CQS + i]);
+        if (t < L) val = __bfloat162float(qs[t * D + i]) * __expf(cq[t * CQS + i]);
         cq[t * CQS + i] = val;
     }
     load_tile(kv, a.v, row0, a.H, L, tid, 0, NT);
@@ -269,13 +289,16 @@ __global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
 #pragma unroll
             for (int s = 0; s < 8; ++s) acc[r][s] = fmaf(ar[r], bv[s], acc[r][s]);
     }
-    const float* Sp = a.ws_S + slot * (int64_t)(D * D);
-    for (int i0 = 0; i0 < D; i0 += SC) {
-        for (int e = tid; e < SC * D / 4; e += NT)
-            reinterpret_cast<float4*>(scr)[e] = reinterpret_cast<const float4*>(Sp + i0 * D)[e];
+    for (int i0 = 0; i0 < D; i0 += SR) {
+#pragma unroll
+        for (int u = 0; u < PF; ++u) reinterpret_cast<float4*>(scr)[tid + u * NT] = pf[u];
         __syncthreads();
+        if (i0 + SR < D) {
+#pragma unroll
+            for (int u = 0; u < PF; ++u) pf[u] = Sp[(i0 + SR) * D / 4 + tid + u * NT];
+        }
 #pragma unroll 4
-        for (int ii = 0; ii < SC; ++ii) {
+        for (int ii = 0; ii < SR; ++ii) {
             float ar[4];
 #pragma unroll
             for (int r = 0; r < 4; ++r) ar[r] = cq[(tr + r) * CQS + i0 + ii];
