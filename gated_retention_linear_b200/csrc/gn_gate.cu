@@ -59,6 +59,7 @@ struct GParams {
     int64_t T;
     int F, D;          // F: output columns (GroupNorm gate: H * 128; projection: 3 H 128 + H)
     int m_blocks, n_blocks, n_tiles;
+    int group_m;       // tile order: runs of group_m row blocks (1 = row-major)
     // projection outputs
     __nv_bfloat16* qkv[3];   // q, k, v: [T, H, 128] bf16
     float* g;                // [T, H] fp32
@@ -73,18 +74,20 @@ __device__ __forceinline__ bool wait_bar(GSmem& sm, uint64_t* bar, uint32_t pari
     return false;
 }
 
-// Tile order: runs of GROUP_M row blocks, and inside a run the row blocks fastest, so that one
+// Tile order: runs of group_m row blocks, and inside a run the row blocks fastest, so that one
 // wave of CTAs shares few rows of X and few column blocks of W and both stay in L2 while the
-// wave runs (a wide W, as in the projection, is otherwise streamed once per few row blocks).
-constexpr int GROUP_M = 16;
-
+// wave runs.  A wide W (the projection's 37 column blocks) is otherwise streamed once per few
+// row blocks; a narrow one (the gate's 12) already fits, and there row-major order (group_m 1)
+// measured faster.
 __device__ __forceinline__ void tile_coords(const GParams& p, int tile, int& mb, int& nb) {
-    const int per_group = GROUP_M * p.n_blocks;
+    const int per_group = p.group_m * p.n_blocks;
     const int grp = tile / per_group, rem = tile - grp * per_group;
-    const int rows = min(GROUP_M, p.m_blocks - grp * GROUP_M);
+    const int rows = min(p.group_m, p.m_blocks - grp * p.group_m);
     nb = rem / rows;
-    mb = grp * GROUP_M + (rem - nb * rows);
+    mb = grp * p.group_m + (rem - nb * rows);
 }
+
+int group_rows(int n_blocks) { return n_blocks > 16 ? 16 : 1; }
 
 __device__ void producer(GSmem& sm, const GParams& p, const CUtensorMap* tx, const CUtensorMap* tw) {
     const int kblocks = p.D / BK;
@@ -392,6 +395,7 @@ gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g, cons
     p.m_blocks = (int)((T + BM - 1) / BM);
     p.n_blocks = F / BN;
     p.n_tiles = p.m_blocks * p.n_blocks;
+    p.group_m = group_rows(p.n_blocks);
     return launch_gemm<EPI_GN_GATE>(tx, tw, p, stream);
 }
 
@@ -427,6 +431,7 @@ gret_status_t launch_qkvg_projection(const void* x, const void* w, int64_t ldw, 
     p.m_blocks = (int)((T + BM - 1) / BM);
     p.n_blocks = (F + BN - 1) / BN;
     p.n_tiles = p.m_blocks * p.n_blocks;
+    p.group_m = group_rows(p.n_blocks);
     return launch_gemm<EPI_PROJECTION>(tx, tw, p, stream);
 }
 

@@ -11,9 +11,10 @@
 //                       scale; element-parallel over the state, serial over chunks)
 //   3. ew_chunk_output  o_t = (q_t * e^{c_t}) S_prev(c) + sum_{m<=t} A[t][m] v_m ,
 //                       A[t][m] = k_scale sum_i q_t[i] k_m[i] e^{c_t[i] - c_m[i]}
-// Inside a 16-token sub-chunk A takes the exponential pair by pair.  Across sub-chunks it
-// splits at p, the last token before t's sub-chunk: e^{c_t - c_p} e^{c_p - c_m}, both factors
-// at most 1, so no scaled operand can overflow whatever the gates.
+// Across sub-chunks A splits at p, the last token before t's sub-chunk: e^{c_t - c_p}
+// e^{c_p - c_m}, both factors at most 1, so no scaled operand can overflow whatever the gates.
+// Inside a 16-token sub-chunk it splits at the token before the sub-chunk when every channel's
+// decay over the sub-chunk is moderate, and takes the exponentials pair by pair otherwise.
 //
 // With a scalar gate the decay of a (t, m) pair is one number, so the head-wise kernel folds it
 // into a masked score matrix and runs every contraction on the tensor cores.  With a gate per
@@ -199,21 +200,61 @@ __global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
     if (tid < D) channel_cumsum(L, tid, cq, CQS);
     __syncthreads();
 
-    // A inside each sub-chunk: one warp per (t, m) pair, lanes over the channels.
-    for (int it = warp; it < (C / SC) * SC * SC; it += NT / 32) {
-        const int s = it / (SC * SC), tt = (it / SC) % SC, mm = it % SC;
-        const int t = s * SC + tt, m = s * SC + mm;
-        if (mm > tt || t >= L) continue;
-        float acc = 0.f;
-#pragma unroll
-        for (int u = 0; u < D / 32; ++u) {
-            const int i = lane + 32 * u;
-            acc += __bfloat162float(qs[t * D + i]) * __bfloat162float(kv[m * D + i]) *
-                   __expf(cq[t * CQS + i] - cq[m * CQS + i]);
+    // A inside each sub-chunk.  With r the token before the sub-chunk (c_r = 0 before the chunk),
+    // e^{c_t - c_m} = e^{c_t - c_r} e^{c_r - c_m}: the block is a dot product of scaled rows, as
+    // across sub-chunks.  The second factor exceeds 1, so the split is taken only while every
+    // channel's decay over the sub-chunk stays within SPAN_MAX (both factors then stay normal
+    // fp32 numbers); otherwise each pair takes its exponentials one by one.
+    constexpr float SPAN_MAX = 80.f;
+    for (int s = 0; s < C / SC && s * SC < L; ++s) {
+        const int r0 = s * SC, last = min(r0 + SC, L) - 1;
+        int wide = 0;
+        if (tid < D) {
+            const float cref = s == 0 ? 0.f : cq[(r0 - 1) * CQS + tid];
+            wide = cref - cq[last * CQS + tid] > SPAN_MAX;
         }
+        if (__syncthreads_or(wide)) {
+            // one warp per (t, m) pair, lanes over the channels
+            for (int it = warp; it < SC * SC; it += NT / 32) {
+                const int tt = it / SC, mm = it % SC;
+                const int t = r0 + tt, m = r0 + mm;
+                if (mm > tt || t >= L) continue;
+                float acc = 0.f;
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-        if (lane == 0) At[m * C + t] = a.k_scale * acc;
+                for (int u = 0; u < D / 32; ++u) {
+                    const int i = lane + 32 * u;
+                    acc += __bfloat162float(qs[t * D + i]) * __bfloat162float(kv[m * D + i]) *
+                           __expf(cq[t * CQS + i] - cq[m * CQS + i]);
+                }
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+                if (lane == 0) At[m * C + t] = a.k_scale * acc;
+            }
+        } else {
+            for (int e = tid; e < 2 * SC * D; e += NT) {
+                const int r = e / D, i = e - r * D;
+                const float cref = s == 0 ? 0.f : cq[(r0 - 1) * CQS + i];
+                const int t = r0 + (r < SC ? r : r - SC);
+                float val = 0.f;
+                if (t < L)
+                    val = r < SC ? __bfloat162float(qs[t * D + i]) * __expf(cq[t * CQS + i] - cref)
+                                 : __bfloat162float(kv[t * D + i]) * __expf(cref - cq[t * CQS + i]);
+                scr[r * SS + i] = val;
+            }
+            __syncthreads();
+            const int r = tid / SC, mm = tid % SC;
+            const float* qr = scr + r * SS;
+            const float* kr = scr + (SC + mm) * SS;
+            float acc = 0.f;
+#pragma unroll 8
+            for (int i = 0; i < D; i += 4) {
+                const float4 x = *reinterpret_cast<const float4*>(qr + i);
+                const float4 y = *reinterpret_cast<const float4*>(kr + i);
+                acc = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc))));
+            }
+            if (mm <= r && r0 + r < L) At[(r0 + mm) * C + r0 + r] = a.k_scale * acc;
+        }
+        __syncthreads();   // scr is reused by the next sub-chunk
     }
 
     // A across sub-chunks: rows of sub-chunk ts against columns of sub-chunk ms < ts, split at
