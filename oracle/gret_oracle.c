@@ -364,3 +364,50 @@ int oracle_gret_recurrent_ew(const double* q, const double* k, const double* v, 
     }
     return 0;
 }
+
+/*
+ * Sliding-window attention, the other Self-Decoder mixer of [P1] (section "路线一：滑动窗口注意力"):
+ * position i attends only to the most recent `window` positions of its own sequence, j in
+ * [i - window + 1, i], with softmax normalisation over exactly those positions:
+ *   o_i = sum_j softmax_j(scale * q_i . k_j) v_j
+ * (the page's formula and mask were stripped; the reading is the causal window mask that is 0
+ * inside the window and -inf outside, with the usual 1/sqrt(d) scale passed as `scale`).
+ * Layout: q, k [T][H][d], v, o [T][H][dv].  Returns 0, or -1 on bad offsets or window < 1.
+ */
+int oracle_swa(const double* q, const double* k, const double* v, double scale, int window,
+               int64_t T, int H, int d, int dv, const int64_t* cu_seqlens, int n_seqs,
+               double* o) {
+    if (check_seqs(cu_seqlens, n_seqs, T) || window < 1) return -1;
+    int64_t units = (int64_t)n_seqs * H;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t u = 0; u < units; ++u) {
+        int s = (int)(u / H), h = (int)(u % H);
+        int64_t a = cu_seqlens[s], e = cu_seqlens[s + 1];
+        double* w = (double*)malloc(sizeof(double) * (size_t)window);
+        for (int64_t i = a; i < e; ++i) {
+            int64_t j0 = i - window + 1 < a ? a : i - window + 1;
+            const double* qi = q + (i * H + h) * d;
+            double mx = -INFINITY;
+            for (int64_t j = j0; j <= i; ++j) {
+                const double* kj = k + (j * H + h) * d;
+                double sc = 0.0;
+                for (int c = 0; c < d; ++c) sc += qi[c] * kj[c];
+                w[j - j0] = scale * sc;
+                if (w[j - j0] > mx) mx = w[j - j0];
+            }
+            double den = 0.0;
+            for (int64_t j = j0; j <= i; ++j) {
+                w[j - j0] = exp(w[j - j0] - mx);
+                den += w[j - j0];
+            }
+            double* oi = o + (i * H + h) * dv;
+            for (int c = 0; c < dv; ++c) oi[c] = 0.0;
+            for (int64_t j = j0; j <= i; ++j) {
+                const double* vj = v + (j * H + h) * dv;
+                for (int c = 0; c < dv; ++c) oi[c] += (w[j - j0] / den) * vj[c];
+            }
+        }
+        free(w);
+    }
+    return 0;
+}

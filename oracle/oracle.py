@@ -44,6 +44,9 @@ def lib():
                                             ctypes.c_int, ctypes.c_int, ctypes.c_int, ip,
                                             ctypes.c_int64, dp]
         L.oracle_groupnorm_gate.restype = ctypes.c_int
+        L.oracle_swa.argtypes = [dp, dp, dp, ctypes.c_double, ctypes.c_int, ctypes.c_int64,
+                                 ctypes.c_int, ctypes.c_int, ctypes.c_int, ip, ctypes.c_int, dp]
+        L.oracle_swa.restype = ctypes.c_int
         L.oracle_log_gamma.argtypes = [ctypes.c_double, ctypes.c_double]
         L.oracle_log_gamma.restype = ctypes.c_double
         _lib = L
@@ -110,6 +113,24 @@ def gret_recurrent_ew(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_
     decays by sigmoid(g[..., i])^(1/tau).  Returns (o [T,H,dv], state [n_seqs,H,dk,dv])."""
     return _run("oracle_gret_recurrent_ew", q, k, v, g, tau, k_scale, cu_seqlens, state_in,
                 g_per_channel=True)
+
+
+def swa(q, k, v, window, scale=None, cu_seqlens=None):
+    """Sliding-window softmax attention ("路线一：滑动窗口注意力"): position i attends to the
+    last `window` positions of its sequence, j in [i - window + 1, i].  q, k [T, H, d],
+    v [T, H, dv]; scale defaults to d^-1/2.  Returns o [T, H, dv]."""
+    q, k, v = _d(q), _d(k), _d(v)
+    T, H, d = q.shape
+    dv = v.shape[2]
+    assert k.shape == (T, H, d) and v.shape == (T, H, dv)
+    cu = _cu(cu_seqlens, T)
+    o = np.zeros((T, H, dv))
+    rc = lib().oracle_swa(_p(q), _p(k), _p(v), float(d ** -0.5 if scale is None else scale),
+                          int(window), T, H, d, dv,
+                          cu.ctypes.data_as(ctypes.POINTER(ctypes.c_int64)), len(cu) - 1, _p(o))
+    if rc != 0:
+        raise ValueError("oracle_swa rejected its arguments (rc=%d)" % rc)
+    return o
 
 
 def gret_parallel(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None):

@@ -406,3 +406,66 @@ def test_ew_closed_gates_keep_current_token(oracle_mod):
     o_ref = 0.5 * np.einsum("thi,thi->th", q, k)[:, :, None] * v
     assert close(o, o_ref)
     assert close(s[0], 0.5 * np.einsum("hi,hj->hij", k[-1], v[-1]))
+
+
+# ---------------------------------------------------------------------------------------------
+# Sliding-window attention ("路线一：滑动窗口注意力"): position i sees positions i-C+1 .. i.
+
+def softmax_rows(s):
+    s = s - s.max(axis=-1, keepdims=True)
+    e = np.exp(s)
+    return e / e.sum(axis=-1, keepdims=True)
+
+
+@pytest.mark.parametrize("window", [1, 3, 7, 40])
+def test_swa_explicit_mask(oracle_mod, window):
+    """Against the matrix form softmax(scale Q K^T + B) V with the causal window mask B written
+    out (0 for i - C < j <= i, -inf elsewhere), per sequence, two sequences packed."""
+    rng = np.random.default_rng(50 + window)
+    T, H, d, dv = 29, 2, 8, 5
+    q, k, v = rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d)), \
+        rng.standard_normal((T, H, dv))
+    cu = [0, 12, T]
+    o = oracle_mod.swa(q, k, v, window, scale=0.3, cu_seqlens=cu)
+    ref = np.zeros_like(o)
+    for a, e in zip(cu[:-1], cu[1:]):
+        n = e - a
+        i, j = np.arange(n)[:, None], np.arange(n)[None, :]
+        B = np.where((j <= i) & (j > i - window), 0.0, -np.inf)
+        for h in range(H):
+            P = softmax_rows(0.3 * q[a:e, h] @ k[a:e, h].T + B)
+            ref[a:e, h] = P @ v[a:e, h]
+    assert close(o, ref)
+
+
+def test_swa_window_one_copies_v(oracle_mod):
+    rng = np.random.default_rng(60)
+    q, k, v = rng.standard_normal((10, 3, 4)), rng.standard_normal((10, 3, 4)), \
+        rng.standard_normal((10, 3, 6))
+    assert close(oracle_mod.swa(q, k, v, 1), v)
+
+
+def test_swa_wide_window_is_causal_attention(oracle_mod):
+    """A window at least the sequence length gives plain causal softmax attention, computed
+    here row by row with a running prefix (a different route from the mask matrix)."""
+    rng = np.random.default_rng(61)
+    T, H, d = 17, 2, 6
+    q, k, v = rng.standard_normal((T, H, d)), rng.standard_normal((T, H, d)), \
+        rng.standard_normal((T, H, d))
+    o = oracle_mod.swa(q, k, v, 1000)
+    ref = np.zeros_like(o)
+    for h in range(H):
+        for i in range(T):
+            w = np.exp(q[i, h] @ k[:i + 1, h].T / np.sqrt(d))
+            ref[i, h] = (w / w.sum()) @ v[:i + 1, h]
+    assert close(o, ref)
+
+
+def test_swa_zero_queries_average_the_window(oracle_mod):
+    """q = 0: every score is 0, so o_i is the plain mean of v over the window."""
+    rng = np.random.default_rng(62)
+    T, H, d, C = 23, 1, 4, 5
+    k, v = rng.standard_normal((T, H, d)), rng.standard_normal((T, H, 3))
+    o = oracle_mod.swa(np.zeros((T, H, d)), k, v, C)
+    ref = np.stack([v[max(0, i - C + 1):i + 1].mean(axis=0) for i in range(T)])
+    assert close(o, ref)
