@@ -296,6 +296,11 @@ def run_gpu(args):
     if not args.no_elementwise:
         ew = run_elementwise(args, rank, world, stream, ms_per_step)
 
+    # ---------------- sliding-window attention, the other Self-Decoder mixer, same shapes
+    swa = None
+    if not args.no_swa:
+        swa = run_swa(args, rank, world, stream, ms_per_step)
+
     # ---------------- one mixer layer: projection GEMM -> prefill -> GroupNorm * gate
     lay = None
     if not args.no_layer:
@@ -385,7 +390,7 @@ def run_gpu(args):
                      "kernel": "prefill_tc_kernel", "launch_ms": launch_ms,
                      "algorithmic_bytes_per_launch": alg_bytes},
         "decode": dec, "varlen_epilogue": epi, "layer": lay,
-        "elementwise_gate": ew, "e2e": e2e, "clocks": clk,
+        "elementwise_gate": ew, "sliding_window": swa, "e2e": e2e, "clocks": clk,
         "gpu_launches": args.steps,
         "cpu_baseline": cpu,
     }
@@ -516,6 +521,54 @@ def run_elementwise(args, rank, world, stream, headwise_ms):
                          "traffic": None,
                          "kernel": "ew_chunk_state + ew_state_scan + ew_chunk_output",
                          "algorithmic_flops_per_launch": flops}}
+
+
+def run_swa(args, rank, world, stream, headwise_ms):
+    """Sliding-window softmax attention (window 1024) on the 3B shapes, 32768 tokens x 24 heads
+    of 128, bf16: one launch per step.  FLOP counted algorithmically, 4 d per (query, visible
+    key) pair (Q K^T and P V)."""
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+    c = SI.SWA_32K
+    Bq, Nq, Hq, W = c["B"], c["N"], c["H"], c["window"]
+    inp = SI.gret_inputs(Bq, Nq, Hq, D, dtype=torch.bfloat16, seed=rank_seed(c["seed"], rank),
+                         device="cuda")
+    q = (inp["q"] * D ** 0.5).to(torch.bfloat16)
+    k = (inp["k"] * D ** 0.5).to(torch.bfloat16)
+    v = inp["v"]
+    del inp
+    o = torch.empty_like(q)
+
+    def step():
+        G.gret_swa_prefill(q, k, v, window=W, o=o)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 10))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    pairs = W * (W + 1) // 2 + (Nq - W) * W if Nq >= W else Nq * (Nq + 1) // 2
+    flops = 4.0 * D * pairs * Hq * Bq
+    tpeak, tkind = measured_tensor_peak()
+    ach = flops / (ms * 1e-3) / 1e12
+    return {"value": Bq * Nq * world / (ms * 1e-3) / 1e6, "unit": "Mtok/s", "tokens": Bq * Nq,
+            "heads": Hq, "window": W, "ms_per_step": ms, "steps": n, "gpu_launches_per_step": 1,
+            "gated_retention_ms_same_shapes": headwise_ms,
+            "l2": "q, k, v, o (805 MB) larger than L2; not flushed",
+            "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
+                         "frac": ach / tpeak, "peak_kind": tkind + " burst",
+                         "mma": "warp-level mma.sync m16n8k16 bf16", "traffic": None,
+                         "kernel": "swa_kernel", "algorithmic_flops_per_launch": flops}}
 
 
 def run_layer(args, rank, world, stream, hbm_peak):
@@ -656,6 +709,7 @@ def main():
     ap.add_argument("--no-epilogue", action="store_true")
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--no-elementwise", action="store_true")
+    ap.add_argument("--no-swa", action="store_true")
     ap.add_argument("--varlen-max-len", type=int, default=65536,
                     help="longest sequence of the varlen + epilogue leg (a smaller value gives "
                          "a small case for profiling)")

@@ -58,6 +58,8 @@ _lib.gret_prefill_elementwise.argtypes = [_vp, _vp, _vp, _vp, _f32, _f32, _i32, 
 _lib.gret_prefill_elementwise.restype = _i32
 _lib.gret_prefill_elementwise_workspace_size.argtypes = [_i32, _i64, _i32, _i32]
 _lib.gret_prefill_elementwise_workspace_size.restype = ctypes.c_size_t
+_lib.gret_swa_prefill.argtypes = [_vp, _vp, _vp, _f32, _i32, _i32, _i64, _i32, _i32, _vp, _vp]
+_lib.gret_swa_prefill.restype = _i32
 
 
 class GretError(RuntimeError):
@@ -275,6 +277,22 @@ def gret_prefill_elementwise(q, k, v, g, tau=16.0, k_scale=1.0, state_in=None, s
         _ptr(state_out), _ptr(o), _ptr(workspace), workspace.numel() * workspace.element_size(),
         _stream(stream)))
     return o, state_out
+
+
+def gret_swa_prefill(q, k, v, window=1024, scale=None, o=None, stream=None):
+    """Sliding-window softmax attention: position i attends to the last `window` positions of
+    its sequence.  q, k, v [B, N, H, 128] bf16 contiguous; scale defaults to d^-1/2.
+    Returns o [B, N, H, 128] bf16."""
+    B, N, H, d = q.shape
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != (B, N, H, d):
+            raise ValueError("q, k, v must be contiguous bfloat16 [B, N, H, d]")
+    if o is None:
+        o = torch.empty_like(q)
+    _check("gret_swa_prefill", _lib.gret_swa_prefill(
+        _ptr(q), _ptr(k), _ptr(v), d ** -0.5 if scale is None else scale, window, B, N, H, d,
+        _ptr(o), _stream(stream)))
+    return o
 
 
 def gret_layer_forward(x, w_qkvg, w_g, H, d=128, cu_seqlens=None, state_in=None, tau=16.0,

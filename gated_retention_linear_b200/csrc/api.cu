@@ -9,6 +9,7 @@
 #include "prefill_tc.cuh"
 #include "gn_gate.cuh"
 #include "prefill_ew.cuh"
+#include "swa.cuh"
 
 using namespace gret;
 
@@ -214,6 +215,26 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
     a.ws_S = static_cast<float*>(workspace);
     a.ws_a = a.ws_S + (size_t)B * H * nch * EW_DIM * EW_DIM;
     return launch_prefill_ew(a, s) == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, float scale,
+                               int window, int B, int64_t N, int H, int d, void* o,
+                               gret_stream_t stream) {
+    if (B < 0 || N < 0 || H < 1 || d < 1 || window < 1 || !isfinite(scale))
+        return GRET_ERR_INVALID_ARG;
+    if (d != SWA_DIM) return GRET_ERR_UNSUPPORTED;
+    if (B > 65535 || H > 65535 || (N + 63) / 64 > 0x7fffffff) return GRET_ERR_UNSUPPORTED;
+    if (B == 0 || N == 0) return GRET_OK;
+    if (!q || !k || !v || !o) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return GRET_ERR_ALIGNMENT;
+    SwaArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.o = static_cast<__nv_bfloat16*>(o);
+    a.scale = scale; a.window = window;
+    a.B = B; a.N = N; a.H = H;
+    return launch_swa(a, (cudaStream_t)stream) == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
 }  // extern "C"

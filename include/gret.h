@@ -218,6 +218,21 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
  * Returns 0 on invalid sizes or d != 128. */
 size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d);
 
+/*
+ * Sliding-window attention prefill, the other Self-Decoder mixer ("路线一：滑动窗口注意力"):
+ * position i attends to the most recent `window` positions of its sequence, itself included,
+ * with softmax over exactly those:
+ *   o_i = sum_{j = max(0, i-window+1) .. i} softmax_j(scale * q_i . k_j) v_j
+ *   q, k, v, o  bf16 [B, N, H, d] contiguous (token-major); each batch row is one sequence.
+ *   scale       score scale (d^-1/2 in the usual reading); window >= 1 (the page's 1024).
+ * bf16 tensor-core products with fp32 accumulation and an fp32 online softmax; o rounded to
+ * bf16 once.  Requires d == 128, B <= 65535, H <= 65535; q, k, v, o 16-byte aligned
+ * (GRET_ERR_ALIGNMENT otherwise).  o must not overlap the inputs.
+ */
+gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, float scale,
+                               int window, int B, int64_t N, int H, int d, void* o,
+                               gret_stream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

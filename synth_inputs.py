@@ -123,6 +123,7 @@ PREFILL_512K = dict(B=1, N=524288, H=24, dk=128, dtype=torch.bfloat16, g_mean=2.
                     seed=3)
 DECODE_BS64 = dict(B=64, prefill_N=4096, steps=256, H=24, dk=128, dtype=torch.bfloat16,
                    g_mean=2.0, g_std=1.0, seed=4)
+SWA_32K = dict(B=1, N=32768, H=24, dk=128, window=1024, seed=8)
 ELEMENTWISE_32K = dict(B=1, N=32768, H=24, dk=128, g_mean=2.0, g_std=1.0, seed=7)
 LAYER_32K = dict(T=32768, D=3072, H=24, dk=128, seed=6)
 VARLEN_EPILOGUE = dict(n_seqs=8, lo=1024, hi=65536, H=24, dk=128, dtype=torch.bfloat16,
