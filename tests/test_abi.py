@@ -87,3 +87,69 @@ def test_decode_and_epilogue_reject_bad_arguments():
     assert lib.gret_groupnorm_gate(*bad) == 0
     bad = list(ep); bad[5] = -1.0
     assert lib.gret_groupnorm_gate(*bad) == 1
+
+
+def test_projection_rejects_bad_arguments_without_launching():
+    import gated_retention_linear_b200 as G
+    lib = G._lib
+
+    def call(**kw):
+        a = dict(x=1024, w=2048, ldw=3 * 2 * 128 + 2 + 6, T=16, H=2, d=128, D=128, q=4096,
+                 k=8192, v=12288, g=16384, stream=None)
+        a.update(kw)
+        return lib.gret_qkvg_projection(*a.values())
+    assert call(ldw=3 * 2 * 128 + 1) == 1     # fewer columns than W_Q, W_K, W_V, W_gamma need
+    assert call(H=0) == 1
+    assert call(T=-1) == 1
+    assert call(d=64, ldw=400) == 2           # only d = 128 has a kernel
+    assert call(H=129, ldw=3 * 129 * 128 + 129 + 7) == 2
+    assert call(D=96) == 2                    # D must be a multiple of 64
+    assert call(T=0) == 0                     # nothing to do
+    assert call(x=None) == 1
+    assert call(x=1026) == 3                  # not 16-byte aligned
+    assert call(ldw=3 * 2 * 128 + 2 + 1) == 3 # rows would not start 16-byte aligned
+    assert call(g=16386) == 3
+
+
+def test_elementwise_prefill_rejects_bad_arguments_without_launching():
+    import gated_retention_linear_b200 as G
+    lib = G._lib
+    assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 128) == (128 * 128 + 128) * 4
+    assert G.gret_prefill_elementwise_workspace_size(1, 65, 2, 128) == 2 * 2 * (128 * 128 + 128) * 4
+    assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 64) == 0
+
+    def call(**kw):
+        a = dict(q=1024, k=2048, v=4096, g=8192, tau=16.0, ks=1.0, B=1, N=64, H=1, d=128,
+                 sin=None, sout=None, o=16384, ws=1 << 20, wsb=1 << 20, stream=None)
+        a.update(kw)
+        return lib.gret_prefill_elementwise(*a.values())
+    assert call(d=64) == 2
+    assert call(H=0) == 1
+    assert call(tau=0.0) == 1
+    assert call(ks=float("inf")) == 1
+    assert call(B=0) == 0
+    assert call(N=0) == 0                     # no tokens and no state to write
+    assert call(q=None) == 1
+    assert call(q=1030) == 3
+    assert call(sin=1028) == 3
+    assert call(wsb=1000) == 4                # workspace smaller than the size query says
+    assert call(ws=None) == 4
+
+
+def test_swa_rejects_bad_arguments_without_launching():
+    import gated_retention_linear_b200 as G
+    lib = G._lib
+
+    def call(**kw):
+        a = dict(q=1024, k=2048, v=4096, scale=0.088, W=1024, B=1, N=64, H=2, d=128, o=8192,
+                 stream=None)
+        a.update(kw)
+        return lib.gret_swa_prefill(*a.values())
+    assert call(W=0) == 1
+    assert call(scale=float("nan")) == 1
+    assert call(H=0) == 1
+    assert call(d=64) == 2
+    assert call(B=0) == 0
+    assert call(N=0) == 0
+    assert call(o=None) == 1
+    assert call(v=4100) == 3
