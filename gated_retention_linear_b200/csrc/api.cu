@@ -172,8 +172,18 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
     return launch_qkvg_projection(x, w, ldw, T, H, D, q, k, v, g, (cudaStream_t)stream);
 }
 
+// Sizes the per-channel gate prefill can take: the scan's grid (B * H * 16 blocks) fits in
+// gridDim.x and the workspace byte count fits in size_t.
+bool ew_sizes_ok(int B, int64_t N, int H) {
+    const int64_t nch = (N + EW_CHUNK - 1) / EW_CHUNK;
+    if (B > 65535 || H > 65535 || nch > 0x7fffffff) return false;
+    if ((int64_t)B * H * 16 > 0x7fffffff) return false;
+    const double bytes = (double)B * H * (double)nch * (EW_DIM * EW_DIM + EW_DIM) * 4.0;
+    return bytes < 9.0e18;
+}
+
 size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d) {
-    if (B < 0 || N < 0 || H < 1 || d != EW_DIM) return 0;
+    if (B < 0 || N < 0 || H < 1 || d != EW_DIM || !ew_sizes_ok(B, N, H)) return 0;
     return ew_workspace_bytes(B, N, H);
 }
 
@@ -186,7 +196,7 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
     if (d != EW_DIM) return GRET_ERR_UNSUPPORTED;
     const int64_t nch = (N + EW_CHUNK - 1) / EW_CHUNK;
-    if (B > 65535 || H > 65535 || nch > 0x7fffffff) return GRET_ERR_UNSUPPORTED;
+    if (!ew_sizes_ok(B, N, H)) return GRET_ERR_UNSUPPORTED;
     if (B == 0) return GRET_OK;
     if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
         return GRET_ERR_ALIGNMENT;

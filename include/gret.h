@@ -204,7 +204,8 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
  *               bytes, 16-byte aligned, owned by the caller; its contents on entry do not
  *               matter and are overwritten.
  * Runs on CUDA cores in fp32 (three launches: chunk states, a scan over chunks, chunk
- * outputs).  Requires d == 128, B <= 65535, H <= 65535; q, k, v, g, o and the states 16-byte
+ * outputs).  Requires d == 128, B <= 65535, H <= 65535, B * H * 16 < 2^31 and a workspace size
+ * below 9e18 bytes (GRET_ERR_UNSUPPORTED otherwise); q, k, v, g, o and the states 16-byte
  * aligned (GRET_ERR_ALIGNMENT otherwise).  N == 0 copies state_in (or zeros) to state_out.
  * o must not overlap the inputs.
  */
@@ -215,7 +216,7 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
                                        size_t workspace_bytes, gret_stream_t stream);
 
 /* Workspace bytes gret_prefill_elementwise needs: B * H * ceil(N / 64) * (d*d + d) * 4.
- * Returns 0 on invalid sizes or d != 128. */
+ * Returns 0 on invalid or unsupported sizes (d != 128 among them). */
 size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d);
 
 /*

@@ -117,6 +117,7 @@ def test_elementwise_prefill_rejects_bad_arguments_without_launching():
     assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 128) == (128 * 128 + 128) * 4
     assert G.gret_prefill_elementwise_workspace_size(1, 65, 2, 128) == 2 * 2 * (128 * 128 + 128) * 4
     assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 64) == 0
+    assert G.gret_prefill_elementwise_workspace_size(65535, 1 << 40, 65535, 128) == 0
 
     def call(**kw):
         a = dict(q=1024, k=2048, v=4096, g=8192, tau=16.0, ks=1.0, B=1, N=64, H=1, d=128,
@@ -134,6 +135,8 @@ def test_elementwise_prefill_rejects_bad_arguments_without_launching():
     assert call(sin=1028) == 3
     assert call(wsb=1000) == 4                # workspace smaller than the size query says
     assert call(ws=None) == 4
+    assert call(B=65535, H=65535) == 2       # the scan's grid would not fit
+    assert call(B=4, H=65535, N=64 << 30) == 2    # workspace bytes past 9e18
 
 
 def test_swa_rejects_bad_arguments_without_launching():
