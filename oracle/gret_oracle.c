@@ -20,13 +20,20 @@
  *        - section "单 token Decode 的实现骨架": the decode update multiplies the old state by
  *          exp(gate) and adds outer(k, v); the gate logit is divided by 16; K is scaled by
  *          d_h^{-1/2}.
+ *        - section "路线一：滑动窗口注意力": the other Self-Decoder mixer, softmax attention in
+ *          which position i sees only the most recent C positions (C = 1024 in the page's
+ *          scaling runs).
+ *        - the same "路线二" section weighs an element-wise gate against the head-wise one.
  *   The display formulas of [P1] were stripped when the page was extracted to text; the
  *   readings taken where the page is silent are listed with each function.
  *
  * Parity pins (tests/test_oracle_pins.py): brute-force parallel form, gamma==1 (causal linear
  * attention), gamma==0 (current token only), a hand-worked example in tests/golden/, chunkwise
  * re-association at many chunk sizes, split prefill, decode-after-prefill, linearity, and the
- * GroupNorm moments.
+ * GroupNorm moments; for the per-channel gate, reduction to the head-wise recurrence, the
+ * brute-force product form, a one-hot query row and closed gates; for sliding-window
+ * attention, the explicit-mask matrix form, window 1, a wide window against causal attention
+ * and zero queries.
  *
  * Layout used by every function here (the test harness converts to it):
  *   q, k  : [T][H][dk]   (token-major, contiguous, fp64)
