@@ -19,7 +19,8 @@
 // With a scalar gate the decay of a (t, m) pair is one number, so the head-wise kernel folds it
 // into a masked score matrix and runs every contraction on the tensor cores.  With a gate per
 // channel the decay sits inside the contraction over i; this path pays for that with the
-// chunk-state round trip through the workspace and with per-pair exponentials.
+// chunk-state round trip through the workspace and with an exponential per channel for every
+// scaled operand (per pair and channel when a sub-chunk's gates are extreme).
 #include <cuda_bf16.h>
 #include <stdint.h>
 
