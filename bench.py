@@ -384,21 +384,53 @@ def run_gpu(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": bench_config(world),
+        "decode": dec, "varlen_epilogue": epi, "layer": lay,
+        "elementwise_gate": ew, "sliding_window": swa,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "traffic": prefill_traffic_from_profile(),
                      "kernel": "prefill_tc_kernel", "launch_ms": launch_ms,
                      "algorithmic_bytes_per_launch": alg_bytes},
-        "decode": dec, "varlen_epilogue": epi, "layer": lay,
-        "elementwise_gate": ew, "sliding_window": swa, "e2e": e2e, "clocks": clk,
-        "gpu_launches": args.steps,
-        "cpu_baseline": cpu,
+        "e2e": e2e, "clocks": clk, "gpu_launches": args.steps, "cpu_baseline": cpu,
+        # last, so that a record which keeps only the end of the line still has every leg
+        "legs": legs_summary(dec, epi, lay, ew, swa),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
         dist.destroy_process_group()
+
+
+def legs_summary(dec, epi, lay, ew, swa):
+    """value, unit and roofline fraction of every secondary leg, rounded, in a few hundred
+    characters."""
+    def r(x, n=4):
+        return None if x is None else float("%.*g" % (n, x))
+    out = {}
+    if dec:
+        out["decode"] = {"v": r(dec["value"]), "u": dec["unit"], "ms": r(dec["ms_per_step"]),
+                         "hbm_frac": r(dec["roofline"]["frac"], 3)}
+    if epi:
+        out["varlen_epilogue"] = {"v": r(epi["value"]), "u": epi["unit"],
+                                  "prefill_hbm_frac": r(epi["prefill_roofline"]["frac"], 3),
+                                  "gemm_tensor_frac": r(epi["roofline"]["frac"], 3)}
+    if lay:
+        out["layer"] = {"v": r(lay["value"]), "u": lay["unit"],
+                        "proj_tensor_frac": r(lay["roofline"]["frac"], 3),
+                        "prefill_hbm_frac": r(lay["prefill_roofline"]["frac"], 3),
+                        "gate_tensor_frac": r(lay["gate_roofline"]["frac"], 3)}
+    if swa:
+        out["sliding_window"] = {"v": r(swa["value"]), "u": swa["unit"],
+                                 "tensor_frac": r(swa["roofline"]["frac"], 3)}
+        if swa.get("decode"):
+            out["sliding_window"]["decode_hbm_frac"] = r(swa["decode"]["roofline"]["frac"], 3)
+    if ew:
+        out["elementwise_gate"] = {"v": r(ew["value"]), "u": ew["unit"],
+                                   "frac": r(ew["roofline"]["frac"], 3),
+                                   "bound": ew["roofline"]["bound"],
+                                   "x_headwise": r(ew["slowdown_vs_headwise"], 3)}
+    return out
 
 
 def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
@@ -658,8 +690,7 @@ def cpu_baseline(q, k, v, g, n_tokens, min_seconds=8.0, max_reps=8):
         reps += 1
     return {"value": n * reps / dt / 1e6, "unit": "Mtok/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": "first %d of 32768 tokens, all 24 heads, fp64 recurrent oracle (OpenMP over "
-                      "heads), %d passes, %.1f s wall" % (n, reps, dt)}
+            "sample": "%d tokens x 24 heads, fp64 recurrent oracle, %d passes, %.1f s" % (n, reps, dt)}
 
 
 def run_reference(args):

@@ -42,6 +42,8 @@ _lib.gret_prefill_chunkwise_noalloc.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp,
                                                 _i32, _vp, _i32, _vp, _vp, _vp, _i64, _i64, _i64,
                                                 _i32, _vp]
 _lib.gret_prefill_chunkwise_noalloc.restype = _i32
+_lib.gret_prefill_noalloc_status.argtypes = [_vp]
+_lib.gret_prefill_noalloc_status.restype = _i32
 _lib.gret_workspace_status.argtypes = [_vp, _vp]
 _lib.gret_workspace_status.restype = _i32
 _lib.gret_decode_step.argtypes = [_vp, _vp, _vp, _vp, _f32, _f32, _i32, _i32, _i32, _i32, _i32,
@@ -112,15 +114,9 @@ def _layout(t, head_major):
     return t.stride(0), t.stride(1), t.stride(2)
 
 
-def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None,
-                           state_out=None, o=None, chunk=0, head_major=False, workspace=None,
-                           stream=None):
-    """Chunkwise gated-retention prefill through the C ABI.
-
-    q, k [B,N,H,dk] (head_major=False) or [B,H,N,dk] (head_major=True); v likewise with dv;
-    packed varlen: q, k, v [T,H,d] with cu_seqlens int32 [n_seqs+1] on the device.
-    g fp32 [B,N,H] or [T,H].  state_in / state_out fp32 [units,H,dk,dv] (state_out=True
-    allocates one).  Returns (o, state_out)."""
+def _prefill_args(q, k, v, g, cu_seqlens, state_out, o, head_major):
+    """Shapes, strides and checks shared by both prefill wrappers.  Returns a dict of the C
+    arguments (sizes and strides) plus the (possibly allocated) o and state_out."""
     if k.stride() != q.stride():
         raise ValueError("q and k must share strides")
     if q.dim() == 3:
@@ -145,17 +141,32 @@ def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, s
     units = n_seqs if cu_seqlens is not None else B
     if state_out is True:
         state_out = torch.empty((units, H, dk, dv), dtype=torch.float32, device=q.device)
-    code = _dtype_code(q)
-    total = N if cu_seqlens is not None else B * N
-    need = int(_lib.gret_prefill_workspace_size(code, total, units, H, dk, dv, chunk))
+    return dict(B=B, N=N, H=H, dk=dk, dv=dv, sb=sb, st=st, sh=sh, vsb=vsb, vst=vst, vsh=vsh,
+                osb=osb, ost=ost, osh=osh, n_seqs=n_seqs, units=units, code=_dtype_code(q),
+                total=N if cu_seqlens is not None else B * N, o=o, state_out=state_out)
+
+
+def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, state_in=None,
+                           state_out=None, o=None, chunk=0, head_major=False, workspace=None,
+                           stream=None):
+    """Chunkwise gated-retention prefill through the C ABI.
+
+    q, k [B,N,H,dk] (head_major=False) or [B,H,N,dk] (head_major=True); v likewise with dv;
+    packed varlen: q, k, v [T,H,d] with cu_seqlens int32 [n_seqs+1] on the device.
+    g fp32 [B,N,H] or [T,H].  state_in / state_out fp32 [units,H,dk,dv] (state_out=True
+    allocates one).  Returns (o, state_out)."""
+    a = _prefill_args(q, k, v, g, cu_seqlens, state_out, o, head_major)
+    o, state_out = a["o"], a["state_out"]
+    need = int(_lib.gret_prefill_workspace_size(a["code"], a["total"], a["units"], a["H"],
+                                                a["dk"], a["dv"], chunk))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=q.device)
     wbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     _check("gret_prefill_chunkwise", _lib.gret_prefill_chunkwise(
-        _ptr(q), _ptr(k), sb, st, sh, _ptr(v), vsb, vst, vsh, _ptr(g), tau, k_scale, code, B,
-        N, H, dk, dv,
-        _ptr(cu_seqlens), n_seqs, _ptr(state_in), _ptr(state_out), _ptr(o), osb, ost, osh,
-        chunk, _ptr(workspace), wbytes, _stream(stream)))
+        _ptr(q), _ptr(k), a["sb"], a["st"], a["sh"], _ptr(v), a["vsb"], a["vst"], a["vsh"],
+        _ptr(g), tau, k_scale, a["code"], a["B"], a["N"], a["H"], a["dk"], a["dv"],
+        _ptr(cu_seqlens), a["n_seqs"], _ptr(state_in), _ptr(state_out), _ptr(o), a["osb"],
+        a["ost"], a["osh"], chunk, _ptr(workspace), wbytes, _stream(stream)))
     return o, state_out
 
 
@@ -164,32 +175,23 @@ def gret_prefill_chunkwise_noalloc(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens
                                    head_major=False, stream=None):
     """gret_prefill_chunkwise through the entry point that needs no workspace and allocates no
     device memory (its scratch is a fixed 8 MiB array inside the library; calls that overlap
-    on the GPU race).  Same arguments and results as gret_prefill_chunkwise; `o` and
+    on the GPU race).  Same arguments, checks and results as gret_prefill_chunkwise; `o` and
     `state_out=True` are allocated here by torch for convenience, so pass them in to allocate
-    nothing at call time."""
-    if k.stride() != q.stride():
-        raise ValueError("q and k must share strides")
-    if q.dim() == 3:
-        B, (N, H, dk) = 1, q.shape
-    elif head_major:
-        B, H, N, dk = q.shape
-    else:
-        B, N, H, dk = q.shape
-    dv = v.shape[-1]
-    sb, st, sh = _layout(q, head_major)
-    vsb, vst, vsh = _layout(v, head_major)
-    if o is None:
-        o = torch.empty(q.shape[:-1] + (dv,), dtype=q.dtype, device=q.device)
-    osb, ost, osh = _layout(o, head_major)
-    n_seqs = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
-    units = n_seqs if cu_seqlens is not None else B
-    if state_out is True:
-        state_out = torch.empty((units, H, dk, dv), dtype=torch.float32, device=q.device)
+    nothing at call time.  gret_prefill_noalloc_status() reports a timed-out wait."""
+    a = _prefill_args(q, k, v, g, cu_seqlens, state_out, o, head_major)
+    o, state_out = a["o"], a["state_out"]
     _check("gret_prefill_chunkwise_noalloc", _lib.gret_prefill_chunkwise_noalloc(
-        _ptr(q), _ptr(k), sb, st, sh, _ptr(v), vsb, vst, vsh, _ptr(g), tau, k_scale,
-        _dtype_code(q), B, N, H, dk, dv, _ptr(cu_seqlens), n_seqs, _ptr(state_in),
-        _ptr(state_out), _ptr(o), osb, ost, osh, chunk, _stream(stream)))
+        _ptr(q), _ptr(k), a["sb"], a["st"], a["sh"], _ptr(v), a["vsb"], a["vst"], a["vsh"],
+        _ptr(g), tau, k_scale, a["code"], a["B"], a["N"], a["H"], a["dk"], a["dv"],
+        _ptr(cu_seqlens), a["n_seqs"], _ptr(state_in), _ptr(state_out), _ptr(o), a["osb"],
+        a["ost"], a["osh"], chunk, _stream(stream)))
     return o, state_out
+
+
+def gret_prefill_noalloc_status(stream=None):
+    """Synchronise and return the status of the latest allocation-free prefill on the current
+    device (0 = OK, 6 = a bounded wait gave up)."""
+    return int(_lib.gret_prefill_noalloc_status(_stream(stream)))
 
 
 def gret_workspace_status(workspace, stream=None):

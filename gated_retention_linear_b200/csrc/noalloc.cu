@@ -22,7 +22,9 @@ constexpr int MAX_DEVICES = 64;
 std::mutex g_mu;
 void* g_ptr[MAX_DEVICES];
 
-// Address of the scratch on the current device, looked up once per device.
+// Address of the scratch on the current device, looked up once per device and kept for the life
+// of the process (a cudaDeviceReset after the first call is therefore not supported: the cached
+// address would then be stale).
 cudaError_t scratch_address(void** out) {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -61,4 +63,18 @@ extern "C" gret_status_t gret_prefill_chunkwise_noalloc(
                                   d_k, d_v, cu_seqlens, n_seqs, state_in, state_out, o,
                                   o_stride_batch, o_stride_tok, o_stride_head, chunk, scratch,
                                   need > 0 ? NOALLOC_SCRATCH_BYTES : 0, stream);
+}
+
+extern "C" gret_status_t gret_prefill_noalloc_status(gret_stream_t stream) {
+    if (cudaStreamSynchronize((cudaStream_t)stream) != cudaSuccess) return GRET_ERR_CUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= MAX_DEVICES) return GRET_ERR_CUDA;
+    void* ptr = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_mu);
+        ptr = g_ptr[dev];
+    }
+    if (!ptr) return GRET_OK;   // no call on this device has used the scratch yet
+    // the error word sits at the start of the scratch, as at the start of every workspace
+    return gret_workspace_status(ptr, stream);
 }

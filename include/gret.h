@@ -123,8 +123,11 @@ gret_status_t gret_prefill_chunkwise(
  *   - Every call shares the one scratch array: calls that overlap on the GPU (other streams, or
  *     other host threads using the same device) race and give wrong results.  The call clears
  *     what must start at zero itself; the array keeps the previous call's contents otherwise.
- *   - The bounded-wait error word lives in the private scratch, so a timed-out wait is not
- *     reported to the caller of this variant.
+ *   - A bounded wait that gives up records GRET_ERR_TIMEOUT in the scratch, where
+ *     gret_prefill_noalloc_status() reads it.  Each call clears the word first, so the status
+ *     describes the latest call on the device.
+ *   - The scratch's device address is kept for the life of the process: calling
+ *     cudaDeviceReset after this entry point has run on a device is not supported.
  */
 gret_status_t gret_prefill_chunkwise_noalloc(
     const void* q, const void* k, int64_t stride_batch, int64_t stride_tok, int64_t stride_head,
@@ -133,6 +136,15 @@ gret_status_t gret_prefill_chunkwise_noalloc(
     int64_t N, int H, int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
     const float* state_in, float* state_out, void* o, int64_t o_stride_batch,
     int64_t o_stride_tok, int64_t o_stride_head, int chunk, gret_stream_t stream);
+
+/*
+ * Status of the latest gret_prefill_chunkwise_noalloc call on the current device: synchronises
+ * `stream` (use the stream that call ran on), then reads the error word of the library's static
+ * scratch.  Returns GRET_OK (also when no call has used the scratch yet), GRET_ERR_TIMEOUT if a
+ * bounded wait of that call gave up (its results are invalid), or GRET_ERR_CUDA.  Blocking; not
+ * for use inside stream capture.  Allocates nothing.  The paper has no counterpart.
+ */
+gret_status_t gret_prefill_noalloc_status(gret_stream_t stream);
 
 /*
  * Synchronises `stream`, then reads the error word that gret_prefill_chunkwise keeps at the

@@ -7,6 +7,16 @@ import synth_inputs as SI
 from oracle import oracle
 from parity import assert_parity
 
+# The tensor-core prefill (bf16, d_k = d_v = 128, chunk 128) carries P, the state copy and the
+# weighted keys as bf16 high + low pairs, which keeps its error near 1e-5 of rms against the
+# fp64 oracle.  This second bar, far below the 1e-2 parity bar, catches a regression of that
+# precision (one dropped low half alone costs about 1e-2).
+TC_TIGHT = 1e-3
+
+
+def tc_path(dtype, dk, dv, chunk):
+    return dtype == torch.bfloat16 and dk == 128 and dv == 128 and chunk in (0, 128)
+
 
 def lib():
     import gated_retention_linear_b200 as G
@@ -40,8 +50,9 @@ def run_dense(B, N, H, dk, dv, dtype, chunk=0, g_mean=2.0, g_std=1.0, seed=0,
         k_scale=k_scale, cu_seqlens=cu, state_in=inp.get("s"))
     bf16 = dtype == torch.bfloat16
     tol = tol if tol is not None else (1e-2 if bf16 else 1e-4)
-    eo = assert_parity("o", token_major(o, head_major), o_ref, tol, stored_bf16=bf16)
-    es = assert_parity("state", s, s_ref, tol, stored_bf16=False)
+    tight = TC_TIGHT if tc_path(dtype, dk, dv, chunk) else None
+    eo = assert_parity("o", token_major(o, head_major), o_ref, tol, stored_bf16=bf16, tight=tight)
+    es = assert_parity("state", s, s_ref, tol, stored_bf16=False, tight=tight)
     return eo, es
 
 
@@ -64,6 +75,7 @@ def run_varlen(lengths, H, dk, dv, dtype, chunk=0, g_mean=0.0, g_std=2.0, seed=0
     o_ref, s_ref = oracle.gret_recurrent(q, k, v, g, cu_seqlens=cu, state_in=s0)
     bf16 = dtype == torch.bfloat16
     tol = tol if tol is not None else (1e-2 if bf16 else 1e-4)
-    eo = assert_parity("o", o, o_ref, tol, stored_bf16=bf16)
-    es = assert_parity("state", s, s_ref, tol, stored_bf16=False)
+    tight = TC_TIGHT if tc_path(dtype, dk, dv, chunk) else None
+    eo = assert_parity("o", o, o_ref, tol, stored_bf16=bf16, tight=tight)
+    es = assert_parity("state", s, s_ref, tol, stored_bf16=False, tight=tight)
     return eo, es

@@ -96,13 +96,27 @@ def test_handworked_matrix_recurrence_with_entry_state(oracle_mod):
         assert np.allclose(a, b, atol=1e-14)
 
 
-def test_state_size_matches_page_count():
-    """The page's 3B hand count: 13 Self layers x 24 heads x 128x128 state, bf16 -> 9.75 MiB."""
+def test_state_size_matches_page_count(oracle_mod):
+    """The page's 3B hand count: 13 Self layers x 24 heads x 128x128 state, bf16 -> 9.75 MiB.
+
+    The oracle is run on one token of one request with the page's head count and widths; the
+    state it returns must hold exactly heads x d_k x d_v numbers, so that 13 such states in bf16
+    come to the page's figure.  A state of another shape (a missing head axis, d_k x d_k, an
+    extra per-token axis) fails the count."""
     with open(os.path.join(GOLDEN, "state_size_3b.json")) as f:
         gold = json.load(f)
-    per_layer = gold["heads"] * gold["d_k"] * gold["d_v"]          # one [H, dk, dv] state
-    mib = gold["self_layers"] * per_layer * gold["bytes_per_elem"] / 2**20
+    H, dk, dv = gold["heads"], gold["d_k"], gold["d_v"]
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((1, H, dk))
+    k = rng.standard_normal((1, H, dk))
+    v = rng.standard_normal((1, H, dv))
+    g = rng.standard_normal((1, H))
+    _, s = oracle_mod.gret_recurrent(q, k, v, g)
+    assert s.shape == (1, H, dk, dv)
+    mib = gold["self_layers"] * s[0].size * gold["bytes_per_elem"] / 2**20
     assert mib == pytest.approx(gold["mib_per_request"], abs=0.005)
+    # with one token from a zero state the state is exactly the first outer product k^T v
+    assert np.allclose(s[0], np.einsum("hi,hj->hij", k[0], v[0]), rtol=0, atol=1e-12)
 
 
 # ---------------------------------------------------------------------------------------------

@@ -6,7 +6,7 @@ import pytest
 import torch
 
 import synth_inputs as SI
-from gpu_cases import lib, run_dense, run_varlen
+from gpu_cases import TC_TIGHT, lib, run_dense, run_varlen
 from oracle import oracle
 from parity import assert_parity
 
@@ -73,7 +73,7 @@ def test_strided_fused_qkv_and_separate_output():
     G.gret_prefill_chunkwise(q, k, v, inp["g"][0].cuda(), cu_seqlens=cu, o=o, state_out=True)
     torch.cuda.synchronize()
     o_ref, _ = oracle.gret_recurrent(inp["q"][0], inp["k"][0], inp["v"][0], inp["g"][0])
-    assert_parity("o", o, o_ref, 1e-2, stored_bf16=True)
+    assert_parity("o", o, o_ref, 1e-2, stored_bf16=True, tight=TC_TIGHT)
     assert torch.count_nonzero(o_store[:, H]) == 0          # the padding column is untouched
 
 
@@ -117,8 +117,8 @@ def test_repeated_multi_span_calls_into_poisoned_output(N):
         _, s = G.gret_prefill_chunkwise(d["q"], d["k"], d["v"], d["g"], state_in=d["s"],
                                         state_out=True, o=o)
         torch.cuda.synchronize()
-        assert_parity("o", o[0], o_ref, 1e-2, stored_bf16=True)
-        assert_parity("state", s, s_ref, 1e-2, stored_bf16=False)
+        assert_parity("o", o[0], o_ref, 1e-2, stored_bf16=True, tight=TC_TIGHT)
+        assert_parity("state", s, s_ref, 1e-2, stored_bf16=False, tight=TC_TIGHT)
 
 
 def _sampled_heads(B, N, H, seed, heads, g_mean=2.0, g_std=1.0):
@@ -134,8 +134,8 @@ def _sampled_heads(B, N, H, seed, heads, g_mean=2.0, g_std=1.0):
     o_ref, s_ref = oracle.gret_recurrent(sel(inp["q"]), sel(inp["k"]), sel(inp["v"]),
                                          inp["g"].reshape(T, H)[:, hs].cpu(),
                                          cu_seqlens=np.arange(B + 1) * N)
-    assert_parity("o", sel(o), o_ref, 1e-2, stored_bf16=True)
-    assert_parity("state", s[:, hs], s_ref, 1e-2, stored_bf16=False)
+    assert_parity("o", sel(o), o_ref, 1e-2, stored_bf16=True, tight=TC_TIGHT)
+    assert_parity("state", s[:, hs], s_ref, 1e-2, stored_bf16=False, tight=TC_TIGHT)
 
 
 def test_prefill_32k_3b_shape_sampled_heads():
@@ -162,5 +162,5 @@ def test_varlen_8_sequences_harsh_gates_sampled_heads():
     hs = [3, 17]
     o_ref, s_ref = oracle.gret_recurrent(q[:, hs].cpu(), k[:, hs].cpu(), v[:, hs].cpu(),
                                          g[:, hs].cpu(), cu_seqlens=cu)
-    assert_parity("o", o[:, hs], o_ref, 1e-2, stored_bf16=True)
-    assert_parity("state", s[:, hs], s_ref, 1e-2, stored_bf16=False)
+    assert_parity("o", o[:, hs], o_ref, 1e-2, stored_bf16=True, tight=TC_TIGHT)
+    assert_parity("state", s[:, hs], s_ref, 1e-2, stored_bf16=False, tight=TC_TIGHT)
