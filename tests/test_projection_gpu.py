@@ -43,8 +43,11 @@ def _check_layer(y, s, rows, ry, rs, ro_rows, x_rows, w_g, H):
     rounding midpoint the two round to neighbouring values, one ulp apart, and GroupNorm and the
     gate carry that ulp into y; parity.gate_o_rounding_allowance bounds it per element (fp64,
     from the oracle's o and the inputs), and it is taken off on top of y's own half-ulp rounding
-    allowance before the 1e-2 rms bar."""
-    assert_parity("state", s, rs, 1e-2, stored_bf16=False, tight=1e-3)
+    allowance before the 1e-2 rms bar.  The state gets no tight bar here: q, k and v reach the
+    prefill rounded to bf16 from the projection's fp32 accumulator on the GPU and from fp64 in
+    the oracle, and the two roundings differ by one ulp where the value lies near a midpoint,
+    which moves the state by a few 1e-3 of rms at the 3B shape."""
+    assert_parity("state", s, rs, 1e-2, stored_bf16=False)
     a = gate_o_rounding_allowance(ro_rows, x_rows, w_g, H)
     yg = y.double().cpu().numpy()
     if rows is not None:
