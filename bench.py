@@ -589,6 +589,8 @@ def run_swa(args, rank, world, stream, headwise_ms):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    del q, k, v, o
+    dec = run_swa_decode(args, rank, world, stream, W)
     pairs = W * (W + 1) // 2 + (Nq - W) * W if Nq >= W else Nq * (Nq + 1) // 2
     flops = 4.0 * D * pairs * Hq * Bq
     tpeak, tkind = measured_tensor_peak()
@@ -599,8 +601,57 @@ def run_swa(args, rank, world, stream, headwise_ms):
             "l2": "q, k, v, o (805 MB) larger than L2; not flushed",
             "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
                          "frac": ach / tpeak, "peak_kind": tkind + " burst",
-                         "mma": "warp-level mma.sync m16n8k16 bf16", "traffic": None,
-                         "kernel": "swa_kernel", "algorithmic_flops_per_launch": flops}}
+                         "mma": "tcgen05 bf16, S and O in TMEM", "traffic": None,
+                         "kernel": "swa_tc_kernel", "algorithmic_flops_per_launch": flops},
+            "decode": dec}
+
+
+SWA_DEC_B, SWA_DEC_STEPS = 64, 64
+
+
+def run_swa_decode(args, rank, world, stream, W):
+    """Sliding-window decode with a full ring-buffer cache: 64 sequences x 24 heads of 128,
+    window W, each step one token per sequence (positions 4096 .. 4096 + steps - 1, so every
+    step reads a whole window).  HBM-bound: per (b, h) and step the window's keys and values
+    (2 W d 2 bytes), q, k, v, o and the cache slot written."""
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+    hbm_peak, peak_kind = measured_peaks()
+    Bq, Hq, S = SWA_DEC_B, H, SWA_DEC_STEPS
+    gen = torch.Generator(device="cuda")
+    gen.manual_seed(rank_seed(9, rank))
+    kc = torch.randn((Bq, Hq, W, D), generator=gen, device="cuda").to(torch.bfloat16)
+    vc = (torch.randn((Bq, Hq, W, D), generator=gen, device="cuda") * D ** -0.5).to(torch.bfloat16)
+    st = SI.gret_inputs(Bq, S, Hq, D, dtype=torch.bfloat16, seed=rank_seed(90, rank),
+                        device="cuda")
+    qs = (st["q"] * D ** 0.5).to(torch.bfloat16).permute(1, 0, 2, 3).contiguous()
+    ks = (st["k"] * D ** 0.5).to(torch.bfloat16).permute(1, 0, 2, 3).contiguous()
+    vs = st["v"].permute(1, 0, 2, 3).contiguous()
+    del st
+    pos = [torch.full((Bq,), 4096 + i, dtype=torch.int32, device="cuda") for i in range(S)]
+    od = torch.empty((Bq, Hq, D), dtype=torch.bfloat16, device="cuda")
+    for i in range(args.warmup):
+        G.gret_swa_decode_step(qs[i], ks[i], vs[i], pos[i], kc, vc, o=od)
+    torch.cuda.synchronize()
+    barrier(world)
+    d0 = torch.cuda.Event(enable_timing=True)
+    d1 = torch.cuda.Event(enable_timing=True)
+    d0.record(stream)
+    for i in range(S):
+        G.gret_swa_decode_step(qs[i], ks[i], vs[i], pos[i], kc, vc, o=od)
+    d1.record(stream)
+    torch.cuda.synchronize()
+    dms = max_over_ranks(d0.elapsed_time(d1), world)
+    per_bh = 2 * W * D * 2 + 4 * D * 2 + 2 * D * 2
+    ach = Bq * Hq * per_bh / (dms / S * 1e-3) / 1e9
+    return {"value": Bq * S * world / (dms * 1e-3), "unit": "tok/s", "ms_per_step": dms / S,
+            "batch": Bq, "window": W, "steps": S, "gpu_launches": S,
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": ach / hbm_peak, "peak_kind": peak_kind, "traffic": None,
+                         "kernel": "swa_decode_kernel",
+                         "algorithmic_bytes_per_launch": Bq * Hq * per_bh}}
 
 
 def run_layer(args, rank, world, stream, hbm_peak):

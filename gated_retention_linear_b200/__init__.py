@@ -42,6 +42,9 @@ _lib.gret_prefill_chunkwise_noalloc.argtypes = [_vp, _vp, _i64, _i64, _i64, _vp,
                                                 _i32, _vp, _i32, _vp, _vp, _vp, _i64, _i64, _i64,
                                                 _i32, _vp]
 _lib.gret_prefill_chunkwise_noalloc.restype = _i32
+_lib.gret_prefill_chunkwise_testing.argtypes = _lib.gret_prefill_chunkwise.argtypes + [
+    ctypes.c_uint64, ctypes.c_uint32]
+_lib.gret_prefill_chunkwise_testing.restype = _i32
 _lib.gret_prefill_noalloc_status.argtypes = [_vp]
 _lib.gret_prefill_noalloc_status.restype = _i32
 _lib.gret_workspace_status.argtypes = [_vp, _vp]
@@ -62,6 +65,9 @@ _lib.gret_prefill_elementwise_workspace_size.argtypes = [_i32, _i64, _i32, _i32]
 _lib.gret_prefill_elementwise_workspace_size.restype = ctypes.c_size_t
 _lib.gret_swa_prefill.argtypes = [_vp, _vp, _vp, _f32, _i32, _i32, _i64, _i32, _i32, _vp, _vp]
 _lib.gret_swa_prefill.restype = _i32
+_lib.gret_swa_decode_step.argtypes = [_vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
+                                      _vp, _vp]
+_lib.gret_swa_decode_step.restype = _i32
 
 
 class GretError(RuntimeError):
@@ -168,6 +174,27 @@ def gret_prefill_chunkwise(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None, s
         _ptr(cu_seqlens), a["n_seqs"], _ptr(state_in), _ptr(state_out), _ptr(o), a["osb"],
         a["ost"], a["osh"], chunk, _ptr(workspace), wbytes, _stream(stream)))
     return o, state_out
+
+
+def gret_prefill_chunkwise_testing(q, k, v, g, wait_ns, first_ticket, tau=16.0, k_scale=1.0,
+                                   cu_seqlens=None, state_in=None, state_out=None, o=None,
+                                   workspace=None, stream=None):
+    """gret_prefill_chunkwise with the failure-path settings of the C entry point of the same
+    name: every bounded wait gives up after wait_ns, and span tickets start at first_ticket.
+    For tests of the timeout path only.  Returns (o, state_out, workspace)."""
+    a = _prefill_args(q, k, v, g, cu_seqlens, state_out, o, False)
+    o, state_out = a["o"], a["state_out"]
+    need = int(_lib.gret_prefill_workspace_size(a["code"], a["total"], a["units"], a["H"],
+                                                a["dk"], a["dv"], 0))
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check("gret_prefill_chunkwise_testing", _lib.gret_prefill_chunkwise_testing(
+        _ptr(q), _ptr(k), a["sb"], a["st"], a["sh"], _ptr(v), a["vsb"], a["vst"], a["vsh"],
+        _ptr(g), tau, k_scale, a["code"], a["B"], a["N"], a["H"], a["dk"], a["dv"],
+        _ptr(cu_seqlens), a["n_seqs"], _ptr(state_in), _ptr(state_out), _ptr(o), a["osb"],
+        a["ost"], a["osh"], 0, _ptr(workspace), workspace.numel(), _stream(stream),
+        int(wait_ns), int(first_ticket)))
+    return o, state_out, workspace
 
 
 def gret_prefill_chunkwise_noalloc(q, k, v, g, tau=16.0, k_scale=1.0, cu_seqlens=None,
@@ -294,6 +321,29 @@ def gret_swa_prefill(q, k, v, window=1024, scale=None, o=None, stream=None):
     _check("gret_swa_prefill", _lib.gret_swa_prefill(
         _ptr(q), _ptr(k), _ptr(v), d ** -0.5 if scale is None else scale, window, B, N, H, d,
         _ptr(o), _stream(stream)))
+    return o
+
+
+def gret_swa_decode_step(q, k, v, pos, k_cache, v_cache, window=None, scale=None, o=None,
+                         stream=None):
+    """One sliding-window attention decode step with a ring-buffer cache: token t = pos[b] of
+    every sequence is written to slot t % window of k_cache / v_cache [B, H, window, 128] and
+    attends to its sequence's last `window` tokens.  q, k, v [B, H, 128] bf16; pos int32 [B] on
+    the device (not advanced here).  Returns o [B, H, 128] bf16."""
+    B, H, d = q.shape
+    W = k_cache.shape[2] if window is None else window
+    for t in (q, k, v, k_cache, v_cache):
+        if t.dtype != torch.bfloat16 or not t.is_contiguous():
+            raise ValueError("q, k, v and the caches must be contiguous bfloat16")
+    if k_cache.shape != (B, H, W, d) or v_cache.shape != (B, H, W, d):
+        raise ValueError("caches must be [B, H, window, d]")
+    if pos.dtype != torch.int32 or pos.shape != (B,):
+        raise ValueError("pos must be int32 [B]")
+    if o is None:
+        o = torch.empty_like(q)
+    _check("gret_swa_decode_step", _lib.gret_swa_decode_step(
+        _ptr(q), _ptr(k), _ptr(v), d ** -0.5 if scale is None else scale, W, B, H, d, _ptr(pos),
+        _ptr(k_cache), _ptr(v_cache), _ptr(o), _stream(stream)))
     return o
 
 

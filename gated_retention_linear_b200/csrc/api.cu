@@ -54,16 +54,21 @@ size_t gret_prefill_workspace_size(gret_dtype_t dtype, int64_t total_tokens, int
     return 0;
 }
 
-gret_status_t gret_prefill_chunkwise(const void* q, const void* k, int64_t stride_batch,
-                                     int64_t stride_tok, int64_t stride_head, const void* v,
-                                     int64_t v_stride_batch, int64_t v_stride_tok,
-                                     int64_t v_stride_head, const float* g, float tau,
-                                     float k_scale, gret_dtype_t dtype, int B, int64_t N, int H,
-                                     int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
-                                     const float* state_in, float* state_out, void* o,
-                                     int64_t o_stride_batch, int64_t o_stride_tok,
-                                     int64_t o_stride_head, int chunk, void* workspace,
-                                     size_t workspace_bytes, gret_stream_t stream) {
+}  // extern "C"
+
+namespace {
+
+gret_status_t prefill_impl(const void* q, const void* k, int64_t stride_batch,
+                           int64_t stride_tok, int64_t stride_head, const void* v,
+                           int64_t v_stride_batch, int64_t v_stride_tok,
+                           int64_t v_stride_head, const float* g, float tau,
+                           float k_scale, gret_dtype_t dtype, int B, int64_t N, int H,
+                           int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
+                           const float* state_in, float* state_out, void* o,
+                           int64_t o_stride_batch, int64_t o_stride_tok,
+                           int64_t o_stride_head, int chunk, void* workspace,
+                           size_t workspace_bytes, gret_stream_t stream, uint64_t test_wait_ns,
+                           uint32_t test_first_ticket) {
     if (dtype != GRET_F32 && dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
     if (!dim_ok(d_k) || !dim_ok(d_v) || H < 1 || B < 0 || N < 0) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
@@ -95,6 +100,8 @@ gret_status_t gret_prefill_chunkwise(const void* q, const void* k, int64_t strid
     a.o = o; a.osb = o_stride_batch; a.ost = o_stride_tok; a.osh = o_stride_head;
     a.workspace = workspace; a.workspace_bytes = workspace_bytes;
     a.stream = (cudaStream_t)stream;
+    a.test_wait_ns = test_wait_ns;
+    a.test_first_ticket = test_first_ticket;
 
     if (choose_path(dtype, d_k, d_v, chunk) == Path::TensorCore) {
         a.chunk = TC_CHUNK;
@@ -116,6 +123,43 @@ gret_status_t gret_prefill_chunkwise(const void* q, const void* k, int64_t strid
     cudaError_t e = launch_prefill_simt(a, dtype == GRET_BF16);
     if (e == cudaErrorInvalidValue) return GRET_ERR_UNSUPPORTED;
     return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+gret_status_t gret_prefill_chunkwise(const void* q, const void* k, int64_t stride_batch,
+                                     int64_t stride_tok, int64_t stride_head, const void* v,
+                                     int64_t v_stride_batch, int64_t v_stride_tok,
+                                     int64_t v_stride_head, const float* g, float tau,
+                                     float k_scale, gret_dtype_t dtype, int B, int64_t N, int H,
+                                     int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
+                                     const float* state_in, float* state_out, void* o,
+                                     int64_t o_stride_batch, int64_t o_stride_tok,
+                                     int64_t o_stride_head, int chunk, void* workspace,
+                                     size_t workspace_bytes, gret_stream_t stream) {
+    return prefill_impl(q, k, stride_batch, stride_tok, stride_head, v, v_stride_batch,
+                        v_stride_tok, v_stride_head, g, tau, k_scale, dtype, B, N, H, d_k, d_v,
+                        cu_seqlens, n_seqs, state_in, state_out, o, o_stride_batch,
+                        o_stride_tok, o_stride_head, chunk, workspace, workspace_bytes, stream, 0,
+                        0);
+}
+
+gret_status_t gret_prefill_chunkwise_testing(
+    const void* q, const void* k, int64_t stride_batch, int64_t stride_tok, int64_t stride_head,
+    const void* v, int64_t v_stride_batch, int64_t v_stride_tok, int64_t v_stride_head,
+    const float* g, float tau, float k_scale, gret_dtype_t dtype, int B, int64_t N, int H,
+    int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs, const float* state_in,
+    float* state_out, void* o, int64_t o_stride_batch, int64_t o_stride_tok,
+    int64_t o_stride_head, int chunk, void* workspace, size_t workspace_bytes,
+    gret_stream_t stream, uint64_t wait_ns, uint32_t first_ticket) {
+    if (wait_ns == 0 || wait_ns > 2000000000ull) return GRET_ERR_INVALID_ARG;
+    return prefill_impl(q, k, stride_batch, stride_tok, stride_head, v, v_stride_batch,
+                        v_stride_tok, v_stride_head, g, tau, k_scale, dtype, B, N, H, d_k, d_v,
+                        cu_seqlens, n_seqs, state_in, state_out, o, o_stride_batch,
+                        o_stride_tok, o_stride_head, chunk, workspace, workspace_bytes, stream,
+                        wait_ns, first_ticket);
 }
 
 gret_status_t gret_workspace_status(const void* workspace, gret_stream_t stream) {
@@ -248,3 +292,28 @@ gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, floa
 }
 
 }  // extern "C"
+
+extern "C" gret_status_t gret_swa_decode_step(const void* q, const void* k, const void* v,
+                                              float scale, int window, int B, int H, int d,
+                                              const int32_t* pos, void* k_cache, void* v_cache,
+                                              void* o, gret_stream_t stream) {
+    if (B < 0 || H < 1 || d < 1 || window < 1 || !isfinite(scale)) return GRET_ERR_INVALID_ARG;
+    if (d != SWA_DIM || window > SWA_DECODE_MAX_WINDOW) return GRET_ERR_UNSUPPORTED;
+    if ((int64_t)B * H > 0x7fffffffLL) return GRET_ERR_UNSUPPORTED;
+    if (B == 0) return GRET_OK;
+    if (!q || !k || !v || !pos || !k_cache || !v_cache || !o) return GRET_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(k_cache) ||
+        !aligned16(v_cache) || (reinterpret_cast<uintptr_t>(pos) & 3u) != 0)
+        return GRET_ERR_ALIGNMENT;
+    SwaDecodeArgs a;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.k = static_cast<const __nv_bfloat16*>(k);
+    a.v = static_cast<const __nv_bfloat16*>(v);
+    a.scale = scale; a.window = window; a.B = B; a.H = H; a.pos = pos;
+    a.k_cache = static_cast<__nv_bfloat16*>(k_cache);
+    a.v_cache = static_cast<__nv_bfloat16*>(v_cache);
+    a.o = static_cast<__nv_bfloat16*>(o);
+    const cudaError_t e = launch_swa_decode(a, (cudaStream_t)stream);
+    if (e == cudaErrorInvalidValue) return GRET_ERR_UNSUPPORTED;
+    return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+}

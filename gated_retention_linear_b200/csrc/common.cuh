@@ -62,6 +62,11 @@ struct PrefillArgs {
     void* workspace;
     size_t workspace_bytes;
     cudaStream_t stream;
+    // Failure-path testing only (gret_prefill_chunkwise_testing): the limit of every bounded
+    // wait of the tensor-core kernel (0 = the default), and the first span ticket handed out
+    // (0 = normal; a value past span 0 of a chain leaves its look-back flag forever unset).
+    uint64_t test_wait_ns = 0;
+    uint32_t test_first_ticket = 0;
 };
 
 cudaError_t launch_prefill_simt(const PrefillArgs& a, bool bf16);

@@ -13,11 +13,19 @@
 // used as a difference inside one chunk, so no exponent can overflow.
 //
 // Precision.  P, the state copy and w K are fp32 values that an MMA needs as bf16.  Rounding
-// each to bf16 once costs up to 2^-8 relative per element and, measured against an fp64
-// reference, left errors of 1-3% of rms on large outputs.  Each is therefore split into a bf16
-// high half and a bf16 low half (x - hi), and both halves go through the MMA: P V and Q S_prev
-// and (w K)^T V are each two MMAs, which keeps them within a few 1e-6 of fp32.  V and Q are used
-// exactly as loaded.
+// each to bf16 once costs up to 2^-8 relative per element and leaves errors near 1e-2 of rms
+// on large outputs.  Each is therefore split into a bf16 high half and a bf16 low half (x - hi),
+// and both halves go through the MMA: P V, Q S_prev and (w K)^T V are each two MMAs, which keeps
+// the result near 1e-5 of rms.  V and Q are used exactly as loaded.
+//
+// Where the operands live.  Shared memory holds two stages of K and V tiles, two Q tiles and
+// the bf16 state copy: 7 x 32 KB.  The weighted keys never go back to shared memory: the
+// converter group reads each key column straight out of the K tile, weights it, splits it into
+// bf16 halves and stores (w K)^T into tensor memory, where dS reads it as its A operand (the
+// same layout P V reads P in).  Tensor memory (512 columns): A / P [0,128), OX [128,256), one
+// region [256,384) that holds dS and then O (dS is folded into the registers of the state group
+// before P V writes O over it), and (w K)^T [384,512).  A chunk's bf16 output tile is staged in
+// its own Q slot (free once Q K^T and Q S have read it) and leaves by TMA store.
 //
 // Parallelism across a sequence.  The chunk chain of one (sequence, head) is sequential, and
 // one 3B-shaped layer has only 24 chains for 148 SMs.  Each chain is therefore cut into spans
@@ -31,31 +39,30 @@
 //           flag in the workspace), entry E = that state (or state_in for s = 0), and publish
 //           the inclusive state exp(L_span) E + Agg for span s+1;
 //   pass B: the full chunk pipeline above from E, writing O.
-// Pass B reads the span's K and V a second time: from L2 when spans are short, from DRAM when
-// the CTAs' spans together outgrow L2 (longer spans still win: fewer look-backs, fuller waves).
 // Inclusive states live in a two-slot ring per chain: span s+2 can only overwrite the slot of
 // span s after span s+1 has consumed it, because it needs span s+1's own inclusive state first.
 // Tickets are taken by running CTAs in increasing order and every span depends only on a smaller
 // ticket, so the chain always progresses.
 //
-// Warp roles (384 threads = 3 warpgroups, one CTA per SM):
-//   warp 0      TMA producer (lane 0): K, V (and Q in pass B) tiles, two pipeline stages;
-//               the whole warp scans the chunk's gate logits into the stage's gate slot
+// Warp roles (512 threads = 4 warpgroups, one CTA per SM):
+//   warp 0      TMA producer (lane 0): K and V tiles (two stages), Q tiles (two slots); the
+//               whole warp scans the chunk's gate logits into the stage's gate slot (in-chunk
+//               cumulative log2-decay, chunk total, key weights)
 //   warp 1      tcgen05 MMA issuer (one thread); owns the 512-column TMEM allocation
-//   warps 2-3   their share of the w K split (3 of the 16 chunks of two rows each)
-//   warps 4-7   "P group": decay mask A -> P (written back into TMEM as bf16 halves), its share
-//               of the w K split (6 chunks of its row), and the output epilogue
-//               O + exp(c_t) OX -> bf16 -> TMA store through the state buffer
-//   warps 8-11  "state group": its share of the w K split (7 chunks of its row), the fp32
-//               state (one row per thread), the look-back, and the bf16 halves of the state
-//               that Q S_prev reads
-// Registers: launched at 168 per thread (384 x 168 = 64512); the first warpgroup drops to 88,
-// the P group to 136 and the state group (128 fp32 state values per thread) rises to 256:
-// 128 x (88 + 136 + 256) = 61440 <= 64512, and each SM sub-partition (one warp of each group)
-// needs 32 x 480 <= 16384.  The host refuses to launch a build whose per-thread register count
-// is not 168, since a request for more registers than the block holds would wait forever.
-// TMEM columns: [0,128) A, then P (bf16 halves, see mma_pv); [128,256) O; [256,384) OX;
-// [384,512) dS.
+//   warps 4-7   P group: decay mask A -> P (bf16 halves in TMEM) and the output epilogue
+//               O + exp(c_t) OX -> bf16 -> the chunk's Q slot -> TMA store
+//   warps 8-11  state group: fp32 state (one row per thread), the look-back, the bf16 halves
+//               of the state that Q S_prev reads
+//   warps 12-15 converter group: (w K)^T in TMEM for every chunk of both passes
+// Per pass-B chunk the MMA issuer runs Q K^T, Q S_hi, dS, Q S_lo, P V; the only step that waits
+// for the previous chunk's state is Q S (after the state group's fold and bf16 writes), and dS
+// and the converter's work depend on nothing but the chunk's own K and V.
+// Registers: launched at 128 per thread (512 x 128 = 65536); warps 0-3 and the converter group
+// drop to 72, the P group rises to 136 and the state group (128 fp32 state values per thread)
+// to 232: 128 x (72 + 136 + 232 + 72) = 65536, and each SM sub-partition (one warp
+// of each group) needs 32 x 512 = 16384.  The host refuses to launch a build whose per-thread
+// register count is not 128, since a request for more registers than the block holds would
+// wait forever.
 // Every wait is bounded (see sm100::mbar_wait); a wait that gives up records GRET_ERR_TIMEOUT in
 // the workspace, and the kernel drains its copies, frees TMEM and exits.
 #include "prefill_tc.cuh"
@@ -77,12 +84,13 @@ constexpr int C = 128;                  // tokens per chunk
 constexpr int D = 128;                  // head width (d_k = d_v)
 constexpr int TILE = C * D * 2;         // one bf16 128x128 tile
 constexpr int SLAB = TILE / 2;          // one 64-column slab
-constexpr int NTHREADS = 384;
+constexpr int NTHREADS = 512;
+constexpr int LAUNCH_REGS = 128;        // 65536 / NTHREADS
 constexpr int ITEM_DEPTH = 4;
 constexpr uint64_t WAIT_NS = 2000000000ull;   // a wait gives up after 2 s
 constexpr uint64_t DRAIN_NS = 200000000ull;   // exit-time drains give up after 0.2 s
 
-constexpr uint32_t TM_A = 0, TM_O = 128, TM_OX = 256, TM_DS = 384;
+constexpr uint32_t TM_A = 0, TM_OX = 128, TM_DO = 256, TM_KT = 384;
 
 struct Item {
     int32_t valid;
@@ -97,31 +105,33 @@ struct Item {
 };
 
 struct __align__(1024) Smem {
-    unsigned char q[2][TILE];  // Q tile; in pass A, and after Q S in pass B, the low half of w K
-    unsigned char k[2][TILE];  // K tile; rewritten in place as the high half of w K
+    unsigned char q[2][TILE];  // Q tiles of pass B; after a chunk's Q S, its bf16 output tile
+    unsigned char k[2][TILE];
     unsigned char v[2][TILE];
-    // bf16 high half, then low half, of the state that Q S_prev reads; between a chunk's Q S_lo
-    // and the next high half, the chunk's bf16 output tile on its way out by TMA store
-    unsigned char sbf[TILE];
-    uint64_t kv_full[2], stage_empty[2];
+    // bf16 high half, then low half, of the state that Q S_prev reads; the look-back stages
+    // the span's entry state through it
+    unsigned char sb[TILE];
+    uint64_t kv_full[2], kv_empty[2];
+    uint64_t q_full[2], q_empty[2];
     uint64_t item_full[ITEM_DEPTH], item_empty[ITEM_DEPTH];
-    // k_ready / kp_ready / kh_ready (per stage): the state group's / the P group's / the helpers'
-    // share of the w K split is written.  Each has one producing group, so arrivals of different groups never mix, and
-    // being per stage, a group can reach the next phase of a stage's barrier only after the MMA
-    // has released that stage -- so no waiter can be left two phases behind.
-    uint64_t k_ready[2], kh_ready[2], kp_ready[2];
-    uint64_t a_full, s3a_done, q_free, p_ready, s_lo_ready, o_full, o_free, ds_full, ds_free,
-        s_ready, sbf_free, drain;
+    uint64_t a_full, p_ready, s_ready, s_hi_done, s_lo_ready, sb_free, kt_ready, kt_free,
+        ds_full, ds_free, o_full, o_free, drain;
+    // per item slot: the span's pass-A gate scans are done and span_L holds its total decay
+    uint64_t span_done[ITEM_DEPTH];
     Item items[ITEM_DEPTH];
-    float gc[2][C];            // per stage: in-chunk inclusive cumulative log2-decay of each token
+    // per stage: in-chunk inclusive cumulative log2-decay of each token, and the key weights
+    // k_scale * 2^(base - c_m) (0 past the end); written as float4 by the gate scan
+    alignas(16) float gc[2][C];
+    alignas(16) float w[2][C];
     float gtot[2];             // per stage: the chunk's total log2-decay
-    // per stage: exponent base of the key weights w_m = k_scale * 2^(gbase - c_m): the chunk
-    // total in pass B, the chunk total plus that of the span's later chunks in pass A
-    float gbase[2];
+    float span_L[ITEM_DEPTH];  // per item slot: log2-decay over the whole span
     uint32_t dec[3][2];        // group-uniform wait decisions (double-buffered)
     uint32_t tmem_base;
     uint32_t abort;
 };
+
+// The dynamic shared memory a block can have on sm_100.
+static_assert(sizeof(Smem) <= 232448, "shared-memory plan exceeds 227 KB");
 
 struct TcParams {
     const float* g;
@@ -143,6 +153,7 @@ struct TcParams {
     int qk_pos_tok, qk_pos_head, qk_pos_b;   // tensor-map dimension of each coordinate
     int v_pos_tok, v_pos_head, v_pos_b;
     int o_pos_tok, o_pos_head, o_pos_b;
+    uint64_t wait_ns;          // limit of every inter-role and inter-block wait
 };
 
 __device__ __forceinline__ float ex2f(float x) {
@@ -174,21 +185,20 @@ __device__ __forceinline__ void mbar_wait_drain(uint64_t* bar, uint32_t parity, 
 struct GroupWait {
     Smem* sm;
     const TcParams* p;
-    int gid;      // 0 = P group, 1 = state group, 2 = split helpers
+    int gid;      // 0 = P group, 1 = state group, 2 = converter group
     int tid;      // thread index within the group
-    int nthreads = 128;
     int flip = 0;
 
     __device__ bool wait(uint64_t* bar, uint32_t parity) {
         if (tid == 0) {
-            bool ok = mbar_wait(bar, parity, &sm->abort, WAIT_NS);
+            bool ok = mbar_wait(bar, parity, &sm->abort, p->wait_ns);
             if (!ok) {
                 if (!sm->abort) set_error(p->err);
                 atomicExch(&sm->abort, 1u);
             }
             sm->dec[gid][flip] = ok ? 0u : 1u;
         }
-        named_sync(1 + gid, nthreads);
+        named_sync(1 + gid);
         bool ok = *reinterpret_cast<volatile uint32_t*>(&sm->dec[gid][flip]) == 0;
         flip ^= 1;
         return ok;
@@ -204,7 +214,7 @@ struct GroupWait {
                 asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(flag) : "memory");
                 if (v == want) { ok = true; break; }
                 if (*reinterpret_cast<volatile uint32_t*>(&sm->abort)) break;
-                if (globaltimer_ns() - t0 > WAIT_NS) break;
+                if (globaltimer_ns() - t0 > p->wait_ns) break;
                 __nanosleep(64);
             }
             if (!ok) {
@@ -284,8 +294,8 @@ __device__ __forceinline__ void gate_load(const TcParams& p, const Item& it, int
 
 // The whole warp computes, for the chunk's 128 tokens, the in-chunk inclusive cumulative
 // log2-decay c_t = sum of logsigmoid(g)/tau * log2(e) over the chunk up to t (0 past the end of
-// the sequence), the chunk total and the weight base `after` + total into the stage's gate slot;
-// returns the chunk total on every lane.
+// the sequence), the chunk total, and the key weights w_t = k_scale * 2^(after + total - c_t)
+// (0 past the end), into the stage's gate slot; returns the chunk total on every lane.
 __device__ __forceinline__ float gate_scan(Smem& sm, const TcParams& p, const Item& it, int c,
                                            int st, int lane, const float (&g4)[4], float after) {
     float lam[4];
@@ -303,25 +313,31 @@ __device__ __forceinline__ float gate_scan(Smem& sm, const TcParams& p, const It
         if (lane >= o) x += y;
     }
     const float excl = x - lam[3];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sm.gc[st][4 * lane + e] = excl + lam[e];
     const float tot = __shfl_sync(0xffffffffu, x, 31);
-    if (lane == 31) {
-        sm.gtot[st] = tot;
-        sm.gbase[st] = after + tot;
+    const float base = after + tot;
+    float4 gc4, w4;
+    float* gcp = &gc4.x;
+    float* wp = &w4.x;
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+        gcp[e] = excl + lam[e];
+        wp[e] = (t0 + e < it.len) ? ex2f(base - gcp[e]) * p.k_scale : 0.f;
     }
+    reinterpret_cast<float4*>(sm.gc[st])[lane] = gc4;
+    reinterpret_cast<float4*>(sm.w[st])[lane] = w4;
+    if (lane == 31) sm.gtot[st] = tot;
     return tot;
 }
 
 __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, const CUtensorMap* tk,
                          const CUtensorMap* tv, uint32_t total, int lane) {
-    int j = 0, it_n = 0;
+    int j = 0, b = 0, it_n = 0;
     bool aborted = false;
     while (!aborted) {
         const int slot = it_n % ITEM_DEPTH;
         int ok = 1;
         if (lane == 0 && it_n >= ITEM_DEPTH)
-            ok = mbar_wait(&sm.item_empty[slot], ((it_n / ITEM_DEPTH) - 1) & 1, &sm.abort, WAIT_NS);
+            ok = mbar_wait(&sm.item_empty[slot], ((it_n / ITEM_DEPTH) - 1) & 1, &sm.abort, p.wait_ns);
         if (!__shfl_sync(0xffffffffu, ok, 0)) {
             aborted = true;
             break;
@@ -337,26 +353,33 @@ __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, con
         }
         ++it_n;
         if (!it.valid) break;
-        // pass A visits the span's chunks last to first (its aggregate is accumulated by the
-        // MMAs with each key weighted by its decay to the end of the span); pass B first to last
         const int n = it.c_end - it.c_begin;
+        if (n == 0 && lane == 0) {   // nothing to scan: the span's total decay is 0
+            sm.span_L[slot] = 0.f;
+            mbar_arrive(&sm.span_done[slot]);
+        }
+        // pass A visits the span's chunks last to first (each key weighted by its decay to the
+        // end of the span); pass B first to last
         float after = 0.f;   // pass A: log2-decay of the chunks after the current one
         for (int jj = 0; jj < 2 * n; ++jj) {
             const bool pass_b = jj >= n;
             const int c = pass_b ? it.c_begin + (jj - n) : it.c_end - 1 - jj;
             const int st = j & 1;
             float g4[4];
-            gate_load(p, it, c, lane, g4);   // in flight while the stage is awaited
+            gate_load(p, it, c, lane, g4);   // in flight while the slots are awaited
             ok = 1;
             if (lane == 0 && j >= 2)
-                ok = mbar_wait(&sm.stage_empty[st], ((j >> 1) - 1) & 1, &sm.abort, WAIT_NS);
+                ok = mbar_wait(&sm.kv_empty[st], ((j >> 1) - 1) & 1, &sm.abort, p.wait_ns);
+            if (pass_b && lane == 0 && ok && b >= 2)
+                ok = mbar_wait(&sm.q_empty[b & 1], ((b >> 1) - 1) & 1, &sm.abort, p.wait_ns);
             if (!__shfl_sync(0xffffffffu, ok, 0)) {
                 aborted = true;
                 break;
             }
             if (lane == 0) {
-                mbar_arrive_expect_tx(&sm.kv_full[st], pass_b ? 3 * TILE : 2 * TILE);
                 const int tok = (int)(it.tok_first + (int64_t)c * C);
+                mbar_arrive_expect_tx(&sm.kv_full[st], 2 * TILE);
+                if (pass_b) mbar_arrive_expect_tx(&sm.q_full[b & 1], TILE);
                 int ck[4], cv[4];
                 for (int half = 0; half < 2; ++half) {
                     set_coord(ck, p.qk_pos_tok, p.qk_pos_head, p.qk_pos_b, half * 64, tok, it.h,
@@ -367,14 +390,21 @@ __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, con
                     tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], cv[0], cv[1], cv[2],
                                 cv[3]);
                     if (pass_b)
-                        tma_load_4d(sm.q[st] + half * SLAB, tq, &sm.kv_full[st], ck[0], ck[1],
-                                    ck[2], ck[3]);
+                        tma_load_4d(sm.q[b & 1] + half * SLAB, tq, &sm.q_full[b & 1], ck[0],
+                                    ck[1], ck[2], ck[3]);
                 }
             }
             const float tot = gate_scan(sm, p, it, c, st, lane, g4, pass_b ? 0.f : after);
             if (!pass_b) after += tot;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.kv_full[st]);
+            if (lane == 0) {
+                mbar_arrive(&sm.kv_full[st]);
+                if (!pass_b && jj == n - 1) {   // the span's total decay, for the look-back
+                    sm.span_L[slot] = after;
+                    mbar_arrive(&sm.span_done[slot]);
+                }
+            }
+            if (pass_b) ++b;
             ++j;
         }
     }
@@ -386,6 +416,8 @@ __device__ void producer(Smem& sm, const TcParams& p, const CUtensorMap* tq, con
         // make sure no TMA write into this CTA's shared memory is still in flight at exit
         for (int jj = (j >= 2 ? j - 2 : 0); jj < j; ++jj)
             mbar_wait_drain(&sm.kv_full[jj & 1], (jj >> 1) & 1, DRAIN_NS);
+        for (int bb = (b >= 2 ? b - 2 : 0); bb < b; ++bb)
+            mbar_wait_drain(&sm.q_full[bb & 1], (bb >> 1) & 1, DRAIN_NS);
     }
 }
 
@@ -408,38 +440,39 @@ __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, 
     }
 }
 
-// D (+)= P V with P (bf16, K-major) in TMEM.  P is stored per 32-token group g = 0..3 as
-// [16 columns of high halves | 16 columns of low halves] at columns 32 g; the K-step of tokens
-// [16 kk, 16 kk + 16) of one half starts at column 32 (kk / 2) + 8 (kk % 2) + 16 * half.
-__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
+// D (+)= X V with X (bf16, K-major) in TMEM and V [token x d_v] in shared memory.  X is stored
+// per 32-token group g = 0..3 as [16 columns of high halves | 16 columns of low halves] at
+// columns 32 g; the K-step of tokens [16 kk, 16 kk + 16) of one half starts at column
+// 32 (kk / 2) + 8 (kk % 2) + 16 * half.  X is P (rows = query tokens) for the inner output and
+// (w K)^T (rows = key channels) for the state update.
+__device__ __forceinline__ void mma_tv(uint32_t d, uint32_t x_base, int half, uint32_t v_base,
                                        bool accumulate) {
     const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
 #pragma unroll 1
     for (int kk = 0; kk < 8; ++kk)
-        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
+        mma_ts(d, x_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
                sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
                (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// dS (+)= (w K)^T V as the sum of its bf16 high half (K slot) and low half (Q slot).
-__device__ __forceinline__ void mma_ds(uint32_t tmem, Smem& sm, int st, bool accumulate) {
-    mma_128(tmem + TM_DS, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, accumulate);
-    mma_128(tmem + TM_DS, smem_u32(sm.q[st]), true, smem_u32(sm.v[st]), true, true);
-}
-
+// Tensor-memory region [256, 384) holds, in turn, each span's aggregate, then per pass-B chunk
+// dS and then O.  The two kinds of content have their own barriers, so that each consumer waits
+// for consecutive phases of one barrier (a parity wait cannot tell phase n from phase n + 2): an
+// aggregate or a dS completes a phase of ds_full and, once folded by the state group, of
+// ds_free; an O completes a phase of o_full and, once read by the P group, of o_free.
 __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
     int j = 0, b = 0, it_n = 0;
-    int dsn = 0;   // dS results handed to the state group so far (phases of ds_full)
+    uint32_t n_ds = 0, n_o = 0;   // aggregates + dS, and O, written so far
     bool ok = true;
     auto W = [&](uint64_t* bar, uint32_t par) {
-        if (ok && !mbar_wait(bar, par, &sm.abort, WAIT_NS)) {
+        if (ok && !mbar_wait(bar, par, &sm.abort, p.wait_ns)) {
             ok = false;
             if (!sm.abort) set_error(p.err);
             atomicExch(&sm.abort, 1u);
         }
         return ok;
     };
-    const uint32_t sbf = smem_u32(sm.sbf);
+    const uint32_t sb = smem_u32(sm.sb);
     while (ok) {
         const int slot = it_n % ITEM_DEPTH;
         if (!W(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
@@ -447,66 +480,66 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
         mbar_arrive(&sm.item_empty[slot]);
         ++it_n;
         if (!it.valid) break;
-        // pass A: the span's aggregate, one dS result accumulated over its chunks (which the
-        // producer delivers last to first, each key weighted by its decay to the span's end)
         const int n = it.c_end - it.c_begin;
+        // pass A: the span's aggregate, one result accumulated over its chunks (delivered last to
+        // first, each key weighted by its decay to the span's end).  The region's previous
+        // content, if any, is the O of the last chunk of an earlier span.
         for (int i = 0; i < n && ok; ++i, ++j) {
             const int st = j & 1;
             if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
-            if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
-            if (!W(&sm.kp_ready[st], (j >> 1) & 1)) break;
-            if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
-            if (i == 0 && dsn > 0 && !W(&sm.ds_free, (dsn - 1) & 1)) break;
+            if (!W(&sm.kt_ready, j & 1)) break;
+            if (i == 0 && n_o > 0 && !W(&sm.o_free, (n_o - 1) & 1)) break;
             tc_fence_after();
-            mma_ds(tmem, sm, st, i > 0);
-            mma_commit(&sm.stage_empty[st]);
+            const uint32_t vb = smem_u32(sm.v[st]);
+            mma_tv(tmem + TM_DO, tmem + TM_KT, 0, vb, i > 0);
+            mma_tv(tmem + TM_DO, tmem + TM_KT, 1, vb, true);
+            mma_commit(&sm.kt_free);
+            mma_commit(&sm.kv_empty[st]);
         }
         if (!ok) break;
         if (n > 0) {
-            mma_commit(&sm.ds_full);
-            ++dsn;
+            mma_commit(&sm.ds_full);   // the aggregate
+            ++n_ds;
         }
-        // pass B: the full chunk.  Order per chunk: Q K^T (issued one chunk ahead), Q S_hi,
-        // Q S_lo (after which the Q slot is free for the low half of w K), P V (which runs while
-        // w K is split), dS (on the state chain, so as soon as the split is done), then Q K^T of
-        // the next chunk once P V has read P out of the tensor memory it overwrites.
-        auto issue_qk = [&](int jj, int bb) {
-            const int st = jj & 1;
-            if (!W(&sm.kv_full[st], (jj >> 1) & 1)) return false;
-            if (bb > 0 && !W(&sm.o_full, (bb - 1) & 1)) return false;   // P of chunk bb-1 used
+        // pass B.  Per chunk: Q K^T (once P V of the previous chunk has read P out of the
+        // tensor memory it overwrites), Q S_hi, dS, Q S_lo, P V.
+        for (int i = 0; i < n && ok; ++i, ++j, ++b) {
+            const int st = j & 1, qs = b & 1;
+            const uint32_t qb = smem_u32(sm.q[qs]), kb = smem_u32(sm.k[st]),
+                           vb = smem_u32(sm.v[st]);
+            if (!W(&sm.kv_full[st], (j >> 1) & 1)) break;
+            if (!W(&sm.q_full[qs], (b >> 1) & 1)) break;
+            if (n_o > 0 && !W(&sm.o_full, (n_o - 1) & 1)) break;    // the last P V is done
             tc_fence_after();
-            mma_128(tmem + TM_A, smem_u32(sm.q[st]), false, smem_u32(sm.k[st]), false, false);
+            mma_128(tmem + TM_A, qb, false, kb, false, false);     // A = Q K^T
             mma_commit(&sm.a_full);
-            return true;
-        };
-        if (it.c_end > it.c_begin && !issue_qk(j, b)) break;
-        for (int c = it.c_begin; c < it.c_end && ok; ++c, ++j, ++b) {
-            const int st = j & 1;
-            const uint32_t qb = smem_u32(sm.q[st]), vb = smem_u32(sm.v[st]);
             if (!W(&sm.s_ready, b & 1)) break;
-            if (b > 0 && !W(&sm.o_free, (b - 1) & 1)) break;     // O, OX read out
+            if (n_o > 0 && !W(&sm.o_free, (n_o - 1) & 1)) break;    // last O and OX read
             tc_fence_after();
-            mma_128(tmem + TM_OX, qb, false, sbf, true, false);   // OX = Q S_hi
-            mma_commit(&sm.s3a_done);
+            mma_128(tmem + TM_OX, qb, false, sb, true, false);     // OX = Q S_hi
+            mma_commit(&sm.s_hi_done);
+            if (!W(&sm.kt_ready, j & 1)) break;
+            // the region's previous content: the aggregate (i = 0, folded) or O of chunk i-1
+            // (read, waited for above)
+            if (i == 0 && !W(&sm.ds_free, (n_ds - 1) & 1)) break;
+            tc_fence_after();
+            mma_tv(tmem + TM_DO, tmem + TM_KT, 0, vb, false);      // dS = (w K)_hi^T V
+            mma_tv(tmem + TM_DO, tmem + TM_KT, 1, vb, true);       //    + (w K)_lo^T V
+            mma_commit(&sm.kt_free);
+            mma_commit(&sm.ds_full);
+            ++n_ds;
             if (!W(&sm.s_lo_ready, b & 1)) break;
             tc_fence_after();
-            mma_128(tmem + TM_OX, qb, false, sbf, true, true);    // OX += Q S_lo
-            mma_commit(&sm.q_free);
+            mma_128(tmem + TM_OX, qb, false, sb, true, true);      // OX += Q S_lo
+            mma_commit(&sm.sb_free);
             if (!W(&sm.p_ready, b & 1)) break;
+            if (!W(&sm.ds_free, (n_ds - 1) & 1)) break;            // dS folded into the state
             tc_fence_after();
-            mma_pv(tmem + TM_O, tmem + TM_A, 0, vb, false);        // O  = P_hi V
-            mma_pv(tmem + TM_O, tmem + TM_A, 1, vb, true);         // O += P_lo V
+            mma_tv(tmem + TM_DO, tmem + TM_A, 0, vb, false);       // O = P_hi V
+            mma_tv(tmem + TM_DO, tmem + TM_A, 1, vb, true);        //   + P_lo V
             mma_commit(&sm.o_full);
-            if (!W(&sm.k_ready[st], (j >> 1) & 1)) break;
-            if (!W(&sm.kp_ready[st], (j >> 1) & 1)) break;
-            if (!W(&sm.kh_ready[st], (j >> 1) & 1)) break;
-            if (dsn > 0 && !W(&sm.ds_free, (dsn - 1) & 1)) break;
-            tc_fence_after();
-            mma_ds(tmem, sm, st, false);
-            mma_commit(&sm.ds_full);
-            mma_commit(&sm.stage_empty[st]);
-            ++dsn;
-            if (c + 1 < it.c_end && !issue_qk(j + 1, b + 1)) break;
+            ++n_o;
+            mma_commit(&sm.kv_empty[st]);
         }
     }
     // all issued MMAs complete before TMEM is released
@@ -527,73 +560,19 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
     lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
-// Chunks [I0, I0 + N) of row r of a swizzled K tile (16 chunks of 8 elements per row; chunk i
-// sits in slab i / 8 at slot (i % 8) ^ (r % 8)): w * K split into a high half written back in
-// place and a low half written to the same position of `lotile`.  All loads are issued before
-// the first store (loads cannot move past stores to the same array).
-template <int I0, int N>
-__device__ __forceinline__ void split_k_chunks(unsigned char* ktile, unsigned char* lotile, int r,
-                                               float w) {
-    uint4 row[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        const int i = I0 + n;
-        row[n] = *reinterpret_cast<const uint4*>(ktile + (i >> 3) * SLAB + r * 128 +
-                                                 (((i & 7) ^ (r & 7)) << 4));
-    }
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        const int i = I0 + n;
-        const int off = (i >> 3) * SLAB + r * 128 + (((i & 7) ^ (r & 7)) << 4);
-        uint32_t* x = reinterpret_cast<uint32_t*>(&row[n]);
-        uint4 lo;
-        uint32_t* l = reinterpret_cast<uint32_t*>(&lo);
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-            const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&x[e]));
-            split2(f.x * w, f.y * w, x[e], l[e]);
-        }
-        *reinterpret_cast<uint4*>(ktile + off) = row[n];
-        *reinterpret_cast<uint4*>(lotile + off) = lo;
-    }
-}
-
-// The split of w K is shared by three groups, by 16-byte chunks of each 128-element row: the state
-// group takes chunks 0-6 of its own row, the P group chunks 7-12 of its own row, and warps 2-3
-// chunks 13-15 of two rows each.
-constexpr int SPLIT_STATE = 7, SPLIT_P = 6;
-constexpr int SPLIT_HELP0 = SPLIT_STATE + SPLIT_P, SPLIT_HELP = 16 - SPLIT_HELP0;
-
-// weight of token r of chunk c: k_scale * exp(c_b - c_r), zero past the end of the sequence
-__device__ __forceinline__ float k_weight(const Smem& sm, const TcParams& p, const Item& it, int c,
-                                          int st, int r) {
-    const bool valid = (int64_t)c * C + r < it.len;
-    return valid ? ex2f(sm.gbase[st] - sm.gc[st][r]) * p.k_scale : 0.f;
-}
-
-// Row r of the state into the MN-major swizzled tile read by Q S: the bf16 high half is
-// written and the low half kept in registers for write_state_lo.
-__device__ __forceinline__ void write_state_hi(unsigned char* tile, int r, const float (&S)[D],
-                                               uint32_t (&lo)[D / 2]) {
+// Row r of the state into the MN-major swizzled tile read by Q S: the bf16 high halves
+// (lo_half = false) or the low halves (lo_half = true) of the split of S.
+template <bool lo_half>
+__device__ __forceinline__ void write_state_half(unsigned char* tile, int r, const float (&S)[D]) {
 #pragma unroll
     for (int cc = 0; cc < 16; ++cc) {
-        uint32_t hi[4];
+        uint32_t hi[4], lo[4];
 #pragma unroll
-        for (int e = 0; e < 4; ++e)
-            split2(S[8 * cc + 2 * e], S[8 * cc + 2 * e + 1], hi[e], lo[4 * cc + e]);
+        for (int e = 0; e < 4; ++e) split2(S[8 * cc + 2 * e], S[8 * cc + 2 * e + 1], hi[e], lo[e]);
         const int half = cc >> 3, c = cc & 7;
+        const uint32_t* x = lo_half ? lo : hi;
         *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(hi[0], hi[1], hi[2], hi[3]);
-    }
-}
-
-__device__ __forceinline__ void write_state_lo(unsigned char* tile, int r,
-                                               const uint32_t (&lo)[D / 2]) {
-#pragma unroll
-    for (int cc = 0; cc < 16; ++cc) {
-        const int half = cc >> 3, c = cc & 7;
-        *reinterpret_cast<uint4*>(tile + half * SLAB + r * 128 + ((c ^ (r & 7)) << 4)) =
-            make_uint4(lo[4 * cc], lo[4 * cc + 1], lo[4 * cc + 2], lo[4 * cc + 3]);
+            make_uint4(x[0], x[1], x[2], x[3]);
     }
 }
 
@@ -610,6 +589,63 @@ __device__ __forceinline__ void fold_ds(uint32_t taddr, float (&S)[D], float eb)
 }
 
 // ----------------------------------------------------------------------------------------------
+// warps 12-15: (w K)^T into tensor memory, for every chunk of both passes
+
+// Thread r (TMEM lane r = key channel r) reads column r of the swizzled K tile (token m at row m;
+// element (m, r) in slab r / 64, 16-byte chunk ((r % 64) / 8) ^ (m % 8), position r % 8), weights
+// token m by w_m, splits into bf16 halves and stores them in the layout mma_tv reads: per
+// 32-token group, 16 columns of high halves then 16 of low halves, two tokens per column.  For a
+// fixed token the 32 lanes of a warp read 64 consecutive bytes of one row: no bank conflict.
+__device__ __forceinline__ void convert_wkt(const Smem& sm, int st, int r, uint32_t taddr) {
+    const unsigned char* kt = sm.k[st] + (r >> 6) * SLAB + ((r & 7) << 1);
+    const int cch = (r & 63) >> 3;
+    const float2* w2 = reinterpret_cast<const float2*>(sm.w[st]);
+#pragma unroll 1
+    for (int jc = 0; jc < 4; ++jc) {
+        uint32_t ph[32];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int m0 = jc * 32 + 2 * i;
+            const float k0 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                kt + m0 * 128 + ((cch ^ (m0 & 7)) << 4)));
+            const float k1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
+                kt + (m0 + 1) * 128 + ((cch ^ ((m0 + 1) & 7)) << 4)));
+            const float2 w = w2[m0 >> 1];
+            split2(k0 * w.x, k1 * w.y, ph[i], ph[16 + i]);
+        }
+        tmem_st32(taddr + jc * 32, ph);
+    }
+    tmem_st_wait();
+}
+
+__device__ void converter(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
+    GroupWait gw{&sm, &p, 2, (warp - 12) * 32 + lane};
+    const int r = (warp & 3) * 32 + lane;
+    const uint32_t taddr = tmem + (((uint32_t)((warp & 3) * 32)) << 16) + TM_KT;
+    int j = 0, it_n = 0;
+    bool ok = true;
+    while (ok) {
+        const int slot = it_n % ITEM_DEPTH;
+        if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
+        const Item it = sm.items[slot];
+        mbar_arrive(&sm.item_empty[slot]);
+        ++it_n;
+        if (!it.valid) break;
+        const int n = it.c_end - it.c_begin;
+        for (int jj = 0; jj < 2 * n; ++jj, ++j) {
+            const int st = j & 1;
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
+            if (j > 0 && !gw.wait(&sm.kt_free, (j - 1) & 1)) { ok = false; break; }
+            tc_fence_after();
+            convert_wkt(sm, st, r, taddr);
+            tc_fence_before();
+            mbar_arrive(&sm.kt_ready);
+            mbar_arrive(&sm.kv_empty[st]);   // this group is done with the stage's K and weights
+        }
+    }
+}
+
+// ----------------------------------------------------------------------------------------------
 // warps 4-7: decay mask (P split into bf16 halves in TMEM) and output epilogue
 
 __device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint32_t tmem, int warp,
@@ -618,108 +654,89 @@ __device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint
     const int q = warp & 3, r = q * 32 + lane;
     const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
     int b = 0, j = 0, it_n = 0;
-    while (true) {
+    bool ok = true;
+    while (ok) {
         const int slot = it_n % ITEM_DEPTH;
         if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
         const Item it = sm.items[slot];
         mbar_arrive(&sm.item_empty[slot]);
         ++it_n;
         if (!it.valid) break;
-        bool ok = true;
         const int n = it.c_end - it.c_begin;
-        // every job of the span: pass A (its share of the w K split only), then pass B
-        for (int jj = 0; jj < 2 * n; ++jj, ++j) {
-            const int st = j & 1;
-            const bool pass_b = jj >= n;
-            const int c = pass_b ? it.c_begin + (jj - n) : it.c_end - 1 - jj;
-            // the stage's gate slot is read before this group's split share is released: after
-            // that the stage may be refilled
-            float cr = 0.f;
-            if (!pass_b) {
-                if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
-            } else {
-                if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
-                if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }  // gate slot
-                cr = sm.gc[st][r];
-                tc_fence_after();
-                // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, split into bf16 halves; each
-                // 32-column group of A is replaced in place by [16 high | 16 low] columns of P.
+        j += n;             // pass A
+        for (int i = 0; i < n; ++i, ++j, ++b) {
+            const int st = j & 1, qs = b & 1, c = it.c_begin + i;
+            if (!gw.wait(&sm.a_full, b & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }   // gate slot
+            const float cr = sm.gc[st][r];
+            tc_fence_after();
+            // P = k_scale * 2^(c_r - c_m) * A[r][m] for m <= r, split into bf16 halves; each
+            // 32-column group of A is replaced in place by [16 high | 16 low] columns of P.
 #pragma unroll 1
-                for (int jc = 0; jc < 4; ++jc) {
-                    uint32_t ph[32];
-                    if (jc <= q) {
-                        float a[32];
-                        tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
-                        tmem_ld_wait();
+            for (int jc = 0; jc < 4; ++jc) {
+                uint32_t ph[32];
+                if (jc <= q) {
+                    float a[32];
+                    tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
+                    tmem_ld_wait();
 #pragma unroll
-                        for (int i = 0; i < 16; ++i) {
-                            const int m0 = jc * 32 + 2 * i;
-                            const float p0 =
-                                (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * p.k_scale * a[2 * i] : 0.f;
-                            const float p1 = (m0 + 1 <= r)
-                                                 ? ex2f(cr - sm.gc[st][m0 + 1]) * p.k_scale * a[2 * i + 1]
-                                                 : 0.f;
-                            split2(p0, p1, ph[i], ph[16 + i]);
-                        }
-                    } else {
-#pragma unroll
-                        for (int i = 0; i < 32; ++i) ph[i] = 0u;
+                    for (int i2 = 0; i2 < 16; ++i2) {
+                        const int m0 = jc * 32 + 2 * i2;
+                        const float p0 =
+                            (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * p.k_scale * a[2 * i2] : 0.f;
+                        const float p1 = (m0 + 1 <= r)
+                                             ? ex2f(cr - sm.gc[st][m0 + 1]) * p.k_scale * a[2 * i2 + 1]
+                                             : 0.f;
+                        split2(p0, p1, ph[i2], ph[16 + i2]);
                     }
-                    tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
+                } else {
+#pragma unroll
+                    for (int i2 = 0; i2 < 32; ++i2) ph[i2] = 0u;
                 }
-                tmem_st_wait();
-                tc_fence_before();
-                mbar_arrive(&sm.p_ready);
-                // both Q S MMAs are done: the Q slot takes the low half of w K
-                if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
+                tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
             }
-            split_k_chunks<SPLIT_STATE, SPLIT_P>(sm.k[st], sm.q[st], r,
-                                                 k_weight(sm, p, it, c, st, r));
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.kp_ready[st]);
-            if (!pass_b) continue;
-            // epilogue: O = O_inner + 2^(c_r) O_cross, rounded to bf16.  A chunk that lies wholly
-            // inside its sequence goes out as one tile: rows into the state buffer (free between
-            // Q S_lo and the next state write) in the swizzled layout, then two TMA stores.  The
-            // rows of a partial chunk are stored one by one, so that nothing past the end of the
-            // sequence (the next packed sequence) is written.
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready);
+            // epilogue: O = O_inner + 2^(c_r) O_cross, rounded to bf16.  o_full for O also means
+            // that every earlier MMA is done, Q K^T and Q S on this chunk's Q slot included.  A
+            // chunk that lies wholly inside its sequence goes out as one tile through that slot:
+            // rows in the swizzled layout, then two TMA stores.  The rows of a partial chunk are
+            // stored one by one, so that nothing past the end of the sequence (the next packed
+            // sequence) is written.
             if (!gw.wait(&sm.o_full, b & 1)) { ok = false; break; }
             tc_fence_after();
             const float ec = ex2f(cr);
             const int64_t t = (int64_t)c * C + r;
             const bool full = (int64_t)(c + 1) * C <= it.len;
-            const bool valid = t < it.len;
-            __nv_bfloat16* orow = p.o + (int64_t)it.b * p.osb + (it.tok_first + t) * p.ost +
-                                  (int64_t)it.h * p.osh;
+            unsigned char* tile = sm.q[qs];
+            uint4* orow = reinterpret_cast<uint4*>(p.o + (int64_t)it.b * p.osb +
+                                                   (it.tok_first + t) * p.ost +
+                                                   (int64_t)it.h * p.osh);
 #pragma unroll 1
             for (int jc = 0; jc < 4; ++jc) {
                 float o[32], ox[32];
-                tmem_ld32(tmem + lane_base + TM_O + jc * 32, o);
+                tmem_ld32(tmem + lane_base + TM_DO + jc * 32, o);
                 tmem_ld32(tmem + lane_base + TM_OX + jc * 32, ox);
                 tmem_ld_wait();
-                uint4 u[4];
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4) {
-                    u[v4].x = pack_bf16x2(fmaf(ec, ox[8 * v4 + 0], o[8 * v4 + 0]),
-                                          fmaf(ec, ox[8 * v4 + 1], o[8 * v4 + 1]));
-                    u[v4].y = pack_bf16x2(fmaf(ec, ox[8 * v4 + 2], o[8 * v4 + 2]),
-                                          fmaf(ec, ox[8 * v4 + 3], o[8 * v4 + 3]));
-                    u[v4].z = pack_bf16x2(fmaf(ec, ox[8 * v4 + 4], o[8 * v4 + 4]),
-                                          fmaf(ec, ox[8 * v4 + 5], o[8 * v4 + 5]));
-                    u[v4].w = pack_bf16x2(fmaf(ec, ox[8 * v4 + 6], o[8 * v4 + 6]),
-                                          fmaf(ec, ox[8 * v4 + 7], o[8 * v4 + 7]));
-                }
-                if (full) {
-                    // columns 32 jc .. 32 jc + 31: 16-byte chunks 4 (jc % 2) + v4 of slab jc / 2
-                    unsigned char* rowp = sm.sbf + (jc >> 1) * SLAB + r * 128;
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4)
-                        *reinterpret_cast<uint4*>(rowp + (((4 * (jc & 1) + v4) ^ (r & 7)) << 4)) =
-                            u[v4];
-                } else if (valid) {
-                    uint4* dst = reinterpret_cast<uint4*>(orow + jc * 32);
-#pragma unroll
-                    for (int v4 = 0; v4 < 4; ++v4) dst[v4] = u[v4];
+                    uint4 u;
+                    u.x = pack_bf16x2(fmaf(ec, ox[8 * v4 + 0], o[8 * v4 + 0]),
+                                      fmaf(ec, ox[8 * v4 + 1], o[8 * v4 + 1]));
+                    u.y = pack_bf16x2(fmaf(ec, ox[8 * v4 + 2], o[8 * v4 + 2]),
+                                      fmaf(ec, ox[8 * v4 + 3], o[8 * v4 + 3]));
+                    u.z = pack_bf16x2(fmaf(ec, ox[8 * v4 + 4], o[8 * v4 + 4]),
+                                      fmaf(ec, ox[8 * v4 + 5], o[8 * v4 + 5]));
+                    u.w = pack_bf16x2(fmaf(ec, ox[8 * v4 + 6], o[8 * v4 + 6]),
+                                      fmaf(ec, ox[8 * v4 + 7], o[8 * v4 + 7]));
+                    // columns 32 jc + 8 v4 .. + 7: 16-byte chunk cc = 4 jc + v4 of the row
+                    const int cc = 4 * jc + v4;
+                    if (full)
+                        *reinterpret_cast<uint4*>(tile + (cc >> 3) * SLAB + r * 128 +
+                                                  (((cc & 7) ^ (r & 7)) << 4)) = u;
+                    else if (t < it.len)
+                        orow[cc] = u;
                 }
             }
             tc_fence_before();
@@ -734,22 +751,22 @@ __device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint
                     for (int half = 0; half < 2; ++half) {
                         set_coord(co, p.o_pos_tok, p.o_pos_head, p.o_pos_b, half * 64, tok, it.h,
                                   it.b);
-                        tma_store_4d(to, sm.sbf + half * SLAB, co[0], co[1], co[2], co[3]);
+                        tma_store_4d(to, tile + half * SLAB, co[0], co[1], co[2], co[3]);
                     }
                     bulk_commit_group();
                     bulk_wait_group_read0();
+                    mbar_arrive(&sm.q_empty[qs]);   // the producer may load the next Q here
                 }
+            } else if (gw.tid == 0) {
+                mbar_arrive(&sm.q_empty[qs]);
             }
-            if (gw.tid == 0) mbar_arrive(&sm.sbf_free);   // the state buffer can be rewritten
-            ++b;
         }
-        if (!ok) break;
     }
     if (gw.tid == 0) bulk_wait_group0();   // the last output tiles are written before exit
 }
 
 // ----------------------------------------------------------------------------------------------
-// warps 8-11: decayed K split, fp32 state, look-back
+// warps 8-11: fp32 state, look-back, bf16 halves of the state for Q S
 
 __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp, int lane) {
     GroupWait gw{&sm, &p, 1, (warp - 8) * 32 + lane};
@@ -757,45 +774,35 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
     const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
     float S[D];
     int j = 0, b = 0, it_n = 0;
-    int dsn = 0;   // dS results taken from the MMA so far (phases of ds_full)
+    uint32_t n_ds = 0;   // aggregates and dS results folded so far (phases of ds_full)
     bool ok = true;
     while (ok) {
         const int slot = it_n % ITEM_DEPTH;
         if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
         const Item& it = sm.items[slot];   // read in place; released at the end of the span
+        const uint32_t use = (uint32_t)(it_n / ITEM_DEPTH);
         ++it_n;
         if (!it.valid) {
             mbar_arrive(&sm.item_empty[slot]);
             break;
         }
         // ---- pass A: the span's aggregate Agg = sum over its keys of (decay to the span's end)
-        // k^T v is accumulated by the dS MMAs over the span's chunks, which arrive last to
-        // first; this group splits its share of w K and sums the span's log2-decay L, then
-        // reads Agg once.
+        // k^T v, accumulated by the MMAs over the span's chunks; the producer sums the span's
+        // log2-decay L.
         const int n = it.c_end - it.c_begin;
 #pragma unroll
         for (int i = 0; i < D; ++i) S[i] = 0.f;
-        float L = 0.f;
-#pragma unroll 1
-        for (int i = 0; i < n; ++i) {
-            const int st = (j + i) & 1;
-            if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
-            L += sm.gtot[st];
-            split_k_chunks<0, SPLIT_STATE>(sm.k[st], sm.q[st], r,
-                                           k_weight(sm, p, it, it.c_end - 1 - i, st, r));
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.k_ready[st]);
-        }
-        j += n;
-        if (!ok) break;
+        if (!gw.wait(&sm.span_done[slot], use & 1)) break;
+        const float L = sm.span_L[slot];
         if (n > 0) {
-            if (!gw.wait(&sm.ds_full, dsn & 1)) break;
+            if (!gw.wait(&sm.ds_full, n_ds & 1)) break;
             tc_fence_after();
-            fold_ds(tmem + lane_base + TM_DS, S, 0.f);   // S = Agg
+            fold_ds(tmem + lane_base + TM_DO, S, 0.f);   // S = Agg
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
-            ++dsn;
+            ++n_ds;
         }
+        j += n;
         // ---- look-back: entry state E of the span; publish exp(L) E + Agg
         const int64_t chain = (int64_t)it.u * p.H + it.h;
         const float* esrc = nullptr;
@@ -810,12 +817,11 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
         const float eL = ex2f(L);
         float4* dst = it.last ? nullptr
                               : reinterpret_cast<float4*>(p.slots + (chain * 2 + (it.s & 1)) * (D * D));
-        // E comes in through the state buffer, free once the previous chunk's output tile has
-        // left it: two rounds of 16 float4 per thread, each thread copying and reading back only
-        // its own elements (no barrier between the rounds), with all 16 copies of a round in
-        // flight.
-        if (b > 0 && !gw.wait(&sm.sbf_free, (b - 1) & 1)) break;
-        float4* ebuf = reinterpret_cast<float4*>(sm.sbf) + r;
+        // E comes in through the state buffer, free once the previous chunk's Q S_lo is done:
+        // two rounds of 16 float4 per thread, each thread copying and reading back only its own
+        // elements (no barrier between the rounds), with all 16 copies of a round in flight.
+        if (b > 0 && !gw.wait(&sm.sb_free, (b - 1) & 1)) break;
+        float4* ebuf = reinterpret_cast<float4*>(sm.sb) + r;
         // float4 j4 of the row: slot layout [j4][row], state_in layout [row][j4]
         const float4* esrc4 =
             reinterpret_cast<const float4*>(esrc) + (from_slot ? r : 0);
@@ -856,39 +862,29 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
             asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(f), "r"((uint32_t)it.s + 1)
                          : "memory");
         }
-        // ---- pass B: running state from E.  Per chunk: the bf16 high half of the state before
-        // it goes into the state buffer (once the previous chunk's output tile has left it) for
-        // Q S_hi, then its low half (kept in registers) once Q S_hi is done, then the chunk's
-        // split of w K (into the Q slot, free after Q S_lo) and the fold of its dS.
+        // ---- pass B: running state from E.  Per chunk: the bf16 high half of the state into
+        // the state buffer for Q S_hi, then (once Q S_hi has read it) the low half for Q S_lo,
+        // then the fold of the chunk's dS.
 #pragma unroll 1
-        for (int i = 0; i < n; ++i) {
-            const int st = (j + i) & 1;
-            uint32_t slo[D / 2];   // bf16 low half of the state row, between its two writes
-            if (b + i > 0 && !gw.wait(&sm.sbf_free, (b + i - 1) & 1)) { ok = false; break; }
-            write_state_hi(sm.sbf, r, S, slo);
+        for (int i = 0; i < n; ++i, ++j, ++b) {
+            const int st = j & 1;
+            if (i > 0 && !gw.wait(&sm.sb_free, (b - 1) & 1)) { ok = false; break; }
+            write_state_half<false>(sm.sb, r, S);
             fence_proxy_async_smem();
             mbar_arrive(&sm.s_ready);
-            if (!gw.wait(&sm.kv_full[st], ((j + i) >> 1) & 1)) { ok = false; break; }
-            if (!gw.wait(&sm.s3a_done, (b + i) & 1)) { ok = false; break; }
-            write_state_lo(sm.sbf, r, slo);
+            if (!gw.wait(&sm.s_hi_done, b & 1)) { ok = false; break; }
+            write_state_half<true>(sm.sb, r, S);
             fence_proxy_async_smem();
             mbar_arrive(&sm.s_lo_ready);
+            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }   // gate slot
             const float tot = sm.gtot[st];
-            // every MMA reading Q has completed: its slot takes the low half of w K
-            if (!gw.wait(&sm.q_free, (b + i) & 1)) { ok = false; break; }
-            split_k_chunks<0, SPLIT_STATE>(sm.k[st], sm.q[st], r,
-                                         k_weight(sm, p, it, it.c_begin + i, st, r));
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.k_ready[st]);
-            if (!gw.wait(&sm.ds_full, dsn & 1)) { ok = false; break; }
+            if (!gw.wait(&sm.ds_full, n_ds & 1)) { ok = false; break; }           // dS
             tc_fence_after();
-            fold_ds(tmem + lane_base + TM_DS, S, ex2f(tot));
+            fold_ds(tmem + lane_base + TM_DO, S, ex2f(tot));
             tc_fence_before();
             mbar_arrive(&sm.ds_free);
-            ++dsn;
+            ++n_ds;
         }
-        j += n;
-        b += n;
         if (!ok) break;
         if (it.last && p.state_out) {
             float4* so = reinterpret_cast<float4*>(p.state_out + (chain * D + r) * D);
@@ -897,42 +893,6 @@ __device__ void state_group(Smem& sm, const TcParams& p, uint32_t tmem, int warp
                 so[j4] = make_float4(S[4 * j4], S[4 * j4 + 1], S[4 * j4 + 2], S[4 * j4 + 3]);
         }
         mbar_arrive(&sm.item_empty[slot]);
-    }
-}
-
-// ----------------------------------------------------------------------------------------------
-// warps 2-3: their share of the w K split (chunks 11-15 of rows 2t and 2t + 1), every chunk
-
-__device__ void split_helper(Smem& sm, const TcParams& p, int warp, int lane) {
-    GroupWait gw{&sm, &p, 2, (warp - 2) * 32 + lane, 64};
-    const int t = (warp - 2) * 32 + lane;
-    int j = 0, b = 0, it_n = 0;
-    bool ok = true;
-    while (ok) {
-        const int slot = it_n % ITEM_DEPTH;
-        if (!gw.wait(&sm.item_full[slot], (it_n / ITEM_DEPTH) & 1)) break;
-        const Item it = sm.items[slot];
-        mbar_arrive(&sm.item_empty[slot]);
-        ++it_n;
-        if (!it.valid) break;
-        const int n_ch = it.c_end - it.c_begin;
-        for (int jj = 0; jj < 2 * n_ch; ++jj, ++j) {
-            const int st = j & 1;
-            const int c = jj < n_ch ? it.c_end - 1 - jj : it.c_begin + (jj - n_ch);
-            if (!gw.wait(&sm.kv_full[st], (j >> 1) & 1)) { ok = false; break; }
-            if (jj >= n_ch) {   // pass B: the Q slot is free once both Q S MMAs are done
-                if (!gw.wait(&sm.q_free, b & 1)) { ok = false; break; }
-                ++b;
-            }
-#pragma unroll 1
-            for (int h = 0; h < 2; ++h) {
-                const int r = 2 * t + h;
-                split_k_chunks<SPLIT_HELP0, SPLIT_HELP>(sm.k[st], sm.q[st], r,
-                                                        k_weight(sm, p, it, c, st, r));
-            }
-            fence_proxy_async_smem();
-            mbar_arrive(&sm.kh_ready[st]);
-        }
     }
 }
 
@@ -949,29 +909,28 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     }
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.kv_full[s], 2);   // TMA bytes + expect_tx arrival, gate arrival
-            mbar_init(&sm.stage_empty[s], 1);
+            mbar_init(&sm.kv_full[s], 2);      // TMA bytes + expect_tx arrival, gate arrival
+            mbar_init(&sm.kv_empty[s], 1 + 128);   // last MMA on the stage, converter group
+            mbar_init(&sm.q_full[s], 1);
+            mbar_init(&sm.q_empty[s], 1);
         }
         for (int s = 0; s < ITEM_DEPTH; ++s) {
             mbar_init(&sm.item_full[s], 1);
-            mbar_init(&sm.item_empty[s], 1 + 128 + 128 + 64);
+            mbar_init(&sm.item_empty[s], 1 + 3 * 128);
+            mbar_init(&sm.span_done[s], 1);
         }
         mbar_init(&sm.a_full, 1);
-        mbar_init(&sm.s3a_done, 1);
-        mbar_init(&sm.q_free, 1);
         mbar_init(&sm.p_ready, 128);
+        mbar_init(&sm.s_ready, 128);
+        mbar_init(&sm.s_hi_done, 1);
         mbar_init(&sm.s_lo_ready, 128);
-        mbar_init(&sm.o_full, 1);
-        mbar_init(&sm.o_free, 128);
-        for (int s = 0; s < 2; ++s) {
-            mbar_init(&sm.k_ready[s], 128);
-            mbar_init(&sm.kp_ready[s], 128);
-            mbar_init(&sm.kh_ready[s], 64);
-        }
+        mbar_init(&sm.sb_free, 1);
+        mbar_init(&sm.kt_ready, 128);
+        mbar_init(&sm.kt_free, 1);
         mbar_init(&sm.ds_full, 1);
         mbar_init(&sm.ds_free, 128);
-        mbar_init(&sm.s_ready, 128);
-        mbar_init(&sm.sbf_free, 1);
+        mbar_init(&sm.o_full, 1);
+        mbar_init(&sm.o_free, 128);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -985,7 +944,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 88;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
         if (warp == 0) {
             if (lane == 0) {
                 tma_prefetch_desc(&tq);
@@ -998,17 +957,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             producer(sm, p, &tq, &tk, &tv, total, lane);
         } else if (warp == 1) {
             if (lane == 0) mma_issuer(sm, p, tmem);
-        } else {
-            split_helper(sm, p, warp, lane);
         }
     } else if (warp < 8) {
-        // 168 -> 136 is a decrease: setmaxnreg.inc must never ask for fewer registers than the
-        // warp holds, and .dec never for more.
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 136;" ::: "memory");
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 136;" ::: "memory");
         p_group(sm, p, &to, tmem, warp, lane);
-    } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 256;" ::: "memory");
+    } else if (warp < 12) {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
         state_group(sm, p, tmem, warp, lane);
+    } else {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 72;" ::: "memory");
+        converter(sm, p, tmem, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -1017,6 +975,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         tmem_dealloc(tmem, 512);
     }
 }
+
+// One 32-bit word of the workspace (the failure-path test's first span ticket).
+__global__ void set_u32_kernel(uint32_t* w, uint32_t value) { *w = value; }
 
 // Varlen: spans per sequence and their exclusive prefix (one CTA).
 __global__ void __launch_bounds__(1024) plan_kernel(const int32_t* __restrict__ cu, int units, int G,
@@ -1175,6 +1136,7 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
     p.G = G;
     const int64_t nc_dense = (a.N + C - 1) / C;
     p.spans_per_unit = (int)std::max<int64_t>(1, (nc_dense + G - 1) / G);
+    p.wait_ns = a.test_wait_ns > 0 ? a.test_wait_ns : WAIT_NS;
 
     const int64_t ntok = a.N;   // dense: tokens per sequence; varlen: packed total
     const int B = varlen ? 1 : a.B;
@@ -1197,6 +1159,10 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
         if (span_bound * (uint64_t)a.H > 0xFFFFFFF0ull) return GRET_ERR_UNSUPPORTED;
     }
     if (cudaMemsetAsync(ws, 0, L.prefix, a.stream) != cudaSuccess) return GRET_ERR_CUDA;
+    if (a.test_first_ticket > 0) {
+        set_u32_kernel<<<1, 1, 0, a.stream>>>(p.ticket, a.test_first_ticket);
+        if (cudaGetLastError() != cudaSuccess) return GRET_ERR_CUDA;
+    }
     if (varlen) {
         plan_kernel<<<1, 1024, 0, a.stream>>>(a.cu_seqlens, units, G, p.prefix);
         if (cudaGetLastError() != cudaSuccess) return GRET_ERR_CUDA;
@@ -1206,14 +1172,14 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
                              (int)smem) != cudaSuccess)
         return GRET_ERR_CUDA;
     {
-        // the in-kernel register split (setmaxnreg) assumes exactly 168 registers per thread
+        // the in-kernel register split (setmaxnreg) assumes exactly LAUNCH_REGS per thread
         static int regs = -1;
         if (regs < 0) {
             cudaFuncAttributes fa;
             if (cudaFuncGetAttributes(&fa, prefill_tc_kernel) != cudaSuccess) return GRET_ERR_CUDA;
             regs = fa.numRegs;
         }
-        if (regs != 168) return GRET_ERR_UNSUPPORTED;
+        if (regs != LAUNCH_REGS) return GRET_ERR_UNSUPPORTED;
     }
     int grid = sm_count();
     if (!varlen && total_dense < (uint64_t)grid) grid = (int)total_dense;

@@ -109,6 +109,27 @@ gret_status_t gret_prefill_chunkwise(
     size_t workspace_bytes, gret_stream_t stream);
 
 /*
+ * gret_prefill_chunkwise with two settings that exist only to test its failure path; production
+ * callers use gret_prefill_chunkwise.  The paper has no counterpart.
+ *   wait_ns       limit of every bounded wait of the tensor-core kernel, in ns (the regular entry
+ *                 point uses 2 s); 1 .. 2e9, else GRET_ERR_INVALID_ARG.
+ *   first_ticket  the first span ticket handed out (0 as in the regular call).  A value past span
+ *                 0 of a chain leaves that span's look-back flag unset, so the waits of the later
+ *                 spans of the chain give up after wait_ns: the call then records
+ *                 GRET_ERR_TIMEOUT for gret_workspace_status, the kernel stops, and its outputs
+ *                 are invalid.  The CUDA context stays usable.
+ * Other arguments, results and errors as gret_prefill_chunkwise.
+ */
+gret_status_t gret_prefill_chunkwise_testing(
+    const void* q, const void* k, int64_t stride_batch, int64_t stride_tok, int64_t stride_head,
+    const void* v, int64_t v_stride_batch, int64_t v_stride_tok, int64_t v_stride_head,
+    const float* g, float tau, float k_scale, gret_dtype_t dtype, int B,
+    int64_t N, int H, int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs,
+    const float* state_in, float* state_out, void* o, int64_t o_stride_batch,
+    int64_t o_stride_tok, int64_t o_stride_head, int chunk, void* workspace,
+    size_t workspace_bytes, gret_stream_t stream, uint64_t wait_ns, uint32_t first_ticket);
+
+/*
  * gret_prefill_chunkwise without a workspace argument and without allocating.  The paper has no
  * counterpart: this entry point exists for callers that cannot allocate device memory when they
  * call, for example a serving process that gives all device memory to its own pool at start-up,
@@ -245,6 +266,27 @@ size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d);
 gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, float scale,
                                int window, int B, int64_t N, int H, int d, void* o,
                                gret_stream_t stream);
+
+/*
+ * One decode step of sliding-window attention ("路线一：滑动窗口注意力": at decode time only the
+ * most recent `window` positions' keys and values are kept).  Each (b, h) keeps a ring of
+ * `window` cache slots, token t in slot t % window.  With t = pos[b], the index of the new token
+ * in sequence b (0 for its first token):
+ *   k_cache[b, h, t % window] = k[b, h] ;  v_cache[b, h, t % window] = v[b, h]
+ *   o[b, h] = sum_{j = max(0, t-window+1) .. t} softmax_j(scale q . k_j) v_j
+ * which is gret_swa_prefill's output at position t.  The slot written held token t - window,
+ * which has just left the window.
+ *   q, k, v, o   bf16 [B, H, d] contiguous.
+ *   pos          device int32 [B], pos[b] >= 0; read only (the caller advances it).
+ *   k_cache, v_cache  bf16 [B, H, window, d] contiguous, owned by the caller and updated in
+ *                place; slots of tokens not yet seen are never read.
+ * Requires d == 128 and window <= 32768 (GRET_ERR_UNSUPPORTED otherwise); pointers 16-byte
+ * aligned, pos 4-byte aligned (GRET_ERR_ALIGNMENT).  fp32 scores and softmax; o rounded to bf16
+ * once.  Memory-bound: the window's keys and values are read once.
+ */
+gret_status_t gret_swa_decode_step(const void* q, const void* k, const void* v, float scale,
+                                   int window, int B, int H, int d, const int32_t* pos,
+                                   void* k_cache, void* v_cache, void* o, gret_stream_t stream);
 
 #ifdef __cplusplus
 }
