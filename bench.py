@@ -245,6 +245,29 @@ def run_gpu(args):
     alg_bytes = B * N * H * BYTES_PER_TOKEN_HEAD
     achieved = alg_bytes / (launch_ms * 1e-3) / 1e9
 
+    # ---------------- the same prefill at every chunk size the library takes
+    sweep = None
+    if args.chunk_sweep:
+        sweep = {}
+        for ch in (16, 32, 64, 128):
+            def stepc():
+                G.gret_prefill_chunkwise(q, k, v, g, state_out=s_out, o=o, workspace=ws, chunk=ch)
+            for _ in range(2):
+                stepc()
+            torch.cuda.synchronize()
+            c0 = torch.cuda.Event(enable_timing=True)
+            c1 = torch.cuda.Event(enable_timing=True)
+            nrep = 3 if ch < 128 else 10
+            c0.record(stream)
+            for _ in range(nrep):
+                stepc()
+            c1.record(stream)
+            torch.cuda.synchronize()
+            cms = c0.elapsed_time(c1) / nrep
+            sweep[str(ch)] = {"ms": cms, "Mtok_s": B * N / (cms * 1e-3) / 1e6,
+                              "hbm_frac": alg_bytes / (cms * 1e-3) / 1e9 / hbm_peak,
+                              "path": "tcgen05" if ch == 128 else "CUDA cores (fp32 FMA)"}
+
     # ---------------- decode at batch 64
     dec = None
     if not args.no_decode:
@@ -384,6 +407,7 @@ def run_gpu(args):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "config": bench_config(world),
+        "chunk_sweep": sweep,
         "decode": dec, "varlen_epilogue": epi, "layer": lay,
         "elementwise_gate": ew, "sliding_window": swa,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
@@ -792,6 +816,9 @@ def main():
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--no-elementwise", action="store_true")
     ap.add_argument("--no-swa", action="store_true")
+    ap.add_argument("--chunk-sweep", action="store_true",
+                    help="also time the 3B-shaped prefill at every chunk size the library takes "
+                         "(16, 32, 64 on CUDA cores, 128 on the tensor cores)")
     ap.add_argument("--varlen-max-len", type=int, default=65536,
                     help="longest sequence of the varlen + epilogue leg (a smaller value gives "
                          "a small case for profiling)")

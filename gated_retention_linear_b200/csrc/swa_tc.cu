@@ -1,0 +1,388 @@
+// swa_tc.cu -- sliding-window softmax attention prefill on the sm_100a tensor cores.
+//
+// Page "YOCO 完全拆解：Decoder-Decoder 架构如何让 KV Cache 只存一次", section
+// "路线一：滑动窗口注意力": position i attends to the most recent W positions of its sequence,
+//   o_i = sum_{j = i-W+1 .. i} softmax_j(scale q_i . k_j) v_j .
+// FlashAttention-style, as the page suggests for this mixer, built on tcgen05:
+//   * one CTA takes two 128-query tiles of one (batch, head), queries q0 .. q0 + 255; the key
+//     tiles of 128 that their windows touch (ten at W = 1024) stream through two TMA stages and
+//     serve both query tiles;
+//   * S = Q K^T for each query tile goes to tensor memory; a softmax warpgroup per query tile
+//     (one query row per thread) masks the window, keeps the running maximum and sum, writes
+//     P = 2^(s - m) back over S as a bf16 high + low pair, and the MMA warp accumulates
+//     O += P_hi V + P_lo V in tensor memory;
+//   * the two warpgroups take turns: while one runs its softmax, the tensor cores run the other
+//     tile's products;
+//   * the running maximum is only moved (and O rescaled) when a tile's maximum exceeds it by
+//     more than 2^8, so rescaling is rare after the first tiles; P then stays below 256;
+//   * the output, O / l in bf16, leaves through the query tile's own shared-memory slot by TMA
+//     store (rows past the sequence end are clipped by the store).
+// P is carried as two bf16 halves because a single bf16 rounding of P over a 1024-key window
+// leaves errors near 1e-2 of rms; the pair keeps the result near 1e-5.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
+// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 and
+// 8-11 the softmax warpgroups of query tiles 0 and 1.  Registers: launched at 168 per thread;
+// warps 0-3 drop to 40 and the softmax groups rise to 232 (128 x (40 + 232 + 232) = 64512).
+// Every wait is bounded; a wait that gives up makes the CTA stop and write NaN into its output
+// rows that are still to be written.
+#include <cuda_bf16.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "swa.cuh"
+#include "tma_host.cuh"
+
+namespace gret {
+
+using namespace sm100;
+
+namespace {
+
+constexpr int D = SWA_DIM;
+constexpr int BM = 128;                  // queries per tile, keys per tile
+constexpr int TILE = BM * D * 2;         // one bf16 128 x 128 tile
+constexpr int SLAB = TILE / 2;
+constexpr int NTHREADS = 384;
+constexpr int LAUNCH_REGS = 168;
+constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_NS = 200000000ull;
+constexpr float RESCALE_LOG2 = 8.f;      // move the running maximum only past this margin
+
+struct __align__(1024) SwaSmem {
+    unsigned char q[2][TILE];            // the two query tiles; later their output tiles
+    unsigned char k[2][TILE];
+    unsigned char v[2][TILE];
+    uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_ready[2], pv_done[2], drain;
+    uint32_t tmem_base;
+    uint32_t abort;
+};
+static_assert(sizeof(SwaSmem) <= 232448, "shared-memory plan exceeds 227 KB");
+
+struct SwaParams {
+    float scale_log2;      // scale * log2(e)
+    int window;
+    int64_t N;
+    int H;
+    int n_qpairs;          // query-tile pairs per sequence
+};
+
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// does query tile w (queries q0 + 128 w .. + 127) see any key of key tile kt?
+__device__ __forceinline__ bool takes_part(int64_t q0, int w, int64_t kt, int window, int64_t N) {
+    const int64_t qa = q0 + BM * w, qb = qa + BM - 1;
+    if (qa >= N) return false;                     // the tile is past the sequence end
+    const int64_t ka = BM * kt, kb = ka + BM - 1;
+    return ka <= qb && kb >= qa - window + 1;
+}
+
+// Exit-time wait for this CTA's own asynchronous work; bounded, and not cut short by an abort.
+__device__ __forceinline__ void mbar_wait_drain_(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
+    uint32_t never = 0;
+    mbar_wait(bar, parity, &never, limit_ns);
+}
+
+__device__ __forceinline__ bool wait_abortable(SwaSmem& sm, uint64_t* bar, uint32_t parity) {
+    if (mbar_wait(bar, parity, &sm.abort, WAIT_NS)) return true;
+    atomicExch(&sm.abort, 1u);
+    return false;
+}
+
+// S (+)= A B over K = 128 with both operands K-major in shared memory (A = Q, B = K).
+__device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a_base, uint32_t b_base) {
+    const uint32_t idesc = idesc_bf16(128, 128, 0, 0);
+#pragma unroll 1
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t off = (kk >> 2) * SLAB + (kk & 3) * 32u;
+        mma_ss(d, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), idesc,
+               kk > 0 ? 1u : 0u);
+    }
+}
+
+// O (+)= P V with P (bf16 halves, K-major) in TMEM: per 32-key group, 16 columns of high halves
+// then 16 of low halves; V [key x d] MN-major in shared memory.
+__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
+                                       bool accumulate) {
+    const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+#pragma unroll 1
+    for (int kk = 0; kk < 8; ++kk)
+        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
+               sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
+}
+
+__global__ void __launch_bounds__(NTHREADS, 1)
+    swa_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
+                  const SwaParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    SwaSmem& sm = *reinterpret_cast<SwaSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if ((smem_u32(smem_raw) & 1023u) != 0) return;   // never: dynamic shared memory starts aligned
+    // the CTA's work: (batch, head, query-tile pair)
+    const int64_t blk = blockIdx.x;
+    const int pair = (int)(blk % p.n_qpairs);
+    const int h = (int)((blk / p.n_qpairs) % p.H);
+    const int b = (int)(blk / ((int64_t)p.n_qpairs * p.H));
+    const int64_t q0 = (int64_t)pair * 2 * BM;
+    const int64_t qlast = (q0 + 2 * BM - 1 < p.N - 1) ? q0 + 2 * BM - 1 : p.N - 1;
+    const int64_t kfirst = (q0 - p.window + 1 > 0) ? q0 - p.window + 1 : 0;
+    const int64_t kt_lo = kfirst / BM, kt_hi = qlast / BM;
+    const int ntiles = (int)(kt_hi - kt_lo + 1);
+
+    if (tid == 0) {
+        mbar_init(&sm.q_full, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.kv_full[s], 1);
+            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.s_full[s], 1);
+            mbar_init(&sm.p_ready[s], 128);
+            mbar_init(&sm.pv_done[s], 1);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.abort = 0;
+        fence_mbar_init();
+    }
+    if (warp == 1) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+
+    if (warp < 4) {
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+        if (warp == 0 && lane == 0) {
+            // ---- producer: both query tiles, then the key / value tiles through two stages
+            tma_prefetch_desc(&tq);
+            tma_prefetch_desc(&tk);
+            tma_prefetch_desc(&tv);
+            tma_prefetch_desc(&to);
+            mbar_arrive_expect_tx(&sm.q_full, 2 * TILE);
+            for (int w = 0; w < 2; ++w)
+                for (int half = 0; half < 2; ++half)
+                    tma_load_4d(sm.q[w] + half * SLAB, &tq, &sm.q_full, half * 64, h,
+                                (int)(q0 + BM * w), b);
+            int i = 0;
+            for (; i < ntiles; ++i) {
+                const int st = i & 1;
+                if (i >= 2 && !wait_abortable(sm, &sm.kv_empty[st], ((i >> 1) - 1) & 1)) break;
+                const int tok = (int)((kt_lo + i) * BM);
+                mbar_arrive_expect_tx(&sm.kv_full[st], 2 * TILE);
+                for (int half = 0; half < 2; ++half) {
+                    tma_load_4d(sm.k[st] + half * SLAB, &tk, &sm.kv_full[st], half * 64, h, tok, b);
+                    tma_load_4d(sm.v[st] + half * SLAB, &tv, &sm.kv_full[st], half * 64, h, tok, b);
+                }
+            }
+            // no TMA write into this CTA's shared memory may be in flight at exit
+            mbar_wait_drain_(&sm.q_full, 0, DRAIN_NS);
+            for (int ii = (i >= 2 ? i - 2 : 0); ii < i; ++ii)
+                mbar_wait_drain_(&sm.kv_full[ii & 1], (ii >> 1) & 1, DRAIN_NS);
+        } else if (warp == 1 && lane == 0) {
+            // ---- MMA issuer
+            bool ok = wait_abortable(sm, &sm.q_full, 0);
+            int cnt[2] = {0, 0};
+            for (int i = 0; i < ntiles && ok; ++i) {
+                const int st = i & 1;
+                const int64_t kt = kt_lo + i;
+                const bool part[2] = {takes_part(q0, 0, kt, p.window, p.N),
+                                      takes_part(q0, 1, kt, p.window, p.N)};
+                if (!(ok = wait_abortable(sm, &sm.kv_full[st], (i >> 1) & 1))) break;
+                tc_fence_after();
+                for (int w = 0; w < 2 && ok; ++w) {
+                    if (!part[w]) continue;
+                    // P of this tile's previous key tile has been read by its P V
+                    if (cnt[w] > 0 && !(ok = wait_abortable(sm, &sm.pv_done[w], (cnt[w] - 1) & 1)))
+                        break;
+                    tc_fence_after();
+                    mma_qk(tmem + BM * w, smem_u32(sm.q[w]), smem_u32(sm.k[st]));
+                    mma_commit(&sm.s_full[w]);
+                }
+                for (int w = 0; w < 2 && ok; ++w) {
+                    if (!part[w]) continue;
+                    if (!(ok = wait_abortable(sm, &sm.p_ready[w], cnt[w] & 1))) break;
+                    tc_fence_after();
+                    const uint32_t vb = smem_u32(sm.v[st]);
+                    mma_pv(tmem + 256 + BM * w, tmem + BM * w, 0, vb, cnt[w] > 0);
+                    mma_pv(tmem + 256 + BM * w, tmem + BM * w, 1, vb, true);
+                    mma_commit(&sm.pv_done[w]);
+                    ++cnt[w];
+                }
+                mma_commit(&sm.kv_empty[st]);
+            }
+            mma_commit(&sm.drain);
+            mbar_wait_drain_(&sm.drain, 0, DRAIN_NS);
+        }
+    } else {
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
+        // ---- softmax warpgroup w: query row r of query tile w
+        const int w = (warp - 4) >> 2;
+        const int q = warp & 3, r = q * 32 + lane;
+        const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
+        const uint32_t s_addr = tmem + lane_base + BM * w;
+        const uint32_t o_addr = tmem + lane_base + 256 + BM * w;
+        const int64_t qi = q0 + BM * w + r;      // this thread's query position
+        float m_ref = -INFINITY, l = 0.f;
+        int cnt = 0;
+        bool ok = true;
+        for (int i = 0; i < ntiles && ok; ++i) {
+            const int64_t kt = kt_lo + i;
+            if (!takes_part(q0, w, kt, p.window, p.N)) continue;
+            // warp-uniform outcome: a warp must not split around the warp-wide TMEM accesses
+            ok = __all_sync(0xffffffffu, wait_abortable(sm, &sm.s_full[w], cnt & 1));
+            if (!ok) break;
+            tc_fence_after();
+            // visible keys of this row in this tile: columns [c_lo, c_hi]
+            const int64_t c_lo64 = qi - p.window + 1 - BM * kt, c_hi64 = qi - BM * kt;
+            const int c_lo = c_lo64 < 0 ? 0 : (c_lo64 > BM ? BM : (int)c_lo64);
+            const int c_hi = c_hi64 > BM - 1 ? BM - 1 : (c_hi64 < -1 ? -1 : (int)c_hi64);
+            float s[BM];
+#pragma unroll
+            for (int jc = 0; jc < 4; ++jc) {
+                float t32[32];
+                tmem_ld32(s_addr + jc * 32, t32);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) s[jc * 32 + e] = t32[e] * p.scale_log2;
+            }
+            float mx = -INFINITY;
+#pragma unroll
+            for (int c = 0; c < BM; ++c)
+                if (c >= c_lo && c <= c_hi) mx = fmaxf(mx, s[c]);
+            // move the reference when this tile's maximum passes it by the margin: O and l
+            // scale by 2^(m_ref - mx).  The tensor-memory accesses are warp-wide instructions,
+            // so the whole warp takes the branch when any of its rows needs it (factor 1 for
+            // the others).
+            const bool move = mx > m_ref + RESCALE_LOG2;
+            const bool rescale = move && l > 0.f;
+            if (__any_sync(0xffffffffu, rescale)) {
+                const float f = rescale ? ex2f(m_ref - mx) : 1.f;
+                l *= f;
+#pragma unroll 1
+                for (int jc = 0; jc < 4; ++jc) {
+                    float t32[32];
+                    tmem_ld32(o_addr + jc * 32, t32);
+                    tmem_ld_wait();
+                    uint32_t u[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(t32[e] * f);
+                    tmem_st32(o_addr + jc * 32, u);
+                }
+            }
+            if (move) m_ref = mx;
+#pragma unroll
+            for (int jc = 0; jc < 4; ++jc) {
+                uint32_t ph[32];
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                    const int c0 = jc * 32 + 2 * e;
+                    const float p0 = (c0 >= c_lo && c0 <= c_hi) ? ex2f(s[c0] - m_ref) : 0.f;
+                    const float p1 =
+                        (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? ex2f(s[c0 + 1] - m_ref) : 0.f;
+                    l += p0 + p1;
+                    split2(p0, p1, ph[e], ph[16 + e]);
+                }
+                tmem_st32(s_addr + jc * 32, ph);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready[w]);
+            ++cnt;
+        }
+        // ---- epilogue: O / l in bf16 through this tile's query slot, then one TMA store
+        if (cnt > 0) {
+            if (ok) ok = __all_sync(0xffffffffu, wait_abortable(sm, &sm.pv_done[w], (cnt - 1) & 1));
+            tc_fence_after();
+            const float inv = ok && l > 0.f ? 1.f / l : __int_as_float(0x7fc00000);
+            unsigned char* tile = sm.q[w];
+#pragma unroll 1
+            for (int jc = 0; jc < 4; ++jc) {
+                float t32[32];
+                tmem_ld32(o_addr + jc * 32, t32);
+                tmem_ld_wait();
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    uint4 u;
+                    u.x = pack_bf16x2(t32[8 * v4 + 0] * inv, t32[8 * v4 + 1] * inv);
+                    u.y = pack_bf16x2(t32[8 * v4 + 2] * inv, t32[8 * v4 + 3] * inv);
+                    u.z = pack_bf16x2(t32[8 * v4 + 4] * inv, t32[8 * v4 + 5] * inv);
+                    u.w = pack_bf16x2(t32[8 * v4 + 6] * inv, t32[8 * v4 + 7] * inv);
+                    const int cc = 4 * jc + v4;
+                    *reinterpret_cast<uint4*>(tile + (cc >> 3) * SLAB + r * 128 +
+                                              (((cc & 7) ^ (r & 7)) << 4)) = u;
+                }
+            }
+            fence_proxy_async_smem();
+            asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");   // the tile is written
+            if (r == 0) {
+                for (int half = 0; half < 2; ++half)
+                    tma_store_4d(&to, tile + half * SLAB, half * 64, h, (int)(q0 + BM * w), b);
+                bulk_commit_group();
+                bulk_wait_group0();
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_swa(const SwaArgs& a, cudaStream_t stream) {
+    // [B, N, H, 128] contiguous: dims (d, head, token, batch), box (64, 1, 128, 1)
+    const uint64_t dims[4] = {(uint64_t)D, (uint64_t)a.H, (uint64_t)a.N, (uint64_t)a.B};
+    const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2,
+                                 (uint64_t)a.N * a.H * D * 2};
+    const uint32_t box[4] = {64, 1, BM, 1};
+    CUtensorMap tq, tk, tv, to;
+    if (!make_bf16_map(&tq, a.q, 4, dims, strides, box) ||
+        !make_bf16_map(&tk, a.k, 4, dims, strides, box) ||
+        !make_bf16_map(&tv, a.v, 4, dims, strides, box) ||
+        !make_bf16_map(&to, a.o, 4, dims, strides, box))
+        return cudaErrorInvalidValue;
+    if (a.N > (int64_t)0x7FFFFE00) return cudaErrorInvalidValue;   // 32-bit token coordinates
+    SwaParams p;
+    p.scale_log2 = a.scale * 1.4426950408889634f;
+    p.window = a.window;
+    p.N = a.N;
+    p.H = a.H;
+    p.n_qpairs = (int)((a.N + 2 * BM - 1) / (2 * BM));
+    const int64_t grid = (int64_t)a.B * a.H * p.n_qpairs;
+    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    const size_t smem = sizeof(SwaSmem);
+    cudaError_t e = cudaFuncSetAttribute(swa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return e;
+    static int regs = -1;
+    if (regs < 0) {
+        cudaFuncAttributes fa;
+        if (cudaFuncGetAttributes(&fa, swa_tc_kernel) != cudaSuccess) return cudaErrorUnknown;
+        regs = fa.numRegs;
+    }
+    // the in-kernel register split (setmaxnreg) assumes exactly LAUNCH_REGS per thread
+    if (regs != LAUNCH_REGS) return cudaErrorInvalidValue;
+    swa_tc_kernel<<<(unsigned)grid, NTHREADS, smem, stream>>>(tq, tk, tv, to, p);
+    return cudaGetLastError();
+}
+
+}  // namespace gret
