@@ -24,7 +24,8 @@
 // 8-11 the softmax warpgroups of query tiles 0 and 1.  Registers: launched at 168 per thread;
 // warps 0-3 drop to 40 and the softmax groups rise to 232 (128 x (40 + 232 + 232) = 64512).
 // Every wait is bounded; a wait that gives up makes the CTA stop and write NaN into its output
-// rows that are still to be written.
+// rows that are still to be written.  In a softmax warpgroup one thread waits while the others
+// sleep at the group's named barrier.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -55,6 +56,7 @@ struct __align__(1024) SwaSmem {
     unsigned char k[2][TILE];
     unsigned char v[2][TILE];
     uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_ready[2], pv_done[2], drain;
+    uint32_t dec[2][2];                  // the softmax groups' shared wait outcomes
     uint32_t tmem_base;
     uint32_t abort;
 };
@@ -100,6 +102,19 @@ __device__ __forceinline__ bool wait_abortable(SwaSmem& sm, uint64_t* bar, uint3
     if (mbar_wait(bar, parity, &sm.abort, WAIT_NS)) return true;
     atomicExch(&sm.abort, 1u);
     return false;
+}
+
+// A softmax warpgroup's wait: one thread polls the barrier, the other 127 sleep at the group's
+// named barrier (no issue slots burned by 128 polling threads), and all take the same branch.
+// The outcome word is double-buffered, so that a fast thread 0 cannot overwrite it for the next
+// wait before a slow thread of the group has read it for this one.
+__device__ __forceinline__ bool group_wait(SwaSmem& sm, uint64_t* bar, uint32_t parity, int w,
+                                           int r, int& flip) {
+    if (r == 0) sm.dec[w][flip] = wait_abortable(sm, bar, parity) ? 1u : 0u;
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+    const bool ok = *reinterpret_cast<volatile uint32_t*>(&sm.dec[w][flip]) != 0;
+    flip ^= 1;
+    return ok;
 }
 
 // S (+)= A B over K = 128 with both operands K-major in shared memory (A = Q, B = K).
@@ -239,13 +254,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t o_addr = tmem + lane_base + 256 + BM * w;
         const int64_t qi = q0 + BM * w + r;      // this thread's query position
         float m_ref = -INFINITY, l = 0.f;
-        int cnt = 0;
+        int cnt = 0, flip = 0;
         bool ok = true;
         for (int i = 0; i < ntiles && ok; ++i) {
             const int64_t kt = kt_lo + i;
             if (!takes_part(q0, w, kt, p.window, p.N)) continue;
-            // warp-uniform outcome: a warp must not split around the warp-wide TMEM accesses
-            ok = __all_sync(0xffffffffu, wait_abortable(sm, &sm.s_full[w], cnt & 1));
+            // group-uniform outcome: no warp may split around the warp-wide TMEM accesses
+            ok = group_wait(sm, &sm.s_full[w], cnt & 1, w, r, flip);
             if (!ok) break;
             tc_fence_after();
             // visible keys of this row in this tile: columns [c_lo, c_hi]
@@ -259,12 +274,24 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 tmem_ld32(s_addr + jc * 32, t32);
                 tmem_ld_wait();
 #pragma unroll
-                for (int e = 0; e < 32; ++e) s[jc * 32 + e] = t32[e] * p.scale_log2;
+                for (int e = 0; e < 32; ++e) s[jc * 32 + e] = t32[e];
             }
-            float mx = -INFINITY;
+            // scores in log2 units are c s; the tile's maximum of c s over the visible keys is
+            // c max(s) for c >= 0 and c min(s) otherwise.  Tiles wholly inside every row's
+            // window (all but the first and the last few) skip the per-key mask.
+            const float c = p.scale_log2;
+            const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == BM - 1);
+            float ext = c >= 0.f ? -INFINITY : INFINITY;
+            if (full) {
 #pragma unroll
-            for (int c = 0; c < BM; ++c)
-                if (c >= c_lo && c <= c_hi) mx = fmaxf(mx, s[c]);
+                for (int cc = 0; cc < BM; ++cc) ext = c >= 0.f ? fmaxf(ext, s[cc]) : fminf(ext, s[cc]);
+            } else {
+#pragma unroll
+                for (int cc = 0; cc < BM; ++cc)
+                    if (cc >= c_lo && cc <= c_hi)
+                        ext = c >= 0.f ? fmaxf(ext, s[cc]) : fminf(ext, s[cc]);
+            }
+            const float mx = (c_lo <= c_hi) ? c * ext : -INFINITY;
             // move the reference when this tile's maximum passes it by the margin: O and l
             // scale by 2^(m_ref - mx).  The tensor-memory accesses are warp-wide instructions,
             // so the whole warp takes the branch when any of its rows needs it (factor 1 for
@@ -286,15 +313,18 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
             }
             if (move) m_ref = mx;
+            const float nm = -m_ref;   // finite whenever a key of the row is visible
 #pragma unroll
             for (int jc = 0; jc < 4; ++jc) {
                 uint32_t ph[32];
 #pragma unroll
                 for (int e = 0; e < 16; ++e) {
                     const int c0 = jc * 32 + 2 * e;
-                    const float p0 = (c0 >= c_lo && c0 <= c_hi) ? ex2f(s[c0] - m_ref) : 0.f;
-                    const float p1 =
-                        (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? ex2f(s[c0 + 1] - m_ref) : 0.f;
+                    float p0 = ex2f(fmaf(s[c0], c, nm)), p1 = ex2f(fmaf(s[c0 + 1], c, nm));
+                    if (!full) {
+                        p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
+                        p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
+                    }
                     l += p0 + p1;
                     split2(p0, p1, ph[e], ph[16 + e]);
                 }
@@ -307,7 +337,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         // ---- epilogue: O / l in bf16 through this tile's query slot, then one TMA store
         if (cnt > 0) {
-            if (ok) ok = __all_sync(0xffffffffu, wait_abortable(sm, &sm.pv_done[w], (cnt - 1) & 1));
+            if (ok) ok = group_wait(sm, &sm.pv_done[w], (cnt - 1) & 1, w, r, flip);
             tc_fence_after();
             const float inv = ok && l > 0.f ? 1.f / l : __int_as_float(0x7fc00000);
             unsigned char* tile = sm.q[w];
