@@ -18,7 +18,8 @@
 //   * the output, O / l in bf16, leaves through the query tile's own shared-memory slot by TMA
 //     store (rows past the sequence end are clipped by the store).
 // P is carried as two bf16 halves because a single bf16 rounding of P over a 1024-key window
-// leaves errors near 1e-2 of rms; the pair keeps the result near 1e-5.
+// leaves errors near 1e-2 of rms; the pair (split by truncation, see split2_trunc) keeps the
+// result near 1e-5.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 and
 // 8-11 the softmax warpgroups of query tiles 0 and 1.  Registers: launched at 168 per thread;
@@ -82,6 +83,18 @@ __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_
     const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
     hi = *reinterpret_cast<const uint32_t*>(&h);
     lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// x = hi + lo in bf16 without the conversion unit: hi keeps the top 16 bits of x (its sign,
+// exponent and 7 fraction bits: truncation), lo = x - hi is exact in fp32 and is truncated the
+// same way.  |hi + lo - x| <= 2^-15 |x|, against 2^-17 with round-to-nearest halves; all of it
+// runs on the integer and FMA pipes (bit masks, one subtraction, one byte permute per pair).
+__device__ __forceinline__ void split2_trunc(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const uint32_t b0 = __float_as_uint(x0), b1 = __float_as_uint(x1);
+    const float l0 = x0 - __uint_as_float(b0 & 0xFFFF0000u);
+    const float l1 = x1 - __uint_as_float(b1 & 0xFFFF0000u);
+    hi = __byte_perm(b0, b1, 0x7632);   // upper halves: x0 in the low 16 bits, x1 in the high
+    lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
 }
 
 // does query tile w (queries q0 + 128 w .. + 127) see any key of key tile kt?
@@ -281,15 +294,34 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             // window (all but the first and the last few) skip the per-key mask.
             const float c = p.scale_log2;
             const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == BM - 1);
-            float ext = c >= 0.f ? -INFINITY : INFINITY;
-            if (full) {
+            // eight independent partial extrema, so that the reduction is not one 128-long
+            // dependency chain
+            float ext;
+            {
+                const bool up = c >= 0.f;
+                float e8[8];
 #pragma unroll
-                for (int cc = 0; cc < BM; ++cc) ext = c >= 0.f ? fmaxf(ext, s[cc]) : fminf(ext, s[cc]);
-            } else {
+                for (int u = 0; u < 8; ++u) e8[u] = up ? -INFINITY : INFINITY;
+                if (full) {
+                    if (up) {
 #pragma unroll
-                for (int cc = 0; cc < BM; ++cc)
-                    if (cc >= c_lo && cc <= c_hi)
-                        ext = c >= 0.f ? fmaxf(ext, s[cc]) : fminf(ext, s[cc]);
+                        for (int cc = 0; cc < BM; ++cc) e8[cc & 7] = fmaxf(e8[cc & 7], s[cc]);
+                    } else {
+#pragma unroll
+                        for (int cc = 0; cc < BM; ++cc) e8[cc & 7] = fminf(e8[cc & 7], s[cc]);
+                    }
+                } else {
+#pragma unroll
+                    for (int cc = 0; cc < BM; ++cc)
+                        if (cc >= c_lo && cc <= c_hi)
+                            e8[cc & 7] = up ? fmaxf(e8[cc & 7], s[cc]) : fminf(e8[cc & 7], s[cc]);
+                }
+#pragma unroll
+                for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+                    for (int v = 0; v < u; ++v)
+                        e8[v] = up ? fmaxf(e8[v], e8[v + u]) : fminf(e8[v], e8[v + u]);
+                ext = e8[0];
             }
             const float mx = (c_lo <= c_hi) ? c * ext : -INFINITY;
             // move the reference when this tile's maximum passes it by the margin: O and l
@@ -314,6 +346,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (move) m_ref = mx;
             const float nm = -m_ref;   // finite whenever a key of the row is visible
+            float l4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
             for (int jc = 0; jc < 4; ++jc) {
                 uint32_t ph[32];
@@ -325,11 +358,12 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                         p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
                         p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
                     }
-                    l += p0 + p1;
-                    split2(p0, p1, ph[e], ph[16 + e]);
+                    l4[e & 3] += p0 + p1;
+                    split2_trunc(p0, p1, ph[e], ph[16 + e]);
                 }
                 tmem_st32(s_addr + jc * 32, ph);
             }
+            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
             tmem_st_wait();
             tc_fence_before();
             mbar_arrive(&sm.p_ready[w]);
