@@ -130,14 +130,22 @@ __device__ __forceinline__ bool group_wait(SwaSmem& sm, uint64_t* bar, uint32_t 
     return ok;
 }
 
+// The MMA issue loops are fully unrolled over constant descriptor offsets: a single thread
+// issues every MMA of the CTA, and per-step descriptor arithmetic in a rolled loop (a chain of
+// dependent integer operations) takes longer than a 128x128x16 MMA takes to execute.  The empty
+// asm statements pin each call's descriptor bases where they are made, so that the compiler
+// does not hoist every unrolled descriptor of every stage out of the key-tile loop (which would
+// need more registers than the issuing warp has).
+
 // S (+)= A B over K = 128 with both operands K-major in shared memory (A = Q, B = K).
 __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a_base, uint32_t b_base) {
-    const uint32_t idesc = idesc_bf16(128, 128, 0, 0);
-#pragma unroll 1
+    constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 0);
+    uint64_t ad = sdesc_sw128(a_base, 16, 1024), bd = sdesc_sw128(b_base, 16, 1024);
+    asm volatile("" : "+l"(ad), "+l"(bd));
+#pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
-        const uint32_t off = (kk >> 2) * SLAB + (kk & 3) * 32u;
-        mma_ss(d, sdesc_sw128(a_base + off, 16, 1024), sdesc_sw128(b_base + off, 16, 1024), idesc,
-               kk > 0 ? 1u : 0u);
+        const uint32_t off = ((kk >> 2) * SLAB + (kk & 3) * 32u) >> 4;
+        mma_ss(d, ad + off, bd + off, idesc, kk > 0 ? 1u : 0u);
     }
 }
 
@@ -145,11 +153,13 @@ __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a_base, uint32_t b_b
 // then 16 of low halves; V [key x d] MN-major in shared memory.
 __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
                                        bool accumulate) {
-    const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
-#pragma unroll 1
+    constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+    uint64_t vd = sdesc_sw128(v_base, SLAB, 1024);
+    uint32_t pb = p_base + 16 * half;
+    asm volatile("" : "+l"(vd), "+r"(pb));
+#pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
-               sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
+        mma_ts(d, pb + 32 * (kk >> 1) + 8 * (kk & 1), vd + ((kk * 2048u) >> 4), idesc,
                (accumulate || kk > 0) ? 1u : 0u);
 }
 

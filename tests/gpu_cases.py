@@ -32,12 +32,15 @@ def token_major(x, head_major):
 
 
 def run_dense(B, N, H, dk, dv, dtype, chunk=0, g_mean=2.0, g_std=1.0, seed=0,
-              head_major=False, state=False, g_fill=None, tau=16.0, k_scale=1.0, tol=None):
+              head_major=False, state=False, g_fill=None, tau=16.0, k_scale=1.0, tol=None,
+              g_edit=None):
     G = lib()
     inp = SI.gret_inputs(B, N, H, dk, dv, dtype=dtype, g_mean=g_mean, g_std=g_std, seed=seed,
                          device="cpu", layout="bhnd" if head_major else "bnhd", with_state=state)
     if g_fill is not None:
         inp["g"].fill_(g_fill)
+    if g_edit is not None:
+        g_edit(inp["g"])
     d = {k: v.cuda() for k, v in inp.items()}
     o, s = G.gret_prefill_chunkwise(d["q"], d["k"], d["v"], d["g"], tau=tau, k_scale=k_scale,
                                     state_in=d.get("s"), state_out=True, chunk=chunk,

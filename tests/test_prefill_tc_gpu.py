@@ -49,6 +49,22 @@ def test_harsh_gates_and_scales():
               state=True)
 
 
+def test_factored_and_unfactored_chunks_in_one_chain():
+    """The kernel factors a chunk's decay mask when the chunk's decay stays within 2^-64 and
+    keeps the per-element form otherwise.  Here chunk c has gates -12 when c % 3 == 1 (decay
+    about 2^-138 over the chunk: unfactored), -5 when c % 3 == 2 (about 2^-58: factored with
+    factors near the limit) and N(2, 1) otherwise, so both forms alternate along each chain and
+    across span boundaries."""
+    def edit(g):   # [B, N, H]
+        n = g.shape[1]
+        for c in range((n + 127) // 128):
+            if c % 3 == 1:
+                g[:, c * 128:(c + 1) * 128] = -12.0
+            elif c % 3 == 2:
+                g[:, c * 128:(c + 1) * 128] = -5.0
+    run_dense(1, 3000, 2, 128, 128, BF, seed=41, state=True, g_edit=edit)
+
+
 def test_varlen_ragged_with_empty_sequences():
     run_varlen([0, 1, 127, 128, 129, 700, 0, 2000], 3, 128, 128, BF, seed=35, state=True)
 
