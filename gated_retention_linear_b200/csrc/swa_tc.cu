@@ -9,8 +9,8 @@
 //     serve both query tiles;
 //   * S = Q K^T for each query tile goes to tensor memory; a softmax warpgroup per query tile
 //     (one query row per thread) masks the window, keeps the running maximum and sum, writes
-//     P = 2^(s - m) back over S as a bf16 high + low pair, and the MMA warp accumulates
-//     O += P_hi V + P_lo V in tensor memory;
+//     P = 2^(s - m) back over S as a bf16 high + low pair, one half of the keys at a time, and
+//     the MMA warp accumulates O += P_hi V + P_lo V in tensor memory as each half arrives;
 //   * the two warpgroups take turns: while one runs its softmax, the tensor cores run the other
 //     tile's products;
 //   * the running maximum is only moved (and O rescaled) when a tile's maximum exceeds it by
@@ -56,7 +56,8 @@ struct __align__(1024) SwaSmem {
     unsigned char q[2][TILE];            // the two query tiles; later their output tiles
     unsigned char k[2][TILE];
     unsigned char v[2][TILE];
-    uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_ready[2], pv_done[2], drain;
+    // p_ready[w][kh]: query tile w's P over keys [64 kh, 64 kh + 64) is in tensor memory
+    uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_ready[2][2], pv_done[2], drain;
     uint32_t dec[2][2];                  // the softmax groups' shared wait outcomes
     uint32_t tmem_base;
     uint32_t abort;
@@ -75,14 +76,6 @@ __device__ __forceinline__ float ex2f(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
-}
-
-__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-    const float2 hf = __bfloat1622float2(h);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-    hi = *reinterpret_cast<const uint32_t*>(&h);
-    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // x = hi + lo in bf16 without the conversion unit: hi keeps the top 16 bits of x (its sign,
@@ -149,18 +142,21 @@ __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a_base, uint32_t b_b
     }
 }
 
-// O (+)= P V with P (bf16 halves, K-major) in TMEM: per 32-key group, 16 columns of high halves
-// then 16 of low halves; V [key x d] MN-major in shared memory.
-__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
+// O (+)= P V over keys [64 kh, 64 kh + 64) with P (bf16 halves, K-major) in TMEM: per 32-key
+// group, 16 columns of high halves then 16 of low halves; V [key x d] MN-major in shared memory.
+// Both halves of P go through: four K-steps of 16 keys each for the high and the low half.
+__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int kh, uint32_t v_base,
                                        bool accumulate) {
     constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 1);
-    uint64_t vd = sdesc_sw128(v_base, SLAB, 1024);
-    uint32_t pb = p_base + 16 * half;
+    uint64_t vd = sdesc_sw128(v_base + kh * 4 * 2048u, SLAB, 1024);
+    uint32_t pb = p_base + 64 * kh;
     asm volatile("" : "+l"(vd), "+r"(pb));
 #pragma unroll
-    for (int kk = 0; kk < 8; ++kk)
-        mma_ts(d, pb + 32 * (kk >> 1) + 8 * (kk & 1), vd + ((kk * 2048u) >> 4), idesc,
-               (accumulate || kk > 0) ? 1u : 0u);
+    for (int half = 0; half < 2; ++half)
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+            mma_ts(d, pb + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half, vd + ((kk * 2048u) >> 4),
+                   idesc, (accumulate || half > 0 || kk > 0) ? 1u : 0u);
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
@@ -188,7 +184,8 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
             mbar_init(&sm.s_full[s], 1);
-            mbar_init(&sm.p_ready[s], 128);
+            mbar_init(&sm.p_ready[s][0], 128);
+            mbar_init(&sm.p_ready[s][1], 128);
             mbar_init(&sm.pv_done[s], 1);
         }
         mbar_init(&sm.drain, 1);
@@ -254,11 +251,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 }
                 for (int w = 0; w < 2 && ok; ++w) {
                     if (!part[w]) continue;
-                    if (!(ok = wait_abortable(sm, &sm.p_ready[w], cnt[w] & 1))) break;
-                    tc_fence_after();
                     const uint32_t vb = smem_u32(sm.v[st]);
-                    mma_pv(tmem + 256 + BM * w, tmem + BM * w, 0, vb, cnt[w] > 0);
-                    mma_pv(tmem + 256 + BM * w, tmem + BM * w, 1, vb, true);
+                    for (int kh = 0; kh < 2 && ok; ++kh) {
+                        if (!(ok = wait_abortable(sm, &sm.p_ready[w][kh], cnt[w] & 1))) break;
+                        tc_fence_after();
+                        mma_pv(tmem + 256 + BM * w, tmem + BM * w, kh, vb, cnt[w] > 0 || kh > 0);
+                    }
+                    if (!ok) break;
                     mma_commit(&sm.pv_done[w]);
                     ++cnt[w];
                 }
@@ -292,13 +291,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             const int c_hi = c_hi64 > BM - 1 ? BM - 1 : (c_hi64 < -1 ? -1 : (int)c_hi64);
             float s[BM];
 #pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                float t32[32];
-                tmem_ld32(s_addr + jc * 32, t32);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) s[jc * 32 + e] = t32[e];
-            }
+            for (int jc = 0; jc < 4; ++jc)
+                tmem_ld32(s_addr + jc * 32, *reinterpret_cast<float(*)[32]>(&s[jc * 32]));
+            tmem_ld_wait();
             // scores in log2 units are c s; the tile's maximum of c s over the visible keys is
             // c max(s) for c >= 0 and c min(s) otherwise.  Tiles wholly inside every row's
             // window (all but the first and the last few) skip the per-key mask.
@@ -356,6 +351,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (move) m_ref = mx;
             const float nm = -m_ref;   // finite whenever a key of the row is visible
+            // P over keys [0, 64), then [64, 128): each half is handed to P V as soon as it is
+            // stored, so that the products of the first half overlap the exponentials of the
+            // second
             float l4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
 #pragma unroll
             for (int jc = 0; jc < 4; ++jc) {
@@ -372,11 +370,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     split2_trunc(p0, p1, ph[e], ph[16 + e]);
                 }
                 tmem_st32(s_addr + jc * 32, ph);
+                if (jc & 1) {
+                    tmem_st_wait();
+                    tc_fence_before();
+                    mbar_arrive(&sm.p_ready[w][jc >> 1]);
+                }
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&sm.p_ready[w]);
             ++cnt;
         }
         // ---- epilogue: O / l in bf16 through this tile's query slot, then one TMA store
