@@ -172,22 +172,32 @@ def kernel_code_digest(path):
     return hashlib.sha256(src.encode()).hexdigest()[:16]
 
 
-def prefill_traffic_from_profile():
-    """DRAM bytes per launch of the prefill kernel from the committed ncu summary, if that
-    summary was taken on the current kernel code (else None)."""
-    src = os.path.join(ROOT, "gated_retention_linear_b200", "csrc", "prefill_tc.cu")
-    summ = os.path.join(ROOT, "profiles", "prefill_tc_kernel_32k.txt")
+def traffic_from_profile(src_name, summary_name, units=None):
+    """DRAM bytes per launch of a kernel from its committed ncu summary under profiles/, if that
+    summary was taken on the current code of csrc/<src_name> (else None).  A summary taken on a
+    smaller case states its `units` (tokens); the bytes are then scaled to `units` of this run,
+    the traffic of these kernels growing in proportion to the tokens they process."""
+    src = os.path.join(ROOT, "gated_retention_linear_b200", "csrc", src_name)
+    summ = os.path.join(ROOT, "profiles", summary_name)
     try:
         kv = {}
         for line in open(summ):
             if ":" in line:
                 k, v = line.split(":", 1)
                 kv[k.strip()] = v.strip()
-        if kv.get("kernel_code_sha256_16") == kernel_code_digest(src):
-            return int(float(kv["dram_bytes_per_launch"]))
+        digest = kv.get("kernel_code_sha256_16", "").split()
+        if digest and digest[0] == kernel_code_digest(src):
+            b = float(kv["dram_bytes_per_launch"].split()[0])
+            if units is not None and "profile_units" in kv:
+                b *= units / float(kv["profile_units"].split()[0])
+            return int(b)
     except Exception:
         pass
     return None
+
+
+def prefill_traffic_from_profile():
+    return traffic_from_profile("prefill_tc.cu", "prefill_tc_kernel_32k.txt")
 
 
 def run_gpu(args):
@@ -305,7 +315,8 @@ def run_gpu(args):
                "gpu_launches": DEC_STEPS,
                "roofline": {"bound": "hbm", "achieved": dec_ach, "peak": hbm_peak,
                             "unit": "GB/s", "frac": dec_ach / hbm_peak,
-                            "peak_kind": peak_kind, "traffic": None},
+                            "peak_kind": peak_kind,
+                            "traffic": traffic_from_profile("decode.cu", "decode_kernel_bs64.txt")},
                "l2": "state (201 MB) larger than L2 (126 MB); not flushed between steps"}
         del qs, ks, vs, gs, state, state0
 
@@ -510,7 +521,9 @@ def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
                                  "peak": hbm_peak, "unit": "GB/s",
                                  "frac": pre_bytes / (pre_ms * 1e-3) / 1e9 / hbm_peak},
             "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
-                         "frac": ach / tpeak, "peak_kind": tkind + " burst", "traffic": None,
+                         "frac": ach / tpeak, "peak_kind": tkind + " burst",
+                         "traffic": traffic_from_profile("gn_gate.cu",
+                                                         "gn_gate_kernel_varlen_T37806.txt", T),
                          "kernel": "gn_gate_kernel", "algorithmic_flops_per_launch": flops}}
 
 
@@ -625,7 +638,8 @@ def run_swa(args, rank, world, stream, headwise_ms):
             "l2": "q, k, v, o (805 MB) larger than L2; not flushed",
             "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
                          "frac": ach / tpeak, "peak_kind": tkind + " burst",
-                         "mma": "tcgen05 bf16, S and O in TMEM", "traffic": None,
+                         "mma": "tcgen05 bf16, S and O in TMEM",
+                         "traffic": traffic_from_profile("swa_tc.cu", "swa_tc_kernel_32k_w1024.txt"),
                          "kernel": "swa_tc_kernel", "algorithmic_flops_per_launch": flops},
             "decode": dec}
 
@@ -673,7 +687,9 @@ def run_swa_decode(args, rank, world, stream, W):
     return {"value": Bq * S * world / (dms * 1e-3), "unit": "tok/s", "ms_per_step": dms / S,
             "batch": Bq, "window": W, "steps": S, "gpu_launches": S,
             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
-                         "frac": ach / hbm_peak, "peak_kind": peak_kind, "traffic": None,
+                         "frac": ach / hbm_peak, "peak_kind": peak_kind,
+                         "traffic": traffic_from_profile("swa_decode.cu",
+                                                         "swa_decode_kernel_bs64_w1024.txt"),
                          "kernel": "swa_decode_kernel",
                          "algorithmic_bytes_per_launch": Bq * Hq * per_bh}}
 
