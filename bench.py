@@ -639,7 +639,8 @@ def run_swa(args, rank, world, stream, headwise_ms):
             "roofline": {"bound": "tensor", "achieved": ach, "peak": tpeak, "unit": "TFLOP/s",
                          "frac": ach / tpeak, "peak_kind": tkind + " burst",
                          "mma": "tcgen05 bf16, S and O in TMEM",
-                         "traffic": traffic_from_profile("swa_tc.cu", "swa_tc_kernel_32k_w1024.txt"),
+                         "traffic": traffic_from_profile("swa_tc.cu",
+                                                         "swa_tc_kernel_32k_w1024.txt"),
                          "kernel": "swa_tc_kernel", "algorithmic_flops_per_launch": flops},
             "decode": dec}
 
@@ -781,7 +782,8 @@ def cpu_baseline(q, k, v, g, n_tokens, min_seconds=8.0, max_reps=8):
         reps += 1
     return {"value": n * reps / dt / 1e6, "unit": "Mtok/s", "cores": oracle.threads(),
             "kind": "oracle",
-            "sample": "%d tokens x 24 heads, fp64 recurrent oracle, %d passes, %.1f s" % (n, reps, dt)}
+            "sample": "%d tokens x 24 heads, fp64 recurrent oracle, %d passes, %.1f s"
+                      % (n, reps, dt)}
 
 
 def run_reference(args):
