@@ -97,16 +97,34 @@ def channel_gates(B, N, H, dk, g_mean=2.0, g_std=1.0, seed=0, device="cpu"):
     return _randn((B, N, H, dk), seed, "gch", device, std=g_std, mean=g_mean)
 
 
-def layer_inputs(T, D, H, d=128, seed=0, device="cpu", pad=0, pad_value=float("nan")):
+def layer_inputs(T, D, H, d=128, seed=0, device="cpu", pad=0, pad_value=float("nan"),
+                 exact_projection=False):
     """One mixer layer's input and weights, bf16: x [T, D], w_qkvg [D, 3 H d + H + pad] (W_Q,
     W_K, W_V and W_gamma side by side; the pad columns, if any, hold pad_value) and
-    w_g [D, H d]."""
+    w_g [D, H d].
+
+    exact_projection: the same distributions drawn on coarse dyadic grids (x on multiples of
+    1/8 within [-4, 4]; the q, k, v weight columns on multiples of 2^-10, the gate-logit columns
+    on 2^-14, their bias row on 2^-5), so that every partial sum of x W is an integer multiple
+    of the grid unit below 2^24 units: the projection is then exact in fp32 and fp64 alike, and
+    both round the same q, k, v to bf16.  For D <= 3072 (the bounds below)."""
     F = 3 * H * d + H
     x = _randn((T, D), seed, "x", device)
     x[:, 0] = 1.0
     w = _randn((D, F + pad), seed, "wqkvg", device, std=D ** -0.5)
     w[:, 3 * H * d:F] *= 0.05
     w[0, 3 * H * d:F] = _randn((H,), seed, "gbias", device, mean=2.0)
+    if exact_projection:
+        # |x| <= 32 units of 1/8; |w| <= 127 units (7 bits, exact in bf16): a q, k, v sum is at
+        # most D * 32 * 127 < 2^24 units of 2^-13, a gate-logit sum at most D * 32 * 127 plus the
+        # bias row's 8 * 127 * 2^9 units of 2^-17
+        assert D <= 3072
+        x = torch.clamp(torch.round(x * 8.0), -32.0, 32.0) / 8.0
+        qkv = w[:, :3 * H * d]
+        w[:, :3 * H * d] = torch.clamp(torch.round(qkv * 1024.0), -127.0, 127.0) / 1024.0
+        gcol = w[1:, 3 * H * d:F]
+        w[1:, 3 * H * d:F] = torch.clamp(torch.round(gcol * 16384.0), -127.0, 127.0) / 16384.0
+        w[0, 3 * H * d:F] = torch.clamp(torch.round(w[0, 3 * H * d:F] * 32.0), -127.0, 127.0) / 32.0
     if pad:
         w[:, F:] = pad_value
     w_g = _randn((D, H * d), seed, "w", device, std=0.02)

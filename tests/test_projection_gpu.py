@@ -36,23 +36,26 @@ def test_projection_matches_oracle(T, H, D):
     assert_parity("g", g, rg, 1e-2, stored_bf16=False)
 
 
-def _check_layer(y, s, rows, ry, rs, ro_rows, x_rows, w_g, H):
+def _check_layer(y, s, rows, ry, rs, ro_rows, x_rows, w_g, H, tight=None):
     """y's rows against the oracle's, after taking off the effect of o's bf16 rounding.
 
     o is stored in bf16 on both sides.  Where the exact o lies within the kernel's error of a
     rounding midpoint the two round to neighbouring values, one ulp apart, and GroupNorm and the
     gate carry that ulp into y; parity.gate_o_rounding_allowance bounds it per element (fp64,
     from the oracle's o and the inputs), and it is taken off on top of y's own half-ulp rounding
-    allowance before the 1e-2 rms bar.  The state gets no tight bar here: q, k and v reach the
-    prefill rounded to bf16 from the projection's fp32 accumulator on the GPU and from fp64 in
-    the oracle, and the two roundings differ by one ulp where the value lies near a midpoint,
-    which moves the state by a few 1e-3 of rms at the 3B shape."""
-    assert_parity("state", s, rs, 1e-2, stored_bf16=False)
+    allowance before the 1e-2 rms bar.  With general inputs q, k and v reach the prefill
+    rounded to bf16 from the projection's fp32 accumulator on the GPU and from fp64 in the
+    oracle, and the two roundings differ by one ulp where the value lies near a midpoint, which
+    moves the state by a few 1e-3 of rms at the 3B shape (and y by about 1e-2).  With inputs
+    whose projection is exact in fp32 (synth_inputs.layer_inputs(exact_projection=True)) both
+    sides round the same q, k, v, and `tight` holds the state and y to the kernels' own
+    error."""
+    assert_parity("state", s, rs, 1e-2, stored_bf16=False, tight=tight)
     a = gate_o_rounding_allowance(ro_rows, x_rows, w_g, H)
     yg = y.double().cpu().numpy()
     if rows is not None:
         yg = yg[np.asarray(rows)]
-    return assert_parity("y", yg, ry, 1e-2, stored_bf16=True, allowance=a)
+    return assert_parity("y", yg, ry, 1e-2, stored_bf16=True, allowance=a, tight=tight)
 
 
 def test_layer_matches_oracle():
@@ -76,12 +79,16 @@ def test_layer_3b_shape_sampled_rows():
     """The layer at the 3B shape the benchmark times: one sequence of 32768 tokens, hidden
     3072, 24 heads of 128 (projection GEMM -> prefill with k scaled by d^-1/2 -> GroupNorm *
     swish(x W_G)).  The oracle runs the whole projection and recurrence in fp64 and the output
-    gate on the first and last row and a seeded sample of rows (rows are independent there)."""
+    gate on the first and last row and a seeded sample of rows (rows are independent there).
+    The inputs are drawn on dyadic grids on which the projection is exact in fp32, so that the
+    GPU and the oracle round the same q, k, v to bf16 and the chain is held to the 1e-3 bar of
+    the tensor-core prefill."""
     G = lib()
     c = SI.LAYER_32K
     T, D, H, d = c["T"], c["D"], c["H"], c["dk"]
     F = 3 * H * d + H
-    li = SI.layer_inputs(T, D, H, d, seed=c["seed"], pad=(-F) % 8, pad_value=0.0)
+    li = SI.layer_inputs(T, D, H, d, seed=c["seed"], pad=(-F) % 8, pad_value=0.0,
+                         exact_projection=True)
     x, w, w_g = li["x"], li["w_qkvg"], li["w_g"]
     y, s = G.gret_layer_forward(x.cuda(), w.cuda(), w_g.cuda(), H, d,
                                 cu_seqlens=torch.tensor([0, T], dtype=torch.int32, device="cuda"))
@@ -90,7 +97,7 @@ def test_layer_3b_shape_sampled_rows():
     rows = sorted(set(rng.integers(0, T, 192).tolist()) | {0, 127, 128, T - 1})
     ry, rs, ro = oracle.layer_forward(x, w[:, :F].float(), w_g, H, d, cu_seqlens=[0, T],
                                       rows=rows, with_o=True)
-    _check_layer(y, s, rows, ry, rs, ro[rows], x[rows], w_g, H)
+    _check_layer(y, s, rows, ry, rs, ro[rows], x[rows], w_g, H, tight=1e-3)
 
 
 def test_projection_rejects_bad_arguments():
