@@ -46,8 +46,8 @@ constexpr int D = SWA_DIM;
 constexpr int BM = 128;                  // queries per tile, keys per tile
 constexpr int TILE = BM * D * 2;         // one bf16 128 x 128 tile
 constexpr int SLAB = TILE / 2;
-constexpr int NTHREADS = 384;
-constexpr int LAUNCH_REGS = 168;
+constexpr int NTHREADS = 640;
+constexpr int LAUNCH_REGS = 96;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
 constexpr float RESCALE_LOG2 = 8.f;      // move the running maximum only past this margin
@@ -58,7 +58,11 @@ struct __align__(1024) SwaSmem {
     unsigned char v[2][TILE];
     // p_ready[w][kh]: query tile w's P over keys [64 kh, 64 kh + 64) is in tensor memory
     uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_ready[2][2], pv_done[2], drain;
-    uint32_t dec[2][2];                  // the softmax groups' shared wait outcomes
+    uint32_t dec[2][2];                  // the softmax pairs' shared wait outcomes
+    // the two halves of a query row exchange their partial maxima (double-buffered by tile) and,
+    // at the end, their partial sums
+    float xmax[2][2][2][BM];             // [tile parity][query tile][key half][row]
+    float xl[2][2][BM];                  // [query tile][key half][row]
     uint32_t tmem_base;
     uint32_t abort;
 };
@@ -110,17 +114,22 @@ __device__ __forceinline__ bool wait_abortable(SwaSmem& sm, uint64_t* bar, uint3
     return false;
 }
 
-// A softmax warpgroup's wait: one thread polls the barrier, the other 127 sleep at the group's
-// named barrier (no issue slots burned by 128 polling threads), and all take the same branch.
-// The outcome word is double-buffered, so that a fast thread 0 cannot overwrite it for the next
-// wait before a slow thread of the group has read it for this one.
-__device__ __forceinline__ bool group_wait(SwaSmem& sm, uint64_t* bar, uint32_t parity, int w,
-                                           int r, int& flip) {
-    if (r == 0) sm.dec[w][flip] = wait_abortable(sm, bar, parity) ? 1u : 0u;
-    asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");
+// A softmax pair's wait (the two warpgroups of one query tile): one thread polls the barrier,
+// the other 255 sleep at the pair's named barrier (no issue slots burned by polling threads),
+// and all take the same branch, so that neither half can leave the tile loop while the other
+// waits at the pair's barrier.  The outcome word is double-buffered, so that a fast thread
+// cannot overwrite it for the next wait before a slow thread of the pair has read it.
+__device__ __forceinline__ bool pair_wait(SwaSmem& sm, uint64_t* bar, uint32_t parity, int w,
+                                          int hf, int r, int& flip) {
+    if (hf == 0 && r == 0) sm.dec[w][flip] = wait_abortable(sm, bar, parity) ? 1u : 0u;
+    asm volatile("bar.sync %0, 256;" ::"r"(1 + w) : "memory");
     const bool ok = *reinterpret_cast<volatile uint32_t*>(&sm.dec[w][flip]) != 0;
     flip ^= 1;
     return ok;
+}
+
+__device__ __forceinline__ void pair_sync(int w) {
+    asm volatile("bar.sync %0, 256;" ::"r"(1 + w) : "memory");
 }
 
 // The MMA issue loops are fully unrolled over constant descriptor offsets: a single thread
@@ -202,7 +211,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem = sm.tmem_base;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 40;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 48;" ::: "memory");
         if (warp == 0 && lane == 0) {
             // ---- producer: both query tiles, then the key / value tiles through two stages
             tma_prefetch_desc(&tq);
@@ -267,13 +276,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             mbar_wait_drain_(&sm.drain, 0, DRAIN_NS);
         }
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 232;" ::: "memory");
-        // ---- softmax warpgroup w: query row r of query tile w
-        const int w = (warp - 4) >> 2;
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
+        // ---- softmax warpgroup (w, hf): query row r of query tile w, keys [64 hf, 64 hf + 64)
+        // of each key tile.  The two halves of a row share its running maximum (exchanged through
+        // shared memory each tile) and add their sums at the end.
+        const int wg = (warp - 4) >> 2;
+        const int w = wg >> 1, hf = wg & 1;
         const int q = warp & 3, r = q * 32 + lane;
         const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
-        const uint32_t s_addr = tmem + lane_base + BM * w;
-        const uint32_t o_addr = tmem + lane_base + 256 + BM * w;
+        const uint32_t s_addr = tmem + lane_base + BM * w + 64 * hf;        // this half of S / P
+        const uint32_t o_addr = tmem + lane_base + 256 + BM * w + 64 * hf;  // this half of O
         const int64_t qi = q0 + BM * w + r;      // this thread's query position
         float m_ref = -INFINITY, l = 0.f;
         int cnt = 0, flip = 0;
@@ -281,65 +293,65 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int i = 0; i < ntiles && ok; ++i) {
             const int64_t kt = kt_lo + i;
             if (!takes_part(q0, w, kt, p.window, p.N)) continue;
-            // group-uniform outcome: no warp may split around the warp-wide TMEM accesses
-            ok = group_wait(sm, &sm.s_full[w], cnt & 1, w, r, flip);
+            // pair-uniform outcome: no warp may split around the warp-wide TMEM accesses, and
+            // neither half may leave while the other waits at the pair's barrier
+            ok = pair_wait(sm, &sm.s_full[w], cnt & 1, w, hf, r, flip);
             if (!ok) break;
             tc_fence_after();
-            // visible keys of this row in this tile: columns [c_lo, c_hi]
-            const int64_t c_lo64 = qi - p.window + 1 - BM * kt, c_hi64 = qi - BM * kt;
-            const int c_lo = c_lo64 < 0 ? 0 : (c_lo64 > BM ? BM : (int)c_lo64);
-            const int c_hi = c_hi64 > BM - 1 ? BM - 1 : (c_hi64 < -1 ? -1 : (int)c_hi64);
-            float s[BM];
-#pragma unroll
-            for (int jc = 0; jc < 4; ++jc)
-                tmem_ld32(s_addr + jc * 32, *reinterpret_cast<float(*)[32]>(&s[jc * 32]));
-            tmem_ld_wait();
-            // scores in log2 units are c s; the tile's maximum of c s over the visible keys is
-            // c max(s) for c >= 0 and c min(s) otherwise.  Tiles wholly inside every row's
-            // window (all but the first and the last few) skip the per-key mask.
+            // visible keys of this row in this half: columns [c_lo, c_hi] of the half
+            const int64_t c_lo64 = qi - p.window + 1 - BM * kt - 64 * hf,
+                          c_hi64 = qi - BM * kt - 64 * hf;
+            const int c_lo = c_lo64 < 0 ? 0 : (c_lo64 > 64 ? 64 : (int)c_lo64);
+            const int c_hi = c_hi64 > 63 ? 63 : (c_hi64 < -1 ? -1 : (int)c_hi64);
+            // scores in log2 units are c s; the half's maximum of c s over its visible keys is
+            // c max(s) for c >= 0 and c min(s) otherwise (eight independent partial extrema),
+            // 32 columns at a time.  Halves wholly inside every row's window skip the per-key
+            // mask.
             const float c = p.scale_log2;
-            const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == BM - 1);
-            // eight independent partial extrema, so that the reduction is not one 128-long
-            // dependency chain
-            float ext;
-            {
-                const bool up = c >= 0.f;
-                float e8[8];
+            const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == 63);
+            const bool up = c >= 0.f;
+            float e8[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) e8[u] = up ? -INFINITY : INFINITY;
+            for (int u = 0; u < 8; ++u) e8[u] = up ? -INFINITY : INFINITY;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                float sg[32];
+                tmem_ld32(s_addr + 32 * g, sg);
+                tmem_ld_wait();
                 if (full) {
-                    if (up) {
 #pragma unroll
-                        for (int cc = 0; cc < BM; ++cc) e8[cc & 7] = fmaxf(e8[cc & 7], s[cc]);
-                    } else {
-#pragma unroll
-                        for (int cc = 0; cc < BM; ++cc) e8[cc & 7] = fminf(e8[cc & 7], s[cc]);
-                    }
+                    for (int e = 0; e < 32; ++e)
+                        e8[e & 7] = up ? fmaxf(e8[e & 7], sg[e]) : fminf(e8[e & 7], sg[e]);
                 } else {
 #pragma unroll
-                    for (int cc = 0; cc < BM; ++cc)
-                        if (cc >= c_lo && cc <= c_hi)
-                            e8[cc & 7] = up ? fmaxf(e8[cc & 7], s[cc]) : fminf(e8[cc & 7], s[cc]);
+                    for (int e = 0; e < 32; ++e)
+                        if (32 * g + e >= c_lo && 32 * g + e <= c_hi)
+                            e8[e & 7] = up ? fmaxf(e8[e & 7], sg[e]) : fminf(e8[e & 7], sg[e]);
                 }
-#pragma unroll
-                for (int u = 4; u > 0; u >>= 1)
-#pragma unroll
-                    for (int v = 0; v < u; ++v)
-                        e8[v] = up ? fmaxf(e8[v], e8[v + u]) : fminf(e8[v], e8[v + u]);
-                ext = e8[0];
             }
-            const float mx = (c_lo <= c_hi) ? c * ext : -INFINITY;
-            // move the reference when this tile's maximum passes it by the margin: O and l
-            // scale by 2^(m_ref - mx).  The tensor-memory accesses are warp-wide instructions,
-            // so the whole warp takes the branch when any of its rows needs it (factor 1 for
-            // the others).
+#pragma unroll
+            for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+                for (int v = 0; v < u; ++v)
+                    e8[v] = up ? fmaxf(e8[v], e8[v + u]) : fminf(e8[v], e8[v + u]);
+            const float ext = e8[0];
+            const float mx_half = (c_lo <= c_hi) ? c * ext : -INFINITY;
+            // the row's maximum over both halves
+            sm.xmax[cnt & 1][w][hf][r] = mx_half;
+            pair_sync(w);
+            const float mx = fmaxf(mx_half, sm.xmax[cnt & 1][w][hf ^ 1][r]);
+            // move the reference when the tile's maximum passes it by the margin: O and l scale
+            // by 2^(m_ref - mx) (both halves take the same decision from the same maximum; each
+            // scales its own columns of O and its own partial sum).  The tensor-memory accesses
+            // are warp-wide instructions, so the whole warp takes the branch when any of its
+            // rows needs it (factor 1 for the others).
             const bool move = mx > m_ref + RESCALE_LOG2;
-            const bool rescale = move && l > 0.f;
+            const bool rescale = move && m_ref > -INFINITY;
             if (__any_sync(0xffffffffu, rescale)) {
                 const float f = rescale ? ex2f(m_ref - mx) : 1.f;
                 l *= f;
 #pragma unroll 1
-                for (int jc = 0; jc < 4; ++jc) {
+                for (int jc = 0; jc < 2; ++jc) {
                     float t32[32];
                     tmem_ld32(o_addr + jc * 32, t32);
                     tmem_ld_wait();
@@ -351,42 +363,56 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             }
             if (move) m_ref = mx;
             const float nm = -m_ref;   // finite whenever a key of the row is visible
-            // P over keys [0, 64), then [64, 128): each half is handed to P V as soon as it is
-            // stored, so that the products of the first half overlap the exponentials of the
-            // second
             float l4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+            // P, one 32-key group at a time, the group's scores read again from tensor memory
+            // (so that the 64 scores of the maximum pass are not held through this one) and
+            // replaced in place by the group's P: 16 columns of high halves, then 16 of low
+            // halves, over the 32 columns the group's scores occupied.
 #pragma unroll
-            for (int jc = 0; jc < 4; ++jc) {
-                uint32_t ph[32];
+            for (int g = 0; g < 2; ++g) {
+                float sg[32];
+                tmem_ld32(s_addr + 32 * g, sg);
+                tmem_ld_wait();
+                // eight key pairs at a time: their high halves to columns 32 g + 8 sub, their
+                // low halves to 32 g + 16 + 8 sub (the group's scores are all in sg already)
 #pragma unroll
-                for (int e = 0; e < 16; ++e) {
-                    const int c0 = jc * 32 + 2 * e;
-                    float p0 = ex2f(fmaf(s[c0], c, nm)), p1 = ex2f(fmaf(s[c0 + 1], c, nm));
-                    if (!full) {
-                        p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
-                        p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
+                for (int sub = 0; sub < 2; ++sub) {
+                    uint32_t hi8[8], lo8[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int k2 = 8 * sub + e;            // key pair within the group
+                        const int c0 = g * 32 + 2 * k2;
+                        float p0 = ex2f(fmaf(sg[2 * k2], c, nm));
+                        float p1 = ex2f(fmaf(sg[2 * k2 + 1], c, nm));
+                        if (!full) {
+                            p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
+                            p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
+                        }
+                        l4[e & 3] += p0 + p1;
+                        split2_trunc(p0, p1, hi8[e], lo8[e]);
                     }
-                    l4[e & 3] += p0 + p1;
-                    split2_trunc(p0, p1, ph[e], ph[16 + e]);
-                }
-                tmem_st32(s_addr + jc * 32, ph);
-                if (jc & 1) {
-                    tmem_st_wait();
-                    tc_fence_before();
-                    mbar_arrive(&sm.p_ready[w][jc >> 1]);
+                    tmem_st8(s_addr + 32 * g + 8 * sub, hi8);
+                    tmem_st8(s_addr + 32 * g + 16 + 8 * sub, lo8);
                 }
             }
             l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready[w][hf]);   // P V over this half's keys may run
             ++cnt;
         }
-        // ---- epilogue: O / l in bf16 through this tile's query slot, then one TMA store
+        // ---- epilogue: O / l in bf16 through this tile's query slot (each half its 64
+        // columns), then one TMA store
         if (cnt > 0) {
-            if (ok) ok = group_wait(sm, &sm.pv_done[w], (cnt - 1) & 1, w, r, flip);
+            if (ok) ok = pair_wait(sm, &sm.pv_done[w], (cnt - 1) & 1, w, hf, r, flip);
             tc_fence_after();
-            const float inv = ok && l > 0.f ? 1.f / l : __int_as_float(0x7fc00000);
-            unsigned char* tile = sm.q[w];
+            sm.xl[w][hf][r] = l;
+            pair_sync(w);
+            const float lt = l + sm.xl[w][hf ^ 1][r];
+            const float inv = ok && lt > 0.f ? 1.f / lt : __int_as_float(0x7fc00000);
+            unsigned char* row = sm.q[w] + hf * SLAB + r * 128;
 #pragma unroll 1
-            for (int jc = 0; jc < 4; ++jc) {
+            for (int jc = 0; jc < 2; ++jc) {
                 float t32[32];
                 tmem_ld32(o_addr + jc * 32, t32);
                 tmem_ld_wait();
@@ -397,16 +423,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                     u.y = pack_bf16x2(t32[8 * v4 + 2] * inv, t32[8 * v4 + 3] * inv);
                     u.z = pack_bf16x2(t32[8 * v4 + 4] * inv, t32[8 * v4 + 5] * inv);
                     u.w = pack_bf16x2(t32[8 * v4 + 6] * inv, t32[8 * v4 + 7] * inv);
-                    const int cc = 4 * jc + v4;
-                    *reinterpret_cast<uint4*>(tile + (cc >> 3) * SLAB + r * 128 +
-                                              (((cc & 7) ^ (r & 7)) << 4)) = u;
+                    const int cc = 4 * jc + v4;   // 16-byte chunk of the half-row
+                    *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) << 4)) = u;
                 }
             }
             fence_proxy_async_smem();
-            asm volatile("bar.sync %0, 128;" ::"r"(1 + w) : "memory");   // the tile is written
-            if (r == 0) {
+            pair_sync(w);   // both halves of the tile are written
+            if (hf == 0 && r == 0) {
                 for (int half = 0; half < 2; ++half)
-                    tma_store_4d(&to, tile + half * SLAB, half * 64, h, (int)(q0 + BM * w), b);
+                    tma_store_4d(&to, sm.q[w] + half * SLAB, half * 64, h, (int)(q0 + BM * w), b);
                 bulk_commit_group();
                 bulk_wait_group0();
             }
