@@ -7,12 +7,13 @@
 //   * one CTA takes two 128-query tiles of one (batch, head), queries q0 .. q0 + 255; the key
 //     tiles of 128 that their windows touch (ten at W = 1024) stream through two TMA stages and
 //     serve both query tiles;
-//   * S = Q K^T for each query tile goes to tensor memory; a softmax warpgroup per query tile
-//     (one query row per thread) masks the window, keeps the running maximum and sum, writes
-//     P = 2^(s - m) back over S as a bf16 high + low pair, one half of the keys at a time, and
-//     the MMA warp accumulates O += P_hi V + P_lo V in tensor memory as each half arrives;
-//   * the two warpgroups take turns: while one runs its softmax, the tensor cores run the other
-//     tile's products;
+//   * S = Q K^T for each query tile goes to tensor memory; two softmax warpgroups per query
+//     tile (one query row per thread, keys [0, 64) and [64, 128) of the key tile) mask the
+//     window, share the row's running maximum through shared memory, keep their partial sums,
+//     and write P = 2^(s - m) back over S as a bf16 high + low pair; the MMA warp accumulates
+//     O += P_hi V + P_lo V in tensor memory as each half of the keys arrives;
+//   * the two query tiles take turns: while one runs its softmax, the tensor cores run the
+//     other tile's products;
 //   * the running maximum is only moved (and O rescaled) when a tile's maximum exceeds it by
 //     more than 2^8, so rescaling is rare after the first tiles; P then stays below 256;
 //   * the output, O / l in bf16, leaves through the query tile's own shared-memory slot by TMA
@@ -21,12 +22,16 @@
 // leaves errors near 1e-2 of rms; the pair (split by truncation, see split2_trunc) keeps the
 // result near 1e-5.
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-7 and
-// 8-11 the softmax warpgroups of query tiles 0 and 1.  Registers: launched at 168 per thread;
-// warps 0-3 drop to 40 and the softmax groups rise to 232 (128 x (40 + 232 + 232) = 64512).
+// Warp roles (640 threads): warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-11 the
+// softmax warpgroups of query tile 0 (keys [0, 64), then [64, 128)), warps 12-19 those of query
+// tile 1.  Registers: launched at 96 per thread; warps 0-3 drop to 48 and the softmax groups
+// rise to 104 (each SM sub-partition holds one warp of each of the five warpgroups:
+// 32 x (48 + 4 x 104) <= 32 x 5 x 96).  A softmax thread reads its 64 scores in two passes (the
+// maximum, then 32 at a time for P) so that it fits its 104 registers.
 // Every wait is bounded; a wait that gives up makes the CTA stop and write NaN into its output
-// rows that are still to be written.  In a softmax warpgroup one thread waits while the others
-// sleep at the group's named barrier.
+// rows that are still to be written.  The two warpgroups of a query tile wait together: one
+// thread waits while the other 255 sleep at the pair's named barrier, so that neither half can
+// leave while the other is at the pair's barrier.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
