@@ -24,9 +24,9 @@
 // Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
 // Warp roles (640 threads): warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-11 the
 // softmax warpgroups of query tile 0 (keys [0, 64), then [64, 128)), warps 12-19 those of query
-// tile 1.  Registers: launched at 96 per thread; warps 0-3 drop to 48 and the softmax groups
+// tile 1.  Registers: launched at 96 per thread; warps 0-3 drop to 56 and the softmax groups
 // rise to 104 (each SM sub-partition holds one warp of each of the five warpgroups:
-// 32 x (48 + 4 x 104) <= 32 x 5 x 96).  A softmax thread reads its 64 scores in two passes (the
+// 32 x (56 + 4 x 104) <= 32 x 5 x 96).  A softmax thread reads its 64 scores in two passes (the
 // maximum, then 32 at a time for P) so that it fits its 104 registers.
 // Every wait is bounded; a wait that gives up makes the CTA stop and write NaN into its output
 // rows that are still to be written.  The two warpgroups of a query tile wait together: one
@@ -216,7 +216,7 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     const uint32_t tmem = sm.tmem_base;
 
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 48;" ::: "memory");
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
         if (warp == 0 && lane == 0) {
             // ---- producer: both query tiles, then the key / value tiles through two stages
             tma_prefetch_desc(&tq);
@@ -244,38 +244,48 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             for (int ii = (i >= 2 ? i - 2 : 0); ii < i; ++ii)
                 mbar_wait_drain_(&sm.kv_full[ii & 1], (ii >> 1) & 1, DRAIN_NS);
         } else if (warp == 1 && lane == 0) {
-            // ---- MMA issuer
+            // ---- MMA issuer.  Query tile 0 runs one step ahead of tile 1: Q_0 K_{i+1}^T is
+            // issued right after P_0 V_i, before P_1 V_i, so that tile 0's next softmax overlaps
+            // tile 1's products instead of both tiles' softmaxes running at the same time.
             bool ok = wait_abortable(sm, &sm.q_full, 0);
             int cnt[2] = {0, 0};
-            for (int i = 0; i < ntiles && ok; ++i) {
-                const int st = i & 1;
-                const int64_t kt = kt_lo + i;
-                const bool part[2] = {takes_part(q0, 0, kt, p.window, p.N),
-                                      takes_part(q0, 1, kt, p.window, p.N)};
-                if (!(ok = wait_abortable(sm, &sm.kv_full[st], (i >> 1) & 1))) break;
+            auto part = [&](int w, int i) { return takes_part(q0, w, kt_lo + i, p.window, p.N); };
+            auto qk = [&](int w, int i) {   // S_w = Q_w K_i^T, once P V has read S_w's last P
+                if (cnt[w] > 0 && !(ok = wait_abortable(sm, &sm.pv_done[w], (cnt[w] - 1) & 1)))
+                    return;
                 tc_fence_after();
-                for (int w = 0; w < 2 && ok; ++w) {
-                    if (!part[w]) continue;
-                    // P of this tile's previous key tile has been read by its P V
-                    if (cnt[w] > 0 && !(ok = wait_abortable(sm, &sm.pv_done[w], (cnt[w] - 1) & 1)))
+                mma_qk(tmem + BM * w, smem_u32(sm.q[w]), smem_u32(sm.k[i & 1]));
+                mma_commit(&sm.s_full[w]);
+            };
+            auto pv = [&](int w, int i) {   // O_w += P_w V_i, one half of the keys at a time
+                const uint32_t vb = smem_u32(sm.v[i & 1]);
+                for (int kh = 0; kh < 2 && ok; ++kh) {
+                    if (!(ok = wait_abortable(sm, &sm.p_ready[w][kh], cnt[w] & 1))) return;
+                    tc_fence_after();
+                    mma_pv(tmem + 256 + BM * w, tmem + BM * w, kh, vb, cnt[w] > 0 || kh > 0);
+                }
+                mma_commit(&sm.pv_done[w]);
+                ++cnt[w];
+            };
+            if (ok && ntiles > 0 && (ok = wait_abortable(sm, &sm.kv_full[0], 0))) {
+                tc_fence_after();
+                if (part(0, 0)) qk(0, 0);
+                if (ok && part(1, 0)) qk(1, 0);
+            }
+            for (int i = 0; i < ntiles && ok; ++i) {
+                const bool nxt = i + 1 < ntiles;
+                if (part(0, i)) pv(0, i);
+                if (ok && nxt) {
+                    if (!(ok = wait_abortable(sm, &sm.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1)))
                         break;
                     tc_fence_after();
-                    mma_qk(tmem + BM * w, smem_u32(sm.q[w]), smem_u32(sm.k[st]));
-                    mma_commit(&sm.s_full[w]);
+                    if (part(0, i + 1)) qk(0, i + 1);
                 }
-                for (int w = 0; w < 2 && ok; ++w) {
-                    if (!part[w]) continue;
-                    const uint32_t vb = smem_u32(sm.v[st]);
-                    for (int kh = 0; kh < 2 && ok; ++kh) {
-                        if (!(ok = wait_abortable(sm, &sm.p_ready[w][kh], cnt[w] & 1))) break;
-                        tc_fence_after();
-                        mma_pv(tmem + 256 + BM * w, tmem + BM * w, kh, vb, cnt[w] > 0 || kh > 0);
-                    }
-                    if (!ok) break;
-                    mma_commit(&sm.pv_done[w]);
-                    ++cnt[w];
-                }
-                mma_commit(&sm.kv_empty[st]);
+                if (ok && part(1, i)) pv(1, i);
+                if (!ok) break;
+                // stage i: its K was read by Q K^T of both tiles and its V by both P V
+                mma_commit(&sm.kv_empty[i & 1]);
+                if (nxt && part(1, i + 1)) qk(1, i + 1);
             }
             mma_commit(&sm.drain);
             mbar_wait_drain_(&sm.drain, 0, DRAIN_NS);
