@@ -4,9 +4,12 @@
 // "路线一：滑动窗口注意力": position i attends to the most recent W positions of its sequence,
 //   o_i = sum_{j = i-W+1 .. i} softmax_j(scale q_i . k_j) v_j .
 // FlashAttention-style, as the page suggests for this mixer, built on tcgen05:
-//   * one CTA takes two 128-query tiles of one (batch, head), queries q0 .. q0 + 255; the key
-//     tiles of 128 that their windows touch (ten at W = 1024) stream through two TMA stages and
-//     serve both query tiles;
+//   * an item of work is two 128-query tiles of one (batch, head), queries q0 .. q0 + 255; the
+//     key tiles of 128 that their windows touch (ten at W = 1024) stream through two TMA stages
+//     and serve both query tiles;
+//   * the kernel is persistent, one CTA per SM taking items round-robin; a query tile's slot is
+//     loaded with the next item's queries as soon as its output has been stored, so the next
+//     item starts while the last one finishes;
 //   * S = Q K^T for each query tile goes to tensor memory; two softmax warpgroups per query
 //     tile (one query row per thread, keys [0, 64) and [64, 128) of the key tile) mask the
 //     window, share the row's running maximum through shared memory, keep their partial sums,
@@ -62,7 +65,10 @@ struct __align__(1024) SwaSmem {
     unsigned char k[2][TILE];
     unsigned char v[2][TILE];
     // p_ready[w][kh]: query tile w's P over keys [64 kh, 64 kh + 64) is in tensor memory
-    uint64_t q_full, kv_full[2], kv_empty[2], s_full[2], p_ready[2][2], pv_done[2], drain;
+    // q_full[w]: query tile w of the item is loaded; q_free[w]: its output has been stored (the
+    // slot may be loaded again); o_free[w]: its O accumulator has been read
+    uint64_t q_full[2], q_free[2], o_free[2];
+    uint64_t kv_full[2], kv_empty[2], s_full[2], p_ready[2][2], pv_done[2], drain;
     uint32_t dec[2][2];                  // the softmax pairs' shared wait outcomes
     // the two halves of a query row exchange their partial maxima (double-buffered by tile) and,
     // at the end, their partial sums
@@ -79,7 +85,28 @@ struct SwaParams {
     int64_t N;
     int H;
     int n_qpairs;          // query-tile pairs per sequence
+    int64_t n_items;       // (batch, head, query-tile pair) items
 };
+
+// One item of work: two 128-query tiles of one (batch, head), queries q0 .. q0 + 255, and the
+// key tiles [kt_lo, kt_lo + ntiles) their windows touch.
+struct SwaItem {
+    int64_t q0, kt_lo;
+    int ntiles, h, b;
+};
+
+__device__ __forceinline__ SwaItem item_of(const SwaParams& p, int64_t t) {
+    SwaItem it;
+    const int pair = (int)(t % p.n_qpairs);
+    it.h = (int)((t / p.n_qpairs) % p.H);
+    it.b = (int)(t / ((int64_t)p.n_qpairs * p.H));
+    it.q0 = (int64_t)pair * 2 * 128;
+    const int64_t qlast = (it.q0 + 2 * 128 - 1 < p.N - 1) ? it.q0 + 2 * 128 - 1 : p.N - 1;
+    const int64_t kfirst = (it.q0 - p.window + 1 > 0) ? it.q0 - p.window + 1 : 0;
+    it.kt_lo = kfirst / 128;
+    it.ntiles = (int)(qlast / 128 - it.kt_lo + 1);
+    return it;
+}
 
 __device__ __forceinline__ float ex2f(float x) {
     float y;
@@ -181,20 +208,11 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     SwaSmem& sm = *reinterpret_cast<SwaSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if ((smem_u32(smem_raw) & 1023u) != 0) return;   // never: dynamic shared memory starts aligned
-    // the CTA's work: (batch, head, query-tile pair)
-    const int64_t blk = blockIdx.x;
-    const int pair = (int)(blk % p.n_qpairs);
-    const int h = (int)((blk / p.n_qpairs) % p.H);
-    const int b = (int)(blk / ((int64_t)p.n_qpairs * p.H));
-    const int64_t q0 = (int64_t)pair * 2 * BM;
-    const int64_t qlast = (q0 + 2 * BM - 1 < p.N - 1) ? q0 + 2 * BM - 1 : p.N - 1;
-    const int64_t kfirst = (q0 - p.window + 1 > 0) ? q0 - p.window + 1 : 0;
-    const int64_t kt_lo = kfirst / BM, kt_hi = qlast / BM;
-    const int ntiles = (int)(kt_hi - kt_lo + 1);
-
     if (tid == 0) {
-        mbar_init(&sm.q_full, 1);
         for (int s = 0; s < 2; ++s) {
+            mbar_init(&sm.q_full[s], 1);
+            mbar_init(&sm.q_free[s], 1);
+            mbar_init(&sm.o_free[s], 256);
             mbar_init(&sm.kv_full[s], 1);
             mbar_init(&sm.kv_empty[s], 1);
             mbar_init(&sm.s_full[s], 1);
@@ -214,78 +232,126 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    // The CTA is persistent: it takes items t = blockIdx.x, blockIdx.x + gridDim.x, ...; every
+    // role walks the same list, and every barrier's phase count runs on across items.
 
     if (warp < 4) {
         asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
         if (warp == 0 && lane == 0) {
-            // ---- producer: both query tiles, then the key / value tiles through two stages
+            // ---- producer: per item, query tile 0, the first key / value tile, query tile 1,
+            // the other key / value tiles (two stages).  A query slot is loaded again once the
+            // previous item's output tile has left it.
             tma_prefetch_desc(&tq);
             tma_prefetch_desc(&tk);
             tma_prefetch_desc(&tv);
             tma_prefetch_desc(&to);
-            mbar_arrive_expect_tx(&sm.q_full, 2 * TILE);
-            for (int w = 0; w < 2; ++w)
+            int g = 0, n = 0;      // key / value tiles and items issued
+            bool ok = true;
+            auto load_q = [&](const SwaItem& it, int w) {
+                if (n > 0 && !(ok = wait_abortable(sm, &sm.q_free[w], (n - 1) & 1))) return;
+                mbar_arrive_expect_tx(&sm.q_full[w], TILE);
                 for (int half = 0; half < 2; ++half)
-                    tma_load_4d(sm.q[w] + half * SLAB, &tq, &sm.q_full, half * 64, h,
-                                (int)(q0 + BM * w), b);
-            int i = 0;
-            for (; i < ntiles; ++i) {
-                const int st = i & 1;
-                if (i >= 2 && !wait_abortable(sm, &sm.kv_empty[st], ((i >> 1) - 1) & 1)) break;
-                const int tok = (int)((kt_lo + i) * BM);
+                    tma_load_4d(sm.q[w] + half * SLAB, &tq, &sm.q_full[w], half * 64, it.h,
+                                (int)(it.q0 + BM * w), it.b);
+            };
+            auto load_kv = [&](const SwaItem& it, int i) {
+                const int st = g & 1;
+                if (g >= 2 && !(ok = wait_abortable(sm, &sm.kv_empty[st], ((g >> 1) - 1) & 1)))
+                    return;
+                const int tok = (int)((it.kt_lo + i) * BM);
                 mbar_arrive_expect_tx(&sm.kv_full[st], 2 * TILE);
                 for (int half = 0; half < 2; ++half) {
-                    tma_load_4d(sm.k[st] + half * SLAB, &tk, &sm.kv_full[st], half * 64, h, tok, b);
-                    tma_load_4d(sm.v[st] + half * SLAB, &tv, &sm.kv_full[st], half * 64, h, tok, b);
+                    tma_load_4d(sm.k[st] + half * SLAB, &tk, &sm.kv_full[st], half * 64, it.h,
+                                tok, it.b);
+                    tma_load_4d(sm.v[st] + half * SLAB, &tv, &sm.kv_full[st], half * 64, it.h,
+                                tok, it.b);
                 }
+                ++g;
+            };
+            for (int64_t t = blockIdx.x; t < p.n_items && ok; t += gridDim.x) {
+                const SwaItem it = item_of(p, t);
+                load_q(it, 0);
+                for (int i = 0; i < it.ntiles && ok; ++i) {
+                    load_kv(it, i);
+                    if (i == 0 && ok) load_q(it, 1);
+                }
+                if (ok) ++n;
             }
             // no TMA write into this CTA's shared memory may be in flight at exit
-            mbar_wait_drain_(&sm.q_full, 0, DRAIN_NS);
-            for (int ii = (i >= 2 ? i - 2 : 0); ii < i; ++ii)
-                mbar_wait_drain_(&sm.kv_full[ii & 1], (ii >> 1) & 1, DRAIN_NS);
+            for (int gg = (g >= 2 ? g - 2 : 0); gg < g; ++gg)
+                mbar_wait_drain_(&sm.kv_full[gg & 1], (gg >> 1) & 1, DRAIN_NS);
+            if (n > 0)
+                for (int w = 0; w < 2; ++w) mbar_wait_drain_(&sm.q_full[w], (n - 1) & 1, DRAIN_NS);
         } else if (warp == 1 && lane == 0) {
             // ---- MMA issuer.  Query tile 0 runs one step ahead of tile 1: Q_0 K_{i+1}^T is
             // issued right after P_0 V_i, before P_1 V_i, so that tile 0's next softmax overlaps
             // tile 1's products instead of both tiles' softmaxes running at the same time.
-            bool ok = wait_abortable(sm, &sm.q_full, 0);
-            int cnt[2] = {0, 0};
-            auto part = [&](int w, int i) { return takes_part(q0, w, kt_lo + i, p.window, p.N); };
-            auto qk = [&](int w, int i) {   // S_w = Q_w K_i^T, once P V has read S_w's last P
-                if (cnt[w] > 0 && !(ok = wait_abortable(sm, &sm.pv_done[w], (cnt[w] - 1) & 1)))
-                    return;
-                tc_fence_after();
-                mma_qk(tmem + BM * w, smem_u32(sm.q[w]), smem_u32(sm.k[i & 1]));
-                mma_commit(&sm.s_full[w]);
-            };
-            auto pv = [&](int w, int i) {   // O_w += P_w V_i, one half of the keys at a time
-                const uint32_t vb = smem_u32(sm.v[i & 1]);
-                for (int kh = 0; kh < 2 && ok; ++kh) {
-                    if (!(ok = wait_abortable(sm, &sm.p_ready[w][kh], cnt[w] & 1))) return;
+            // Every item waits each tile's q_full phase once and (after the first item) each
+            // tile's o_free phase once, before the first use or at the item's end.
+            bool ok = true;
+            int cnt[2] = {0, 0};   // P V products issued per query tile (all items)
+            int g = 0, n = 0;      // key / value tiles and items consumed
+            for (int64_t t = blockIdx.x; t < p.n_items && ok; t += gridDim.x) {
+                const SwaItem it = item_of(p, t);
+                bool need_q[2] = {true, true}, need_o[2] = {n > 0, n > 0}, first[2] = {true, true};
+                auto part = [&](int w, int i) {
+                    return takes_part(it.q0, w, it.kt_lo + i, p.window, p.N);
+                };
+                auto qk = [&](int w, int i) {   // S_w = Q_w K_i^T, once P V has read the last P
+                    if (need_q[w]) {
+                        if (!(ok = wait_abortable(sm, &sm.q_full[w], n & 1))) return;
+                        need_q[w] = false;
+                    }
+                    if (cnt[w] > 0 && !(ok = wait_abortable(sm, &sm.pv_done[w], (cnt[w] - 1) & 1)))
+                        return;
                     tc_fence_after();
-                    mma_pv(tmem + 256 + BM * w, tmem + BM * w, kh, vb, cnt[w] > 0 || kh > 0);
+                    mma_qk(tmem + BM * w, smem_u32(sm.q[w]), smem_u32(sm.k[(g + i) & 1]));
+                    mma_commit(&sm.s_full[w]);
+                };
+                auto pv = [&](int w, int i) {   // O_w += P_w V_i, one half of the keys at a time
+                    if (need_o[w]) {   // the previous item's O_w has been read
+                        if (!(ok = wait_abortable(sm, &sm.o_free[w], (n - 1) & 1))) return;
+                        need_o[w] = false;
+                    }
+                    const uint32_t vb = smem_u32(sm.v[(g + i) & 1]);
+                    for (int kh = 0; kh < 2 && ok; ++kh) {
+                        if (!(ok = wait_abortable(sm, &sm.p_ready[w][kh], cnt[w] & 1))) return;
+                        tc_fence_after();
+                        mma_pv(tmem + 256 + BM * w, tmem + BM * w, kh, vb, !first[w] || kh > 0);
+                    }
+                    first[w] = false;
+                    mma_commit(&sm.pv_done[w]);
+                    ++cnt[w];
+                };
+                auto kv_wait = [&](int i) {
+                    const int gi = g + i;
+                    if ((ok = wait_abortable(sm, &sm.kv_full[gi & 1], (gi >> 1) & 1))) tc_fence_after();
+                };
+                if (it.ntiles > 0) {
+                    kv_wait(0);
+                    if (ok && part(0, 0)) qk(0, 0);
+                    if (ok && part(1, 0)) qk(1, 0);
                 }
-                mma_commit(&sm.pv_done[w]);
-                ++cnt[w];
-            };
-            if (ok && ntiles > 0 && (ok = wait_abortable(sm, &sm.kv_full[0], 0))) {
-                tc_fence_after();
-                if (part(0, 0)) qk(0, 0);
-                if (ok && part(1, 0)) qk(1, 0);
-            }
-            for (int i = 0; i < ntiles && ok; ++i) {
-                const bool nxt = i + 1 < ntiles;
-                if (part(0, i)) pv(0, i);
-                if (ok && nxt) {
-                    if (!(ok = wait_abortable(sm, &sm.kv_full[(i + 1) & 1], ((i + 1) >> 1) & 1)))
-                        break;
-                    tc_fence_after();
-                    if (part(0, i + 1)) qk(0, i + 1);
+                for (int i = 0; i < it.ntiles && ok; ++i) {
+                    const bool nxt = i + 1 < it.ntiles;
+                    if (part(0, i)) pv(0, i);
+                    if (ok && nxt) {
+                        kv_wait(i + 1);
+                        if (ok && part(0, i + 1)) qk(0, i + 1);
+                    }
+                    if (ok && part(1, i)) pv(1, i);
+                    if (!ok) break;
+                    // this stage: its K was read by Q K^T of both tiles and its V by both P V
+                    mma_commit(&sm.kv_empty[(g + i) & 1]);
+                    if (nxt && part(1, i + 1)) qk(1, i + 1);
                 }
-                if (ok && part(1, i)) pv(1, i);
-                if (!ok) break;
-                // stage i: its K was read by Q K^T of both tiles and its V by both P V
-                mma_commit(&sm.kv_empty[i & 1]);
-                if (nxt && part(1, i + 1)) qk(1, i + 1);
+                // the phases this item did not need
+                for (int w = 0; w < 2 && ok; ++w) {
+                    if (need_q[w]) ok = wait_abortable(sm, &sm.q_full[w], n & 1);
+                    if (ok && need_o[w]) ok = wait_abortable(sm, &sm.o_free[w], (n - 1) & 1);
+                }
+                g += it.ntiles;
+                ++n;
             }
             mma_commit(&sm.drain);
             mbar_wait_drain_(&sm.drain, 0, DRAIN_NS);
@@ -301,12 +367,22 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
         const uint32_t s_addr = tmem + lane_base + BM * w + 64 * hf;        // this half of S / P
         const uint32_t o_addr = tmem + lane_base + 256 + BM * w + 64 * hf;  // this half of O
-        const int64_t qi = q0 + BM * w + r;      // this thread's query position
-        float m_ref = -INFINITY, l = 0.f;
-        int cnt = 0, flip = 0;
+        int cnt = 0, flip = 0;   // key tiles taken part in (all items): the barriers' phases
         bool ok = true;
+        for (int64_t t = blockIdx.x; t < p.n_items && ok; t += gridDim.x) {
+        // token positions fit in 32 bits (the host checks N)
+        int q0, kt_lo, ntiles;
+        {
+            const SwaItem it = item_of(p, t);
+            q0 = (int)it.q0;
+            kt_lo = (int)it.kt_lo;
+            ntiles = it.ntiles;
+        }
+        const int qi = q0 + BM * w + r;          // this thread's query position
+        float m_ref = -INFINITY, l = 0.f;
+        int cnt_item = 0;
         for (int i = 0; i < ntiles && ok; ++i) {
-            const int64_t kt = kt_lo + i;
+            const int kt = kt_lo + i;
             if (!takes_part(q0, w, kt, p.window, p.N)) continue;
             // pair-uniform outcome: no warp may split around the warp-wide TMEM accesses, and
             // neither half may leave while the other waits at the pair's barrier
@@ -314,10 +390,9 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             if (!ok) break;
             tc_fence_after();
             // visible keys of this row in this half: columns [c_lo, c_hi] of the half
-            const int64_t c_lo64 = qi - p.window + 1 - BM * kt - 64 * hf,
-                          c_hi64 = qi - BM * kt - 64 * hf;
-            const int c_lo = c_lo64 < 0 ? 0 : (c_lo64 > 64 ? 64 : (int)c_lo64);
-            const int c_hi = c_hi64 > 63 ? 63 : (c_hi64 < -1 ? -1 : (int)c_hi64);
+            const int c_lo64 = qi - p.window + 1 - BM * kt - 64 * hf, c_hi64 = qi - BM * kt - 64 * hf;
+            const int c_lo = c_lo64 < 0 ? 0 : (c_lo64 > 64 ? 64 : c_lo64);
+            const int c_hi = c_hi64 > 63 ? 63 : (c_hi64 < -1 ? -1 : c_hi64);
             // scores in log2 units are c s; the half's maximum of c s over its visible keys is
             // c max(s) for c >= 0 and c min(s) otherwise (eight independent partial extrema),
             // 32 columns at a time.  Halves wholly inside every row's window skip the per-key
@@ -415,10 +490,13 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             tc_fence_before();
             mbar_arrive(&sm.p_ready[w][hf]);   // P V over this half's keys may run
             ++cnt;
+            ++cnt_item;
         }
         // ---- epilogue: O / l in bf16 through this tile's query slot (each half its 64
-        // columns), then one TMA store
-        if (cnt > 0) {
+        // columns), then one TMA store.  O_w is released (o_free) once read, the query slot
+        // (q_free) once the store has read it; both once per item, also for a tile that took
+        // no part.
+        if (cnt_item > 0) {
             if (ok) ok = pair_wait(sm, &sm.pv_done[w], (cnt - 1) & 1, w, hf, r, flip);
             tc_fence_after();
             sm.xl[w][hf][r] = l;
@@ -431,6 +509,10 @@ __global__ void __launch_bounds__(NTHREADS, 1)
                 float t32[32];
                 tmem_ld32(o_addr + jc * 32, t32);
                 tmem_ld_wait();
+                if (jc == 1) {
+                    tc_fence_before();
+                    mbar_arrive(&sm.o_free[w]);
+                }
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4) {
                     uint4 u;
@@ -445,12 +527,19 @@ __global__ void __launch_bounds__(NTHREADS, 1)
             fence_proxy_async_smem();
             pair_sync(w);   // both halves of the tile are written
             if (hf == 0 && r == 0) {
+                const SwaItem it = item_of(p, t);
                 for (int half = 0; half < 2; ++half)
-                    tma_store_4d(&to, sm.q[w] + half * SLAB, half * 64, h, (int)(q0 + BM * w), b);
+                    tma_store_4d(&to, sm.q[w] + half * SLAB, half * 64, it.h, q0 + BM * w, it.b);
                 bulk_commit_group();
-                bulk_wait_group0();
+                bulk_wait_group_read0();
+                mbar_arrive(&sm.q_free[w]);
             }
+        } else {
+            mbar_arrive(&sm.o_free[w]);
+            if (hf == 0 && r == 0) mbar_arrive(&sm.q_free[w]);
         }
+        }   // items
+        if (hf == 0 && r == 0) bulk_wait_group0();   // the last stores have completed
     }
     tc_fence_before();
     __syncthreads();
@@ -481,8 +570,15 @@ cudaError_t launch_swa(const SwaArgs& a, cudaStream_t stream) {
     p.N = a.N;
     p.H = a.H;
     p.n_qpairs = (int)((a.N + 2 * BM - 1) / (2 * BM));
-    const int64_t grid = (int64_t)a.B * a.H * p.n_qpairs;
-    if (grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+    p.n_items = (int64_t)a.B * a.H * p.n_qpairs;
+    // persistent: one CTA per SM (at most one per item)
+    int dev = 0, n_sm = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&n_sm, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess ||
+        n_sm < 1)
+        return cudaErrorUnknown;
+    const int64_t grid = p.n_items < n_sm ? p.n_items : n_sm;
+    if (grid == 0) return cudaSuccess;   // nothing to do
     const size_t smem = sizeof(SwaSmem);
     cudaError_t e = cudaFuncSetAttribute(swa_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
