@@ -527,19 +527,16 @@ def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
                          "kernel": "gn_gate_kernel", "algorithmic_flops_per_launch": flops}}
 
 
-# fp32 FMA peak of the CUDA-core path: 148 SMs x 128 fp32 lanes x 2 FLOP x 1.965 GHz (the
-# maximum SM clock); FLOP per token and head of the per-channel-gate prefill at chunk 64:
-# chunk state 2 d^2, cross-chunk output 2 d^2, in-chunk scores and A V 2 d (C + 1) / 2 each,
-# scan 2 d^2 / C.
-FP32_FMA_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12
-EW_FLOP_PER_TOKEN_HEAD = 2 * D * D + 2 * D * D + 2 * (2 * D * (64 + 1) // 2) + 2 * D * D // 64
+# Algorithmic bytes per token and head of the per-channel-gate prefill: q, k, v, o in bf16 and
+# one fp32 gate logit per key channel.
+EW_BYTES_PER_TOKEN_HEAD = 4 * D * 2 + 4 * D
 
 
 def run_elementwise(args, rank, world, stream, headwise_ms):
-    """The per-key-channel-gate prefill (three CUDA-core launches: chunk states, scan over
-    chunks, chunk outputs) on the 3B shapes, 32768 tokens x 24 heads, bf16 q, k, v and one fp32
-    gate logit per key channel.  Also reports the head-wise kernel's time on the same shapes
-    over this variant's: the hardware-efficiency cost of a gate per channel."""
+    """The per-key-channel-gate prefill (three launches: range aggregates on the tensor cores,
+    scan over ranges, range outputs on the tensor cores) on the 3B shapes, 32768 tokens x 24
+    heads, bf16 q, k, v and one fp32 gate logit per key channel.  Also reports the head-wise
+    kernel's time on the same shapes over this variant's: the cost of a gate per channel."""
     import torch
 
     import gated_retention_linear_b200 as G
@@ -573,23 +570,25 @@ def run_elementwise(args, rank, world, stream, headwise_ms):
     e1.record(stream)
     torch.cuda.synchronize()
     ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    if G.gret_workspace_status(ws) != 0:
+        raise RuntimeError("per-channel prefill reported a timed-out wait")
     tokens = Bq * Nq
-    flops = float(EW_FLOP_PER_TOKEN_HEAD) * tokens * Hq
-    ach = flops / (ms * 1e-3) / 1e12
+    alg = float(EW_BYTES_PER_TOKEN_HEAD) * tokens * Hq
+    ach = alg / (ms * 1e-3) / 1e9
+    peak, kind = measured_peaks()
     return {"value": tokens * world / (ms * 1e-3) / 1e6, "unit": "Mtok/s", "tokens": tokens,
             "heads": Hq, "ms_per_step": ms, "steps": n, "gpu_launches_per_step": 3,
             "gate": "one logit per key channel, g ~ N(2, 1)",
             "headwise_ms_same_shapes": headwise_ms,
             "slowdown_vs_headwise": ms / headwise_ms,
             "workspace_bytes": ws.numel(),
-            "l2": "inputs (1.2 GB) and the 812 MB chunk-state workspace larger than L2; "
-                  "not flushed",
-            "roofline": {"bound": "alu", "achieved": ach, "peak": FP32_FMA_PEAK_TFLOPS,
-                         "unit": "TFLOP/s", "frac": ach / FP32_FMA_PEAK_TFLOPS,
-                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 x 1.965 GHz",
-                         "traffic": None,
-                         "kernel": "ew_chunk_state + ew_state_scan + ew_chunk_output",
-                         "algorithmic_flops_per_launch": flops}}
+            "l2": "inputs and outputs (1.2 GB) larger than L2; not flushed",
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
+                         "frac": ach / peak, "peak_kind": kind,
+                         "traffic": traffic_from_profile("prefill_ew.cu",
+                                                         "ew_kernels_32k.txt"),
+                         "kernel": "ew_range_state + ew_state_scan + ew_range_output",
+                         "algorithmic_bytes_per_launch": alg}}
 
 
 def run_swa(args, rank, world, stream, headwise_ms):

@@ -216,11 +216,11 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
     return launch_qkvg_projection(x, w, ldw, T, H, D, q, k, v, g, (cudaStream_t)stream);
 }
 
-// Sizes the per-channel gate prefill can take: the scan's grid (B * H * 16 blocks) fits in
-// gridDim.x and the workspace byte count fits in size_t.
+// Sizes the per-channel gate prefill can take: the range kernels' grid (ranges, H, B) and the
+// scan's (B * H * 16 blocks) fit their limits, and the workspace byte count fits in size_t.
 bool ew_sizes_ok(int B, int64_t N, int H) {
     const int64_t nch = (N + EW_CHUNK - 1) / EW_CHUNK;
-    if (B > 65535 || H > 65535 || nch > 0x7fffffff) return false;
+    if (B > 65535 || H > 65535 || nch > 0x7fffffff || N > (int64_t)0x7FFFFF00) return false;
     if ((int64_t)B * H * 16 > 0x7fffffff) return false;
     const double bytes = (double)B * H * (double)nch * (EW_DIM * EW_DIM + EW_DIM) * 4.0;
     return bytes < 9.0e18;
@@ -239,7 +239,6 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
     if (B < 0 || N < 0 || H < 1 || d < 1) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
     if (d != EW_DIM) return GRET_ERR_UNSUPPORTED;
-    const int64_t nch = (N + EW_CHUNK - 1) / EW_CHUNK;
     if (!ew_sizes_ok(B, N, H)) return GRET_ERR_UNSUPPORTED;
     if (B == 0) return GRET_OK;
     if ((state_in && !aligned16(state_in)) || (state_out && !aligned16(state_out)))
@@ -263,12 +262,13 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
     a.k = static_cast<const __nv_bfloat16*>(k);
     a.v = static_cast<const __nv_bfloat16*>(v);
     a.g = g; a.tau = tau; a.k_scale = k_scale;
-    a.B = B; a.N = N; a.H = H; a.nch = (int)nch;
+    a.B = B; a.N = N; a.H = H;
     a.state_in = state_in; a.state_out = state_out;
     a.o = static_cast<__nv_bfloat16*>(o);
-    a.ws_S = static_cast<float*>(workspace);
-    a.ws_a = a.ws_S + (size_t)B * H * nch * EW_DIM * EW_DIM;
-    return launch_prefill_ew(a, s) == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+    a.workspace = workspace;
+    const cudaError_t e = launch_prefill_ew(a, s);
+    if (e == cudaErrorInvalidValue) return GRET_ERR_UNSUPPORTED;   // a tensor map was refused
+    return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
 gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, float scale,

@@ -1,172 +1,337 @@
-// prefill_ew.cu -- chunkwise prefill of gated retention with one gate per key channel: the
-// element-wise gate that "路线二：Multi-Head Gated Retention" weighs against the head-wise
-// scalar gate YOCO keeps.  CUDA cores, fp32 arithmetic on bf16 q, k, v.
+// prefill_ew.cu -- chunkwise prefill of gated retention with one gate per key channel (the
+// element-wise gate that "路线二：Multi-Head Gated Retention" weighs against the head-wise scalar
+// gate YOCO keeps), on the sm_100a tensor cores.
 //
 // Per sequence and head, with alpha_t[i] = sigmoid(g_t[i])^(1/tau) for key channel i:
 //   S_t[i][:] = alpha_t[i] S_{t-1}[i][:] + k_scale k_t[i] v_t ,   o_t = q_t S_t
-// Chunks of C = 64 tokens; c_t[i] is channel i's inclusive cumulative log-decay in the chunk
-// (the chunkwise re-association of "Prefill 与 Decode 为什么使用两种计算形态", per channel):
-//   1. ew_chunk_state   dS_c = sum_m (k_scale k_m * e^{c_last - c_m})^T v_m ,  a_c = e^{c_last}
-//   2. ew_state_scan    S_prev(0) = S_in,  S_prev(c+1) = a_c * S_prev(c) + dS_c  (row-wise
-//                       scale; element-parallel over the state, serial over chunks)
-//   3. ew_chunk_output  o_t = (q_t * e^{c_t}) S_prev(c) + sum_{m<=t} A[t][m] v_m ,
-//                       A[t][m] = k_scale sum_i q_t[i] k_m[i] e^{c_t[i] - c_m[i]}
-// Across sub-chunks A splits at p, the last token before t's sub-chunk: e^{c_t - c_p}
-// e^{c_p - c_m}, both factors at most 1, so no scaled operand can overflow whatever the gates.
-// Inside a 16-token sub-chunk it splits at the token before the sub-chunk when every channel's
-// decay over the sub-chunk is moderate, and takes the exponentials pair by pair otherwise.
+// Chunks of C = 128 tokens; c_t[i] is channel i's inclusive cumulative log2-decay inside the
+// chunk and c_L[i] its chunk total (the chunkwise form of "Prefill 与 Decode 为什么使用两种计算
+// 形态", one decay per channel).  With a scalar gate the decay of a (query, key) pair is one
+// number that can scale the score matrix after Q K^T; with a gate per channel it sits inside the
+// contraction over i, so here it is folded into the operands before the MMAs:
+//   K~[m][i] = k_scale k_m[i] 2^(c_L[i] - c_m[i])          (<= |k_scale k|: always finite)
+//   Q^[t][i] = q_t[i] 2^(c_t[i] - c_L[i])                   (>= |q|: bounded by the check below)
+//   S'       = diag(2^c_L) S_prev                           (the state decayed over the chunk)
+// so that, with the intra-chunk pair decay 2^(c_t - c_m) = 2^(c_t - c_L) 2^(c_L - c_m),
+//   P   = mask_{m <= t}( Q^ K~^T )                          (scores, decay included)
+//   o   = Q^ S' + P V                                       (cross-chunk + inner terms)
+//   S   = S' + K~^T V                                       (next chunk's state)
+// Every factored operand is an fp32 value split into a bf16 high half and a bf16 low half; the
+// products take hi*hi + lo*hi + hi*lo (Q^ K~^T, Q^ S') or both halves against an exact bf16
+// operand (P V, K~^T V), which keeps the result near 1e-5 of rms.
 //
-// With a scalar gate the decay of a (t, m) pair is one number, so the head-wise kernel folds it
-// into a masked score matrix and runs every contraction on the tensor cores.  With a gate per
-// channel the decay sits inside the contraction over i; this path pays for that with the
-// chunk-state round trip through the workspace and with an exponential per channel for every
-// scaled operand (per pair and channel when a sub-chunk's gates are extreme).
-#include <cuda_bf16.h>
-#include <stdint.h>
-
-#include "common.cuh"
+// Range of the factorisation.  Q^ grows with the chunk's decay: when some channel decays by more
+// than 2^-SPAN2 over the chunk the masked (m > t) scores could overflow and Q^ loses meaning.
+// Such a chunk takes the safe form: the scores come pairwise on CUDA cores,
+//   P[t][m] = k_scale sum_i q_t[i] k_m[i] 2^(c_t[i] - c_m[i])   (every exponent <= 0)
+// and the cross term uses Q~ = q 2^c_t (<= |q|) against the undecayed state.  Gates that decay
+// that fast (below about 2^-0.5 per token per channel) are rare; the path exists for exactness.
+//
+// Parallelism.  A sequence's chunks are grouped into ranges of G chunks (G from a wave model on
+// the host).  Three launches:
+//   ew_range_state   one CTA per range: the range's aggregate sum over its keys of
+//                    (decay to the range end) k^T v, one tensor-memory accumulator over the
+//                    range (keys weighted by their decay to the range end: always <= 1), and
+//                    the range's total decay per channel
+//   ew_state_scan    per (sequence, head), serial over ranges: entry state of every range
+//   ew_range_output  one CTA per range, chunks in order from the range's entry state: the
+//                    outputs above, and the state carried to the next chunk of the range
+// The range kernels are synchronous per CTA (one block-wide phase after another; one thread
+// issues the MMAs) and take a whole SM each (224 KB of shared memory).
 #include "prefill_ew.cuh"
 
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tma_host.cuh"
+
 namespace gret {
+
+using namespace sm100;
+
 namespace {
 
-constexpr int C = EW_CHUNK;   // tokens per chunk
-constexpr int SC = 16;        // tokens per sub-chunk
-constexpr int D = EW_DIM;     // d_k = d_v
-constexpr int NT = 256;       // threads per block of the chunk kernels
-constexpr int CQS = D + 1;    // row stride (floats) of the log-decay / scaled-q tile
-constexpr int SS = D + 4;     // row stride (floats) of the scaled q / k rows of a sub-chunk pair
+constexpr int C = EW_CHUNK;             // tokens per chunk
+constexpr int D = EW_DIM;               // d_k = d_v
+constexpr int NT = 256;                 // threads of the range kernels
+constexpr int TILE = C * D * 2;         // one bf16 128 x 128 tile
+constexpr int SLAB = TILE / 2;          // one 64-column slab of it
+constexpr int GTILE = C * D * 4;        // the chunk's fp32 gate logits
+constexpr float SPAN2 = 64.f;           // largest chunk log2-decay of the factored form
+constexpr uint64_t WAIT_NS = 2000000000ull;
+constexpr uint64_t DRAIN_NS = 200000000ull;
+constexpr uint32_t TM_A = 0, TM_O = 128, TM_S = 256;   // scores / P, output, state update
+constexpr size_t WS_HEAD = 256;          // status word, then the range slots
 
-constexpr size_t SMEM_STATE = (size_t)C * D * 4 + (size_t)C * D * 2 + D * 4;
-constexpr size_t SMEM_OUT = (size_t)C * CQS * 4 + 2 * (size_t)C * D * 2 + (size_t)C * C * 4 +
-                            (size_t)2 * SC * SS * 4;
+struct EwParams {
+    float inv_tau_log2e;   // log2(e) / tau
+    float k_scale;
+    int64_t N;
+    int H, R, G;           // heads, ranges per sequence, chunks per range
+    float* ws_S;           // [B][H][R][D][D]: range aggregates, then range entry states
+    float* ws_a;           // [B][H][R][D]: range decays
+    uint32_t* err;
+    __nv_bfloat16* o;
+};
 
-__device__ __forceinline__ void unpack4(uint2 u, float* f) {
-    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.x));
-    const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&u.y));
-    f[0] = a.x; f[1] = a.y; f[2] = b.x; f[3] = b.y;
+struct __align__(1024) OutSmem {
+    unsigned char q[TILE];   // q, then the high half of the query operand (in place)
+    unsigned char k[TILE];   // k, then the high half of K~ (in place)
+    unsigned char v[TILE];
+    unsigned char x[TILE];   // low half of the query operand; then the output tile
+    unsigned char y[TILE];   // low half of K~  (x and y: fp32 P of a pairwise chunk)
+    float g[C * D];          // gate logits -> cumulative log2-decay -> state operand hi | lo
+    float tot[2][D];         // per channel: log2-decay of tokens [0, 64) and [64, 128)
+    uint64_t ld_full, mma_done, drain;
+    uint32_t tmem_base;
+};
+
+struct __align__(1024) StateSmem {
+    unsigned char k[TILE];   // k, then the high half of the weighted keys (in place)
+    unsigned char v[TILE];
+    unsigned char y[TILE];   // low half of the weighted keys
+    float g[C * D];          // gate logits -> per-token log2-decay
+    float tot[2][D];
+    uint64_t ld_full, mma_done, drain;
+    uint32_t tmem_base;
+};
+
+static_assert(sizeof(OutSmem) <= 232448, "shared-memory plan exceeds 227 KB");
+static_assert(sizeof(StateSmem) <= 232448, "shared-memory plan exceeds 227 KB");
+
+__host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
+
+__device__ __forceinline__ float ex2f(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
 }
 
-__device__ __forceinline__ uint2 pack4(float a, float b, float c, float d) {
-    __nv_bfloat162 lo = __floats2bfloat162_rn(a, b), hi = __floats2bfloat162_rn(c, d);
-    return make_uint2(*reinterpret_cast<uint32_t*>(&lo), *reinterpret_cast<uint32_t*>(&hi));
+// log(sigmoid(x)) = min(x, 0) - log(1 + exp(-|x|)) with the fast exponential and logarithm
+// (absolute error near 1e-7, which is what a cumulative sum of these sees).
+__device__ __forceinline__ float logsigmoid_fast(float x) {
+    return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
 }
 
-// Copy rows [0, L) of a [C][D] bf16 chunk tile into shared memory, zeros in rows [L, C).
-__device__ __forceinline__ void load_tile(__nv_bfloat16* dst, const __nv_bfloat16* src,
-                                          int64_t row0, int H, int L, int tid, int first,
-                                          int nthreads) {
-    for (int p = tid - first; p < C * D / 8; p += nthreads) {
-        const int t = p / (D / 8), col = (p % (D / 8)) * 8;
-        uint4 val = make_uint4(0u, 0u, 0u, 0u);
-        if (t < L) val = *reinterpret_cast<const uint4*>(src + (row0 + (int64_t)t * H) * D + col);
-        *reinterpret_cast<uint4*>(dst + t * D + col) = val;
+__device__ __forceinline__ float bf16_at(const unsigned char* tile, uint32_t off) {
+    return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
+}
+
+// x = hi + lo, hi = bf16(x), lo = bf16(x - hi)
+__device__ __forceinline__ void split1(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+    hi = __float2bfloat16_rn(x);
+    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+}
+
+__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
+// Every thread of the block waits on the barrier itself; the block agrees on the outcome, and a
+// wait that gave up records GRET_ERR_TIMEOUT in the workspace.
+__device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+    uint32_t never = 0;
+    const bool ok = mbar_wait(bar, parity, &never, WAIT_NS);
+    const int bad = __syncthreads_or(!ok);
+    if (bad && threadIdx.x == 0) atomicExch(err, WS_ERR_TIMEOUT);
+    return bad == 0;
+}
+
+// D (+)= A B over K = 128: eight K-steps of 16, bf16 operands in shared memory (64-column slabs,
+// 128-byte swizzle).  a_mn / b_mn: the operand is stored MN-major (M or N contiguous).
+__device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, uint32_t b_base,
+                                        bool b_mn, bool accumulate) {
+    const uint32_t idesc = idesc_bf16(128, 128, a_mn, b_mn);
+#pragma unroll 1
+    for (int kk = 0; kk < 8; ++kk) {
+        const uint32_t aoff = a_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
+        const uint32_t boff = b_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
+        const uint64_t ad = a_mn ? sdesc_sw128(a_base + aoff, SLAB, 1024)
+                                 : sdesc_sw128(a_base + aoff, 16, 1024);
+        const uint64_t bd = b_mn ? sdesc_sw128(b_base + boff, SLAB, 1024)
+                                 : sdesc_sw128(b_base + boff, 16, 1024);
+        mma_ss(d, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
     }
 }
 
-// Log-decays logsigmoid(g) / tau of tokens [0, L) of the chunk into c[t * stride + i], by all
-// threads of the block (no barrier inside).
-__device__ __forceinline__ void log_decays(const EwArgs& a, int64_t row0, int L, int tid,
-                                           float* c, int stride) {
-    const float inv_tau = 1.f / a.tau;
-    for (int e = tid; e < L * D; e += NT) {
-        const int t = e / D, i = e - t * D;
-        c[t * stride + i] = logsigmoidf_(a.g[(row0 + (int64_t)t * a.H) * D + i]) * inv_tau;
-    }
+// D += P V with P (bf16 halves, K-major) in tensor memory: per 32-token group g the columns
+// [32 g, 32 g + 16) hold the high halves and [32 g + 16, 32 g + 32) the low halves, two tokens
+// per column; V [token x d_v] in shared memory.
+__device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
+                                       bool accumulate) {
+    const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
+#pragma unroll 1
+    for (int kk = 0; kk < 8; ++kk)
+        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
+               sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
+               (accumulate || kk > 0) ? 1u : 0u);
 }
 
-// Thread `tid` < D: turn channel tid's log-decays into the inclusive cumulative sum over the
-// chunk, in place.  Returns the chunk total.
-__device__ __forceinline__ float channel_cumsum(int L, int tid, float* c, int stride) {
-    float cum = 0.f;
-#pragma unroll 16
-    for (int t = 0; t < L; ++t) {
-        cum += c[t * stride + tid];
-        c[t * stride + tid] = cum;
+// Loads of one chunk: bf16 tiles as two 64-column slabs each, the gate logits as one fp32 box.
+// Coordinates of every map: (column, head, token, batch); rows past the sequence read as zero.
+__device__ __forceinline__ void load_tiles(unsigned char* q, unsigned char* k, unsigned char* v,
+                                           float* g, const CUtensorMap* tq, const CUtensorMap* tk,
+                                           const CUtensorMap* tv, const CUtensorMap* tg,
+                                           uint64_t* bar, int tok, int h, int b) {
+    const uint32_t bytes = (q ? TILE : 0) + 2 * TILE + GTILE;
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        if (q) tma_load_4d(q + half * SLAB, tq, bar, half * 64, h, tok, b);
+        tma_load_4d(k + half * SLAB, tk, bar, half * 64, h, tok, b);
+        tma_load_4d(v + half * SLAB, tv, bar, half * 64, h, tok, b);
     }
-    return cum;
+    tma_load_4d(g, tg, bar, 0, h, tok, b);
 }
 
-// 1. Chunk state and chunk decay.  Block (chunk, head, batch).
-__global__ void __launch_bounds__(NT) ew_chunk_state(EwArgs a) {
-    extern __shared__ float4 smem_f4[];
-    float* kt = reinterpret_cast<float*>(smem_f4);                        // [C][D]
-    __nv_bfloat16* vs = reinterpret_cast<__nv_bfloat16*>(kt + C * D);      // [C][D]
-    float* clast = reinterpret_cast<float*>(vs + C * D);                  // [D]
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int64_t t0 = (int64_t)c * C;
-    const int L = (int)min((int64_t)C, a.N - t0);
-    const int64_t row0 = ((int64_t)b * a.N + t0) * a.H + h;
-    const int64_t slot = ((int64_t)b * a.H + h) * a.nch + c;
+// ----------------------------------------------------------------------------------------------
+// 1. Range aggregates.  Block (range, head, batch).  The range's chunks are visited last to
+// first so that each key's weight, its log2-decay to the end of the range, is a running suffix
+// sum; every K~^T V MMA of the range accumulates into one tensor-memory result.
 
-    load_tile(vs, a.v, row0, a.H, L, tid, 0, NT);
-    log_decays(a, row0, L, tid, kt, D);                      // kt holds c_t for now
+__global__ void __launch_bounds__(NT, 1)
+    ew_range_state(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
+                   const __grid_constant__ CUtensorMap tg, const EwParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    StateSmem& sm = *reinterpret_cast<StateSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if ((smem_u32(smem_raw) & 1023u) != 0) {   // the swizzled tiles need 1 KB alignment
+        if (tid == 0) atomicExch(p.err, WS_ERR_TIMEOUT);
+        return;
+    }
+    const int64_t nch = (p.N + C - 1) / C;
+    const int c0 = r * p.G;
+    const int c1 = (int)min64(nch, (int64_t)c0 + p.G);
+    if (tid == 0) {
+        mbar_init(&sm.ld_full, 1);
+        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 128);
+        tmem_relinquish();
+    }
+    tc_fence_before();
     __syncthreads();
-    if (tid < D) clast[tid] = channel_cumsum(L, tid, kt, D);
-    __syncthreads();
-    for (int e = tid; e < L * D; e += NT) {
-        const int t = e / D, i = e - t * D;
-        const float kv = __bfloat162float(a.k[(row0 + (int64_t)t * a.H) * D + i]);
-        kt[e] = a.k_scale * kv * __expf(clast[i] - kt[e]);
-    }
-    if (tid < D) a.ws_a[slot * D + tid] = expf(clast[tid]);
-    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    const int i = tid & 127, hh = tid >> 7;           // channel, token half (also TMEM lane, column half)
+    const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
 
-    // dS[i][j] = sum_m kt[m][i] v[m][j]: rows {ri..ri+3, 64+ri..}, columns {cj..cj+3, 64+cj..}
-    const int ri = (tid >> 4) * 4, cj = (tid & 15) * 4;
-    float acc[8][8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int s = 0; s < 8; ++s) acc[r][s] = 0.f;
-    for (int m = 0; m < L; ++m) {
-        const float4 a0 = *reinterpret_cast<const float4*>(kt + m * D + ri);
-        const float4 a1 = *reinterpret_cast<const float4*>(kt + m * D + 64 + ri);
-        const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
-        float bv[8];
-        unpack4(*reinterpret_cast<const uint2*>(vs + m * D + cj), bv);
-        unpack4(*reinterpret_cast<const uint2*>(vs + m * D + 64 + cj), bv + 4);
-#pragma unroll
-        for (int r = 0; r < 8; ++r)
-#pragma unroll
-            for (int s = 0; s < 8; ++s) acc[r][s] = fmaf(av[r], bv[s], acc[r][s]);
+    if (tid == 0) load_tiles(nullptr, sm.k, sm.v, sm.g, nullptr, &tk, &tv, &tg, &sm.ld_full,
+                             (c1 - 1) * C, h, b);
+    float R = 0.f;   // log2-decay of the tokens after the current chunk, to the range end
+    uint32_t n_ld = 1, n_mma = 0;
+    bool ok = true;
+    for (int c = c1 - 1; c >= c0; --c) {
+        const int L = (int)min64(C, p.N - (int64_t)c * C);
+        if (!(ok = block_wait(&sm.ld_full, (n_ld - 1) & 1, p.err))) break;
+        // per-token log2-decays of channel i over this thread's half, in place
+        float sum = 0.f;
+#pragma unroll 8
+        for (int t = 64 * hh; t < 64 * hh + 64; ++t) {
+            float* gp = &sm.g[t * D + i];
+            const float lam = t < L ? logsigmoid_fast(*gp) * p.inv_tau_log2e : 0.f;
+            *gp = lam;
+            sum += lam;
+        }
+        sm.tot[hh][i] = sum;
+        __syncthreads();
+        const float t0 = sm.tot[0][i], t1 = sm.tot[1][i];
+        // weights 2^(suffix) k_scale, suffix = log2-decay from after token t to the range end
+        float s = R + (hh == 0 ? t1 : 0.f);
+#pragma unroll 4
+        for (int t = 64 * hh + 63; t >= 64 * hh; --t) {
+            const uint32_t off = sw128_offset(t, i, SLAB);
+            const float kw = bf16_at(sm.k, off) * ex2f(s) * p.k_scale;
+            __nv_bfloat16 hi, lo;
+            split1(kw, hi, lo);
+            *reinterpret_cast<__nv_bfloat16*>(sm.k + off) = hi;
+            *reinterpret_cast<__nv_bfloat16*>(sm.y + off) = lo;
+            s += sm.g[t * D + i];
+        }
+        R += t0 + t1;
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // Agg (+)= K~_hi^T V + K~_lo^T V: A = K~^T (channels x tokens) stored token-major
+            mma_128(tmem, smem_u32(sm.k), true, smem_u32(sm.v), true, c != c1 - 1);
+            mma_128(tmem, smem_u32(sm.y), true, smem_u32(sm.v), true, true);
+            mma_commit(&sm.mma_done);
+        }
+        ++n_mma;
+        if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
+        if (c > c0 && tid == 0) {
+            load_tiles(nullptr, sm.k, sm.v, sm.g, nullptr, &tk, &tv, &tg, &sm.ld_full,
+                       (c - 1) * C, h, b);
+        }
+        if (c > c0) ++n_ld;
     }
-    float* dS = a.ws_S + slot * (int64_t)(D * D);
+    if (ok) {
+        tc_fence_after();
+        const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
+        float* dst = p.ws_S + slot * (D * D) + (int64_t)i * D + 64 * hh;
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int i = r < 4 ? ri + r : 64 + ri + (r - 4);
-        *reinterpret_cast<float4*>(dS + i * D + cj) =
-            make_float4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-        *reinterpret_cast<float4*>(dS + i * D + 64 + cj) =
-            make_float4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+        for (int jc = 0; jc < 2; ++jc) {
+            float a[32];
+            tmem_ld32(tmem + lane_base + 64 * hh + 32 * jc, a);
+            tmem_ld_wait();
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+                reinterpret_cast<float4*>(dst + 32 * jc)[e] =
+                    make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
+        }
+        if (hh == 0) p.ws_a[slot * D + i] = ex2f(R);
+    } else if (tid == 0) {
+        // a wait gave up: let the issued MMAs and any load in flight finish before exit
+        mma_commit(&sm.drain);
+        uint32_t never = 0;
+        mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
+        mbar_wait(&sm.ld_full, (n_ld - 1) & 1, &never, DRAIN_NS);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 128);
     }
 }
 
-// 2. Scan over chunks.  Block: one (batch, head) and 8 state rows; thread: one row, 4 columns.
-// The chunk-state slot c is overwritten with the state entering chunk c.
-__global__ void __launch_bounds__(256) ew_state_scan(EwArgs a) {
-    constexpr int U = 8;   // chunks whose loads are issued together
+// ----------------------------------------------------------------------------------------------
+// 2. Scan over ranges.  Block: one (batch, head) and 8 state rows; thread: one row, 4 columns.
+// The aggregate slot of range r is overwritten with the state entering range r.
+__global__ void __launch_bounds__(256) ew_state_scan(EwParams p, const float* state_in,
+                                                     float* state_out) {
+    constexpr int U = 8;   // ranges whose loads are issued together
     const int64_t bh = blockIdx.x / 16;
     const int i = (blockIdx.x % 16) * 8 + threadIdx.x / 32;
     const int j = (threadIdx.x % 32) * 4;
     const int64_t off = (int64_t)i * D + j;
     float4 S = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (a.state_in) S = *reinterpret_cast<const float4*>(a.state_in + bh * D * D + off);
-    float* base = a.ws_S + bh * a.nch * (int64_t)(D * D) + off;
-    const float* abase = a.ws_a + bh * a.nch * (int64_t)D + i;
-    for (int c0 = 0; c0 < a.nch; c0 += U) {
+    if (state_in) S = *reinterpret_cast<const float4*>(state_in + bh * D * D + off);
+    float* base = p.ws_S + bh * p.R * (int64_t)(D * D) + off;
+    const float* abase = p.ws_a + bh * p.R * (int64_t)D + i;
+    for (int c0 = 0; c0 < p.R; c0 += U) {
         float4 d[U];
         float al[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (c0 + u < a.nch) {
+            if (c0 + u < p.R) {
                 d[u] = *reinterpret_cast<const float4*>(base + (int64_t)(c0 + u) * (D * D));
                 al[u] = abase[(int64_t)(c0 + u) * D];
             }
         }
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            if (c0 + u < a.nch) {
+            if (c0 + u < p.R) {
                 *reinterpret_cast<float4*>(base + (int64_t)(c0 + u) * (D * D)) = S;
                 S.x = fmaf(al[u], S.x, d[u].x);
                 S.y = fmaf(al[u], S.y, d[u].y);
@@ -175,215 +340,391 @@ __global__ void __launch_bounds__(256) ew_state_scan(EwArgs a) {
             }
         }
     }
-    if (a.state_out) *reinterpret_cast<float4*>(a.state_out + bh * D * D + off) = S;
+    if (state_out) *reinterpret_cast<float4*>(state_out + bh * D * D + off) = S;
 }
 
-// 3. Chunk output.  Block (chunk, head, batch).
-__global__ void __launch_bounds__(NT) ew_chunk_output(EwArgs a) {
-    extern __shared__ float4 smem_f4[];
-    float* cq = reinterpret_cast<float*>(smem_f4);                       // [C][CQS]: c, then q*e^c
-    __nv_bfloat16* qs = reinterpret_cast<__nv_bfloat16*>(cq + C * CQS);   // [C][D]
-    __nv_bfloat16* kv = qs + C * D;                                      // [C][D]: k, then v
-    float* At = reinterpret_cast<float*>(kv + C * D);                    // [C][C]: At[m][t] = A[t][m]
-    float* scr = At + C * C;                                             // [2 SC][SS], or S rows
-    const int c = blockIdx.x, h = blockIdx.y, b = blockIdx.z, tid = threadIdx.x;
-    const int warp = tid >> 5, lane = tid & 31;
-    const int64_t t0 = (int64_t)c * C;
-    const int L = (int)min((int64_t)C, a.N - t0);
-    const int64_t row0 = ((int64_t)b * a.N + t0) * a.H + h;
-    const int64_t slot = ((int64_t)b * a.H + h) * a.nch + c;
+// ----------------------------------------------------------------------------------------------
+// 3. Outputs.  Block (range, head, batch); chunks in order from the range's entry state.
 
-    load_tile(qs, a.q, row0, a.H, L, tid, 0, NT);
-    load_tile(kv, a.k, row0, a.H, L, tid, 0, NT);
-    for (int e = tid; e < C * C; e += NT) At[e] = 0.f;
-    log_decays(a, row0, L, tid, cq, CQS);
+// Scores of a chunk whose decay is too fast for the factored form, pairwise on CUDA cores (every
+// exponent c_t - c_m <= 0), into P^T [m][t] fp32 over the x and y tiles; then P into tensor
+// memory as bf16 halves.  Needs the chunk's raw q and k tiles and the cumulative log2-decays
+// over the whole chunk in sm.g.
+__device__ void pairwise_scores(OutSmem& sm, const EwParams& p, uint32_t tmem, int L) {
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* Pt = reinterpret_cast<float*>(sm.x);
+    for (int e = tid; e < C * C; e += NT) Pt[e] = 0.f;
     __syncthreads();
-    if (tid < D) channel_cumsum(L, tid, cq, CQS);
-    __syncthreads();
-
-    // A inside each sub-chunk.  With r the token before the sub-chunk (c_r = 0 before the chunk),
-    // e^{c_t - c_m} = e^{c_t - c_r} e^{c_r - c_m}: the block is a dot product of scaled rows, as
-    // across sub-chunks.  The second factor exceeds 1, so the split is taken only while every
-    // channel's decay over the sub-chunk stays within SPAN_MAX (both factors then stay normal
-    // fp32 numbers); otherwise each pair takes its exponentials one by one.
-    constexpr float SPAN_MAX = 80.f;
-    for (int s = 0; s < C / SC && s * SC < L; ++s) {
-        const int r0 = s * SC, last = min(r0 + SC, L) - 1;
-        int wide = 0;
-        if (tid < D) {
-            const float cref = s == 0 ? 0.f : cq[(r0 - 1) * CQS + tid];
-            wide = cref - cq[last * CQS + tid] > SPAN_MAX;
+    for (int pr = warp; pr < C * C; pr += NT / 32) {
+        const int t = pr >> 7, m = pr & (C - 1);
+        if (m > t || t >= L) continue;   // warp-uniform
+        float acc = 0.f;
+#pragma unroll
+        for (int u = 0; u < D / 32; ++u) {
+            const int ch = lane + 32 * u;
+            acc += bf16_at(sm.q, sw128_offset(t, ch, SLAB)) * bf16_at(sm.k, sw128_offset(m, ch, SLAB)) *
+                   ex2f(sm.g[t * D + ch] - sm.g[m * D + ch]);
         }
-        if (__syncthreads_or(wide)) {
-            // one warp per (t, m) pair, lanes over the channels
-            for (int it = warp; it < SC * SC; it += NT / 32) {
-                const int tt = it / SC, mm = it % SC;
-                const int t = r0 + tt, m = r0 + mm;
-                if (mm > tt || t >= L) continue;
-                float acc = 0.f;
 #pragma unroll
-                for (int u = 0; u < D / 32; ++u) {
-                    const int i = lane + 32 * u;
-                    acc += __bfloat162float(qs[t * D + i]) * __bfloat162float(kv[m * D + i]) *
-                           __expf(cq[t * CQS + i] - cq[m * CQS + i]);
-                }
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (lane == 0) Pt[m * C + t] = acc * p.k_scale;
+    }
+    __syncthreads();
+    const int row = (warp & 3) * 32 + lane, hh = warp >> 2;
+    const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
+#pragma unroll 1
+    for (int jc = 2 * hh; jc < 2 * hh + 2; ++jc) {
+        uint32_t ph[32];
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
-                if (lane == 0) At[m * C + t] = a.k_scale * acc;
-            }
-        } else {
-            for (int e = tid; e < 2 * SC * D; e += NT) {
-                const int r = e / D, i = e - r * D;
-                const float cref = s == 0 ? 0.f : cq[(r0 - 1) * CQS + i];
-                const int t = r0 + (r < SC ? r : r - SC);
-                float val = 0.f;
-                if (t < L)
-                    val = r < SC ? __bfloat162float(qs[t * D + i]) * __expf(cq[t * CQS + i] - cref)
-                                 : __bfloat162float(kv[t * D + i]) * __expf(cref - cq[t * CQS + i]);
-                scr[r * SS + i] = val;
-            }
+        for (int i2 = 0; i2 < 16; ++i2) {
+            const int m0 = jc * 32 + 2 * i2;
+            split2(Pt[m0 * C + row], Pt[(m0 + 1) * C + row], ph[i2], ph[16 + i2]);
+        }
+        tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
+    }
+    tmem_st_wait();
+    tc_fence_before();
+    __syncthreads();
+}
+
+__global__ void __launch_bounds__(NT, 1)
+    ew_range_output(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
+                    const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap tg,
+                    const __grid_constant__ CUtensorMap to, const EwParams p) {
+    extern __shared__ __align__(1024) unsigned char smem_raw[];
+    OutSmem& sm = *reinterpret_cast<OutSmem*>(smem_raw);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int r = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+    if ((smem_u32(smem_raw) & 1023u) != 0) {
+        if (tid == 0) atomicExch(p.err, WS_ERR_TIMEOUT);
+        return;
+    }
+    const int64_t nch = (p.N + C - 1) / C;
+    const int c0 = r * p.G;
+    const int c1 = (int)min64(nch, (int64_t)c0 + p.G);
+    if (tid == 0) {
+        mbar_init(&sm.ld_full, 1);
+        mbar_init(&sm.mma_done, 1);
+        mbar_init(&sm.drain, 1);
+        fence_mbar_init();
+    }
+    if (warp == 0) {
+        tmem_alloc(&sm.tmem_base, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    // thread (i, hh): channel / state row i = TMEM lane, column half (token half in the
+    // per-channel passes) hh
+    const int i = tid & 127, hh = tid >> 7;
+    const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
+    const uint32_t qb = smem_u32(sm.q), kb = smem_u32(sm.k), vb = smem_u32(sm.v),
+                   xb = smem_u32(sm.x), yb = smem_u32(sm.y), shb = smem_u32(sm.g),
+                   slb = shb + TILE;
+
+    if (tid == 0) load_tiles(sm.q, sm.k, sm.v, sm.g, &tq, &tk, &tv, &tg, &sm.ld_full, c0 * C, h, b);
+    // entry state of the range: row i, columns [64 hh, 64 hh + 64)
+    const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
+    float S[64];
+    {
+        const float4* src =
+            reinterpret_cast<const float4*>(p.ws_S + slot * (D * D) + (int64_t)i * D + 64 * hh);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+            const float4 x = src[e];
+            S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
+        }
+    }
+    uint32_t n_ld = 1, n_mma = 0;
+    bool ok = true;
+    for (int c = c0; c < c1; ++c) {
+        const int L = (int)min64(C, p.N - (int64_t)c * C);
+        const bool last = c == c1 - 1;
+        if (c > c0) {   // the previous output tile has left x
+            if (tid == 0) bulk_wait_group_read0();
             __syncthreads();
-            const int r = tid / SC, mm = tid % SC;
-            const float* qr = scr + r * SS;
-            const float* kr = scr + (SC + mm) * SS;
-            float acc = 0.f;
-#pragma unroll 8
-            for (int i = 0; i < D; i += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(qr + i);
-                const float4 y = *reinterpret_cast<const float4*>(kr + i);
-                acc = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc))));
-            }
-            if (mm <= r && r0 + r < L) At[(r0 + mm) * C + r0 + r] = a.k_scale * acc;
         }
-        __syncthreads();   // scr is reused by the next sub-chunk
-    }
-
-    // A across sub-chunks: rows of sub-chunk ts against columns of sub-chunk ms < ts, split at
-    // p = ts * SC - 1:  q_t e^{c_t - c_p}  .  k_m e^{c_p - c_m}.
-    for (int ts = 1; ts < C / SC && ts * SC < L; ++ts) {
-        const int p = ts * SC - 1;
-        for (int ms = 0; ms < ts; ++ms) {
-            __syncthreads();   // previous readers of scr are done
-            for (int e = tid; e < 2 * SC * D; e += NT) {
-                const int r = e / D, i = e - r * D;
-                float val = 0.f;
-                if (r < SC) {
-                    const int t = ts * SC + r;
-                    if (t < L)
-                        val = __bfloat162float(qs[t * D + i]) *
-                              __expf(cq[t * CQS + i] - cq[p * CQS + i]);
-                } else {
-                    const int m = ms * SC + (r - SC);
-                    val = __bfloat162float(kv[m * D + i]) *
-                          __expf(cq[p * CQS + i] - cq[m * CQS + i]);
-                }
-                scr[r * SS + i] = val;
-            }
-            __syncthreads();
-            const int r = tid / SC, mm = tid % SC;
-            const float* qr = scr + r * SS;
-            const float* kr = scr + (SC + mm) * SS;
-            float acc = 0.f;
+        if (!(ok = block_wait(&sm.ld_full, (n_ld - 1) & 1, p.err))) break;
+        // cumulative log2-decay of channel i over this thread's token half, in place
+        float cum = 0.f;
 #pragma unroll 8
-            for (int i = 0; i < D; i += 4) {
-                const float4 x = *reinterpret_cast<const float4*>(qr + i);
-                const float4 y = *reinterpret_cast<const float4*>(kr + i);
-                acc = fmaf(x.x, y.x, fmaf(x.y, y.y, fmaf(x.z, y.z, fmaf(x.w, y.w, acc))));
-            }
-            if (ts * SC + r < L) At[(ms * SC + mm) * C + ts * SC + r] = a.k_scale * acc;
+        for (int t = 64 * hh; t < 64 * hh + 64; ++t) {
+            float* gp = &sm.g[t * D + i];
+            cum += t < L ? logsigmoid_fast(*gp) * p.inv_tau_log2e : 0.f;
+            *gp = cum;
         }
-    }
-    __syncthreads();   // all of A written; k and the log-decays no longer needed as such
-
-    // The entry state of the chunk is read in slices of SR rows, each fetched into registers
-    // one slice ahead of its use; the first fetch overlaps the work below.
-    constexpr int SR = 2 * SC, PF = SR * D / 4 / NT;
-    const float4* Sp = reinterpret_cast<const float4*>(a.ws_S + slot * (int64_t)(D * D));
-    float4 pf[PF];
-#pragma unroll
-    for (int u = 0; u < PF; ++u) pf[u] = Sp[tid + u * NT];
-
-    // q * e^{c} in place (zero rows past L), and v into the k tile.
-    for (int e = tid; e < C * D; e += NT) {
-        const int t = e / D, i = e - t * D;
-        float val = 0.f;
-        if (t < L) val = __bfloat162float(qs[t * D + i]) * __expf(cq[t * CQS + i]);
-        cq[t * CQS + i] = val;
-    }
-    load_tile(kv, a.v, row0, a.H, L, tid, 0, NT);
-    __syncthreads();
-
-    // o[t][j] for rows {tr..tr+3}, columns {cj..cj+3, 64+cj..}
-    const int tr = (tid >> 4) * 4, cj = (tid & 15) * 4;
-    float acc[4][8];
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int s = 0; s < 8; ++s) acc[r][s] = 0.f;
-    for (int m = 0; m < L; ++m) {
-        const float4 av = *reinterpret_cast<const float4*>(At + m * C + tr);
-        const float ar[4] = {av.x, av.y, av.z, av.w};
-        float bv[8];
-        unpack4(*reinterpret_cast<const uint2*>(kv + m * D + cj), bv);
-        unpack4(*reinterpret_cast<const uint2*>(kv + m * D + 64 + cj), bv + 4);
-#pragma unroll
-        for (int r = 0; r < 4; ++r)
-#pragma unroll
-            for (int s = 0; s < 8; ++s) acc[r][s] = fmaf(ar[r], bv[s], acc[r][s]);
-    }
-    for (int i0 = 0; i0 < D; i0 += SR) {
-#pragma unroll
-        for (int u = 0; u < PF; ++u) reinterpret_cast<float4*>(scr)[tid + u * NT] = pf[u];
+        sm.tot[hh][i] = cum;
         __syncthreads();
-        if (i0 + SR < D) {
-#pragma unroll
-            for (int u = 0; u < PF; ++u) pf[u] = Sp[(i0 + SR) * D / 4 + tid + u * NT];
+        const float t0 = sm.tot[0][i], cL = t0 + sm.tot[1][i];
+        const bool pairwise = __syncthreads_or(cL < -SPAN2) != 0;
+        if (pairwise) {
+            if (hh == 1) {
+#pragma unroll 8
+                for (int t = 64; t < C; ++t) sm.g[t * D + i] += t0;
+            }
+            __syncthreads();
+            pairwise_scores(sm, p, tmem, L);
         }
+        // operands: query (factored: 2^(c_t - c_L); pairwise: 2^(c_t)) and K~ = k_scale k
+        // 2^(c_L - c_t), each as bf16 high half in place and low half in x / y
+        {
+            const float off = (hh == 1 && !pairwise) ? t0 : 0.f;
+            const float qshift = pairwise ? 0.f : -cL;
 #pragma unroll 4
-        for (int ii = 0; ii < SR; ++ii) {
-            float ar[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) ar[r] = cq[(tr + r) * CQS + i0 + ii];
-            const float4 b0 = *reinterpret_cast<const float4*>(scr + ii * D + cj);
-            const float4 b1 = *reinterpret_cast<const float4*>(scr + ii * D + 64 + cj);
-            const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
-#pragma unroll
-            for (int r = 0; r < 4; ++r)
-#pragma unroll
-                for (int s = 0; s < 8; ++s) acc[r][s] = fmaf(ar[r], bv[s], acc[r][s]);
+            for (int t = 64 * hh; t < 64 * hh + 64; ++t) {
+                const float ct = sm.g[t * D + i] + off;
+                const uint32_t o = sw128_offset(t, i, SLAB);
+                const float qs = bf16_at(sm.q, o) * ex2f(ct + qshift);
+                const float ks = bf16_at(sm.k, o) * ex2f(cL - ct) * p.k_scale;
+                __nv_bfloat16 qh, ql, kh, kl;
+                split1(qs, qh, ql);
+                split1(ks, kh, kl);
+                *reinterpret_cast<__nv_bfloat16*>(sm.q + o) = qh;
+                *reinterpret_cast<__nv_bfloat16*>(sm.x + o) = ql;
+                *reinterpret_cast<__nv_bfloat16*>(sm.k + o) = kh;
+                *reinterpret_cast<__nv_bfloat16*>(sm.y + o) = kl;
+            }
         }
-        __syncthreads();
-    }
+        __syncthreads();   // every read of the log2-decays is done: sm.g takes the state operand
+        // state operand: 2^c_L S (factored) or S (pairwise), row i, slab hh of the MN-major
+        // high-half and low-half tiles
+        {
+            const float sc = pairwise ? 1.f : ex2f(cL);
+            unsigned char* shi = reinterpret_cast<unsigned char*>(sm.g);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int t = tr + r;
-        if (t >= L) continue;
-        __nv_bfloat16* dst = a.o + (row0 + (int64_t)t * a.H) * D;
-        *reinterpret_cast<uint2*>(dst + cj) = pack4(acc[r][0], acc[r][1], acc[r][2], acc[r][3]);
-        *reinterpret_cast<uint2*>(dst + 64 + cj) =
-            pack4(acc[r][4], acc[r][5], acc[r][6], acc[r][7]);
+            for (int cc = 0; cc < 8; ++cc) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    split2(sc * S[8 * cc + 2 * e], sc * S[8 * cc + 2 * e + 1], hi[e], lo[e]);
+                const uint32_t off = hh * SLAB + i * 128 + ((cc ^ (i & 7)) << 4);
+                *reinterpret_cast<uint4*>(shi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(shi + TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
+        }
+        fence_proxy_async_smem();
+        __syncthreads();
+        if (!pairwise) {
+            if (tid == 0) {
+                tc_fence_after();
+                mma_128(tmem + TM_A, qb, false, kb, false, false);   // Q_hi K~_hi^T
+                mma_128(tmem + TM_A, xb, false, kb, false, true);    //  + Q_lo K~_hi^T
+                mma_128(tmem + TM_A, qb, false, yb, false, true);    //  + Q_hi K~_lo^T
+                mma_commit(&sm.mma_done);
+            }
+            ++n_mma;
+            if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
+            tc_fence_after();
+            // causal mask, P split into bf16 halves in place: row = lane, 64 columns per thread
+            const int row = (warp & 3) * 32 + lane;
+#pragma unroll 1
+            for (int jc = 2 * hh; jc < 2 * hh + 2; ++jc) {
+                float a[32];
+                tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
+                tmem_ld_wait();
+                uint32_t ph[32];
+#pragma unroll
+                for (int i2 = 0; i2 < 16; ++i2) {
+                    const int m0 = jc * 32 + 2 * i2;
+                    split2(m0 <= row ? a[2 * i2] : 0.f, m0 + 1 <= row ? a[2 * i2 + 1] : 0.f,
+                           ph[i2], ph[16 + i2]);
+                }
+                tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            __syncthreads();
+        }
+        if (tid == 0) {
+            tc_fence_after();
+            mma_128(tmem + TM_O, qb, false, shb, true, false);   // O = Q_hi S_hi
+            mma_128(tmem + TM_O, xb, false, shb, true, true);    //   + Q_lo S_hi
+            mma_128(tmem + TM_O, qb, false, slb, true, true);    //   + Q_hi S_lo
+            mma_pv(tmem + TM_O, tmem + TM_A, 0, vb, true);       //   + P_hi V
+            mma_pv(tmem + TM_O, tmem + TM_A, 1, vb, true);       //   + P_lo V
+            if (!last) {
+                mma_128(tmem + TM_S, kb, true, vb, true, false); // dS = K~_hi^T V
+                mma_128(tmem + TM_S, yb, true, vb, true, true);  //    + K~_lo^T V
+            }
+            mma_commit(&sm.mma_done);
+        }
+        ++n_mma;
+        if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
+        tc_fence_after();
+        if (!last) {   // every tile but x is free: the next chunk's loads go now
+            if (tid == 0)
+                load_tiles(sm.q, sm.k, sm.v, sm.g, &tq, &tk, &tv, &tg, &sm.ld_full, (c + 1) * C, h, b);
+            ++n_ld;
+        }
+        // output rows: a chunk inside the sequence goes out as one tile through x (rows in the
+        // swizzled layout, two TMA stores); the rows of a partial chunk one by one
+        const int row = (warp & 3) * 32 + lane;
+        const bool full = L == C;
+        const int64_t tok = (int64_t)c * C + row;
+        uint4* orow = reinterpret_cast<uint4*>(p.o + (((int64_t)b * p.N + tok) * p.H + h) * D);
+#pragma unroll 1
+        for (int jc = 2 * hh; jc < 2 * hh + 2; ++jc) {
+            float o[32];
+            tmem_ld32(tmem + lane_base + TM_O + jc * 32, o);
+            tmem_ld_wait();
+#pragma unroll
+            for (int v4 = 0; v4 < 4; ++v4) {
+                uint4 u;
+                u.x = pack_bf16x2(o[8 * v4 + 0], o[8 * v4 + 1]);
+                u.y = pack_bf16x2(o[8 * v4 + 2], o[8 * v4 + 3]);
+                u.z = pack_bf16x2(o[8 * v4 + 4], o[8 * v4 + 5]);
+                u.w = pack_bf16x2(o[8 * v4 + 6], o[8 * v4 + 7]);
+                const int cc = 4 * jc + v4;   // 16-byte chunk of the row
+                if (full)
+                    *reinterpret_cast<uint4*>(sm.x + (cc >> 3) * SLAB + row * 128 +
+                                              (((cc & 7) ^ (row & 7)) << 4)) = u;
+                else if (row < L)
+                    orow[cc] = u;
+            }
+        }
+        // the state carried to the next chunk: S = 2^c_L S + dS
+        if (!last) {
+            const float eL = ex2f(cL);
+#pragma unroll
+            for (int jc = 0; jc < 2; ++jc) {
+                float d[32];
+                tmem_ld32(tmem + lane_base + TM_S + 64 * hh + 32 * jc, d);
+                tmem_ld_wait();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) S[32 * jc + e] = fmaf(eL, S[32 * jc + e], d[e]);
+            }
+        }
+        tc_fence_before();
+        if (full) fence_proxy_async_smem();
+        __syncthreads();
+        if (full && tid == 0) {
+#pragma unroll
+            for (int half = 0; half < 2; ++half)
+                tma_store_4d(&to, sm.x + half * SLAB, half * 64, h, c * C, b);
+            bulk_commit_group();
+        }
     }
+    if (tid == 0) {
+        if (!ok) {   // a wait gave up: the issued MMAs and any load in flight finish first
+            mma_commit(&sm.drain);
+            uint32_t never = 0;
+            mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
+            mbar_wait(&sm.ld_full, (n_ld - 1) & 1, &never, DRAIN_NS);
+        }
+        bulk_wait_group0();
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+// ----------------------------------------------------------------------------------------------
+// host side
+
+int sm_count_ew() {
+    static int cached[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) dev = 0;
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        int n = 0;
+        if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) n = 0;
+        cached[dev] = n > 0 ? n : 148;
+    }
+    return cached[dev];
+}
+
+// [B, N, H, 128] contiguous, coordinates (column, head, token, batch); bf16 with 64-column
+// swizzled boxes, or fp32 with one unswizzled 128-column box.
+bool make_ew_map(CUtensorMap* map, const void* base, bool fp32, int B, int64_t N, int H) {
+    EncodeTiledFn fn = encode_tiled_fn();
+    if (!fn) return false;
+    const uint64_t es = fp32 ? 4 : 2;
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)H, (cuuint64_t)N, (cuuint64_t)B};
+    cuuint64_t strides[3] = {D * es, (cuuint64_t)H * D * es, (cuuint64_t)N * H * D * es};
+    cuuint32_t box[4] = {fp32 ? (cuuint32_t)D : 64u, 1u, (cuuint32_t)C, 1u};
+    cuuint32_t estr[4] = {1, 1, 1, 1};
+    return fn(map, fp32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4,
+              const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+              fp32 ? CU_TENSOR_MAP_SWIZZLE_NONE : CU_TENSOR_MAP_SWIZZLE_128B,
+              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
-size_t ew_workspace_bytes(int B, int64_t N, int H) {
+// Chunks per range.  A range kernel runs ceil(B H R / SMs) waves of CTAs (R = ceil(chunks / G)
+// ranges per sequence), each about G + 1 chunk-times long: its chunks plus a start (the first
+// loads and the entry state, exposed since a CTA has its SM to itself).  G minimises that, and
+// among equal costs the largest G wins (fewer ranges: less workspace traffic, a shorter scan).
+int ew_range_chunks(int B, int64_t N, int H) {
     const int64_t nch = (N + C - 1) / C;
-    return (size_t)B * H * nch * (size_t)(D * D + D) * sizeof(float);
+    if (nch <= 1 || B < 1 || H < 1) return 1;
+    const int64_t grid = sm_count_ew();
+    const int64_t units = (int64_t)B * H;
+    int best = 1;
+    int64_t best_cost = -1;
+    const int64_t gmax = std::min<int64_t>(nch, 1 << 20);
+    for (int64_t g = 1; g <= gmax; ++g) {
+        const int64_t ranges = (nch + g - 1) / g;
+        if (g > 1 && ranges == (nch + g - 2) / (g - 1)) continue;   // same R as g - 1
+        const int64_t cost = ((units * ranges + grid - 1) / grid) * (g + 1);
+        if (best_cost < 0 || cost <= best_cost) {
+            best = (int)g;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+int64_t ew_ranges(int B, int64_t N, int H) {
+    const int64_t nch = (N + C - 1) / C;
+    const int G = ew_range_chunks(B, N, H);
+    return (nch + G - 1) / G;
+}
+
+size_t ew_workspace_bytes(int B, int64_t N, int H) {
+    const int64_t R = ew_ranges(B, N, H);
+    return WS_HEAD + (size_t)B * H * R * (size_t)(D * D + D) * sizeof(float);
 }
 
 cudaError_t launch_prefill_ew(const EwArgs& a, cudaStream_t stream) {
-    cudaError_t e = cudaFuncSetAttribute(ew_chunk_state,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)SMEM_STATE);
+    const int G = ew_range_chunks(a.B, a.N, a.H);
+    const int64_t R = ew_ranges(a.B, a.N, a.H);
+    unsigned char* ws = static_cast<unsigned char*>(a.workspace);
+    EwParams p;
+    p.inv_tau_log2e = 1.4426950408889634f / a.tau;
+    p.k_scale = a.k_scale;
+    p.N = a.N;
+    p.H = a.H;
+    p.R = (int)R;
+    p.G = G;
+    p.err = reinterpret_cast<uint32_t*>(ws);
+    p.ws_S = reinterpret_cast<float*>(ws + WS_HEAD);
+    p.ws_a = p.ws_S + (size_t)a.B * a.H * R * D * D;
+    p.o = a.o;
+    CUtensorMap tq, tk, tv, tg, to;
+    if (!make_ew_map(&tq, a.q, false, a.B, a.N, a.H) || !make_ew_map(&tk, a.k, false, a.B, a.N, a.H) ||
+        !make_ew_map(&tv, a.v, false, a.B, a.N, a.H) || !make_ew_map(&tg, a.g, true, a.B, a.N, a.H) ||
+        !make_ew_map(&to, a.o, false, a.B, a.N, a.H))
+        return cudaErrorInvalidValue;
+    cudaError_t e = cudaMemsetAsync(ws, 0, WS_HEAD, stream);
     if (e != cudaSuccess) return e;
-    e = cudaFuncSetAttribute(ew_chunk_output, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_OUT);
+    e = cudaFuncSetAttribute(ew_range_state, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(StateSmem));
     if (e != cudaSuccess) return e;
-    const dim3 grid((unsigned)a.nch, (unsigned)a.H, (unsigned)a.B);
-    ew_chunk_state<<<grid, NT, SMEM_STATE, stream>>>(a);
-    ew_state_scan<<<(unsigned)((int64_t)a.B * a.H * 16), 256, 0, stream>>>(a);
-    ew_chunk_output<<<grid, NT, SMEM_OUT, stream>>>(a);
+    e = cudaFuncSetAttribute(ew_range_output, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sizeof(OutSmem));
+    if (e != cudaSuccess) return e;
+    const dim3 grid((unsigned)R, (unsigned)a.H, (unsigned)a.B);
+    ew_range_state<<<grid, NT, sizeof(StateSmem), stream>>>(tk, tv, tg, p);
+    ew_state_scan<<<(unsigned)((int64_t)a.B * a.H * 16), 256, 0, stream>>>(p, a.state_in,
+                                                                           a.state_out);
+    ew_range_output<<<grid, NT, sizeof(OutSmem), stream>>>(tq, tk, tv, tg, to, p);
     return cudaGetLastError();
 }
 

@@ -8,7 +8,7 @@
 
 namespace gret {
 
-constexpr int EW_CHUNK = 64;   // tokens per chunk
+constexpr int EW_CHUNK = 128;  // tokens per chunk (one M = 128 tensor-core tile)
 constexpr int EW_DIM = 128;    // d_k = d_v
 
 struct EwArgs {
@@ -20,14 +20,16 @@ struct EwArgs {
     int B;
     int64_t N;
     int H;
-    int nch;                   // chunks per sequence, ceil(N / EW_CHUNK)
     const float* state_in;     // [B, H, 128, 128] or nullptr (zero)
     float* state_out;          // [B, H, 128, 128] or nullptr
     __nv_bfloat16* o;          // [B, N, H, 128]
-    float* ws_S;               // [B, H, nch, 128, 128]: chunk states, then entry states
-    float* ws_a;               // [B, H, nch, 128]: chunk decays
+    void* workspace;           // ew_workspace_bytes(B, N, H) bytes, 16-byte aligned
 };
 
+// Chunks per range (the unit of one CTA of the range kernels) for this shape on the current
+// device, and the number of ranges per sequence.
+int ew_range_chunks(int B, int64_t N, int H);
+int64_t ew_ranges(int B, int64_t N, int H);
 size_t ew_workspace_bytes(int B, int64_t N, int H);
 cudaError_t launch_prefill_ew(const EwArgs& a, cudaStream_t stream);
 

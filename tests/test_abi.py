@@ -114,8 +114,14 @@ def test_projection_rejects_bad_arguments_without_launching():
 def test_elementwise_prefill_rejects_bad_arguments_without_launching():
     import gated_retention_linear_b200 as G
     lib = G._lib
-    assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 128) == (128 * 128 + 128) * 4
-    assert G.gret_prefill_elementwise_workspace_size(1, 65, 2, 128) == 2 * 2 * (128 * 128 + 128) * 4
+    # a 256-byte status head, then per (batch, head, range of chunks) one fp32 state slot and
+    # one decay row; one 128-token chunk per range while the ranges fill one wave of 148 SMs
+    slot = (128 * 128 + 128) * 4
+    assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 128) == 256 + slot
+    assert G.gret_prefill_elementwise_workspace_size(1, 129, 2, 128) == 256 + 2 * 2 * slot
+    assert G.gret_prefill_elementwise_workspace_size(1, 1000, 4, 128) == 256 + 4 * 8 * slot
+    # 256 chunks x 24 heads: ranges of 43 chunks, 6 per head (144 CTAs, one wave)
+    assert G.gret_prefill_elementwise_workspace_size(1, 32768, 24, 128) == 256 + 24 * 6 * slot
     assert G.gret_prefill_elementwise_workspace_size(1, 64, 1, 64) == 0
     assert G.gret_prefill_elementwise_workspace_size(65535, 1 << 40, 65535, 128) == 0
 
@@ -136,7 +142,7 @@ def test_elementwise_prefill_rejects_bad_arguments_without_launching():
     assert call(wsb=1000) == 4                # workspace smaller than the size query says
     assert call(ws=None) == 4
     assert call(B=65535, H=65535) == 2       # the scan's grid would not fit
-    assert call(B=4, H=65535, N=64 << 30) == 2    # workspace bytes past 9e18
+    assert call(B=4, H=65535, N=64 << 30) == 2    # token coordinates past 32 bits
 
 
 def test_swa_rejects_bad_arguments_without_launching():
