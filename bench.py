@@ -543,6 +543,8 @@ def run_elementwise(args, rank, world, stream, headwise_ms):
     import synth_inputs as SI
     c = SI.ELEMENTWISE_32K
     Bq, Nq, Hq = c["B"], c["N"], c["H"]
+    if args.elementwise_tokens:
+        Nq = args.elementwise_tokens
     inp = SI.gret_inputs(Bq, Nq, Hq, D, dtype=torch.bfloat16, seed=rank_seed(c["seed"], rank),
                          device="cuda")
     q, k, v = inp["q"], inp["k"], inp["v"]
@@ -586,7 +588,7 @@ def run_elementwise(args, rank, world, stream, headwise_ms):
             "roofline": {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s",
                          "frac": ach / peak, "peak_kind": kind,
                          "traffic": traffic_from_profile("prefill_ew.cu",
-                                                         "ew_kernels_32k.txt"),
+                                                         "ew_kernels_32k.txt", Nq),
                          "kernel": "ew_range_state + ew_state_scan + ew_range_output",
                          "algorithmic_bytes_per_launch": alg}}
 
@@ -833,6 +835,9 @@ def main():
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--no-elementwise", action="store_true")
     ap.add_argument("--no-swa", action="store_true")
+    ap.add_argument("--elementwise-tokens", type=int, default=None,
+                    help="tokens of the per-channel-gate leg (default: the 32768 of its "
+                         "workload; smaller values are for profiling captures)")
     ap.add_argument("--chunk-sweep", action="store_true",
                     help="also time the 3B-shaped prefill at every chunk size the library takes "
                          "(16, 32, 64 on CUDA cores, 128 on the tensor cores)")

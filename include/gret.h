@@ -235,12 +235,15 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
  *               state_out may alias state_in.
  *   workspace   device memory of at least gret_prefill_elementwise_workspace_size(B, N, H, d)
  *               bytes, 16-byte aligned, owned by the caller; its contents on entry do not
- *               matter and are overwritten.
- * Runs on CUDA cores in fp32 (three launches: chunk states, a scan over chunks, chunk
- * outputs).  Requires d == 128, B <= 65535, H <= 65535, B * H * 16 < 2^31 and a workspace size
- * below 9e18 bytes (GRET_ERR_UNSUPPORTED otherwise); q, k, v, g, o and the states 16-byte
- * aligned (GRET_ERR_ALIGNMENT otherwise).  N == 0 copies state_in (or zeros) to state_out.
- * o must not overlap the inputs.
+ *               matter and are overwritten.  Its first word is the status word that
+ *               gret_workspace_status reads (GRET_ERR_TIMEOUT if a bounded wait gave up).
+ * Runs on the tensor cores (three launches: per range of chunks the decayed sum of k^T v, a
+ * scan over ranges, the outputs range by range) with each channel's decay folded into bf16
+ * high/low operand pairs; chunks whose decay is too fast for that take their in-chunk scores
+ * pairwise on CUDA cores.  Requires d == 128, B <= 65535, H <= 65535, N <= 2^31 - 256,
+ * B * H * 16 < 2^31 and a workspace size below 9e18 bytes (GRET_ERR_UNSUPPORTED otherwise);
+ * q, k, v, g, o and the states 16-byte aligned (GRET_ERR_ALIGNMENT otherwise).  N == 0 copies
+ * state_in (or zeros) to state_out.  o must not overlap the inputs.
  */
 gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void* v,
                                        const float* g, float tau, float k_scale, int B,
@@ -248,8 +251,10 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
                                        float* state_out, void* o, void* workspace,
                                        size_t workspace_bytes, gret_stream_t stream);
 
-/* Workspace bytes gret_prefill_elementwise needs: B * H * ceil(N / 64) * (d*d + d) * 4.
- * Returns 0 on invalid or unsupported sizes (d != 128 among them). */
+/* Workspace bytes gret_prefill_elementwise needs: 256 + B * H * R * (d*d + d) * 4, with R the
+ * ranges of chunks per sequence that the launch uses on the current device (a wave model over
+ * its SM count: R = 6 at N = 32768, H = 24 on 148 SMs).  Query it on the device that runs the
+ * call.  Returns 0 on invalid or unsupported sizes (d != 128 among them). */
 size_t gret_prefill_elementwise_workspace_size(int B, int64_t N, int H, int d);
 
 /*
