@@ -65,6 +65,7 @@ constexpr uint32_t TM_A = 0, TM_O = 128, TM_S = 256;   // scores / P, output, st
 constexpr size_t WS_HEAD = 256;          // status word, then the range slots
 
 struct EwParams {
+    const float* g;        // [B][N][H][D] gate logits (read directly by the range aggregates)
     float inv_tau_log2e;   // log2(e) / tau
     float k_scale;
     int64_t N;
@@ -83,17 +84,16 @@ struct __align__(1024) OutSmem {
     unsigned char y[TILE];   // low half of K~  (x and y: fp32 P of a pairwise chunk)
     float g[C * D];          // gate logits -> cumulative log2-decay -> state operand hi | lo
     float tot[2][D];         // per channel: log2-decay of tokens [0, 64) and [64, 128)
-    uint64_t ld_full, mma_done, drain;
+    uint64_t k_full, r_full, mma_done, drain;   // k tile; q, v, g tiles; MMA groups; exit
     uint32_t tmem_base;
 };
 
 struct __align__(1024) StateSmem {
-    unsigned char k[TILE];   // k, then the high half of the weighted keys (in place)
-    unsigned char v[TILE];
-    unsigned char y[TILE];   // low half of the weighted keys
-    float g[C * D];          // gate logits -> per-token log2-decay
+    unsigned char k[2][TILE];   // k (two stages), then the high half of the weighted keys in place
+    unsigned char v[2][TILE];
+    unsigned char y[TILE];      // low half of the weighted keys
     float tot[2][D];
-    uint64_t ld_full, mma_done, drain;
+    uint64_t kv_full[2], mma_done, drain;
     uint32_t tmem_base;
 };
 
@@ -113,6 +113,19 @@ __device__ __forceinline__ float ex2f(float x) {
 __device__ __forceinline__ float logsigmoid_fast(float x) {
     return fminf(x, 0.f) - __logf(1.f + __expf(-fabsf(x)));
 }
+
+// Element (t, col) of a swizzled bf16 tile for rows t = t8 + u, t8 a multiple of 8: the
+// column's slab and byte position are fixed per thread, the 16-byte chunk index is
+// (col % 64) / 8 xor u.
+struct ColOffset {
+    uint32_t base, chunk;
+    __device__ __forceinline__ explicit ColOffset(int col)
+        : base((uint32_t)(col >> 6) * SLAB + (uint32_t)(col & 7) * 2u),
+          chunk((uint32_t)(col & 63) >> 3) {}
+    __device__ __forceinline__ uint32_t at(int t8, int u) const {
+        return base + (uint32_t)(t8 + u) * 128u + ((chunk ^ (uint32_t)u) << 4);
+    }
+};
 
 __device__ __forceinline__ float bf16_at(const unsigned char* tile, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
@@ -143,19 +156,21 @@ __device__ __forceinline__ bool block_wait(uint64_t* bar, uint32_t parity, uint3
 }
 
 // D (+)= A B over K = 128: eight K-steps of 16, bf16 operands in shared memory (64-column slabs,
-// 128-byte swizzle).  a_mn / b_mn: the operand is stored MN-major (M or N contiguous).
+// 128-byte swizzle).  a_mn / b_mn: the operand is stored MN-major (M or N contiguous).  The steps
+// are unrolled with each step's descriptors formed just before its MMA (the empty asm keeps the
+// compiler from computing all of them up front), so that one thread issues them back to back.
 __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, uint32_t b_base,
                                         bool b_mn, bool accumulate) {
     const uint32_t idesc = idesc_bf16(128, 128, a_mn, b_mn);
-#pragma unroll 1
+    const uint64_t ad = sdesc_sw128(a_base, a_mn ? SLAB : 16, 1024);
+    const uint64_t bd = sdesc_sw128(b_base, b_mn ? SLAB : 16, 1024);
+#pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         const uint32_t aoff = a_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
         const uint32_t boff = b_mn ? kk * 2048u : (kk >> 2) * SLAB + (kk & 3) * 32u;
-        const uint64_t ad = a_mn ? sdesc_sw128(a_base + aoff, SLAB, 1024)
-                                 : sdesc_sw128(a_base + aoff, 16, 1024);
-        const uint64_t bd = b_mn ? sdesc_sw128(b_base + boff, SLAB, 1024)
-                                 : sdesc_sw128(b_base + boff, 16, 1024);
-        mma_ss(d, ad, bd, idesc, (accumulate || kk > 0) ? 1u : 0u);
+        uint64_t a = ad + (aoff >> 4), bb = bd + (boff >> 4);
+        asm volatile("" : "+l"(a), "+l"(bb));
+        mma_ss(d, a, bb, idesc, (accumulate || kk > 0) ? 1u : 0u);
     }
 }
 
@@ -165,25 +180,35 @@ __device__ __forceinline__ void mma_128(uint32_t d, uint32_t a_base, bool a_mn, 
 __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, uint32_t v_base,
                                        bool accumulate) {
     const uint32_t idesc = idesc_bf16(128, 128, 0, 1);
-#pragma unroll 1
-    for (int kk = 0; kk < 8; ++kk)
-        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half,
-               sdesc_sw128(v_base + kk * 2048u, SLAB, 1024), idesc,
+    const uint64_t vd = sdesc_sw128(v_base, SLAB, 1024);
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk) {
+        uint64_t bb = vd + ((kk * 2048u) >> 4);
+        asm volatile("" : "+l"(bb));
+        mma_ts(d, p_base + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half, bb, idesc,
                (accumulate || kk > 0) ? 1u : 0u);
+    }
 }
 
-// Loads of one chunk: bf16 tiles as two 64-column slabs each, the gate logits as one fp32 box.
-// Coordinates of every map: (column, head, token, batch); rows past the sequence read as zero.
-__device__ __forceinline__ void load_tiles(unsigned char* q, unsigned char* k, unsigned char* v,
-                                           float* g, const CUtensorMap* tq, const CUtensorMap* tk,
-                                           const CUtensorMap* tv, const CUtensorMap* tg,
-                                           uint64_t* bar, int tok, int h, int b) {
-    const uint32_t bytes = (q ? TILE : 0) + 2 * TILE + GTILE;
-    mbar_arrive_expect_tx(bar, bytes);
+// Loads of one chunk, coordinates (column, head, token, batch) in every map, rows past the
+// sequence read as zero: the k tile (two 64-column swizzled slabs), and the q and v tiles with
+// the gate logits (one unswizzled fp32 box of 128 columns).
+__device__ __forceinline__ void load_k_tile(unsigned char* k, const CUtensorMap* tk, uint64_t* bar,
+                                            int tok, int h, int b) {
+    mbar_arrive_expect_tx(bar, TILE);
+#pragma unroll
+    for (int half = 0; half < 2; ++half)
+        tma_load_4d(k + half * SLAB, tk, bar, half * 64, h, tok, b);
+}
+
+__device__ __forceinline__ void load_qvg_tiles(unsigned char* q, unsigned char* v, float* g,
+                                               const CUtensorMap* tq, const CUtensorMap* tv,
+                                               const CUtensorMap* tg, uint64_t* bar, int tok,
+                                               int h, int b) {
+    mbar_arrive_expect_tx(bar, 2 * TILE + GTILE);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
-        if (q) tma_load_4d(q + half * SLAB, tq, bar, half * 64, h, tok, b);
-        tma_load_4d(k + half * SLAB, tk, bar, half * 64, h, tok, b);
+        tma_load_4d(q + half * SLAB, tq, bar, half * 64, h, tok, b);
         tma_load_4d(v + half * SLAB, tv, bar, half * 64, h, tok, b);
     }
     tma_load_4d(g, tg, bar, 0, h, tok, b);
@@ -192,11 +217,31 @@ __device__ __forceinline__ void load_tiles(unsigned char* q, unsigned char* k, u
 // ----------------------------------------------------------------------------------------------
 // 1. Range aggregates.  Block (range, head, batch).  The range's chunks are visited last to
 // first so that each key's weight, its log2-decay to the end of the range, is a running suffix
-// sum; every K~^T V MMA of the range accumulates into one tensor-memory result.
+// sum; every K~^T V MMA of the range accumulates into one tensor-memory result.  k and v tiles
+// come by TMA through a two-stage ring, the next chunk's issued as soon as its stage is free;
+// thread (i, hh) reads the gate logits of channel i for its token half straight into registers,
+// one chunk ahead.
+
+__device__ __forceinline__ void load_kv(StateSmem& sm, int st, const CUtensorMap* tk,
+                                        const CUtensorMap* tv, int tok, int h, int b) {
+    mbar_arrive_expect_tx(&sm.kv_full[st], 2 * TILE);
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+        tma_load_4d(sm.k[st] + half * SLAB, tk, &sm.kv_full[st], half * 64, h, tok, b);
+        tma_load_4d(sm.v[st] + half * SLAB, tv, &sm.kv_full[st], half * 64, h, tok, b);
+    }
+}
+
+// Gate logits of tokens [t0, t0 + 64) of one (batch, head) row at channel i (0 past the end).
+__device__ __forceinline__ void load_gate64(const float* grow, int64_t gstride, int64_t t0,
+                                            int64_t N, float (&x)[64]) {
+#pragma unroll
+    for (int u = 0; u < 64; ++u) x[u] = t0 + u < N ? __ldg(grow + (t0 + u) * gstride) : 0.f;
+}
 
 __global__ void __launch_bounds__(NT, 1)
     ew_range_state(const __grid_constant__ CUtensorMap tk, const __grid_constant__ CUtensorMap tv,
-                   const __grid_constant__ CUtensorMap tg, const EwParams p) {
+                   const EwParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     StateSmem& sm = *reinterpret_cast<StateSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5;
@@ -208,8 +253,10 @@ __global__ void __launch_bounds__(NT, 1)
     const int64_t nch = (p.N + C - 1) / C;
     const int c0 = r * p.G;
     const int c1 = (int)min64(nch, (int64_t)c0 + p.G);
+    const int n_ch = c1 - c0;
     if (tid == 0) {
-        mbar_init(&sm.ld_full, 1);
+        mbar_init(&sm.kv_full[0], 1);
+        mbar_init(&sm.kv_full[1], 1);
         mbar_init(&sm.mma_done, 1);
         mbar_init(&sm.drain, 1);
         fence_mbar_init();
@@ -222,40 +269,62 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int i = tid & 127, hh = tid >> 7;           // channel, token half (also TMEM lane, column half)
+    const int i = tid & 127, hh = tid >> 7;   // channel (TMEM lane), token half (column half)
     const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
+    const float* grow = p.g + ((int64_t)b * p.N * p.H + h) * D + i;
+    const int64_t gstride = (int64_t)p.H * D;
+    const ColOffset co(i);
 
-    if (tid == 0) load_tiles(nullptr, sm.k, sm.v, sm.g, nullptr, &tk, &tv, &tg, &sm.ld_full,
-                             (c1 - 1) * C, h, b);
+    if (tid == 0) load_kv(sm, 0, &tk, &tv, (c1 - 1) * C, h, b);
+    float gcur[64], gnext[64];
+    load_gate64(grow, gstride, (int64_t)(c1 - 1) * C + 64 * hh, p.N, gcur);
     float R = 0.f;   // log2-decay of the tokens after the current chunk, to the range end
-    uint32_t n_ld = 1, n_mma = 0;
+    int issued = 1, consumed = 0;
+    uint32_t n_mma = 0;
     bool ok = true;
-    for (int c = c1 - 1; c >= c0; --c) {
+#pragma unroll 1
+    for (int n = 0; n < n_ch; ++n) {
+        const int c = c1 - 1 - n, st = n & 1;
         const int L = (int)min64(C, p.N - (int64_t)c * C);
-        if (!(ok = block_wait(&sm.ld_full, (n_ld - 1) & 1, p.err))) break;
-        // per-token log2-decays of channel i over this thread's half, in place
+        // the previous chunk's MMAs are done: its stage and the low-half tile are free
+        if (n > 0 && !(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
+        if (n + 1 < n_ch) {
+            if (tid == 0) load_kv(sm, st ^ 1, &tk, &tv, (c - 1) * C, h, b);
+            ++issued;
+            load_gate64(grow, gstride, (int64_t)(c - 1) * C + 64 * hh, p.N, gnext);
+        }
+        // per-token log2-decays of channel i over this thread's half
         float sum = 0.f;
-#pragma unroll 8
-        for (int t = 64 * hh; t < 64 * hh + 64; ++t) {
-            float* gp = &sm.g[t * D + i];
-            const float lam = t < L ? logsigmoid_fast(*gp) * p.inv_tau_log2e : 0.f;
-            *gp = lam;
-            sum += lam;
+#pragma unroll
+        for (int u = 0; u < 64; ++u) {
+            gcur[u] = 64 * hh + u < L ? logsigmoid_fast(gcur[u]) * p.inv_tau_log2e : 0.f;
+            sum += gcur[u];
         }
         sm.tot[hh][i] = sum;
         __syncthreads();
         const float t0 = sm.tot[0][i], t1 = sm.tot[1][i];
-        // weights 2^(suffix) k_scale, suffix = log2-decay from after token t to the range end
+        if (!(ok = block_wait(&sm.kv_full[st], (n >> 1) & 1, p.err))) break;
+        ++consumed;
+        // weights 2^(suffix) k_scale, suffix = log2-decay from after token t to the range end,
+        // last token first, in batches of 8
         float s = R + (hh == 0 ? t1 : 0.f);
-#pragma unroll 4
-        for (int t = 64 * hh + 63; t >= 64 * hh; --t) {
-            const uint32_t off = sw128_offset(t, i, SLAB);
-            const float kw = bf16_at(sm.k, off) * ex2f(s) * p.k_scale;
-            __nv_bfloat16 hi, lo;
-            split1(kw, hi, lo);
-            *reinterpret_cast<__nv_bfloat16*>(sm.k + off) = hi;
-            *reinterpret_cast<__nv_bfloat16*>(sm.y + off) = lo;
-            s += sm.g[t * D + i];
+#pragma unroll
+        for (int ub = 56; ub >= 0; ub -= 8) {
+            float kv[8], sw[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) kv[u] = bf16_at(sm.k[st], co.at(64 * hh + ub, u));
+#pragma unroll
+            for (int u = 7; u >= 0; --u) {
+                sw[u] = s;
+                s += gcur[ub + u];
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                __nv_bfloat16 hi, lo;
+                split1(kv[u] * ex2f(sw[u]) * p.k_scale, hi, lo);
+                *reinterpret_cast<__nv_bfloat16*>(sm.k[st] + co.at(64 * hh + ub, u)) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(sm.y + co.at(64 * hh + ub, u)) = lo;
+            }
         }
         R += t0 + t1;
         fence_proxy_async_smem();
@@ -263,18 +332,15 @@ __global__ void __launch_bounds__(NT, 1)
         if (tid == 0) {
             tc_fence_after();
             // Agg (+)= K~_hi^T V + K~_lo^T V: A = K~^T (channels x tokens) stored token-major
-            mma_128(tmem, smem_u32(sm.k), true, smem_u32(sm.v), true, c != c1 - 1);
-            mma_128(tmem, smem_u32(sm.y), true, smem_u32(sm.v), true, true);
+            mma_128(tmem, smem_u32(sm.k[st]), true, smem_u32(sm.v[st]), true, n > 0);
+            mma_128(tmem, smem_u32(sm.y), true, smem_u32(sm.v[st]), true, true);
             mma_commit(&sm.mma_done);
         }
         ++n_mma;
-        if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
-        if (c > c0 && tid == 0) {
-            load_tiles(nullptr, sm.k, sm.v, sm.g, nullptr, &tk, &tv, &tg, &sm.ld_full,
-                       (c - 1) * C, h, b);
-        }
-        if (c > c0) ++n_ld;
+#pragma unroll
+        for (int u = 0; u < 64; ++u) gcur[u] = gnext[u];
     }
+    if (ok) ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err);
     if (ok) {
         tc_fence_after();
         const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
@@ -291,11 +357,12 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (hh == 0) p.ws_a[slot * D + i] = ex2f(R);
     } else if (tid == 0) {
-        // a wait gave up: let the issued MMAs and any load in flight finish before exit
+        // a wait gave up: let the issued MMAs and the loads in flight finish before exit
         mma_commit(&sm.drain);
         uint32_t never = 0;
         mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
-        mbar_wait(&sm.ld_full, (n_ld - 1) & 1, &never, DRAIN_NS);
+        for (int j = consumed; j < issued; ++j)
+            mbar_wait(&sm.kv_full[j & 1], (j >> 1) & 1, &never, DRAIN_NS);
     }
     tc_fence_before();
     __syncthreads();
@@ -403,7 +470,8 @@ __global__ void __launch_bounds__(NT, 1)
     const int c0 = r * p.G;
     const int c1 = (int)min64(nch, (int64_t)c0 + p.G);
     if (tid == 0) {
-        mbar_init(&sm.ld_full, 1);
+        mbar_init(&sm.k_full, 1);
+        mbar_init(&sm.r_full, 1);
         mbar_init(&sm.mma_done, 1);
         mbar_init(&sm.drain, 1);
         fence_mbar_init();
@@ -424,7 +492,10 @@ __global__ void __launch_bounds__(NT, 1)
                    xb = smem_u32(sm.x), yb = smem_u32(sm.y), shb = smem_u32(sm.g),
                    slb = shb + TILE;
 
-    if (tid == 0) load_tiles(sm.q, sm.k, sm.v, sm.g, &tq, &tk, &tv, &tg, &sm.ld_full, c0 * C, h, b);
+    if (tid == 0) {
+        load_k_tile(sm.k, &tk, &sm.k_full, c0 * C, h, b);
+        load_qvg_tiles(sm.q, sm.v, sm.g, &tq, &tv, &tg, &sm.r_full, c0 * C, h, b);
+    }
     // entry state of the range: row i, columns [64 hh, 64 hh + 64)
     const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
     float S[64];
@@ -437,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1)
             S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
         }
     }
-    uint32_t n_ld = 1, n_mma = 0;
+    uint32_t n_ld = 1, n_k = 1, n_mma = 0;   // q/v/g and k loads issued, MMA groups committed
     bool ok = true;
     for (int c = c0; c < c1; ++c) {
         const int L = (int)min64(C, p.N - (int64_t)c * C);
@@ -446,14 +517,24 @@ __global__ void __launch_bounds__(NT, 1)
             if (tid == 0) bulk_wait_group_read0();
             __syncthreads();
         }
-        if (!(ok = block_wait(&sm.ld_full, (n_ld - 1) & 1, p.err))) break;
-        // cumulative log2-decay of channel i over this thread's token half, in place
+        if (!(ok = block_wait(&sm.r_full, (n_ld - 1) & 1, p.err))) break;
+        if (!(ok = block_wait(&sm.k_full, (n_k - 1) & 1, p.err))) break;
+        // cumulative log2-decay of channel i over this thread's token half, in place (batches
+        // of 16 tokens)
         float cum = 0.f;
-#pragma unroll 8
-        for (int t = 64 * hh; t < 64 * hh + 64; ++t) {
-            float* gp = &sm.g[t * D + i];
-            cum += t < L ? logsigmoid_fast(*gp) * p.inv_tau_log2e : 0.f;
-            *gp = cum;
+#pragma unroll 1
+        for (int tb = 64 * hh; tb < 64 * hh + 64; tb += 16) {
+            float x[16];
+#pragma unroll
+            for (int u = 0; u < 16; ++u) x[u] = sm.g[(tb + u) * D + i];
+#pragma unroll
+            for (int u = 0; u < 16; ++u)
+                x[u] = tb + u < L ? logsigmoid_fast(x[u]) * p.inv_tau_log2e : 0.f;
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                cum += x[u];
+                sm.g[(tb + u) * D + i] = cum;
+            }
         }
         sm.tot[hh][i] = cum;
         __syncthreads();
@@ -472,19 +553,27 @@ __global__ void __launch_bounds__(NT, 1)
         {
             const float off = (hh == 1 && !pairwise) ? t0 : 0.f;
             const float qshift = pairwise ? 0.f : -cL;
-#pragma unroll 4
-            for (int t = 64 * hh; t < 64 * hh + 64; ++t) {
-                const float ct = sm.g[t * D + i] + off;
-                const uint32_t o = sw128_offset(t, i, SLAB);
-                const float qs = bf16_at(sm.q, o) * ex2f(ct + qshift);
-                const float ks = bf16_at(sm.k, o) * ex2f(cL - ct) * p.k_scale;
-                __nv_bfloat16 qh, ql, kh, kl;
-                split1(qs, qh, ql);
-                split1(ks, kh, kl);
-                *reinterpret_cast<__nv_bfloat16*>(sm.q + o) = qh;
-                *reinterpret_cast<__nv_bfloat16*>(sm.x + o) = ql;
-                *reinterpret_cast<__nv_bfloat16*>(sm.k + o) = kh;
-                *reinterpret_cast<__nv_bfloat16*>(sm.y + o) = kl;
+            const ColOffset co(i);
+#pragma unroll 1
+            for (int tb = 64 * hh; tb < 64 * hh + 64; tb += 8) {
+                float ct[8], qv[8], kv[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    ct[u] = sm.g[(tb + u) * D + i] + off;
+                    qv[u] = bf16_at(sm.q, co.at(tb, u));
+                    kv[u] = bf16_at(sm.k, co.at(tb, u));
+                }
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    __nv_bfloat16 qh, ql, kh, kl;
+                    split1(qv[u] * ex2f(ct[u] + qshift), qh, ql);
+                    split1(kv[u] * ex2f(cL - ct[u]) * p.k_scale, kh, kl);
+                    const uint32_t o = co.at(tb, u);
+                    *reinterpret_cast<__nv_bfloat16*>(sm.q + o) = qh;
+                    *reinterpret_cast<__nv_bfloat16*>(sm.x + o) = ql;
+                    *reinterpret_cast<__nv_bfloat16*>(sm.k + o) = kh;
+                    *reinterpret_cast<__nv_bfloat16*>(sm.y + o) = kl;
+                }
             }
         }
         __syncthreads();   // every read of the log2-decays is done: sm.g takes the state operand
@@ -506,17 +595,31 @@ __global__ void __launch_bounds__(NT, 1)
         }
         fence_proxy_async_smem();
         __syncthreads();
-        if (!pairwise) {
+        // first MMA group: the scores (factored chunks) and the state update dS = K~^T V (all
+        // chunks but the range's last); after it the k and y tiles are free
+        if (!pairwise || !last) {
             if (tid == 0) {
                 tc_fence_after();
-                mma_128(tmem + TM_A, qb, false, kb, false, false);   // Q_hi K~_hi^T
-                mma_128(tmem + TM_A, xb, false, kb, false, true);    //  + Q_lo K~_hi^T
-                mma_128(tmem + TM_A, qb, false, yb, false, true);    //  + Q_hi K~_lo^T
+                if (!pairwise) {
+                    mma_128(tmem + TM_A, qb, false, kb, false, false);   // Q_hi K~_hi^T
+                    mma_128(tmem + TM_A, xb, false, kb, false, true);    //  + Q_lo K~_hi^T
+                    mma_128(tmem + TM_A, qb, false, yb, false, true);    //  + Q_hi K~_lo^T
+                }
+                if (!last) {
+                    mma_128(tmem + TM_S, kb, true, vb, true, false);     // dS = K~_hi^T V
+                    mma_128(tmem + TM_S, yb, true, vb, true, true);      //    + K~_lo^T V
+                }
                 mma_commit(&sm.mma_done);
             }
             ++n_mma;
             if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
             tc_fence_after();
+        }
+        if (!last) {
+            if (tid == 0) load_k_tile(sm.k, &tk, &sm.k_full, (c + 1) * C, h, b);
+            ++n_k;
+        }
+        if (!pairwise) {
             // causal mask, P split into bf16 halves in place: row = lane, 64 columns per thread
             const int row = (warp & 3) * 32 + lane;
 #pragma unroll 1
@@ -537,6 +640,7 @@ __global__ void __launch_bounds__(NT, 1)
             tc_fence_before();
             __syncthreads();
         }
+        // second group: the output O = Q S' + P V
         if (tid == 0) {
             tc_fence_after();
             mma_128(tmem + TM_O, qb, false, shb, true, false);   // O = Q_hi S_hi
@@ -544,18 +648,14 @@ __global__ void __launch_bounds__(NT, 1)
             mma_128(tmem + TM_O, qb, false, slb, true, true);    //   + Q_hi S_lo
             mma_pv(tmem + TM_O, tmem + TM_A, 0, vb, true);       //   + P_hi V
             mma_pv(tmem + TM_O, tmem + TM_A, 1, vb, true);       //   + P_lo V
-            if (!last) {
-                mma_128(tmem + TM_S, kb, true, vb, true, false); // dS = K~_hi^T V
-                mma_128(tmem + TM_S, yb, true, vb, true, true);  //    + K~_lo^T V
-            }
             mma_commit(&sm.mma_done);
         }
         ++n_mma;
         if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
         tc_fence_after();
-        if (!last) {   // every tile but x is free: the next chunk's loads go now
+        if (!last) {   // every tile but x is free: the rest of the next chunk's loads go now
             if (tid == 0)
-                load_tiles(sm.q, sm.k, sm.v, sm.g, &tq, &tk, &tv, &tg, &sm.ld_full, (c + 1) * C, h, b);
+                load_qvg_tiles(sm.q, sm.v, sm.g, &tq, &tv, &tg, &sm.r_full, (c + 1) * C, h, b);
             ++n_ld;
         }
         // output rows: a chunk inside the sequence goes out as one tile through x (rows in the
@@ -611,7 +711,8 @@ __global__ void __launch_bounds__(NT, 1)
             mma_commit(&sm.drain);
             uint32_t never = 0;
             mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
-            mbar_wait(&sm.ld_full, (n_ld - 1) & 1, &never, DRAIN_NS);
+            mbar_wait(&sm.k_full, (n_k - 1) & 1, &never, DRAIN_NS);
+            mbar_wait(&sm.r_full, (n_ld - 1) & 1, &never, DRAIN_NS);
         }
         bulk_wait_group0();
     }
@@ -697,6 +798,7 @@ cudaError_t launch_prefill_ew(const EwArgs& a, cudaStream_t stream) {
     const int64_t R = ew_ranges(a.B, a.N, a.H);
     unsigned char* ws = static_cast<unsigned char*>(a.workspace);
     EwParams p;
+    p.g = a.g;
     p.inv_tau_log2e = 1.4426950408889634f / a.tau;
     p.k_scale = a.k_scale;
     p.N = a.N;
@@ -721,7 +823,7 @@ cudaError_t launch_prefill_ew(const EwArgs& a, cudaStream_t stream) {
                              (int)sizeof(OutSmem));
     if (e != cudaSuccess) return e;
     const dim3 grid((unsigned)R, (unsigned)a.H, (unsigned)a.B);
-    ew_range_state<<<grid, NT, sizeof(StateSmem), stream>>>(tk, tv, tg, p);
+    ew_range_state<<<grid, NT, sizeof(StateSmem), stream>>>(tk, tv, p);
     ew_state_scan<<<(unsigned)((int64_t)a.B * a.H * 16), 256, 0, stream>>>(p, a.state_in,
                                                                            a.state_out);
     ew_range_output<<<grid, NT, sizeof(OutSmem), stream>>>(tq, tk, tv, tg, to, p);
