@@ -8,21 +8,29 @@
 //     n_j = (o_j - mean) / sqrt(var + eps) * gn_w + gn_b     (o = O_t[h*d_v .. h*d_v + d_v))
 //     y_j = n_j * z_j * sigmoid(z_j)
 //
-// The GEMM dominates (2 D H d_v FLOP per token): a persistent tcgen05 kernel, one CTA per SM,
-// output tiles of 128 tokens x 256 columns (two heads), K in blocks of 64 through a 4-stage
-// TMA ring, fp32 accumulators in TMEM, two accumulator buffers so the epilogue of one tile runs
-// under the MMAs of the next.  The epilogue is fused: GroupNorm statistics of the O row, swish
-// of the accumulator, the product, bf16 out; z never goes to memory.
+// The GEMM dominates (2 D H d_v FLOP per token): a persistent tcgen05 kernel run by pairs of
+// CTAs (clusters of two, one CTA per SM).  A pair computes output tiles of 256 tokens x 256
+// columns (two heads) with cta_group::2 MMAs: each CTA loads its 128 rows of X and its 128
+// columns of W per K block of 64 through a 6-stage TMA ring into its own shared memory, the even
+// CTA issues the MMAs for both, and each CTA's tensor memory receives its 128 rows x 256
+// columns in fp32.  Against single-CTA 128 x 256 tiles this cuts the operand bytes each SM
+// pulls from L2 per MMA by a third (32 KB instead of 48 KB per K block), the bound of that
+// version.  Two accumulator buffers let the epilogue of one tile run under the MMAs of the
+// next.  The epilogue is fused: GroupNorm statistics of the O row, swish of the accumulator,
+// the product, bf16 out; z never goes to memory.
 //
 // The same GEMM, with a plain epilogue, is the layer's input projection: X W_qkvg with
 // W_qkvg = [W_Q | W_K | W_V | W_gamma] gives q, k, v (bf16, [T, H, d] each) and the gate logits
 // g (fp32, [T, H]) in one pass over X (qkvg_projection below).
 //
-// Warp roles (384 threads): warp 0 TMA producer, warp 1 MMA issuer (owns TMEM), warps 2-3 idle,
-// warps 4-7 epilogue for the first head of a tile, warps 8-11 for the second.  Tiles are
-// assigned round-robin (tile = blockIdx.x + i * gridDim.x), M-block major, so the CTAs working
-// at one time share a few X row-blocks and all of W_G (9.4 MB at D = 3072) through L2.
-// Every wait is bounded; a wait that gives up makes every role exit.
+// Warp roles (384 threads per CTA): warp 0 TMA producer (both CTAs; the odd CTA's loads count
+// on the even CTA's stage barrier), warp 1 MMA issuer (even CTA; warp 1 of both CTAs allocates
+// the pair's TMEM), warps 2-3 idle, warps 4-7 epilogue for the first head of the CTA's rows of a
+// tile, warps 8-11 for the second; the epilogue threads of both CTAs release an accumulator
+// buffer on the even CTA's barrier.  Tiles are assigned round-robin over pairs, in the grouped
+// order of tile_coords, so the pairs working at one time share a few X row-blocks and column
+// blocks of W through L2.  Every wait is bounded; a wait that gives up makes every role exit,
+// and the two CTAs leave together (cluster barrier) once the even CTA's MMAs have drained.
 #include "gn_gate.cuh"
 
 #include "sm100.cuh"
@@ -34,9 +42,11 @@ using namespace sm100;
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 64, STAGES = 4;
+constexpr int BM = 128;                         // rows per CTA; a pair's tile has 2 BM
+constexpr int BN = 256, BK = 64, STAGES = 6;    // columns per tile; each CTA loads BN / 2 of W
+constexpr int PM = 2 * BM;                      // rows per pair tile
 constexpr int A_BYTES = BM * BK * 2;            // 16 KB
-constexpr int B_BYTES = BN * BK * 2;            // 32 KB
+constexpr int B_BYTES = (BN / 2) * BK * 2;      // 16 KB
 constexpr int NTHREADS = 384;
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
@@ -58,7 +68,7 @@ struct GParams {
     float eps;
     int64_t T;
     int F, D;          // F: output columns (GroupNorm gate: H * 128; projection: 3 H 128 + H)
-    int m_blocks, n_blocks, n_tiles;
+    int m_blocks, n_blocks, n_tiles;   // in pair tiles (PM rows x BN columns)
     int group_m;       // tile order: runs of group_m row blocks (1 = row-major)
     // projection outputs
     __nv_bfloat16* qkv[3];   // q, k, v: [T, H, 128] bf16
@@ -89,11 +99,16 @@ __device__ __forceinline__ void tile_coords(const GParams& p, int tile, int& mb,
 
 int group_rows(int n_blocks) { return n_blocks > 16 ? 16 : 1; }
 
-__device__ void producer(GSmem& sm, const GParams& p, const CUtensorMap* tx, const CUtensorMap* tw) {
+// Both CTAs: this CTA's rows of X (rows PM mb + BM rank) and its half of the column block of W
+// (columns BN nb + (BN / 2) rank), into its own stage; the bytes count on the even CTA's stage
+// barrier, which expects both CTAs' loads.  A stage is reused once the pair's MMAs on it are done
+// (the even CTA's commit arrives on the empty barrier of both CTAs).
+__device__ void producer(GSmem& sm, const GParams& p, const CUtensorMap* tx, const CUtensorMap* tw,
+                         uint32_t rank, int pair, int n_pairs) {
     const int kblocks = p.D / BK;
     int it = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x) {
+    for (int tile = pair; tile < p.n_tiles && ok; tile += n_pairs) {
         int mb, nb;
         tile_coords(p, tile, mb, nb);
         for (int kb = 0; kb < kblocks; ++kb, ++it) {
@@ -102,25 +117,30 @@ __device__ void producer(GSmem& sm, const GParams& p, const CUtensorMap* tx, con
                 ok = false;
                 break;
             }
-            mbar_arrive_expect_tx(&sm.full[s], A_BYTES + B_BYTES);
-            tma_load_2d(sm.a[s], tx, &sm.full[s], kb * BK, mb * BM);
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 2 * (A_BYTES + B_BYTES));
+            const uint32_t fb = mapa_shared(&sm.full[s], 0);
+            tma_load_2d_pair(sm.a[s], tx, fb, kb * BK, mb * PM + (int)rank * BM);
 #pragma unroll
-            for (int j = 0; j < BN / 64; ++j)
-                tma_load_2d(sm.b[s] + j * (BK * 128), tw, &sm.full[s], nb * BN + j * 64, kb * BK);
+            for (int j = 0; j < BN / 128; ++j)
+                tma_load_2d_pair(sm.b[s] + j * (BK * 128), tw, fb,
+                                 nb * BN + (int)rank * (BN / 2) + j * 64, kb * BK);
         }
     }
-    // no TMA write may be in flight when the CTA exits
+    // no TMA write into this CTA may be in flight when it exits: wait until the pair's MMAs have
+    // consumed the last stages (the stage's empty barrier)
     uint32_t never = 0;
     for (int jj = (it >= STAGES ? it - STAGES : 0); jj < it; ++jj)
-        mbar_wait(&sm.full[jj % STAGES], (jj / STAGES) & 1, &never, DRAIN_NS);
+        mbar_wait(&sm.empty[jj % STAGES], (jj / STAGES) & 1, &never, DRAIN_NS);
 }
 
-__device__ void mma_issuer(GSmem& sm, const GParams& p, uint32_t tmem) {
+// Even CTA, one thread: the pair's MMAs, M = 256 (128 rows from each CTA), N = 256 (128 columns
+// from each CTA's half of W), into accumulator buffer buf of both CTAs' tensor memory.
+__device__ void mma_issuer(GSmem& sm, const GParams& p, uint32_t tmem, int pair, int n_pairs) {
     const int kblocks = p.D / BK;
-    const uint32_t idesc = idesc_bf16(BM, BN, 0, 1);
+    const uint32_t idesc = idesc_bf16(PM, BN, 0, 1);
     int it = 0, t_local = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < p.n_tiles && ok; tile += gridDim.x, ++t_local) {
+    for (int tile = pair; tile < p.n_tiles && ok; tile += n_pairs, ++t_local) {
         const int buf = t_local & 1;
         if (t_local >= 2 && !wait_bar(sm, &sm.acc_empty[buf], ((t_local >> 1) - 1) & 1)) break;
         tc_fence_after();
@@ -132,16 +152,16 @@ __device__ void mma_issuer(GSmem& sm, const GParams& p, uint32_t tmem) {
             const uint32_t ab = smem_u32(sm.a[s]), bb = smem_u32(sm.b[s]);
 #pragma unroll
             for (int kk = 0; kk < BK / 16; ++kk)
-                mma_ss(d, sdesc_sw128(ab + kk * 32, 16, 1024),
-                       sdesc_sw128(bb + kk * 2048, BK * 128, 1024), idesc,
-                       (kb > 0 || kk > 0) ? 1u : 0u);
-            mma_commit(&sm.empty[s]);
+                mma_ss_pair(d, sdesc_sw128(ab + kk * 32, 16, 1024),
+                            sdesc_sw128(bb + kk * 2048, BK * 128, 1024), idesc,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
+            mma_commit_pair(&sm.empty[s], 0x3);
         }
         if (!ok) break;
-        mma_commit(&sm.acc_full[buf]);
+        mma_commit_pair(&sm.acc_full[buf], 0x3);
     }
     uint32_t never = 0;
-    mma_commit(&sm.drain);
+    mma_commit_pair(&sm.drain, 0x1);
     mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
 }
 
@@ -186,16 +206,20 @@ __device__ __forceinline__ void store_projection(const GParams& p, uint32_t tadd
 
 // One epilogue thread: token row r of the tile, one head (128 columns) of it.
 template <int MODE>
-__device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, int lane) {
+__device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, int lane,
+                         uint32_t rank, int pair, int n_pairs) {
     const int q = warp & 3, r = q * 32 + lane;
     const int half = (warp - 4) >> 2;                    // which head of the 256-column tile
     const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
+    // the even CTA's release barriers
+    const uint32_t acc_empty_even0 = mapa_shared(&sm.acc_empty[0], 0);
+    const uint32_t acc_empty_even1 = mapa_shared(&sm.acc_empty[1], 0);
     int t_local = 0;
-    for (int tile = blockIdx.x; tile < p.n_tiles; tile += gridDim.x, ++t_local) {
+    for (int tile = pair; tile < p.n_tiles; tile += n_pairs, ++t_local) {
         const int buf = t_local & 1;
         int mb, nb;
         tile_coords(p, tile, mb, nb);
-        const int64_t t = (int64_t)mb * BM + r;
+        const int64_t t = (int64_t)mb * PM + (int64_t)rank * BM + r;
         const int col0 = nb * BN + half * 128;
         const bool valid = t < p.T;
         if (MODE == EPI_PROJECTION) {
@@ -206,7 +230,7 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
             tc_fence_after();
             store_projection(p, tmem + lane_base + buf * BN + half * 128, t, col0, valid);
             tc_fence_before();
-            mbar_arrive(&sm.acc_empty[buf]);
+            mbar_arrive_cluster(buf ? acc_empty_even1 : acc_empty_even0);
             continue;
         }
         // GroupNorm statistics of this head's slice of O, computed while the MMAs run; the row
@@ -284,18 +308,22 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
             }
         }
         tc_fence_before();
-        mbar_arrive(&sm.acc_empty[buf]);
+        mbar_arrive_cluster(buf ? acc_empty_even1 : acc_empty_even0);
     }
 }
 
 template <int MODE>
-__global__ void __launch_bounds__(NTHREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(NTHREADS, 1)
     gn_gate_kernel(const __grid_constant__ CUtensorMap tx, const __grid_constant__ CUtensorMap tw,
                    const GParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     GSmem& sm = *reinterpret_cast<GSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    if ((smem_u32(smem_raw) & 1023u) != 0) return;   // the swizzled tiles need 1 KB alignment
+    const uint32_t rank = cluster_ctarank();
+    const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+    // the swizzled tiles need 1 KB alignment; both CTAs of a pair see the same layout, so they
+    // take this exit together, before any cluster-wide step
+    if ((smem_u32(smem_raw) & 1023u) != 0) return;
     if (tid == 0) {
         for (int s = 0; s < STAGES; ++s) {
             mbar_init(&sm.full[s], 1);
@@ -303,15 +331,16 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
-            mbar_init(&sm.acc_empty[b], 256);
+            mbar_init(&sm.acc_empty[b], 2 * 256);   // the epilogue threads of both CTAs
         }
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
     }
+    cluster_sync();   // every barrier of the pair is initialised before the other CTA uses it
     if (warp == 1) {
-        tmem_alloc(&sm.tmem_base, 512);
-        tmem_relinquish();
+        tmem_alloc_pair(&sm.tmem_base, 512);
+        tmem_relinquish_pair();
     }
     tc_fence_before();
     __syncthreads();
@@ -321,18 +350,21 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         if (lane == 0) {
             tma_prefetch_desc(&tx);
             tma_prefetch_desc(&tw);
-            producer(sm, p, &tx, &tw);
+            producer(sm, p, &tx, &tw, rank, pair, n_pairs);
         }
     } else if (warp == 1) {
-        if (lane == 0) mma_issuer(sm, p, tmem);
+        if (lane == 0 && rank == 0) mma_issuer(sm, p, tmem, pair, n_pairs);
     } else if (warp >= 4) {
-        epilogue<MODE>(sm, p, tmem, warp, lane);
+        epilogue<MODE>(sm, p, tmem, warp, lane, rank, pair, n_pairs);
     }
     tc_fence_before();
     __syncthreads();
+    // the even CTA's MMAs have drained (its issuer waited for them before the barrier above):
+    // neither CTA leaves while the pair's MMAs could still touch its memory
+    cluster_sync();
     if (warp == 1) {
         tc_fence_after();
-        tmem_dealloc(tmem, 512);
+        tmem_dealloc_pair(tmem, 512);
     }
 }
 
@@ -349,6 +381,33 @@ int sm_count() {
     return cached[dev];
 }
 
+// Pairs resident at once on this device (clusters of two need two SMs of one GPC).
+template <int MODE>
+int max_pairs(size_t smem) {
+    static int cached[64] = {0};
+    int dev = 0;
+    cudaGetDevice(&dev);
+    if (dev < 0 || dev >= 64) dev = 0;
+    if (!cached[dev]) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (unsigned)(sm_count() / 2), 1, 1);
+        cfg.blockDim = dim3(NTHREADS, 1, 1);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = 2;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaOccupancyMaxActiveClusters(&n, gn_gate_kernel<MODE>, &cfg) != cudaSuccess || n < 1)
+            n = sm_count() / 2;
+        cached[dev] = n;
+    }
+    return cached[dev];
+}
+
 template <int MODE>
 gret_status_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const GParams& p,
                           cudaStream_t stream) {
@@ -356,9 +415,10 @@ gret_status_t launch_gemm(const CUtensorMap& tx, const CUtensorMap& tw, const GP
     if (cudaFuncSetAttribute(gn_gate_kernel<MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem) != cudaSuccess)
         return GRET_ERR_CUDA;
-    int grid = sm_count();
-    if (p.n_tiles < grid) grid = p.n_tiles;
-    gn_gate_kernel<MODE><<<grid, NTHREADS, smem, stream>>>(tx, tw, p);
+    int pairs = max_pairs<MODE>(smem);
+    if (p.n_tiles < pairs) pairs = p.n_tiles;
+    if (pairs < 1) pairs = 1;
+    gn_gate_kernel<MODE><<<2 * pairs, NTHREADS, smem, stream>>>(tx, tw, p);
     return cudaGetLastError() == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
@@ -369,7 +429,7 @@ gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g, cons
                              void* y, cudaStream_t stream) {
     const int F = H * d_v;
     if (d_v != 128 || F % BN != 0 || D % BK != 0) return GRET_ERR_UNSUPPORTED;
-    if (T > ((int64_t)1 << 31) - BM) return GRET_ERR_UNSUPPORTED;
+    if (T > ((int64_t)1 << 31) - PM) return GRET_ERR_UNSUPPORTED;
     CUtensorMap tx, tw;
     {
         uint64_t dims[2] = {(uint64_t)D, (uint64_t)T};
@@ -392,7 +452,7 @@ gret_status_t launch_gn_gate(const void* o, const void* x, const void* w_g, cons
     p.T = T;
     p.F = F;
     p.D = D;
-    p.m_blocks = (int)((T + BM - 1) / BM);
+    p.m_blocks = (int)((T + PM - 1) / PM);
     p.n_blocks = F / BN;
     p.n_tiles = p.m_blocks * p.n_blocks;
     p.group_m = group_rows(p.n_blocks);
@@ -404,7 +464,7 @@ gret_status_t launch_qkvg_projection(const void* x, const void* w, int64_t ldw, 
                                      cudaStream_t stream) {
     const int F = 3 * H * 128 + H;
     if (H < 1 || H > 128 || D % BK != 0) return GRET_ERR_UNSUPPORTED;
-    if (T > ((int64_t)1 << 31) - BM) return GRET_ERR_UNSUPPORTED;
+    if (T > ((int64_t)1 << 31) - PM) return GRET_ERR_UNSUPPORTED;
     CUtensorMap tx, tw;
     {
         uint64_t dims[2] = {(uint64_t)D, (uint64_t)T};
@@ -428,7 +488,7 @@ gret_status_t launch_qkvg_projection(const void* x, const void* w, int64_t ldw, 
     p.qkv[1] = (__nv_bfloat16*)k;
     p.qkv[2] = (__nv_bfloat16*)v;
     p.g = g;
-    p.m_blocks = (int)((T + BM - 1) / BM);
+    p.m_blocks = (int)((T + PM - 1) / PM);
     p.n_blocks = (F + BN - 1) / BN;
     p.n_tiles = p.m_blocks * p.n_blocks;
     p.group_m = group_rows(p.n_blocks);
