@@ -258,20 +258,29 @@ def gret_groupnorm_gate(o, x, w_g, H, gn_weight=None, gn_bias=None, eps=1e-5, y=
     return y
 
 
-def gret_qkvg_projection(x, w, H, d=128, stream=None):
+def gret_qkvg_projection(x, w, H, d=128, out=None, stream=None):
     """[q | k | v | g] = x @ w in one GEMM: x [T, D] bf16, w [D, >= 3*H*d + H] bf16 (W_Q, W_K,
     W_V, W_gamma side by side; extra columns, if any, are padding).  Returns q, k, v bf16
-    [T, H, d] and the gate logits g fp32 [T, H]."""
+    [T, H, d] and the gate logits g fp32 [T, H], written into `out` = (q, k, v, g) when given
+    (contiguous tensors of those shapes and types)."""
     T, D = x.shape
     for t in (x, w):
         if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
             raise ValueError("x and w must be bfloat16 with contiguous rows")
     if x.stride(0) != D:
         raise ValueError("x must be contiguous")
-    q = torch.empty((T, H, d), dtype=torch.bfloat16, device=x.device)
-    k = torch.empty_like(q)
-    v = torch.empty_like(q)
-    g = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    if out is None:
+        q = torch.empty((T, H, d), dtype=torch.bfloat16, device=x.device)
+        k = torch.empty_like(q)
+        v = torch.empty_like(q)
+        g = torch.empty((T, H), dtype=torch.float32, device=x.device)
+    else:
+        q, k, v, g = out
+        for t in (q, k, v):
+            if t.dtype != torch.bfloat16 or not t.is_contiguous() or t.shape != (T, H, d):
+                raise ValueError("q, k, v outputs must be contiguous bfloat16 [T, H, d]")
+        if g.dtype != torch.float32 or not g.is_contiguous() or g.shape != (T, H):
+            raise ValueError("g output must be contiguous float32 [T, H]")
     _check("gret_qkvg_projection", _lib.gret_qkvg_projection(
         _ptr(x), _ptr(w), w.stride(0), T, H, d, D, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
         _stream(stream)))

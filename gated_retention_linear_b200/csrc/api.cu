@@ -139,6 +139,7 @@ gret_status_t gret_prefill_chunkwise(const void* q, const void* k, int64_t strid
                                      int64_t o_stride_batch, int64_t o_stride_tok,
                                      int64_t o_stride_head, int chunk, void* workspace,
                                      size_t workspace_bytes, gret_stream_t stream) {
+    const NvtxRange range("gret_prefill_chunkwise");
     return prefill_impl(q, k, stride_batch, stride_tok, stride_head, v, v_stride_batch,
                         v_stride_tok, v_stride_head, g, tau, k_scale, dtype, B, N, H, d_k, d_v,
                         cu_seqlens, n_seqs, state_in, state_out, o, o_stride_batch,
@@ -154,6 +155,7 @@ gret_status_t gret_prefill_chunkwise_testing(
     float* state_out, void* o, int64_t o_stride_batch, int64_t o_stride_tok,
     int64_t o_stride_head, int chunk, void* workspace, size_t workspace_bytes,
     gret_stream_t stream, uint64_t wait_ns, uint32_t first_ticket) {
+    const NvtxRange range("gret_prefill_chunkwise_testing");
     if (wait_ns == 0 || wait_ns > 2000000000ull) return GRET_ERR_INVALID_ARG;
     return prefill_impl(q, k, stride_batch, stride_tok, stride_head, v, v_stride_batch,
                         v_stride_tok, v_stride_head, g, tau, k_scale, dtype, B, N, H, d_k, d_v,
@@ -174,6 +176,7 @@ gret_status_t gret_workspace_status(const void* workspace, gret_stream_t stream)
 gret_status_t gret_decode_step(const void* q, const void* k, const void* v, const float* g,
                                float tau, float k_scale, gret_dtype_t dtype, int B, int H,
                                int d_k, int d_v, float* state, void* o, gret_stream_t stream) {
+    const NvtxRange range("gret_decode_step");
     if (dtype != GRET_F32 && dtype != GRET_BF16) return GRET_ERR_INVALID_ARG;
     if (!dim_ok(d_k) || !dim_ok(d_v) || B < 0 || H < 0) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
@@ -191,6 +194,7 @@ gret_status_t gret_groupnorm_gate(const void* o, const void* x, const void* w_g,
                                   const float* gn_weight, const float* gn_bias, float eps,
                                   int64_t T, int H, int d_v, int D, void* y,
                                   gret_stream_t stream) {
+    const NvtxRange range("gret_groupnorm_gate");
     if (T < 0 || H < 1 || D < 1 || !(eps >= 0.f) || !isfinite(eps)) return GRET_ERR_INVALID_ARG;
     if (d_v != 128 || D % 64 != 0) return GRET_ERR_UNSUPPORTED;
     if (T == 0) return GRET_OK;
@@ -204,6 +208,7 @@ gret_status_t gret_groupnorm_gate(const void* o, const void* x, const void* w_g,
 gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, int64_t T, int H,
                                    int d, int D, void* q, void* k, void* v, float* g,
                                    gret_stream_t stream) {
+    const NvtxRange range("gret_qkvg_projection");
     if (T < 0 || H < 1 || D < 1 || d < 1) return GRET_ERR_INVALID_ARG;
     const int64_t F = 3 * (int64_t)H * d + H;
     if (ldw < F) return GRET_ERR_INVALID_ARG;
@@ -236,6 +241,7 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
                                        int64_t N, int H, int d, const float* state_in,
                                        float* state_out, void* o, void* workspace,
                                        size_t workspace_bytes, gret_stream_t stream) {
+    const NvtxRange range("gret_prefill_elementwise");
     if (B < 0 || N < 0 || H < 1 || d < 1) return GRET_ERR_INVALID_ARG;
     if (!(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale)) return GRET_ERR_INVALID_ARG;
     if (d != EW_DIM) return GRET_ERR_UNSUPPORTED;
@@ -274,6 +280,7 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
 gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, float scale,
                                int window, int B, int64_t N, int H, int d, void* o,
                                gret_stream_t stream) {
+    const NvtxRange range("gret_swa_prefill");
     if (B < 0 || N < 0 || H < 1 || d < 1 || window < 1 || !isfinite(scale))
         return GRET_ERR_INVALID_ARG;
     if (d != SWA_DIM) return GRET_ERR_UNSUPPORTED;
@@ -297,6 +304,7 @@ extern "C" gret_status_t gret_swa_decode_step(const void* q, const void* k, cons
                                               float scale, int window, int B, int H, int d,
                                               const int32_t* pos, void* k_cache, void* v_cache,
                                               void* o, gret_stream_t stream) {
+    const NvtxRange range("gret_swa_decode_step");
     if (B < 0 || H < 1 || d < 1 || window < 1 || !isfinite(scale)) return GRET_ERR_INVALID_ARG;
     if (d != SWA_DIM || window > SWA_DECODE_MAX_WINDOW) return GRET_ERR_UNSUPPORTED;
     if ((int64_t)B * H > 0x7fffffffLL) return GRET_ERR_UNSUPPORTED;

@@ -38,6 +38,21 @@ enum : uint32_t { WS_ERR_NONE = 0, WS_ERR_TIMEOUT = 1 };
 
 }  // namespace gret
 
+// Host side: an NVTX range over the scope (the header-only NVTX v3 API; with no tool attached a
+// push or pop is a no-op), so that profilers show each ABI call by name around its launches.
+#include <nvtx3/nvToolsExt.h>
+
+namespace gret {
+
+struct NvtxRange {
+    explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+    ~NvtxRange() { nvtxRangePop(); }
+    NvtxRange(const NvtxRange&) = delete;
+    NvtxRange& operator=(const NvtxRange&) = delete;
+};
+
+}  // namespace gret
+
 // Host-side launchers (defined in the kernel files, called from api.cu).
 namespace gret {
 

@@ -50,6 +50,7 @@ extern "C" gret_status_t gret_prefill_chunkwise_noalloc(
     int d_k, int d_v, const int32_t* cu_seqlens, int n_seqs, const float* state_in,
     float* state_out, void* o, int64_t o_stride_batch, int64_t o_stride_tok,
     int64_t o_stride_head, int chunk, gret_stream_t stream) {
+    const gret::NvtxRange range("gret_prefill_chunkwise_noalloc");
     // size check on the host, before any CUDA call
     const int units = cu_seqlens ? n_seqs : B;
     const int64_t tokens = cu_seqlens ? N : (int64_t)B * N;
