@@ -63,6 +63,12 @@ _lib.gret_prefill_elementwise.argtypes = [_vp, _vp, _vp, _vp, _f32, _f32, _i32, 
 _lib.gret_prefill_elementwise.restype = _i32
 _lib.gret_prefill_elementwise_workspace_size.argtypes = [_i32, _i64, _i32, _i32]
 _lib.gret_prefill_elementwise_workspace_size.restype = ctypes.c_size_t
+_lib.gret_layer_forward.argtypes = [_vp, _vp, _i64, _vp, _vp, _vp, _f32, _f32, _f32, _i64, _i32,
+                                    _i32, _i32, _vp, _i32, _vp, _vp, _vp, _vp, ctypes.c_size_t,
+                                    _vp]
+_lib.gret_layer_forward.restype = _i32
+_lib.gret_layer_workspace_size.argtypes = [_i64, _i32, _i32, _i32]
+_lib.gret_layer_workspace_size.restype = ctypes.c_size_t
 _lib.gret_swa_prefill.argtypes = [_vp, _vp, _vp, _f32, _i32, _i32, _i64, _i32, _i32, _vp, _vp]
 _lib.gret_swa_prefill.restype = _i32
 _lib.gret_swa_decode_step.argtypes = [_vp, _vp, _vp, _f32, _i32, _i32, _i32, _i32, _vp, _vp, _vp,
@@ -356,21 +362,38 @@ def gret_swa_decode_step(q, k, v, pos, k_cache, v_cache, window=None, scale=None
     return o
 
 
+def gret_layer_workspace_size(T, n_seqs, H, d=128):
+    return int(_lib.gret_layer_workspace_size(T, n_seqs, H, d))
+
+
 def gret_layer_forward(x, w_qkvg, w_g, H, d=128, cu_seqlens=None, state_in=None, tau=16.0,
-                       k_scale=None, gn_weight=None, gn_bias=None, eps=1e-5, stream=None):
-    """One gated-retention mixer layer through the library's kernels: the q / k / v / gate-logit
-    projection of x, the chunkwise prefill (k scaled by d^-1/2 unless k_scale is given), and the
-    per-head GroupNorm * swish(x @ w_g) output gate.  x [T, D] bf16 is one packed batch
-    (cu_seqlens marks its sequences; None means one sequence).  Returns y [T, H*d] bf16 and the
-    final fp32 states [n_seqs, H, d, d]."""
-    T = x.shape[0]
-    q, k, v, g = gret_qkvg_projection(x, w_qkvg, H, d, stream=stream)
-    if cu_seqlens is None:
-        cu_seqlens = torch.tensor([0, T], dtype=torch.int32, device=x.device)
-    o, state = gret_prefill_chunkwise(q, k, v, g, tau=tau,
-                                      k_scale=d ** -0.5 if k_scale is None else k_scale,
-                                      cu_seqlens=cu_seqlens, state_in=state_in, state_out=True,
-                                      stream=stream)
-    y = gret_groupnorm_gate(o.view(T, H * d), x, w_g, H, gn_weight=gn_weight, gn_bias=gn_bias,
-                            eps=eps, stream=stream)
-    return y, state
+                       k_scale=None, gn_weight=None, gn_bias=None, eps=1e-5, y=None,
+                       state_out=True, workspace=None, stream=None):
+    """One gated-retention mixer layer through the C entry point gret_layer_forward: the
+    q / k / v / gate-logit projection of x, the chunkwise prefill (k scaled by d^-1/2 unless
+    k_scale is given), and the per-head GroupNorm * swish(x @ w_g) output gate.  x [T, D] bf16 is
+    one packed batch (cu_seqlens marks its sequences; None means one sequence).  Returns y
+    [T, H*d] bf16 and the final fp32 states [n_seqs, H, d, d] (state_out=True allocates them,
+    None skips them).  The workspace holds the intermediates; it is allocated here unless given."""
+    T, D = x.shape
+    for t in (x, w_qkvg, w_g):
+        if t.dtype != torch.bfloat16 or t.stride(-1) != 1:
+            raise ValueError("x, w_qkvg and w_g must be bfloat16 with contiguous rows")
+    if x.stride(0) != D or not w_g.is_contiguous():
+        raise ValueError("x and w_g must be contiguous")
+    if cu_seqlens is not None and (cu_seqlens.dtype != torch.int32 or cu_seqlens.dim() != 1):
+        raise ValueError("cu_seqlens must be 1-D int32")
+    n_seqs = 1 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if y is None:
+        y = torch.empty((T, H * d), dtype=torch.bfloat16, device=x.device)
+    if state_out is True:
+        state_out = torch.empty((n_seqs, H, d, d), dtype=torch.float32, device=x.device)
+    if workspace is None:
+        workspace = torch.empty(max(16, gret_layer_workspace_size(T, n_seqs, H, d)),
+                                dtype=torch.uint8, device=x.device)
+    _check("gret_layer_forward", _lib.gret_layer_forward(
+        _ptr(x), _ptr(w_qkvg), w_qkvg.stride(0), _ptr(w_g), _ptr(gn_weight), _ptr(gn_bias), eps,
+        tau, d ** -0.5 if k_scale is None else k_scale, T, H, d, D, _ptr(cu_seqlens), n_seqs,
+        _ptr(state_in), _ptr(state_out), _ptr(y), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream(stream)))
+    return y, state_out

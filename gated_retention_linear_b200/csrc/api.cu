@@ -277,6 +277,71 @@ gret_status_t gret_prefill_elementwise(const void* q, const void* k, const void*
     return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
 }
 
+// Workspace of gret_layer_forward: the prefill's workspace first (its status word at byte 0),
+// then q, k, v, o (bf16 [T, H, d]) and g (fp32 [T, H]), each 256-byte aligned.
+struct LayerWs {
+    size_t prefill, q, k, v, o, g, total;
+};
+
+LayerWs layer_ws(int64_t T, int n_seqs, int H, int d) {
+    auto up = [](size_t x) { return (x + 255) & ~size_t(255); };
+    LayerWs l = {};
+    l.prefill = gret_prefill_workspace_size(GRET_BF16, T, n_seqs, H, d, d, 0);
+    if (l.prefill == 0) return l;
+    const size_t act = (size_t)T * H * d * 2;
+    l.q = up(l.prefill);
+    l.k = l.q + up(act);
+    l.v = l.k + up(act);
+    l.o = l.v + up(act);
+    l.g = l.o + up(act);
+    l.total = l.g + up((size_t)T * H * 4);
+    return l;
+}
+
+size_t gret_layer_workspace_size(int64_t T, int n_seqs, int H, int d) {
+    if (T < 0 || n_seqs < 1 || H < 1 || d != 128) return 0;
+    return layer_ws(T, n_seqs, H, d).total;
+}
+
+gret_status_t gret_layer_forward(const void* x, const void* w_qkvg, int64_t ldw, const void* w_g,
+                                 const float* gn_weight, const float* gn_bias, float eps,
+                                 float tau, float k_scale, int64_t T, int H, int d, int D,
+                                 const int32_t* cu_seqlens, int n_seqs, const float* state_in,
+                                 float* state_out, void* y, void* workspace,
+                                 size_t workspace_bytes, gret_stream_t stream) {
+    const NvtxRange range("gret_layer_forward");
+    if (T < 0 || H < 1 || d < 1 || D < 1 || n_seqs < 1) return GRET_ERR_INVALID_ARG;
+    if (!cu_seqlens && n_seqs != 1) return GRET_ERR_INVALID_ARG;
+    if (d != 128) return GRET_ERR_UNSUPPORTED;
+    const LayerWs l = layer_ws(T, n_seqs, H, d);
+    if (l.total == 0) return GRET_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < l.total) return GRET_ERR_WORKSPACE;
+    if (!aligned16(workspace)) return GRET_ERR_ALIGNMENT;
+    if (T == 0) {   // no tokens: the final states are the entry states, y is empty
+        if (!state_out || state_out == state_in) return GRET_OK;
+        const size_t bytes = (size_t)n_seqs * H * d * d * sizeof(float);
+        const cudaStream_t s = (cudaStream_t)stream;
+        const cudaError_t e =
+            state_in ? cudaMemcpyAsync(state_out, state_in, bytes, cudaMemcpyDeviceToDevice, s)
+                     : cudaMemsetAsync(state_out, 0, bytes, s);
+        return e == cudaSuccess ? GRET_OK : GRET_ERR_CUDA;
+    }
+    unsigned char* ws = static_cast<unsigned char*>(workspace);
+    void* q = ws + l.q;
+    void* k = ws + l.k;
+    void* v = ws + l.v;
+    void* o = ws + l.o;
+    float* g = reinterpret_cast<float*>(ws + l.g);
+    gret_status_t st = gret_qkvg_projection(x, w_qkvg, ldw, T, H, d, D, q, k, v, g, stream);
+    if (st != GRET_OK) return st;
+    const int64_t td = (int64_t)H * d;   // token stride of q, k, v, o
+    st = gret_prefill_chunkwise(q, k, 0, td, d, v, 0, td, d, g, tau, k_scale, GRET_BF16, 1, T, H,
+                                d, d, cu_seqlens, cu_seqlens ? n_seqs : 0, state_in, state_out, o,
+                                0, td, d, 0, ws, l.prefill, stream);
+    if (st != GRET_OK) return st;
+    return gret_groupnorm_gate(o, x, w_g, gn_weight, gn_bias, eps, T, H, d, D, y, stream);
+}
+
 gret_status_t gret_swa_prefill(const void* q, const void* k, const void* v, float scale,
                                int window, int B, int64_t N, int H, int d, void* o,
                                gret_stream_t stream) {

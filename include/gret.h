@@ -221,6 +221,38 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
                                    gret_stream_t stream);
 
 /*
+ * One gated-retention mixer layer in one call: the input projection (gret_qkvg_projection), the
+ * chunkwise prefill (gret_prefill_chunkwise, tensor-core path) and the per-head GroupNorm and
+ * swish output gate (gret_groupnorm_gate), chained on one stream in the order the page
+ * "路线二：Multi-Head Gated Retention" draws the mixer:
+ *   [q | k | v | g] = X W_qkvg,   o = gRet(q, k_scale k, v; gamma = sigmoid(g)^(1/tau)),
+ *   y = GN_h(o) * swish(X W_G)
+ *   x        bf16 [T, D] row-major; one packed batch of sequences.
+ *   w_qkvg   bf16 [D, ldw] as in gret_qkvg_projection (3 H d + H used columns).
+ *   w_g      bf16 [D, H d];  gn_weight, gn_bias fp32 [H d] or NULL;  eps > 0.
+ *   cu_seqlens  int32 [n_seqs + 1] on the device (offsets into x), or NULL for one sequence
+ *               (n_seqs must then be 1).
+ *   state_in / state_out  fp32 [n_seqs, H, d, d] or NULL (zero entry state / no final state).
+ *   y        bf16 [T, H d].
+ *   workspace  at least gret_layer_workspace_size(T, n_seqs, H, d) bytes of device memory,
+ *              16-byte aligned, owned by the caller; it holds the intermediates q, k, v, g and o
+ *              and, at its start, the prefill's workspace (gret_workspace_status reads it).
+ * Requires d == 128 and what the three calls require (H <= 128, D a multiple of 64, H d a
+ * multiple of 256, 16-byte aligned pointers and ldw a multiple of 8); the first call that
+ * refuses its arguments returns its status and the later ones are not launched.  y must not
+ * overlap x or the workspace.
+ */
+gret_status_t gret_layer_forward(const void* x, const void* w_qkvg, int64_t ldw, const void* w_g,
+                                 const float* gn_weight, const float* gn_bias, float eps,
+                                 float tau, float k_scale, int64_t T, int H, int d, int D,
+                                 const int32_t* cu_seqlens, int n_seqs, const float* state_in,
+                                 float* state_out, void* y, void* workspace,
+                                 size_t workspace_bytes, gret_stream_t stream);
+
+/* Workspace bytes gret_layer_forward needs; 0 for invalid or unsupported sizes. */
+size_t gret_layer_workspace_size(int64_t T, int n_seqs, int H, int d);
+
+/*
  * Chunkwise prefill with one gate per key channel: the element-wise alternative that
  * "路线二：Multi-Head Gated Retention" weighs against the head-wise scalar gate (YOCO keeps the
  * head-wise one because it keeps every contraction a plain matrix product).  Per sequence and

@@ -162,3 +162,33 @@ def test_swa_rejects_bad_arguments_without_launching():
     assert call(N=0) == 0
     assert call(o=None) == 1
     assert call(v=4100) == 3
+
+
+def test_layer_forward_rejects_bad_arguments_without_launching():
+    import gated_retention_linear_b200 as G
+    lib = G._lib
+    need = G.gret_layer_workspace_size(300, 1, 2, 128)
+    # the prefill's workspace, then q, k, v, o (bf16) and g (fp32), each 256-byte aligned
+    up = lambda x: (x + 255) // 256 * 256
+    pre = G.gret_prefill_workspace_size(torch_bf16_code(G), 300, 1, 2, 128, 128)
+    assert need == up(pre) + 4 * up(300 * 2 * 128 * 2) + up(300 * 2 * 4)
+    assert G.gret_layer_workspace_size(300, 1, 2, 64) == 0
+    assert G.gret_layer_workspace_size(300, 0, 2, 128) == 0
+
+    def call(**kw):
+        a = dict(x=1024, w=2048, ldw=776, wg=4096, gnw=None, gnb=None, eps=1e-5, tau=16.0,
+                 ks=1.0, T=300, H=2, d=128, D=128, cu=None, n=1, sin=None, sout=None, y=8192,
+                 ws=1 << 20, wsb=need, stream=None)
+        a.update(kw)
+        return lib.gret_layer_forward(*a.values())
+    assert call(d=64) == 2                     # no kernel for d = 64
+    assert call(n=2) == 1                      # two sequences need cu_seqlens
+    assert call(H=0) == 1
+    assert call(wsb=need - 1) == 4             # workspace smaller than the size query says
+    assert call(ws=None) == 4
+    assert call(ws=(1 << 20) + 8) == 3         # workspace not 16-byte aligned
+
+
+def torch_bf16_code(G):
+    import torch
+    return G._dtype_code(torch.empty(0, dtype=torch.bfloat16))

@@ -130,3 +130,16 @@ def test_guards_sliding_window():
     kc.check("k_cache")
     vc.check("v_cache")
     od.check("o")
+
+
+def test_guards_layer_forward():
+    G = lib()
+    T, H, D = 300, 2, 128
+    lay = SI.layer_inputs(T, D, H, seed=51, device="cuda", pad=6)
+    cu = torch.tensor([0, 100, 300], dtype=torch.int32, device="cuda")
+    y = Guarded((T, H * 128), torch.bfloat16)
+    s = Guarded((2, H, 128, 128), torch.float32)
+    G.gret_layer_forward(lay["x"], lay["w_qkvg"], lay["w_g"], H, cu_seqlens=cu, y=y.t,
+                         state_out=s.t)
+    y.check("y")
+    s.check("state_out")
