@@ -54,7 +54,7 @@ namespace {
 
 constexpr int C = EW_CHUNK;             // tokens per chunk
 constexpr int D = EW_DIM;               // d_k = d_v
-constexpr int NT = 256;                 // threads of the range kernels
+constexpr int NT = 512;                 // threads of the range kernels
 constexpr int TILE = C * D * 2;         // one bf16 128 x 128 tile
 constexpr int SLAB = TILE / 2;          // one 64-column slab of it
 constexpr int GTILE = C * D * 4;        // the chunk's fp32 gate logits
@@ -83,7 +83,7 @@ struct __align__(1024) OutSmem {
     unsigned char x[TILE];   // low half of the query operand; then the output tile
     unsigned char y[TILE];   // low half of K~  (x and y: fp32 P of a pairwise chunk)
     float g[C * D];          // gate logits -> cumulative log2-decay -> state operand hi | lo
-    float tot[2][D];         // per channel: log2-decay of tokens [0, 64) and [64, 128)
+    float tot[4][D];         // per channel: log2-decay of tokens [32 q, 32 q + 32)
     uint64_t k_full, r_full, mma_done, drain;   // k tile; q, v, g tiles; MMA groups; exit
     uint32_t tmem_base;
 };
@@ -92,7 +92,7 @@ struct __align__(1024) StateSmem {
     unsigned char k[2][TILE];   // k (two stages), then the high half of the weighted keys in place
     unsigned char v[2][TILE];
     unsigned char y[TILE];      // low half of the weighted keys
-    float tot[2][D];
+    float tot[4][D];
     uint64_t kv_full[2], mma_done, drain;
     uint32_t tmem_base;
 };
@@ -219,7 +219,7 @@ __device__ __forceinline__ void load_qvg_tiles(unsigned char* q, unsigned char* 
 // first so that each key's weight, its log2-decay to the end of the range, is a running suffix
 // sum; every K~^T V MMA of the range accumulates into one tensor-memory result.  k and v tiles
 // come by TMA through a two-stage ring, the next chunk's issued as soon as its stage is free;
-// thread (i, hh) reads the gate logits of channel i for its token half straight into registers,
+// thread (i, qq) reads the gate logits of channel i for its 32 tokens straight into registers,
 // one chunk ahead.
 
 __device__ __forceinline__ void load_kv(StateSmem& sm, int st, const CUtensorMap* tk,
@@ -232,11 +232,11 @@ __device__ __forceinline__ void load_kv(StateSmem& sm, int st, const CUtensorMap
     }
 }
 
-// Gate logits of tokens [t0, t0 + 64) of one (batch, head) row at channel i (0 past the end).
-__device__ __forceinline__ void load_gate64(const float* grow, int64_t gstride, int64_t t0,
-                                            int64_t N, float (&x)[64]) {
+// Gate logits of tokens [t0, t0 + 32) of one (batch, head) row at channel i (0 past the end).
+__device__ __forceinline__ void load_gate32(const float* grow, int64_t gstride, int64_t t0,
+                                            int64_t N, float (&x)[32]) {
 #pragma unroll
-    for (int u = 0; u < 64; ++u) x[u] = t0 + u < N ? __ldg(grow + (t0 + u) * gstride) : 0.f;
+    for (int u = 0; u < 32; ++u) x[u] = t0 + u < N ? __ldg(grow + (t0 + u) * gstride) : 0.f;
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -269,15 +269,15 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int i = tid & 127, hh = tid >> 7;   // channel (TMEM lane), token half (column half)
+    const int i = tid & 127, qq = tid >> 7;   // channel (TMEM lane), token / column quarter
     const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
     const float* grow = p.g + ((int64_t)b * p.N * p.H + h) * D + i;
     const int64_t gstride = (int64_t)p.H * D;
     const ColOffset co(i);
 
     if (tid == 0) load_kv(sm, 0, &tk, &tv, (c1 - 1) * C, h, b);
-    float gcur[64], gnext[64];
-    load_gate64(grow, gstride, (int64_t)(c1 - 1) * C + 64 * hh, p.N, gcur);
+    float gcur[32], gnext[32];
+    load_gate32(grow, gstride, (int64_t)(c1 - 1) * C + 32 * qq, p.N, gcur);
     float R = 0.f;   // log2-decay of the tokens after the current chunk, to the range end
     int issued = 1, consumed = 0;
     uint32_t n_mma = 0;
@@ -291,28 +291,34 @@ __global__ void __launch_bounds__(NT, 1)
         if (n + 1 < n_ch) {
             if (tid == 0) load_kv(sm, st ^ 1, &tk, &tv, (c - 1) * C, h, b);
             ++issued;
-            load_gate64(grow, gstride, (int64_t)(c - 1) * C + 64 * hh, p.N, gnext);
+            load_gate32(grow, gstride, (int64_t)(c - 1) * C + 32 * qq, p.N, gnext);
         }
-        // per-token log2-decays of channel i over this thread's half
+        // per-token log2-decays of channel i over this thread's 32 tokens
         float sum = 0.f;
 #pragma unroll
-        for (int u = 0; u < 64; ++u) {
-            gcur[u] = 64 * hh + u < L ? logsigmoid_fast(gcur[u]) * p.inv_tau_log2e : 0.f;
+        for (int u = 0; u < 32; ++u) {
+            gcur[u] = 32 * qq + u < L ? logsigmoid_fast(gcur[u]) * p.inv_tau_log2e : 0.f;
             sum += gcur[u];
         }
-        sm.tot[hh][i] = sum;
+        sm.tot[qq][i] = sum;
         __syncthreads();
-        const float t0 = sm.tot[0][i], t1 = sm.tot[1][i];
+        float after = 0.f, total = 0.f;   // log2-decay of the later quarters, and of the chunk
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float t = sm.tot[q4][i];
+            if (q4 > qq) after += t;
+            total += t;
+        }
         if (!(ok = block_wait(&sm.kv_full[st], (n >> 1) & 1, p.err))) break;
         ++consumed;
         // weights 2^(suffix) k_scale, suffix = log2-decay from after token t to the range end,
         // last token first, in batches of 8
-        float s = R + (hh == 0 ? t1 : 0.f);
+        float s = R + after;
 #pragma unroll
-        for (int ub = 56; ub >= 0; ub -= 8) {
+        for (int ub = 24; ub >= 0; ub -= 8) {
             float kv[8], sw[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) kv[u] = bf16_at(sm.k[st], co.at(64 * hh + ub, u));
+            for (int u = 0; u < 8; ++u) kv[u] = bf16_at(sm.k[st], co.at(32 * qq + ub, u));
 #pragma unroll
             for (int u = 7; u >= 0; --u) {
                 sw[u] = s;
@@ -322,11 +328,11 @@ __global__ void __launch_bounds__(NT, 1)
             for (int u = 0; u < 8; ++u) {
                 __nv_bfloat16 hi, lo;
                 split1(kv[u] * ex2f(sw[u]) * p.k_scale, hi, lo);
-                *reinterpret_cast<__nv_bfloat16*>(sm.k[st] + co.at(64 * hh + ub, u)) = hi;
-                *reinterpret_cast<__nv_bfloat16*>(sm.y + co.at(64 * hh + ub, u)) = lo;
+                *reinterpret_cast<__nv_bfloat16*>(sm.k[st] + co.at(32 * qq + ub, u)) = hi;
+                *reinterpret_cast<__nv_bfloat16*>(sm.y + co.at(32 * qq + ub, u)) = lo;
             }
         }
-        R += t0 + t1;
+        R += total;
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
@@ -338,24 +344,21 @@ __global__ void __launch_bounds__(NT, 1)
         }
         ++n_mma;
 #pragma unroll
-        for (int u = 0; u < 64; ++u) gcur[u] = gnext[u];
+        for (int u = 0; u < 32; ++u) gcur[u] = gnext[u];
     }
     if (ok) ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err);
     if (ok) {
         tc_fence_after();
         const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
-        float* dst = p.ws_S + slot * (D * D) + (int64_t)i * D + 64 * hh;
+        float* dst = p.ws_S + slot * (D * D) + (int64_t)i * D + 32 * qq;
+        float a[32];
+        tmem_ld32(tmem + lane_base + 32 * qq, a);
+        tmem_ld_wait();
 #pragma unroll
-        for (int jc = 0; jc < 2; ++jc) {
-            float a[32];
-            tmem_ld32(tmem + lane_base + 64 * hh + 32 * jc, a);
-            tmem_ld_wait();
-#pragma unroll
-            for (int e = 0; e < 8; ++e)
-                reinterpret_cast<float4*>(dst + 32 * jc)[e] =
-                    make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
-        }
-        if (hh == 0) p.ws_a[slot * D + i] = ex2f(R);
+        for (int e = 0; e < 8; ++e)
+            reinterpret_cast<float4*>(dst)[e] =
+                make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
+        if (qq == 0) p.ws_a[slot * D + i] = ex2f(R);
     } else if (tid == 0) {
         // a wait gave up: let the issued MMAs and the loads in flight finish before exit
         mma_commit(&sm.drain);
@@ -437,10 +440,9 @@ __device__ void pairwise_scores(OutSmem& sm, const EwParams& p, uint32_t tmem, i
         if (lane == 0) Pt[m * C + t] = acc * p.k_scale;
     }
     __syncthreads();
-    const int row = (warp & 3) * 32 + lane, hh = warp >> 2;
+    const int row = (warp & 3) * 32 + lane, jc = warp >> 2;   // 32 columns per thread
     const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
-#pragma unroll 1
-    for (int jc = 2 * hh; jc < 2 * hh + 2; ++jc) {
+    {
         uint32_t ph[32];
 #pragma unroll
         for (int i2 = 0; i2 < 16; ++i2) {
@@ -484,9 +486,9 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // thread (i, hh): channel / state row i = TMEM lane, column half (token half in the
-    // per-channel passes) hh
-    const int i = tid & 127, hh = tid >> 7;
+    // thread (i, qq): channel / state row i = TMEM lane, quarter qq: tokens [32 qq, 32 qq + 32)
+    // in the per-channel passes, columns [32 qq, 32 qq + 32) of the state and of the output
+    const int i = tid & 127, qq = tid >> 7;
     const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
     const uint32_t qb = smem_u32(sm.q), kb = smem_u32(sm.k), vb = smem_u32(sm.v),
                    xb = smem_u32(sm.x), yb = smem_u32(sm.y), shb = smem_u32(sm.g),
@@ -496,14 +498,14 @@ __global__ void __launch_bounds__(NT, 1)
         load_k_tile(sm.k, &tk, &sm.k_full, c0 * C, h, b);
         load_qvg_tiles(sm.q, sm.v, sm.g, &tq, &tv, &tg, &sm.r_full, c0 * C, h, b);
     }
-    // entry state of the range: row i, columns [64 hh, 64 hh + 64)
+    // entry state of the range: row i, columns [32 qq, 32 qq + 32)
     const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
-    float S[64];
+    float S[32];
     {
         const float4* src =
-            reinterpret_cast<const float4*>(p.ws_S + slot * (D * D) + (int64_t)i * D + 64 * hh);
+            reinterpret_cast<const float4*>(p.ws_S + slot * (D * D) + (int64_t)i * D + 32 * qq);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
+        for (int e = 0; e < 8; ++e) {
             const float4 x = src[e];
             S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
         }
@@ -519,11 +521,11 @@ __global__ void __launch_bounds__(NT, 1)
         }
         if (!(ok = block_wait(&sm.r_full, (n_ld - 1) & 1, p.err))) break;
         if (!(ok = block_wait(&sm.k_full, (n_k - 1) & 1, p.err))) break;
-        // cumulative log2-decay of channel i over this thread's token half, in place (batches
-        // of 16 tokens)
+        // cumulative log2-decay of channel i over this thread's 32 tokens, in place (batches of
+        // 16 tokens: every load of a batch before its arithmetic)
         float cum = 0.f;
 #pragma unroll 1
-        for (int tb = 64 * hh; tb < 64 * hh + 64; tb += 16) {
+        for (int tb = 32 * qq; tb < 32 * qq + 32; tb += 16) {
             float x[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u) x[u] = sm.g[(tb + u) * D + i];
@@ -536,14 +538,20 @@ __global__ void __launch_bounds__(NT, 1)
                 sm.g[(tb + u) * D + i] = cum;
             }
         }
-        sm.tot[hh][i] = cum;
+        sm.tot[qq][i] = cum;
         __syncthreads();
-        const float t0 = sm.tot[0][i], cL = t0 + sm.tot[1][i];
+        float before = 0.f, cL = 0.f;   // log2-decay of the quarters before this one, and total
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const float t = sm.tot[q4][i];
+            if (q4 < qq) before += t;
+            cL += t;
+        }
         const bool pairwise = __syncthreads_or(cL < -SPAN2) != 0;
         if (pairwise) {
-            if (hh == 1) {
+            if (qq > 0) {
 #pragma unroll 8
-                for (int t = 64; t < C; ++t) sm.g[t * D + i] += t0;
+                for (int t = 32 * qq; t < 32 * qq + 32; ++t) sm.g[t * D + i] += before;
             }
             __syncthreads();
             pairwise_scores(sm, p, tmem, L);
@@ -551,11 +559,11 @@ __global__ void __launch_bounds__(NT, 1)
         // operands: query (factored: 2^(c_t - c_L); pairwise: 2^(c_t)) and K~ = k_scale k
         // 2^(c_L - c_t), each as bf16 high half in place and low half in x / y
         {
-            const float off = (hh == 1 && !pairwise) ? t0 : 0.f;
+            const float off = pairwise ? 0.f : before;
             const float qshift = pairwise ? 0.f : -cL;
             const ColOffset co(i);
 #pragma unroll 1
-            for (int tb = 64 * hh; tb < 64 * hh + 64; tb += 8) {
+            for (int tb = 32 * qq; tb < 32 * qq + 32; tb += 8) {
                 float ct[8], qv[8], kv[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
@@ -577,18 +585,20 @@ __global__ void __launch_bounds__(NT, 1)
             }
         }
         __syncthreads();   // every read of the log2-decays is done: sm.g takes the state operand
-        // state operand: 2^c_L S (factored) or S (pairwise), row i, slab hh of the MN-major
-        // high-half and low-half tiles
+        // state operand: 2^c_L S (factored) or S (pairwise), row i, columns [32 qq, 32 qq + 32)
+        // of the MN-major high-half and low-half tiles (slab qq / 2, 16-byte chunks
+        // 4 (qq % 2) .. 4 (qq % 2) + 3 of the row)
         {
             const float sc = pairwise ? 1.f : ex2f(cL);
             unsigned char* shi = reinterpret_cast<unsigned char*>(sm.g);
 #pragma unroll
-            for (int cc = 0; cc < 8; ++cc) {
+            for (int cc = 0; cc < 4; ++cc) {
                 uint32_t hi[4], lo[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e)
                     split2(sc * S[8 * cc + 2 * e], sc * S[8 * cc + 2 * e + 1], hi[e], lo[e]);
-                const uint32_t off = hh * SLAB + i * 128 + ((cc ^ (i & 7)) << 4);
+                const int chunk = 4 * (qq & 1) + cc;
+                const uint32_t off = (qq >> 1) * SLAB + i * 128 + ((chunk ^ (i & 7)) << 4);
                 *reinterpret_cast<uint4*>(shi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
                 *reinterpret_cast<uint4*>(shi + TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
             }
@@ -619,23 +629,20 @@ __global__ void __launch_bounds__(NT, 1)
             if (tid == 0) load_k_tile(sm.k, &tk, &sm.k_full, (c + 1) * C, h, b);
             ++n_k;
         }
+        const int row = (warp & 3) * 32 + lane;   // == i: this thread's TMEM lane
         if (!pairwise) {
-            // causal mask, P split into bf16 halves in place: row = lane, 64 columns per thread
-            const int row = (warp & 3) * 32 + lane;
-#pragma unroll 1
-            for (int jc = 2 * hh; jc < 2 * hh + 2; ++jc) {
-                float a[32];
-                tmem_ld32(tmem + lane_base + TM_A + jc * 32, a);
-                tmem_ld_wait();
-                uint32_t ph[32];
+            // causal mask, P split into bf16 halves in place: row = lane, columns [32 qq, +32)
+            float a[32];
+            tmem_ld32(tmem + lane_base + TM_A + qq * 32, a);
+            tmem_ld_wait();
+            uint32_t ph[32];
 #pragma unroll
-                for (int i2 = 0; i2 < 16; ++i2) {
-                    const int m0 = jc * 32 + 2 * i2;
-                    split2(m0 <= row ? a[2 * i2] : 0.f, m0 + 1 <= row ? a[2 * i2 + 1] : 0.f,
-                           ph[i2], ph[16 + i2]);
-                }
-                tmem_st32(tmem + lane_base + TM_A + jc * 32, ph);
+            for (int i2 = 0; i2 < 16; ++i2) {
+                const int m0 = qq * 32 + 2 * i2;
+                split2(m0 <= row ? a[2 * i2] : 0.f, m0 + 1 <= row ? a[2 * i2 + 1] : 0.f, ph[i2],
+                       ph[16 + i2]);
             }
+            tmem_st32(tmem + lane_base + TM_A + qq * 32, ph);
             tmem_st_wait();
             tc_fence_before();
             __syncthreads();
@@ -660,14 +667,14 @@ __global__ void __launch_bounds__(NT, 1)
         }
         // output rows: a chunk inside the sequence goes out as one tile through x (rows in the
         // swizzled layout, two TMA stores); the rows of a partial chunk one by one
-        const int row = (warp & 3) * 32 + lane;
         const bool full = L == C;
         const int64_t tok = (int64_t)c * C + row;
         uint4* orow = reinterpret_cast<uint4*>(p.o + (((int64_t)b * p.N + tok) * p.H + h) * D);
-#pragma unroll 1
-        for (int jc = 2 * hh; jc < 2 * hh + 2; ++jc) {
+        {
             float o[32];
-            tmem_ld32(tmem + lane_base + TM_O + jc * 32, o);
+            tmem_ld32(tmem + lane_base + TM_O + qq * 32, o);
+            float d[32];
+            if (!last) tmem_ld32(tmem + lane_base + TM_S + qq * 32, d);
             tmem_ld_wait();
 #pragma unroll
             for (int v4 = 0; v4 < 4; ++v4) {
@@ -676,24 +683,18 @@ __global__ void __launch_bounds__(NT, 1)
                 u.y = pack_bf16x2(o[8 * v4 + 2], o[8 * v4 + 3]);
                 u.z = pack_bf16x2(o[8 * v4 + 4], o[8 * v4 + 5]);
                 u.w = pack_bf16x2(o[8 * v4 + 6], o[8 * v4 + 7]);
-                const int cc = 4 * jc + v4;   // 16-byte chunk of the row
+                const int cc = 4 * qq + v4;   // 16-byte chunk of the row
                 if (full)
                     *reinterpret_cast<uint4*>(sm.x + (cc >> 3) * SLAB + row * 128 +
                                               (((cc & 7) ^ (row & 7)) << 4)) = u;
                 else if (row < L)
                     orow[cc] = u;
             }
-        }
-        // the state carried to the next chunk: S = 2^c_L S + dS
-        if (!last) {
-            const float eL = ex2f(cL);
+            // the state carried to the next chunk: S = 2^c_L S + dS
+            if (!last) {
+                const float eL = ex2f(cL);
 #pragma unroll
-            for (int jc = 0; jc < 2; ++jc) {
-                float d[32];
-                tmem_ld32(tmem + lane_base + TM_S + 64 * hh + 32 * jc, d);
-                tmem_ld_wait();
-#pragma unroll
-                for (int e = 0; e < 32; ++e) S[32 * jc + e] = fmaf(eL, S[32 * jc + e], d[e]);
+                for (int e = 0; e < 32; ++e) S[e] = fmaf(eL, S[e], d[e]);
             }
         }
         tc_fence_before();
