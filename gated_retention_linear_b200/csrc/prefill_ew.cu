@@ -78,13 +78,14 @@ struct EwParams {
 
 struct __align__(1024) OutSmem {
     unsigned char q[TILE];   // q, then the high half of the query operand (in place)
-    unsigned char k[TILE];   // k, then the high half of K~ (in place)
+    unsigned char k[TILE];   // k, then the high half of K~ (in place), then that of the state operand
     unsigned char v[TILE];
     unsigned char x[TILE];   // low half of the query operand; then the output tile
-    unsigned char y[TILE];   // low half of K~  (x and y: fp32 P of a pairwise chunk)
-    float g[C * D];          // gate logits -> cumulative log2-decay -> state operand hi | lo
+    unsigned char y[TILE];   // low half of K~, then that of the state operand  (x and y: fp32 P
+                             // of a pairwise chunk)
+    float g[C * D];          // gate logits -> cumulative log2-decay
     float tot[4][D];         // per channel: log2-decay of tokens [32 q, 32 q + 32)
-    uint64_t k_full, r_full, mma_done, drain;   // k tile; q, v, g tiles; MMA groups; exit
+    uint64_t g_full, r_full, mma_done, drain;   // gate tile; q, k, v tiles; MMA groups; exit
     uint32_t tmem_base;
 };
 
@@ -191,27 +192,25 @@ __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int half, ui
 }
 
 // Loads of one chunk, coordinates (column, head, token, batch) in every map, rows past the
-// sequence read as zero: the k tile (two 64-column swizzled slabs), and the q and v tiles with
-// the gate logits (one unswizzled fp32 box of 128 columns).
-__device__ __forceinline__ void load_k_tile(unsigned char* k, const CUtensorMap* tk, uint64_t* bar,
-                                            int tok, int h, int b) {
-    mbar_arrive_expect_tx(bar, TILE);
-#pragma unroll
-    for (int half = 0; half < 2; ++half)
-        tma_load_4d(k + half * SLAB, tk, bar, half * 64, h, tok, b);
+// sequence read as zero: the gate logits (one unswizzled fp32 box of 128 columns), and the q, k
+// and v tiles (two 64-column swizzled slabs each).
+__device__ __forceinline__ void load_gate_tile(float* g, const CUtensorMap* tg, uint64_t* bar,
+                                               int tok, int h, int b) {
+    mbar_arrive_expect_tx(bar, GTILE);
+    tma_load_4d(g, tg, bar, 0, h, tok, b);
 }
 
-__device__ __forceinline__ void load_qvg_tiles(unsigned char* q, unsigned char* v, float* g,
-                                               const CUtensorMap* tq, const CUtensorMap* tv,
-                                               const CUtensorMap* tg, uint64_t* bar, int tok,
+__device__ __forceinline__ void load_qkv_tiles(unsigned char* q, unsigned char* k, unsigned char* v,
+                                               const CUtensorMap* tq, const CUtensorMap* tk,
+                                               const CUtensorMap* tv, uint64_t* bar, int tok,
                                                int h, int b) {
-    mbar_arrive_expect_tx(bar, 2 * TILE + GTILE);
+    mbar_arrive_expect_tx(bar, 3 * TILE);
 #pragma unroll
     for (int half = 0; half < 2; ++half) {
         tma_load_4d(q + half * SLAB, tq, bar, half * 64, h, tok, b);
+        tma_load_4d(k + half * SLAB, tk, bar, half * 64, h, tok, b);
         tma_load_4d(v + half * SLAB, tv, bar, half * 64, h, tok, b);
     }
-    tma_load_4d(g, tg, bar, 0, h, tok, b);
 }
 
 // ----------------------------------------------------------------------------------------------
@@ -472,7 +471,7 @@ __global__ void __launch_bounds__(NT, 1)
     const int c0 = r * p.G;
     const int c1 = (int)min64(nch, (int64_t)c0 + p.G);
     if (tid == 0) {
-        mbar_init(&sm.k_full, 1);
+        mbar_init(&sm.g_full, 1);
         mbar_init(&sm.r_full, 1);
         mbar_init(&sm.mma_done, 1);
         mbar_init(&sm.drain, 1);
@@ -491,12 +490,11 @@ __global__ void __launch_bounds__(NT, 1)
     const int i = tid & 127, qq = tid >> 7;
     const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
     const uint32_t qb = smem_u32(sm.q), kb = smem_u32(sm.k), vb = smem_u32(sm.v),
-                   xb = smem_u32(sm.x), yb = smem_u32(sm.y), shb = smem_u32(sm.g),
-                   slb = shb + TILE;
+                   xb = smem_u32(sm.x), yb = smem_u32(sm.y);
 
     if (tid == 0) {
-        load_k_tile(sm.k, &tk, &sm.k_full, c0 * C, h, b);
-        load_qvg_tiles(sm.q, sm.v, sm.g, &tq, &tv, &tg, &sm.r_full, c0 * C, h, b);
+        load_gate_tile(sm.g, &tg, &sm.g_full, c0 * C, h, b);
+        load_qkv_tiles(sm.q, sm.k, sm.v, &tq, &tk, &tv, &sm.r_full, c0 * C, h, b);
     }
     // entry state of the range: row i, columns [32 qq, 32 qq + 32)
     const int64_t slot = ((int64_t)b * p.H + h) * p.R + r;
@@ -510,7 +508,7 @@ __global__ void __launch_bounds__(NT, 1)
             S[4 * e] = x.x; S[4 * e + 1] = x.y; S[4 * e + 2] = x.z; S[4 * e + 3] = x.w;
         }
     }
-    uint32_t n_ld = 1, n_k = 1, n_mma = 0;   // q/v/g and k loads issued, MMA groups committed
+    uint32_t n_g = 1, n_ld = 1, n_mma = 0;   // gate and q/k/v loads issued, MMA groups committed
     bool ok = true;
     for (int c = c0; c < c1; ++c) {
         const int L = (int)min64(C, p.N - (int64_t)c * C);
@@ -519,8 +517,7 @@ __global__ void __launch_bounds__(NT, 1)
             if (tid == 0) bulk_wait_group_read0();
             __syncthreads();
         }
-        if (!(ok = block_wait(&sm.r_full, (n_ld - 1) & 1, p.err))) break;
-        if (!(ok = block_wait(&sm.k_full, (n_k - 1) & 1, p.err))) break;
+        if (!(ok = block_wait(&sm.g_full, (n_g - 1) & 1, p.err))) break;
         // cumulative log2-decay of channel i over this thread's 32 tokens, in place (batches of
         // 16 tokens: every load of a batch before its arithmetic)
         float cum = 0.f;
@@ -548,6 +545,7 @@ __global__ void __launch_bounds__(NT, 1)
             cL += t;
         }
         const bool pairwise = __syncthreads_or(cL < -SPAN2) != 0;
+        if (!(ok = block_wait(&sm.r_full, (n_ld - 1) & 1, p.err))) break;
         if (pairwise) {
             if (qq > 0) {
 #pragma unroll 8
@@ -584,24 +582,10 @@ __global__ void __launch_bounds__(NT, 1)
                 }
             }
         }
-        __syncthreads();   // every read of the log2-decays is done: sm.g takes the state operand
-        // state operand: 2^c_L S (factored) or S (pairwise), row i, columns [32 qq, 32 qq + 32)
-        // of the MN-major high-half and low-half tiles (slab qq / 2, 16-byte chunks
-        // 4 (qq % 2) .. 4 (qq % 2) + 3 of the row)
-        {
-            const float sc = pairwise ? 1.f : ex2f(cL);
-            unsigned char* shi = reinterpret_cast<unsigned char*>(sm.g);
-#pragma unroll
-            for (int cc = 0; cc < 4; ++cc) {
-                uint32_t hi[4], lo[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    split2(sc * S[8 * cc + 2 * e], sc * S[8 * cc + 2 * e + 1], hi[e], lo[e]);
-                const int chunk = 4 * (qq & 1) + cc;
-                const uint32_t off = (qq >> 1) * SLAB + i * 128 + ((chunk ^ (i & 7)) << 4);
-                *reinterpret_cast<uint4*>(shi + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                *reinterpret_cast<uint4*>(shi + TILE + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
-            }
+        __syncthreads();   // every read of the log2-decays is done: the next gate tile may come
+        if (!last) {
+            if (tid == 0) load_gate_tile(sm.g, &tg, &sm.g_full, (c + 1) * C, h, b);
+            ++n_g;
         }
         fence_proxy_async_smem();
         __syncthreads();
@@ -625,9 +609,22 @@ __global__ void __launch_bounds__(NT, 1)
             if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
             tc_fence_after();
         }
-        if (!last) {
-            if (tid == 0) load_k_tile(sm.k, &tk, &sm.k_full, (c + 1) * C, h, b);
-            ++n_k;
+        // state operand into the k (high halves) and y (low halves) tiles: 2^c_L S (factored) or
+        // S (pairwise), row i, columns [32 qq, 32 qq + 32) of the MN-major tiles (slab qq / 2,
+        // 16-byte chunks 4 (qq % 2) .. 4 (qq % 2) + 3 of the row)
+        {
+            const float sc = pairwise ? 1.f : ex2f(cL);
+#pragma unroll
+            for (int cc = 0; cc < 4; ++cc) {
+                uint32_t hi[4], lo[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    split2(sc * S[8 * cc + 2 * e], sc * S[8 * cc + 2 * e + 1], hi[e], lo[e]);
+                const int chunk = 4 * (qq & 1) + cc;
+                const uint32_t off = (qq >> 1) * SLAB + i * 128 + ((chunk ^ (i & 7)) << 4);
+                *reinterpret_cast<uint4*>(sm.k + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                *reinterpret_cast<uint4*>(sm.y + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+            }
         }
         const int row = (warp & 3) * 32 + lane;   // == i: this thread's TMEM lane
         if (!pairwise) {
@@ -644,15 +641,16 @@ __global__ void __launch_bounds__(NT, 1)
             }
             tmem_st32(tmem + lane_base + TM_A + qq * 32, ph);
             tmem_st_wait();
-            tc_fence_before();
-            __syncthreads();
         }
+        tc_fence_before();
+        fence_proxy_async_smem();
+        __syncthreads();
         // second group: the output O = Q S' + P V
         if (tid == 0) {
             tc_fence_after();
-            mma_128(tmem + TM_O, qb, false, shb, true, false);   // O = Q_hi S_hi
-            mma_128(tmem + TM_O, xb, false, shb, true, true);    //   + Q_lo S_hi
-            mma_128(tmem + TM_O, qb, false, slb, true, true);    //   + Q_hi S_lo
+            mma_128(tmem + TM_O, qb, false, kb, true, false);    // O = Q_hi S_hi
+            mma_128(tmem + TM_O, xb, false, kb, true, true);     //   + Q_lo S_hi
+            mma_128(tmem + TM_O, qb, false, yb, true, true);     //   + Q_hi S_lo
             mma_pv(tmem + TM_O, tmem + TM_A, 0, vb, true);       //   + P_hi V
             mma_pv(tmem + TM_O, tmem + TM_A, 1, vb, true);       //   + P_lo V
             mma_commit(&sm.mma_done);
@@ -660,9 +658,9 @@ __global__ void __launch_bounds__(NT, 1)
         ++n_mma;
         if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
         tc_fence_after();
-        if (!last) {   // every tile but x is free: the rest of the next chunk's loads go now
+        if (!last) {   // q, k, v are free: the next chunk's tiles go now
             if (tid == 0)
-                load_qvg_tiles(sm.q, sm.v, sm.g, &tq, &tv, &tg, &sm.r_full, (c + 1) * C, h, b);
+                load_qkv_tiles(sm.q, sm.k, sm.v, &tq, &tk, &tv, &sm.r_full, (c + 1) * C, h, b);
             ++n_ld;
         }
         // output rows: a chunk inside the sequence goes out as one tile through x (rows in the
@@ -712,7 +710,7 @@ __global__ void __launch_bounds__(NT, 1)
             mma_commit(&sm.drain);
             uint32_t never = 0;
             mbar_wait(&sm.drain, 0, &never, DRAIN_NS);
-            mbar_wait(&sm.k_full, (n_k - 1) & 1, &never, DRAIN_NS);
+            mbar_wait(&sm.g_full, (n_g - 1) & 1, &never, DRAIN_NS);
             mbar_wait(&sm.r_full, (n_ld - 1) & 1, &never, DRAIN_NS);
         }
         bulk_wait_group0();
