@@ -84,7 +84,7 @@ struct __align__(1024) OutSmem {
     unsigned char y[TILE];   // low half of K~, then that of the state operand  (x and y: fp32 P
                              // of a pairwise chunk)
     float g[C * D];          // gate logits -> cumulative log2-decay
-    float tot[4][D];         // per channel: log2-decay of tokens [32 q, 32 q + 32)
+    float cls[D];            // per channel: the chunk's total log2-decay c_L
     uint64_t g_full, r_full, mma_done, drain;   // gate tile; q, k, v tiles; MMA groups; exit
     uint32_t tmem_base;
 };
@@ -93,7 +93,8 @@ struct __align__(1024) StateSmem {
     unsigned char k[2][TILE];   // k (two stages), then the high half of the weighted keys in place
     unsigned char v[2][TILE];
     unsigned char y[TILE];      // low half of the weighted keys
-    float tot[4][D];
+    float tot[8][D];         // per channel: log2-decay of tokens [16 s, 16 s + 16)
+    float rs[D];             // per channel: log2-decay from the range's first chunk to its end
     uint64_t kv_full[2], mma_done, drain;
     uint32_t tmem_base;
 };
@@ -130,6 +131,10 @@ struct ColOffset {
 
 __device__ __forceinline__ float bf16_at(const unsigned char* tile, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(tile + off));
+}
+
+__device__ __forceinline__ float2 bf16x2_at(const unsigned char* tile, uint32_t off) {
+    return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tile + off));
 }
 
 // x = hi + lo, hi = bf16(x), lo = bf16(x - hi)
@@ -218,7 +223,7 @@ __device__ __forceinline__ void load_qkv_tiles(unsigned char* q, unsigned char* 
 // first so that each key's weight, its log2-decay to the end of the range, is a running suffix
 // sum; every K~^T V MMA of the range accumulates into one tensor-memory result.  k and v tiles
 // come by TMA through a two-stage ring, the next chunk's issued as soon as its stage is free;
-// thread (i, qq) reads the gate logits of channel i for its 32 tokens straight into registers,
+// thread (cp, seg) reads the gate logits of its channel pair for its 16 tokens straight into registers,
 // one chunk ahead.
 
 __device__ __forceinline__ void load_kv(StateSmem& sm, int st, const CUtensorMap* tk,
@@ -231,11 +236,14 @@ __device__ __forceinline__ void load_kv(StateSmem& sm, int st, const CUtensorMap
     }
 }
 
-// Gate logits of tokens [t0, t0 + 32) of one (batch, head) row at channel i (0 past the end).
-__device__ __forceinline__ void load_gate32(const float* grow, int64_t gstride, int64_t t0,
-                                            int64_t N, float (&x)[32]) {
+// Gate logits of tokens [t0, t0 + 16) of one (batch, head) row at a pair of adjacent channels
+// (0 past the end).
+__device__ __forceinline__ void load_gate16x2(const float* grow, int64_t gstride, int64_t t0,
+                                              int64_t N, float2 (&x)[16]) {
 #pragma unroll
-    for (int u = 0; u < 32; ++u) x[u] = t0 + u < N ? __ldg(grow + (t0 + u) * gstride) : 0.f;
+    for (int u = 0; u < 16; ++u)
+        x[u] = t0 + u < N ? __ldg(reinterpret_cast<const float2*>(grow + (t0 + u) * gstride))
+                          : make_float2(0.f, 0.f);
 }
 
 __global__ void __launch_bounds__(NT, 1)
@@ -268,16 +276,20 @@ __global__ void __launch_bounds__(NT, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    const int i = tid & 127, qq = tid >> 7;   // channel (TMEM lane), token / column quarter
+    // per-channel passes: thread (cp, seg) takes channels 2 cp, 2 cp + 1 over tokens
+    // [16 seg, 16 seg + 16); the aggregate is read out by thread (i, qq): TMEM lane i, columns
+    // [32 qq, 32 qq + 32)
+    const int cp = tid & 63, seg = tid >> 6, ch = 2 * cp;
+    const int i = tid & 127, qq = tid >> 7;
     const uint32_t lane_base = ((uint32_t)(warp & 3) * 32u) << 16;
-    const float* grow = p.g + ((int64_t)b * p.N * p.H + h) * D + i;
+    const float* grow = p.g + ((int64_t)b * p.N * p.H + h) * D + ch;
     const int64_t gstride = (int64_t)p.H * D;
-    const ColOffset co(i);
+    const ColOffset co(ch);   // channels ch, ch + 1: one aligned 4-byte pair
 
     if (tid == 0) load_kv(sm, 0, &tk, &tv, (c1 - 1) * C, h, b);
-    float gcur[32], gnext[32];
-    load_gate32(grow, gstride, (int64_t)(c1 - 1) * C + 32 * qq, p.N, gcur);
-    float R = 0.f;   // log2-decay of the tokens after the current chunk, to the range end
+    float2 gcur[16], gnext[16];
+    load_gate16x2(grow, gstride, (int64_t)(c1 - 1) * C + 16 * seg, p.N, gcur);
+    float2 R = make_float2(0.f, 0.f);   // log2-decay after the current chunk, to the range end
     int issued = 1, consumed = 0;
     uint32_t n_mma = 0;
     bool ok = true;
@@ -290,48 +302,58 @@ __global__ void __launch_bounds__(NT, 1)
         if (n + 1 < n_ch) {
             if (tid == 0) load_kv(sm, st ^ 1, &tk, &tv, (c - 1) * C, h, b);
             ++issued;
-            load_gate32(grow, gstride, (int64_t)(c - 1) * C + 32 * qq, p.N, gnext);
+            load_gate16x2(grow, gstride, (int64_t)(c - 1) * C + 16 * seg, p.N, gnext);
         }
-        // per-token log2-decays of channel i over this thread's 32 tokens
-        float sum = 0.f;
+        // per-token log2-decays of both channels over this thread's 16 tokens
+        float2 sum = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int u = 0; u < 32; ++u) {
-            gcur[u] = 32 * qq + u < L ? logsigmoid_fast(gcur[u]) * p.inv_tau_log2e : 0.f;
-            sum += gcur[u];
+        for (int u = 0; u < 16; ++u) {
+            const bool in = 16 * seg + u < L;
+            gcur[u].x = in ? logsigmoid_fast(gcur[u].x) * p.inv_tau_log2e : 0.f;
+            gcur[u].y = in ? logsigmoid_fast(gcur[u].y) * p.inv_tau_log2e : 0.f;
+            sum.x += gcur[u].x;
+            sum.y += gcur[u].y;
         }
-        sm.tot[qq][i] = sum;
+        *reinterpret_cast<float2*>(&sm.tot[seg][ch]) = sum;
         __syncthreads();
-        float after = 0.f, total = 0.f;   // log2-decay of the later quarters, and of the chunk
+        float2 after = make_float2(0.f, 0.f), total = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const float t = sm.tot[q4][i];
-            if (q4 > qq) after += t;
-            total += t;
+        for (int s8 = 0; s8 < 8; ++s8) {
+            const float2 t = *reinterpret_cast<const float2*>(&sm.tot[s8][ch]);
+            if (s8 > seg) {
+                after.x += t.x;
+                after.y += t.y;
+            }
+            total.x += t.x;
+            total.y += t.y;
         }
         if (!(ok = block_wait(&sm.kv_full[st], (n >> 1) & 1, p.err))) break;
         ++consumed;
         // weights 2^(suffix) k_scale, suffix = log2-decay from after token t to the range end,
         // last token first, in batches of 8
-        float s = R + after;
+        float2 s2 = make_float2(R.x + after.x, R.y + after.y);
 #pragma unroll
-        for (int ub = 24; ub >= 0; ub -= 8) {
-            float kv[8], sw[8];
+        for (int ub = 8; ub >= 0; ub -= 8) {
+            float2 kv[8], sw[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) kv[u] = bf16_at(sm.k[st], co.at(32 * qq + ub, u));
+            for (int u = 0; u < 8; ++u) kv[u] = bf16x2_at(sm.k[st], co.at(16 * seg + ub, u));
 #pragma unroll
             for (int u = 7; u >= 0; --u) {
-                sw[u] = s;
-                s += gcur[ub + u];
+                sw[u] = s2;
+                s2.x += gcur[ub + u].x;
+                s2.y += gcur[ub + u].y;
             }
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                __nv_bfloat16 hi, lo;
-                split1(kv[u] * ex2f(sw[u]) * p.k_scale, hi, lo);
-                *reinterpret_cast<__nv_bfloat16*>(sm.k[st] + co.at(32 * qq + ub, u)) = hi;
-                *reinterpret_cast<__nv_bfloat16*>(sm.y + co.at(32 * qq + ub, u)) = lo;
+                uint32_t hi, lo;
+                split2(kv[u].x * ex2f(sw[u].x) * p.k_scale, kv[u].y * ex2f(sw[u].y) * p.k_scale,
+                       hi, lo);
+                *reinterpret_cast<uint32_t*>(sm.k[st] + co.at(16 * seg + ub, u)) = hi;
+                *reinterpret_cast<uint32_t*>(sm.y + co.at(16 * seg + ub, u)) = lo;
             }
         }
-        R += total;
+        R.x += total.x;
+        R.y += total.y;
         fence_proxy_async_smem();
         __syncthreads();
         if (tid == 0) {
@@ -343,8 +365,9 @@ __global__ void __launch_bounds__(NT, 1)
         }
         ++n_mma;
 #pragma unroll
-        for (int u = 0; u < 32; ++u) gcur[u] = gnext[u];
+        for (int u = 0; u < 16; ++u) gcur[u] = gnext[u];
     }
+    if (seg == 0) *reinterpret_cast<float2*>(&sm.rs[ch]) = R;   // read after the next barrier
     if (ok) ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err);
     if (ok) {
         tc_fence_after();
@@ -357,7 +380,7 @@ __global__ void __launch_bounds__(NT, 1)
         for (int e = 0; e < 8; ++e)
             reinterpret_cast<float4*>(dst)[e] =
                 make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
-        if (qq == 0) p.ws_a[slot * D + i] = ex2f(R);
+        if (qq == 0) p.ws_a[slot * D + i] = ex2f(sm.rs[i]);
     } else if (tid == 0) {
         // a wait gave up: let the issued MMAs and the loads in flight finish before exit
         mma_commit(&sm.drain);
@@ -518,38 +541,55 @@ __global__ void __launch_bounds__(NT, 1)
             __syncthreads();
         }
         if (!(ok = block_wait(&sm.g_full, (n_g - 1) & 1, p.err))) break;
-        // cumulative log2-decay of channel i over this thread's 32 tokens, in place (batches of
-        // 16 tokens: every load of a batch before its arithmetic)
-        float cum = 0.f;
-#pragma unroll 1
-        for (int tb = 32 * qq; tb < 32 * qq + 32; tb += 16) {
-            float x[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u) x[u] = sm.g[(tb + u) * D + i];
+        // per-channel passes: thread (cp, seg) takes channels 2 cp, 2 cp + 1 over tokens
+        // [16 seg, 16 seg + 16), with paired shared-memory accesses (float2, bf16x2)
+        const int cp = tid & 63, seg = tid >> 6, ch = 2 * cp;
+        // cumulative log2-decay of both channels over the segment, in place (every load first)
+        float2 cum = make_float2(0.f, 0.f);
+        {
+            float2 x[16];
 #pragma unroll
             for (int u = 0; u < 16; ++u)
-                x[u] = tb + u < L ? logsigmoid_fast(x[u]) * p.inv_tau_log2e : 0.f;
+                x[u] = *reinterpret_cast<const float2*>(&sm.g[(16 * seg + u) * D + ch]);
 #pragma unroll
             for (int u = 0; u < 16; ++u) {
-                cum += x[u];
-                sm.g[(tb + u) * D + i] = cum;
+                const bool in = 16 * seg + u < L;
+                x[u].x = in ? logsigmoid_fast(x[u].x) * p.inv_tau_log2e : 0.f;
+                x[u].y = in ? logsigmoid_fast(x[u].y) * p.inv_tau_log2e : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 16; ++u) {
+                cum.x += x[u].x;
+                cum.y += x[u].y;
+                *reinterpret_cast<float2*>(&sm.g[(16 * seg + u) * D + ch]) = cum;
             }
         }
-        sm.tot[qq][i] = cum;
+        float* tot = reinterpret_cast<float*>(sm.y);   // [8][D] segment totals; y is idle here
+        *reinterpret_cast<float2*>(&tot[seg * D + ch]) = cum;
         __syncthreads();
-        float before = 0.f, cL = 0.f;   // log2-decay of the quarters before this one, and total
+        float2 before = make_float2(0.f, 0.f), cl2 = make_float2(0.f, 0.f);
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-            const float t = sm.tot[q4][i];
-            if (q4 < qq) before += t;
-            cL += t;
+        for (int s8 = 0; s8 < 8; ++s8) {
+            const float2 t = *reinterpret_cast<const float2*>(&tot[s8 * D + ch]);
+            if (s8 < seg) {
+                before.x += t.x;
+                before.y += t.y;
+            }
+            cl2.x += t.x;
+            cl2.y += t.y;
         }
-        const bool pairwise = __syncthreads_or(cL < -SPAN2) != 0;
+        if (seg == 0) *reinterpret_cast<float2*>(&sm.cls[ch]) = cl2;
+        // (also the barrier after which y may be written again)
+        const bool pairwise = __syncthreads_or(fminf(cl2.x, cl2.y) < -SPAN2) != 0;
         if (!(ok = block_wait(&sm.r_full, (n_ld - 1) & 1, p.err))) break;
         if (pairwise) {
-            if (qq > 0) {
-#pragma unroll 8
-                for (int t = 32 * qq; t < 32 * qq + 32; ++t) sm.g[t * D + i] += before;
+            if (seg > 0) {
+#pragma unroll 4
+                for (int t = 16 * seg; t < 16 * seg + 16; ++t) {
+                    float2* gp = reinterpret_cast<float2*>(&sm.g[t * D + ch]);
+                    const float2 c2 = *gp;
+                    *gp = make_float2(c2.x + before.x, c2.y + before.y);
+                }
             }
             __syncthreads();
             pairwise_scores(sm, p, tmem, L);
@@ -557,28 +597,30 @@ __global__ void __launch_bounds__(NT, 1)
         // operands: query (factored: 2^(c_t - c_L); pairwise: 2^(c_t)) and K~ = k_scale k
         // 2^(c_L - c_t), each as bf16 high half in place and low half in x / y
         {
-            const float off = pairwise ? 0.f : before;
-            const float qshift = pairwise ? 0.f : -cL;
-            const ColOffset co(i);
+            const float2 off = pairwise ? make_float2(0.f, 0.f) : before;
+            const float qsx = pairwise ? 0.f : -cl2.x, qsy = pairwise ? 0.f : -cl2.y;
+            const ColOffset co(ch);   // channels ch, ch + 1: one aligned 4-byte pair
 #pragma unroll 1
-            for (int tb = 32 * qq; tb < 32 * qq + 32; tb += 8) {
-                float ct[8], qv[8], kv[8];
+            for (int tb = 16 * seg; tb < 16 * seg + 16; tb += 8) {
+                float2 ct[8], qv[8], kv[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    ct[u] = sm.g[(tb + u) * D + i] + off;
-                    qv[u] = bf16_at(sm.q, co.at(tb, u));
-                    kv[u] = bf16_at(sm.k, co.at(tb, u));
+                    const float2 c2 = *reinterpret_cast<const float2*>(&sm.g[(tb + u) * D + ch]);
+                    ct[u] = make_float2(c2.x + off.x, c2.y + off.y);
+                    qv[u] = bf16x2_at(sm.q, co.at(tb, u));
+                    kv[u] = bf16x2_at(sm.k, co.at(tb, u));
                 }
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
-                    __nv_bfloat16 qh, ql, kh, kl;
-                    split1(qv[u] * ex2f(ct[u] + qshift), qh, ql);
-                    split1(kv[u] * ex2f(cL - ct[u]) * p.k_scale, kh, kl);
+                    uint32_t qh, ql, kh, kl;
+                    split2(qv[u].x * ex2f(ct[u].x + qsx), qv[u].y * ex2f(ct[u].y + qsy), qh, ql);
+                    split2(kv[u].x * ex2f(cl2.x - ct[u].x) * p.k_scale,
+                           kv[u].y * ex2f(cl2.y - ct[u].y) * p.k_scale, kh, kl);
                     const uint32_t o = co.at(tb, u);
-                    *reinterpret_cast<__nv_bfloat16*>(sm.q + o) = qh;
-                    *reinterpret_cast<__nv_bfloat16*>(sm.x + o) = ql;
-                    *reinterpret_cast<__nv_bfloat16*>(sm.k + o) = kh;
-                    *reinterpret_cast<__nv_bfloat16*>(sm.y + o) = kl;
+                    *reinterpret_cast<uint32_t*>(sm.q + o) = qh;
+                    *reinterpret_cast<uint32_t*>(sm.x + o) = ql;
+                    *reinterpret_cast<uint32_t*>(sm.k + o) = kh;
+                    *reinterpret_cast<uint32_t*>(sm.y + o) = kl;
                 }
             }
         }
@@ -609,6 +651,7 @@ __global__ void __launch_bounds__(NT, 1)
             if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
             tc_fence_after();
         }
+        const float cL = sm.cls[i];   // row i's channel total (the state rows below)
         // state operand into the k (high halves) and y (low halves) tiles: 2^c_L S (factored) or
         // S (pairwise), row i, columns [32 qq, 32 qq + 32) of the MN-major tiles (slab qq / 2,
         // 16-byte chunks 4 (qq % 2) .. 4 (qq % 2) + 3 of the row)
