@@ -37,7 +37,14 @@
 //   ew_range_output  one CTA per range, chunks in order from the range's entry state: the
 //                    outputs above, and the state carried to the next chunk of the range
 // The range kernels are synchronous per CTA (one block-wide phase after another; one thread
-// issues the MMAs) and take a whole SM each (224 KB of shared memory).
+// issues the MMAs) and take a whole SM each: 512 threads, 224 KB of shared memory.  In the
+// per-channel passes a thread takes a pair of adjacent channels over 16 tokens, so that its
+// shared-memory accesses and bf16 conversions come in pairs; in the state and output phases a
+// thread takes a quarter (32 columns) of one TMEM lane.  Loads run ahead of the phases as far
+// as the shared-memory plan allows: in the outputs kernel the next chunk's gate tile right after
+// the operand build (the state operand goes into the k and y tiles once the first MMA group has
+// read them) and its q, k, v after the second group; in the aggregates kernel a two-stage k / v
+// ring and the gate logits read into registers one chunk ahead.
 #include "prefill_ew.cuh"
 
 #include <algorithm>
