@@ -335,6 +335,11 @@ def run_gpu(args):
     if not args.no_swa:
         swa = run_swa(args, rank, world, stream, ms_per_step)
 
+    # ---------------- the long-context prefill: one 524288-token sequence, 24 heads
+    long_ctx = None
+    if not args.no_long:
+        long_ctx = run_long_context(args, rank, world, stream, hbm_peak, peak_kind)
+
     # ---------------- varlen prefill + GroupNorm * swish(X W_G) epilogue
     epi = None
     if not args.no_epilogue:
@@ -425,7 +430,7 @@ def run_gpu(args):
         "config": bench_config(world),
         "chunk_sweep": sweep,
         "decode": dec, "varlen_epilogue": epi, "layer": lay,
-        "elementwise_gate": ew, "sliding_window": swa,
+        "elementwise_gate": ew, "sliding_window": swa, "long_context": long_ctx,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm_peak, "unit": "GB/s",
                      "frac": achieved / hbm_peak, "peak_kind": peak_kind,
                      "traffic": prefill_traffic_from_profile(),
@@ -433,7 +438,7 @@ def run_gpu(args):
                      "algorithmic_bytes_per_launch": alg_bytes},
         "e2e": e2e, "clocks": clk, "gpu_launches": args.steps, "cpu_baseline": cpu,
         # last, so that a record which keeps only the end of the line still has every leg
-        "legs": legs_summary(dec, epi, lay, ew, swa),
+        "legs": legs_summary(dec, epi, lay, ew, swa, long_ctx),
     }
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -442,7 +447,7 @@ def run_gpu(args):
         dist.destroy_process_group()
 
 
-def legs_summary(dec, epi, lay, ew, swa):
+def legs_summary(dec, epi, lay, ew, swa, long_ctx=None):
     """value, unit and roofline fraction of every secondary leg, rounded, in a few hundred
     characters."""
     def r(x, n=4):
@@ -465,12 +470,63 @@ def legs_summary(dec, epi, lay, ew, swa):
                                  "tensor_frac": r(swa["roofline"]["frac"], 3)}
         if swa.get("decode"):
             out["sliding_window"]["decode_hbm_frac"] = r(swa["decode"]["roofline"]["frac"], 3)
+    if long_ctx:
+        out["long_context"] = {"v": r(long_ctx["value"]), "u": long_ctx["unit"],
+                               "ms": r(long_ctx["ms_per_step"]),
+                               "hbm_frac": r(long_ctx["roofline"]["frac"], 3)}
     if ew:
         out["elementwise_gate"] = {"v": r(ew["value"]), "u": ew["unit"],
                                    "frac": r(ew["roofline"]["frac"], 3),
                                    "bound": ew["roofline"]["bound"],
                                    "x_headwise": r(ew["slowdown_vs_headwise"], 3)}
     return out
+
+
+def run_long_context(args, rank, world, stream, hbm_peak, peak_kind):
+    """The long-context configuration: one sequence of 524288 tokens (4096 chunks), 24 heads of
+    128, bf16 q, k, v ~ N(0, 1)/sqrt(128), g ~ N(2, 1), tau 16, the fp32 state carried through
+    every chunk; the same kernel and roofline as the headline prefill."""
+    import torch
+
+    import gated_retention_linear_b200 as G
+    import synth_inputs as SI
+    Nl = 524288
+    inp = SI.gret_inputs(1, Nl, H, D, dtype=torch.bfloat16, g_mean=2.0, g_std=1.0,
+                         seed=rank_seed(3, rank), device="cuda")
+    q, k, v, g = inp["q"], inp["k"], inp["v"], inp["g"]
+    del inp
+    o = torch.empty_like(q)
+    s_out = torch.empty((1, H, D, D), dtype=torch.float32, device="cuda")
+    ws = torch.empty(G.gret_prefill_workspace_size(torch.bfloat16, Nl, 1, H, D, D, 0),
+                     dtype=torch.uint8, device="cuda")
+
+    def step():
+        G.gret_prefill_chunkwise(q, k, v, g, state_out=s_out, o=o, workspace=ws)
+
+    for _ in range(max(2, min(args.warmup, 3))):
+        step()
+    torch.cuda.synchronize()
+    n = max(1, min(args.steps, 5))
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / n, world)
+    if G.gret_workspace_status(ws) != 0:
+        raise RuntimeError("long-context prefill reported a timed-out wait")
+    alg = float(Nl * H * BYTES_PER_TOKEN_HEAD)
+    ach = alg / (ms * 1e-3) / 1e9
+    del q, k, v, g, o, ws
+    return {"value": Nl * world / (ms * 1e-3) / 1e6, "unit": "Mtok/s", "tokens": Nl, "heads": H,
+            "ms_per_step": ms, "steps": n, "gpu_launches_per_step": 1,
+            "l2": "inputs and outputs (12.9 GB) far larger than L2; not flushed",
+            "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm_peak, "unit": "GB/s",
+                         "frac": ach / hbm_peak, "peak_kind": peak_kind, "traffic": None,
+                         "kernel": "prefill_tc_kernel", "algorithmic_bytes_per_launch": alg}}
 
 
 def run_varlen_epilogue(args, rank, world, stream, hbm_peak):
@@ -840,6 +896,8 @@ def main():
     ap.add_argument("--no-layer", action="store_true")
     ap.add_argument("--no-elementwise", action="store_true")
     ap.add_argument("--no-swa", action="store_true")
+    ap.add_argument("--no-long", action="store_true",
+                    help="skip the long-context leg (524288 tokens x 24 heads, 13 GB)")
     ap.add_argument("--elementwise-tokens", type=int, default=None,
                     help="tokens of the per-channel-gate leg (default: the 32768 of its "
                          "workload; smaller values are for profiling captures)")
