@@ -313,10 +313,24 @@ gret_status_t gret_layer_forward(const void* x, const void* w_qkvg, int64_t ldw,
     if (T < 0 || H < 1 || d < 1 || D < 1 || n_seqs < 1) return GRET_ERR_INVALID_ARG;
     if (!cu_seqlens && n_seqs != 1) return GRET_ERR_INVALID_ARG;
     if (d != 128) return GRET_ERR_UNSUPPORTED;
+    // the three steps' requirements, checked before anything is launched, so that a call that
+    // one step would refuse has no effect on the device
+    if (!(eps >= 0.f) || !isfinite(eps) || !(tau > 0.f) || !isfinite(tau) || !isfinite(k_scale))
+        return GRET_ERR_INVALID_ARG;
+    if (ldw < 3 * (int64_t)H * d + H) return GRET_ERR_INVALID_ARG;
+    if (H > 128 || D % 64 != 0 || (H * d) % 256 != 0) return GRET_ERR_UNSUPPORTED;
+    if (T > ((int64_t)1 << 31) - 256) return GRET_ERR_UNSUPPORTED;
     const LayerWs l = layer_ws(T, n_seqs, H, d);
     if (l.total == 0) return GRET_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < l.total) return GRET_ERR_WORKSPACE;
     if (!aligned16(workspace)) return GRET_ERR_ALIGNMENT;
+    if (T > 0) {
+        if (!x || !w_qkvg || !w_g || !y) return GRET_ERR_INVALID_ARG;
+        if (!aligned16(x) || !aligned16(w_qkvg) || !aligned16(w_g) || !aligned16(y) ||
+            ldw % 8 != 0 || (state_in && !aligned16(state_in)) ||
+            (state_out && !aligned16(state_out)))
+            return GRET_ERR_ALIGNMENT;
+    }
     if (T == 0) {   // no tokens: the final states are the entry states, y is empty
         if (!state_out || state_out == state_in) return GRET_OK;
         const size_t bytes = (size_t)n_seqs * H * d * d * sizeof(float);

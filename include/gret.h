@@ -238,9 +238,9 @@ gret_status_t gret_qkvg_projection(const void* x, const void* w, int64_t ldw, in
  *              16-byte aligned, owned by the caller; it holds the intermediates q, k, v, g and o
  *              and, at its start, the prefill's workspace (gret_workspace_status reads it).
  * Requires d == 128 and what the three calls require (H <= 128, D a multiple of 64, H d a
- * multiple of 256, 16-byte aligned pointers and ldw a multiple of 8); the first call that
- * refuses its arguments returns its status and the later ones are not launched.  y must not
- * overlap x or the workspace.
+ * multiple of 256, 16-byte aligned pointers and ldw a multiple of 8).  These are all checked
+ * before the first launch, so a refused call has no effect on the device.  y must not overlap
+ * x or the workspace.
  */
 gret_status_t gret_layer_forward(const void* x, const void* w_qkvg, int64_t ldw, const void* w_g,
                                  const float* gn_weight, const float* gn_bias, float eps,

@@ -192,3 +192,25 @@ def test_layer_forward_rejects_bad_arguments_without_launching():
 def torch_bf16_code(G):
     import torch
     return G._dtype_code(torch.empty(0, dtype=torch.bfloat16))
+
+
+def test_layer_forward_refuses_before_any_launch():
+    """Arguments that only the later steps (the prefill, the GroupNorm gate) would refuse are
+    refused up front: none of these calls launches anything (no GPU here)."""
+    import gated_retention_linear_b200 as G
+    lib = G._lib
+    need = G.gret_layer_workspace_size(300, 1, 2, 128)
+
+    def call(**kw):
+        a = dict(x=1024, w=2048, ldw=776, wg=4096, gnw=None, gnb=None, eps=1e-5, tau=16.0,
+                 ks=1.0, T=300, H=2, d=128, D=128, cu=None, n=1, sin=None, sout=None, y=8192,
+                 ws=1 << 20, wsb=need, stream=None)
+        a.update(kw)
+        return lib.gret_layer_forward(*a.values())
+    assert call(eps=-1.0) == 1                 # the gate's eps
+    assert call(tau=0.0) == 1                  # the prefill's tau
+    assert call(ldw=700) == 1                  # narrower than the projection's columns
+    assert call(D=96) == 2                     # the GEMMs' K blocks
+    assert call(H=3, ldw=3 * 3 * 128 + 3 + 5, wsb=G.gret_layer_workspace_size(300, 1, 3, 128)) == 2
+    assert call(ldw=777) == 3                  # rows of W not 16-byte aligned
+    assert call(y=8200) == 3
