@@ -144,12 +144,7 @@ __device__ __forceinline__ float2 bf16x2_at(const unsigned char* tile, uint32_t 
     return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(tile + off));
 }
 
-// x = hi + lo, hi = bf16(x), lo = bf16(x - hi)
-__device__ __forceinline__ void split1(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-    hi = __float2bfloat16_rn(x);
-    lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-}
-
+// (x0, x1) = hi + lo per element, hi = bf16(x), lo = bf16(x - hi), each pair packed
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
     const float2 hf = __bfloat1622float2(h);
