@@ -1077,8 +1077,8 @@ bool make_map(CUtensorMap* map, const void* base, int64_t st, int64_t sh, int64_
 // Chunks per span.  Spans run in waves of `grid` CTAs; a span costs about G chunk-times plus a
 // fixed overhead of about 1.5 (its look-back and the switches between passes), and the
 // look-backs of one chain run one after another at about half a chunk-time each.  G minimises
-// the larger of the two over [2, 128]; measured at 32K x 24 heads this picks 22 (two waves) and
-// at 512K x 24 heads 96 (both within 2% of the best span size found by sweeping).
+// the larger of the two over [2, 128]: at 32K x 24 heads it picks 43 (144 spans, one wave; the
+// fastest span size of a measured sweep), at 512K x 24 heads 111.
 // GRET_SPAN_CHUNKS overrides the choice.
 int span_chunks(int64_t chunks_per_unit, int64_t chains, int grid) {
     static int forced = -2;
