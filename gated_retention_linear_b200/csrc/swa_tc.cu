@@ -4,37 +4,37 @@
 // "路线一：滑动窗口注意力": position i attends to the most recent W positions of its sequence,
 //   o_i = sum_{j = i-W+1 .. i} softmax_j(scale q_i . k_j) v_j .
 // FlashAttention-style, as the page suggests for this mixer, built on tcgen05:
-//   * an item of work is two 128-query tiles of one (batch, head), queries q0 .. q0 + 255; the
-//     key tiles of 128 that their windows touch (ten at W = 1024) stream through two TMA stages
-//     and serve both query tiles;
-//   * the kernel is persistent, one CTA per SM taking items round-robin; a query tile's slot is
-//     loaded with the next item's queries as soon as its output has been stored, so the next
-//     item starts while the last one finishes;
-//   * S = Q K^T for each query tile goes to tensor memory; two softmax warpgroups per query
-//     tile (one query row per thread, keys [0, 64) and [64, 128) of the key tile) mask the
-//     window, share the row's running maximum through shared memory, keep their partial sums,
-//     and write P = 2^(s - m) back over S as a bf16 high + low pair; the MMA warp accumulates
-//     O += P_hi V + P_lo V in tensor memory as each half of the keys arrives;
-//   * the two query tiles take turns: while one runs its softmax, the tensor cores run the
-//     other tile's products;
-//   * the running maximum is only moved (and O rescaled) when a tile's maximum exceeds it by
-//     more than 2^8, so rescaling is rare after the first tiles; P then stays below 256;
-//   * the output, O / l in bf16, leaves through the query tile's own shared-memory slot by TMA
-//     store (rows past the sequence end are clipped by the store).
+//   * an item of work is one 128-query tile of one (batch, head); the key tiles of 128 that its
+//     window touches (nine at W = 1024) stream through shared memory (two K stages, three V
+//     stages).  The kernel is persistent: one CTA per SM takes items round-robin, consecutive
+//     items being neighbouring query tiles of one head (their key tiles meet in L2);
+//   * every key tile j of the CTA (numbered across items) has its own score buffer S[j % 3] in
+//     tensor memory and its own softmax warpgroup j % 3, so that Q K^T runs up to three key
+//     tiles ahead of P V and three softmaxes overlap the products, instead of one tile's
+//     Q K^T -> softmax -> P V chain setting the pace;
+//   * a softmax thread owns one query row of its tile (all 128 keys): it masks the window,
+//     takes the row's maximum, writes P = 2^(s - m) back over S as a bf16 high + low pair, and
+//     the MMA warp accumulates O += P_hi V + P_lo V as each half of the keys arrives;
+//   * the row's reference maximum m is handed from tile to tile (through shared memory, one
+//     mbarrier per tile parity): it only moves, and O and the running sum are rescaled, when a
+//     tile's maximum exceeds it by more than 2^8, so rescaling is rare after the first tiles and
+//     P stays below 256.  The running sum l is handed on the same way, one tile later;
+//   * the warpgroup of an item's last key tile writes O / l in bf16 straight from its
+//     registers to HBM (16-byte stores, rows past the sequence end skipped).  An item's query
+//     slot is freed by the completion of its last Q K^T, so no Q K^T ever waits for a P V (with
+//     Q K^T three tiles ahead, a slot freed by the output would deadlock behind items of fewer
+//     than three key tiles).
 // P is carried as two bf16 halves because a single bf16 rounding of P over a 1024-key window
 // leaves errors near 1e-2 of rms; the pair (split by truncation, see split2_trunc) keeps the
 // result near 1e-5.
-// Tensor memory (512 columns): S0 [0,128), S1 [128,256), O0 [256,384), O1 [384,512).
-// Warp roles (640 threads): warp 0 TMA producer, warp 1 MMA issuer (one thread), warps 4-11 the
-// softmax warpgroups of query tile 0 (keys [0, 64), then [64, 128)), warps 12-19 those of query
-// tile 1.  Registers: launched at 96 per thread; warps 0-3 drop to 56 and the softmax groups
-// rise to 104 (each SM sub-partition holds one warp of each of the five warpgroups:
-// 32 x (56 + 4 x 104) <= 32 x 5 x 96).  A softmax thread reads its 64 scores in two passes (the
-// maximum, then 32 at a time for P) so that it fits its 104 registers.
-// Every wait is bounded; a wait that gives up makes the CTA stop and write NaN into its output
-// rows that are still to be written.  The two warpgroups of a query tile wait together: one
-// thread waits while the other 255 sleep at the pair's named barrier, so that neither half can
-// leave while the other is at the pair's barrier.
+// Tensor memory (512 columns): S0 [0,128), S1 [128,256), S2 [256,384), O [384,512).
+// Warp roles (512 threads): warp 0 TMA producer, warp 1 MMA issuer (one elected lane), warps 4-7,
+// 8-11 and 12-15 the softmax warpgroups 0, 1, 2.  Registers: launched at 128 per thread; warps
+// 0-3 drop to 80 and the softmax warpgroups rise to 144: 32 x (4 x 80 + 12 x 144) = 65536.
+// Every wait is bounded; a wait that gives up makes every role of the CTA stop (the item in
+// progress gets NaN rows if its last warpgroup still reaches the output).  A warpgroup waits as
+// one: one thread polls the barrier while the other 127 sleep at the group's named barrier, and
+// all take the same branch.
 #include <cuda_bf16.h>
 #include <math.h>
 #include <stdint.h>
@@ -54,42 +54,45 @@ constexpr int D = SWA_DIM;
 constexpr int BM = 128;                  // queries per tile, keys per tile
 constexpr int TILE = BM * D * 2;         // one bf16 128 x 128 tile
 constexpr int SLAB = TILE / 2;
-constexpr int NTHREADS = 640;
-constexpr int LAUNCH_REGS = 96;
+constexpr int NTHREADS = 512;
+constexpr int LAUNCH_REGS = 128;
+constexpr int NBUF = 3;                  // score buffers = softmax warpgroups = V stages
+constexpr uint32_t TM_O = 384;           // O's first tensor-memory column
 constexpr uint64_t WAIT_NS = 2000000000ull;
 constexpr uint64_t DRAIN_NS = 200000000ull;
-constexpr float RESCALE_LOG2 = 8.f;      // move the running maximum only past this margin
+constexpr float RESCALE_LOG2 = 8.f;      // move the reference maximum only past this margin
 
 struct __align__(1024) SwaSmem {
-    unsigned char q[2][TILE];            // the two query tiles; later their output tiles
-    unsigned char k[2][TILE];
-    unsigned char v[2][TILE];
-    // p_ready[w][kh]: query tile w's P over keys [64 kh, 64 kh + 64) is in tensor memory
-    // q_full[w]: query tile w of the item is loaded; q_free[w]: its output has been stored (the
-    // slot may be loaded again); o_free[w]: its O accumulator has been read
-    uint64_t q_full[2], q_free[2], o_free[2];
-    uint64_t kv_full[2], kv_empty[2], s_full[2], p_ready[2][2], pv_done[2], drain;
-    uint32_t dec[2][2];                  // the softmax pairs' shared wait outcomes
-    // the two halves of a query row exchange their partial maxima (double-buffered by tile) and,
-    // at the end, their partial sums
-    float xmax[2][2][2][BM];             // [tile parity][query tile][key half][row]
-    float xl[2][2][BM];                  // [query tile][key half][row]
+    unsigned char q[2][TILE];            // query tile of item n in slot n % 2
+    unsigned char k[2][TILE];            // key tile j in stage j % 2
+    unsigned char v[NBUF][TILE];         // value tile j in stage j % 3
+    // q_full / q_free: an item's query tile is loaded / read by the item's last Q K^T
+    uint64_t q_full[2], q_free[2], k_full[2], k_empty[2], v_full[NBUF], v_empty[NBUF];
+    // s_full[b]: Q K^T of the key tile in buffer b is done; p_ready[b][h]: its P over keys
+    // [64 h, 64 h + 64) is in tensor memory; pv_done[b]: P V of that tile is done
+    uint64_t s_full[NBUF], p_ready[NBUF][2], pv_done[NBUF];
+    // dec_full[j % 2] / l_full[j % 2]: key tile j's reference maximum / running sum is posted
+    uint64_t dec_full[2], l_full[2], o_free, drain;
+    uint32_t dec[NBUF][2];               // the warpgroups' shared wait outcomes
+    float mref[2][BM];                   // [key tile parity][row]
+    float lsum[2][BM];
     uint32_t tmem_base;
     uint32_t abort;
 };
 static_assert(sizeof(SwaSmem) <= 232448, "shared-memory plan exceeds 227 KB");
 
 struct SwaParams {
+    __nv_bfloat16* o;      // [B, N, H, 128]
     float scale_log2;      // scale * log2(e)
     int window;
     int64_t N;
     int H;
-    int n_qpairs;          // query-tile pairs per sequence
-    int64_t n_items;       // (batch, head, query-tile pair) items
+    int n_qt;              // query tiles per sequence
+    int64_t n_items;       // (batch, head, query tile) items
 };
 
-// One item of work: two 128-query tiles of one (batch, head), queries q0 .. q0 + 255, and the
-// key tiles [kt_lo, kt_lo + ntiles) their windows touch.
+// One item of work: the 128-query tile q0 .. q0 + 127 of one (batch, head), and the key tiles
+// [kt_lo, kt_lo + ntiles) its window touches.
 struct SwaItem {
     int64_t q0, kt_lo;
     int ntiles, h, b;
@@ -97,16 +100,37 @@ struct SwaItem {
 
 __device__ __forceinline__ SwaItem item_of(const SwaParams& p, int64_t t) {
     SwaItem it;
-    const int pair = (int)(t % p.n_qpairs);
-    it.h = (int)((t / p.n_qpairs) % p.H);
-    it.b = (int)(t / ((int64_t)p.n_qpairs * p.H));
-    it.q0 = (int64_t)pair * 2 * 128;
-    const int64_t qlast = (it.q0 + 2 * 128 - 1 < p.N - 1) ? it.q0 + 2 * 128 - 1 : p.N - 1;
+    const int qt = (int)(t % p.n_qt);
+    it.h = (int)((t / p.n_qt) % p.H);
+    it.b = (int)(t / ((int64_t)p.n_qt * p.H));
+    it.q0 = (int64_t)qt * BM;
+    const int64_t qlast = (it.q0 + BM - 1 < p.N - 1) ? it.q0 + BM - 1 : p.N - 1;
     const int64_t kfirst = (it.q0 - p.window + 1 > 0) ? it.q0 - p.window + 1 : 0;
-    it.kt_lo = kfirst / 128;
-    it.ntiles = (int)(qlast / 128 - it.kt_lo + 1);
+    it.kt_lo = kfirst / BM;
+    it.ntiles = (int)(qlast / BM - it.kt_lo + 1);
     return it;
 }
+
+// Walks this CTA's items (t = blockIdx.x, blockIdx.x + gridDim.x, ...) and their key tiles,
+// numbered across items: key tile j belongs to item number n, whose first tile is jbase.
+struct TileWalk {
+    int64_t t;
+    int n, jbase;
+    SwaItem it;
+    __device__ explicit TileWalk(const SwaParams& p) : t(blockIdx.x), n(0), jbase(0) {
+        if (t < p.n_items) it = item_of(p, t);
+    }
+    // moves to the item that holds key tile j (j never decreases); false past the last item
+    __device__ bool seek(const SwaParams& p, int j) {
+        while (t < p.n_items && j >= jbase + it.ntiles) {
+            jbase += it.ntiles;
+            ++n;
+            t += gridDim.x;
+            if (t < p.n_items) it = item_of(p, t);
+        }
+        return t < p.n_items;
+    }
+};
 
 __device__ __forceinline__ float ex2f(float x) {
     float y;
@@ -126,14 +150,6 @@ __device__ __forceinline__ void split2_trunc(float x0, float x1, uint32_t& hi, u
     lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
 }
 
-// does query tile w (queries q0 + 128 w .. + 127) see any key of key tile kt?
-__device__ __forceinline__ bool takes_part(int64_t q0, int w, int64_t kt, int window, int64_t N) {
-    const int64_t qa = q0 + BM * w, qb = qa + BM - 1;
-    if (qa >= N) return false;                     // the tile is past the sequence end
-    const int64_t ka = BM * kt, kb = ka + BM - 1;
-    return ka <= qb && kb >= qa - window + 1;
-}
-
 // Exit-time wait for this CTA's own asynchronous work; bounded, and not cut short by an abort.
 __device__ __forceinline__ void mbar_wait_drain_(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     uint32_t never = 0;
@@ -146,32 +162,45 @@ __device__ __forceinline__ bool wait_abortable(SwaSmem& sm, uint64_t* bar, uint3
     return false;
 }
 
-// A softmax pair's wait (the two warpgroups of one query tile): one thread polls the barrier,
-// the other 255 sleep at the pair's named barrier (no issue slots burned by polling threads),
-// and all take the same branch, so that neither half can leave the tile loop while the other
-// waits at the pair's barrier.  The outcome word is double-buffered, so that a fast thread
-// cannot overwrite it for the next wait before a slow thread of the pair has read it.
-__device__ __forceinline__ bool pair_wait(SwaSmem& sm, uint64_t* bar, uint32_t parity, int w,
-                                          int hf, int r, int& flip) {
-    if (hf == 0 && r == 0) sm.dec[w][flip] = wait_abortable(sm, bar, parity) ? 1u : 0u;
-    asm volatile("bar.sync %0, 256;" ::"r"(1 + w) : "memory");
-    const bool ok = *reinterpret_cast<volatile uint32_t*>(&sm.dec[w][flip]) != 0;
+__device__ __forceinline__ void group_sync(int gid) {
+    asm volatile("bar.sync %0, 128;" ::"r"(1 + gid) : "memory");
+}
+
+// A softmax warpgroup's wait: thread 0 of the group polls the barrier, the other 127 sleep at
+// the group's named barrier, and all take the same branch.  The outcome word is
+// double-buffered, so that thread 0 cannot overwrite it for the next wait before a slow thread
+// of the group has read it.
+__device__ __forceinline__ bool group_wait(SwaSmem& sm, uint64_t* bar, uint32_t parity, int gid,
+                                           int r, int& flip) {
+    if (r == 0) sm.dec[gid][flip] = wait_abortable(sm, bar, parity) ? 1u : 0u;
+    group_sync(gid);
+    const bool ok = *reinterpret_cast<volatile uint32_t*>(&sm.dec[gid][flip]) != 0;
     flip ^= 1;
     return ok;
 }
 
-__device__ __forceinline__ void pair_sync(int w) {
-    asm volatile("bar.sync %0, 256;" ::"r"(1 + w) : "memory");
+// true on every thread of the warpgroup when x holds on any of them
+__device__ __forceinline__ bool group_any(bool x, int gid) {
+    uint32_t res;
+    asm volatile(
+        "{\n\t.reg .pred p, q;\n\t"
+        "setp.ne.u32 p, %1, 0;\n\t"
+        "bar.red.or.pred q, %2, 128, p;\n\t"
+        "selp.u32 %0, 1, 0, q;\n\t}"
+        : "=r"(res)
+        : "r"((uint32_t)x), "r"(1 + gid)
+        : "memory");
+    return res != 0;
 }
 
-// The MMA issue loops are fully unrolled over constant descriptor offsets: a single thread
-// issues every MMA of the CTA, and per-step descriptor arithmetic in a rolled loop (a chain of
-// dependent integer operations) takes longer than a 128x128x16 MMA takes to execute.  The empty
-// asm statements pin each call's descriptor bases where they are made, so that the compiler
-// does not hoist every unrolled descriptor of every stage out of the key-tile loop (which would
-// need more registers than the issuing warp has).
+// The MMA issue loops are fully unrolled over constant descriptor offsets, and the whole of
+// warp 1 runs them (one elected lane issues each instruction), so that the operands stay in
+// uniform registers: per-step descriptor arithmetic, or operands moved into uniform registers
+// per instruction, takes longer than a 128x128x16 MMA takes to execute.  The empty asm
+// statements pin each call's descriptor bases where they are made, so that the compiler does
+// not hoist every unrolled descriptor of every stage out of the key-tile loop.
 
-// S (+)= A B over K = 128 with both operands K-major in shared memory (A = Q, B = K).
+// S = Q K^T over K = 128 with both operands K-major in shared memory.
 __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a_base, uint32_t b_base) {
     constexpr uint32_t idesc = idesc_bf16(128, 128, 0, 0);
     uint64_t ad = sdesc_sw128(a_base, 16, 1024), bd = sdesc_sw128(b_base, 16, 1024);
@@ -179,7 +208,7 @@ __device__ __forceinline__ void mma_qk(uint32_t d, uint32_t a_base, uint32_t b_b
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk) {
         const uint32_t off = ((kk >> 2) * SLAB + (kk & 3) * 32u) >> 4;
-        mma_ss(d, ad + off, bd + off, idesc, kk > 0 ? 1u : 0u);
+        mma_ss_w(d, ad + off, bd + off, idesc, kk > 0 ? 1u : 0u);
     }
 }
 
@@ -196,14 +225,293 @@ __device__ __forceinline__ void mma_pv(uint32_t d, uint32_t p_base, int kh, uint
     for (int half = 0; half < 2; ++half)
 #pragma unroll
         for (int kk = 0; kk < 4; ++kk)
-            mma_ts(d, pb + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half, vd + ((kk * 2048u) >> 4),
+            mma_ts_w(d, pb + 32 * (kk >> 1) + 8 * (kk & 1) + 16 * half, vd + ((kk * 2048u) >> 4),
                    idesc, (accumulate || half > 0 || kk > 0) ? 1u : 0u);
+}
+
+// ---- warp 0: TMA producer.  Per item its query tile (slot n % 2, once item n - 2's last
+// Q K^T has read the slot) ahead of its first key tile; key tiles j in K stage j % 2 and V stage
+// j % 3.  The K stream runs one tile ahead of the V stream: K stage j % 2 is freed by Q K^T of
+// tile j - 2, which completes before P V of tile j - 4 frees the V stage of tile j - 1.
+__device__ void producer(SwaSmem& sm, const SwaParams& p, const CUtensorMap* tq,
+                         const CUtensorMap* tk, const CUtensorMap* tv) {
+    tma_prefetch_desc(tq);
+    tma_prefetch_desc(tk);
+    tma_prefetch_desc(tv);
+    TileWalk wk(p), wv(p);
+    int jk = 0, jv = 0, nq = 0;   // key tiles, value tiles and query tiles issued
+    bool ok = true;
+    auto load = [&](const CUtensorMap* map, unsigned char* dst, uint64_t* bar, const SwaItem& it,
+                    int tok) {
+        mbar_arrive_expect_tx(bar, TILE);
+        for (int half = 0; half < 2; ++half)
+            tma_load_4d(dst + half * SLAB, map, bar, half * 64, it.h, tok, it.b);
+    };
+    while (ok) {
+        const bool more_k = wk.seek(p, jk);
+        if (more_k) {
+            const int i = jk - wk.jbase;
+            if (i == 0) {   // the item's query tile
+                const int n = wk.n, qs = n & 1;
+                if (n >= 2 && !(ok = wait_abortable(sm, &sm.q_free[qs], ((n >> 1) - 1) & 1)))
+                    break;
+                load(tq, sm.q[qs], &sm.q_full[qs], wk.it, (int)wk.it.q0);
+                nq = n + 1;
+            }
+            const int ks = jk & 1;
+            if (jk >= 2 && !(ok = wait_abortable(sm, &sm.k_empty[ks], ((jk >> 1) - 1) & 1))) break;
+            load(tk, sm.k[ks], &sm.k_full[ks], wk.it, (int)((wk.it.kt_lo + i) * BM));
+            ++jk;
+        }
+        if (jv < jk - (more_k ? 1 : 0)) {
+            wv.seek(p, jv);
+            const int vs = jv % NBUF;
+            if (jv >= NBUF && !(ok = wait_abortable(sm, &sm.v_empty[vs], (jv / NBUF - 1) & 1)))
+                break;
+            load(tv, sm.v[vs], &sm.v_full[vs], wv.it, (int)((wv.it.kt_lo + jv - wv.jbase) * BM));
+            ++jv;
+        } else if (!more_k) {
+            break;
+        }
+    }
+    // no TMA write into this CTA's shared memory may be in flight at exit
+    for (int jj = (jk >= 2 ? jk - 2 : 0); jj < jk; ++jj)
+        mbar_wait_drain_(&sm.k_full[jj & 1], (jj >> 1) & 1, DRAIN_NS);
+    for (int jj = (jv >= NBUF ? jv - NBUF : 0); jj < jv; ++jj)
+        mbar_wait_drain_(&sm.v_full[jj % NBUF], (jj / NBUF) & 1, DRAIN_NS);
+    for (int nn = (nq >= 2 ? nq - 2 : 0); nn < nq; ++nn)
+        mbar_wait_drain_(&sm.q_full[nn & 1], (nn >> 1) & 1, DRAIN_NS);
+}
+
+// ---- warp 1: the MMA issuer (the whole warp, converged; one elected lane issues).  Q K^T of
+// key tile j into S[j % 3] once P V of tile j - 3 has read that buffer; P V of tile j as its
+// softmax hands P over, half the keys at a time.  Issue order: Q K^T of tiles 0, 1, 2, then per
+// tile j: P V_j, Q K^T_{j+3}.
+__device__ void mma_issuer(SwaSmem& sm, const SwaParams& p, uint32_t tmem) {
+    TileWalk wq(p), wp(p);   // the Q K^T and the P V streams
+    int jq = 0, jp = 0;
+    bool ok = true;
+    auto W = [&](uint64_t* bar, uint32_t parity) {   // warp-uniform outcome (lane 0's)
+        if (ok) ok = __shfl_sync(0xffffffffu, wait_abortable(sm, bar, parity) ? 1 : 0, 0) != 0;
+        return ok;
+    };
+    auto issue_qk = [&](int j) {
+        const int i = j - wq.jbase, n = wq.n, b = j % NBUF;
+        if (i == 0 && !W(&sm.q_full[n & 1], (n >> 1) & 1)) return;
+        if (!W(&sm.k_full[j & 1], (j >> 1) & 1)) return;
+        if (j >= NBUF && !W(&sm.pv_done[b], (j / NBUF - 1) & 1)) return;
+        tc_fence_after();
+        mma_qk(tmem + BM * b, smem_u32(sm.q[n & 1]), smem_u32(sm.k[j & 1]));
+        mma_commit_w(&sm.s_full[b]);
+        mma_commit_w(&sm.k_empty[j & 1]);
+        if (i + 1 == wq.it.ntiles) mma_commit_w(&sm.q_free[n & 1]);   // the item's last Q K^T
+    };
+    auto issue_pv = [&](int j) {
+        const int i = j - wp.jbase, n = wp.n, b = j % NBUF;
+        const uint32_t use = (uint32_t)(j / NBUF);
+        if (i == 0 && n > 0 && !W(&sm.o_free, (n - 1) & 1)) return;   // last item's O read
+        if (!W(&sm.v_full[b], use & 1)) return;
+        const uint32_t vb = smem_u32(sm.v[b]);
+        for (int kh = 0; kh < 2; ++kh) {
+            if (!W(&sm.p_ready[b][kh], use & 1)) return;
+            tc_fence_after();
+            mma_pv(tmem + TM_O, tmem + BM * b, kh, vb, i > 0 || kh > 0);
+        }
+        mma_commit_w(&sm.pv_done[b]);
+        mma_commit_w(&sm.v_empty[b]);
+    };
+    while (ok) {
+        while (ok && jq < jp + NBUF && wq.seek(p, jq)) issue_qk(jq++);
+        if (!ok || !wp.seek(p, jp)) break;
+        issue_pv(jp++);
+    }
+    // all issued MMAs complete before tensor memory is released
+    mma_commit_w(&sm.drain);
+    mbar_wait_drain_(&sm.drain, 0, DRAIN_NS);
+}
+
+// ---- softmax warpgroup gid: key tiles j = gid, gid + 3, ... (score buffer S[gid], V stage
+// gid); thread r owns query row r of the tile's item.
+__device__ void softmax_group(SwaSmem& sm, const SwaParams& p, uint32_t tmem, int gid, int warp,
+                              int lane) {
+    const int q = warp & 3, r = q * 32 + lane;
+    const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
+    const uint32_t s_addr = tmem + lane_base + BM * gid;   // this row of S / P
+    const uint32_t o_addr = tmem + lane_base + TM_O;       // this row of O
+    const float c = p.scale_log2;
+    const bool up = c >= 0.f;
+    TileWalk wk(p);
+    int flip = 0;
+    bool ok = true;
+    for (int j = gid; ok && wk.seek(p, j); j += NBUF) {
+        const int i = j - wk.jbase;
+        const uint32_t use = (uint32_t)(j / NBUF);
+        // token positions fit in 32 bits (the host checks N)
+        const int qi = (int)wk.it.q0 + r;            // this thread's query position
+        const int kt = (int)wk.it.kt_lo + i;
+        if (!(ok = group_wait(sm, &sm.s_full[gid], use & 1, gid, r, flip))) break;
+        tc_fence_after();
+        // visible keys of this row in this key tile: columns [c_lo, c_hi]
+        const int lo128 = qi - p.window + 1 - BM * kt, hi128 = qi - BM * kt;
+        const int c_lo = lo128 < 0 ? 0 : (lo128 > BM ? BM : lo128);
+        const int c_hi = hi128 > BM - 1 ? BM - 1 : (hi128 < -1 ? -1 : hi128);
+        const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == BM - 1);
+        // scores in log2 units are c s; the row's maximum of c s over its visible keys is
+        // c max(s) for c >= 0 and c min(s) otherwise (eight independent partial extrema)
+        float e8[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) e8[u] = up ? -INFINITY : INFINITY;
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+            float sg[32];
+            tmem_ld32(s_addr + 32 * g, sg);
+            tmem_ld_wait();
+            if (full) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    e8[e & 7] = up ? fmaxf(e8[e & 7], sg[e]) : fminf(e8[e & 7], sg[e]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 32; ++e)
+                    if (32 * g + e >= c_lo && 32 * g + e <= c_hi)
+                        e8[e & 7] = up ? fmaxf(e8[e & 7], sg[e]) : fminf(e8[e & 7], sg[e]);
+            }
+        }
+#pragma unroll
+        for (int u = 4; u > 0; u >>= 1)
+#pragma unroll
+            for (int v = 0; v < u; ++v)
+                e8[v] = up ? fmaxf(e8[v], e8[v + u]) : fminf(e8[v], e8[v + u]);
+        const float mx = (c_lo <= c_hi) ? c * e8[0] : -INFINITY;
+        // the reference maximum after the previous key tile (every tile waits for it, also the
+        // first of an item, whose reference starts afresh, so that the barrier's phases stay
+        // in step)
+        float m_prev = -INFINITY;
+        if (j > 0) {
+            if (!(ok = group_wait(sm, &sm.dec_full[(j - 1) & 1], ((j - 1) >> 1) & 1, gid, r, flip)))
+                break;
+            if (i > 0) m_prev = sm.mref[(j - 1) & 1][r];
+        }
+        const bool move = mx > m_prev + RESCALE_LOG2;
+        const float m = move ? mx : m_prev;
+        const bool rescale = move && m_prev > -INFINITY;
+        sm.mref[j & 1][r] = m;
+        mbar_arrive(&sm.dec_full[j & 1]);
+        // O holds the rows' sums over the item's earlier key tiles relative to m_prev; rows that
+        // move scale them by 2^(m_prev - m) once P V of tile j - 1 is done, and P V of this tile
+        // may only start after that.  The wait comes after this tile's P is written, so that it
+        // overlaps the previous tile's products.
+        const bool any_rescale = group_any(rescale, gid);
+        // P, one 32-key group at a time, the group's scores read again from tensor memory and
+        // replaced in place by the group's P: 16 columns of high halves, then 16 of low halves.
+        // P V over the first 64 keys may start once their P is written (unless O is rescaled).
+        const float nm = -m;   // finite whenever a key of the row is visible
+        float l4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+#pragma unroll 1
+        for (int g = 0; g < 4; ++g) {
+            float sg[32];
+            tmem_ld32(s_addr + 32 * g, sg);
+            tmem_ld_wait();
+#pragma unroll
+            for (int sub = 0; sub < 2; ++sub) {
+                uint32_t hi8[8], lo8[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int k2 = 8 * sub + e;            // key pair within the group
+                    const int c0 = g * 32 + 2 * k2;
+                    float p0 = ex2f(fmaf(sg[2 * k2], c, nm));
+                    float p1 = ex2f(fmaf(sg[2 * k2 + 1], c, nm));
+                    if (!full) {
+                        p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
+                        p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
+                    }
+                    l4[e & 3] += p0 + p1;
+                    split2_trunc(p0, p1, hi8[e], lo8[e]);
+                }
+                tmem_st8(s_addr + 32 * g + 8 * sub, hi8);
+                tmem_st8(s_addr + 32 * g + 16 + 8 * sub, lo8);
+            }
+            if (g == 1 && !any_rescale) {
+                tmem_st_wait();
+                tc_fence_before();
+                mbar_arrive(&sm.p_ready[gid][0]);
+            }
+        }
+        if (any_rescale) {
+            // a warp rescales (by 1 for its other rows) when any of its rows moves: the tensor
+            // memory accesses are warp-wide instructions
+            if (!(ok = group_wait(sm, &sm.pv_done[(j - 1) % NBUF], ((j - 1) / NBUF) & 1, gid, r,
+                                  flip)))
+                break;
+            tc_fence_after();
+            if (__any_sync(0xffffffffu, rescale)) {
+                const float f = rescale ? ex2f(m_prev - m) : 1.f;
+#pragma unroll 1
+                for (int jc = 0; jc < 4; ++jc) {
+                    float t32[32];
+                    tmem_ld32(o_addr + jc * 32, t32);
+                    tmem_ld_wait();
+                    uint32_t u[32];
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(t32[e] * f);
+                    tmem_st32(o_addr + jc * 32, u);
+                }
+            }
+            tmem_st_wait();
+            tc_fence_before();
+            mbar_arrive(&sm.p_ready[gid][0]);
+        } else {
+            tmem_st_wait();
+            tc_fence_before();
+        }
+        mbar_arrive(&sm.p_ready[gid][1]);
+        // the running sum: the previous tile's, relative to m_prev, plus this tile's
+        float l_prev = 0.f;
+        if (j > 0) {
+            if (!(ok = group_wait(sm, &sm.l_full[(j - 1) & 1], ((j - 1) >> 1) & 1, gid, r, flip)))
+                break;
+            if (i > 0) l_prev = sm.lsum[(j - 1) & 1][r];
+        }
+        const float l = (rescale ? l_prev * ex2f(m_prev - m) : l_prev) +
+                        ((l4[0] + l4[1]) + (l4[2] + l4[3]));
+        sm.lsum[j & 1][r] = l;
+        mbar_arrive(&sm.l_full[j & 1]);
+        if (i + 1 < wk.it.ntiles) continue;
+        // ---- the item's last key tile: O / l in bf16, row r straight to HBM.  O is released
+        // (o_free) once read.
+        ok = group_wait(sm, &sm.pv_done[gid], use & 1, gid, r, flip);
+        tc_fence_after();
+        const float inv = ok && l > 0.f ? 1.f / l : __int_as_float(0x7fc00000);
+        const bool in = (int64_t)qi < p.N;
+        uint4* orow = reinterpret_cast<uint4*>(
+            p.o + (((int64_t)wk.it.b * p.N + (in ? qi : 0)) * p.H + wk.it.h) * D);
+#pragma unroll 1
+        for (int jc = 0; jc < 4; ++jc) {
+            float t32[32];
+            tmem_ld32(o_addr + jc * 32, t32);
+            tmem_ld_wait();
+            if (jc == 3) {
+                tc_fence_before();
+                mbar_arrive(&sm.o_free);
+            }
+            if (in) {
+#pragma unroll
+                for (int v4 = 0; v4 < 4; ++v4) {
+                    uint4 u;
+                    u.x = pack_bf16x2(t32[8 * v4 + 0] * inv, t32[8 * v4 + 1] * inv);
+                    u.y = pack_bf16x2(t32[8 * v4 + 2] * inv, t32[8 * v4 + 3] * inv);
+                    u.z = pack_bf16x2(t32[8 * v4 + 4] * inv, t32[8 * v4 + 5] * inv);
+                    u.w = pack_bf16x2(t32[8 * v4 + 6] * inv, t32[8 * v4 + 7] * inv);
+                    orow[4 * jc + v4] = u;
+                }
+            }
+        }
+    }
 }
 
 __global__ void __launch_bounds__(NTHREADS, 1)
     swa_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                  const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
-                  const SwaParams p) {
+                  const __grid_constant__ CUtensorMap tv, const SwaParams p) {
     extern __shared__ __align__(1024) unsigned char smem_raw[];
     SwaSmem& sm = *reinterpret_cast<SwaSmem*>(smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -212,14 +520,20 @@ __global__ void __launch_bounds__(NTHREADS, 1)
         for (int s = 0; s < 2; ++s) {
             mbar_init(&sm.q_full[s], 1);
             mbar_init(&sm.q_free[s], 1);
-            mbar_init(&sm.o_free[s], 256);
-            mbar_init(&sm.kv_full[s], 1);
-            mbar_init(&sm.kv_empty[s], 1);
+            mbar_init(&sm.k_full[s], 1);
+            mbar_init(&sm.k_empty[s], 1);
+            mbar_init(&sm.dec_full[s], 128);
+            mbar_init(&sm.l_full[s], 128);
+        }
+        for (int s = 0; s < NBUF; ++s) {
+            mbar_init(&sm.v_full[s], 1);
+            mbar_init(&sm.v_empty[s], 1);
             mbar_init(&sm.s_full[s], 1);
             mbar_init(&sm.p_ready[s][0], 128);
             mbar_init(&sm.p_ready[s][1], 128);
             mbar_init(&sm.pv_done[s], 1);
         }
+        mbar_init(&sm.o_free, 128);
         mbar_init(&sm.drain, 1);
         sm.abort = 0;
         fence_mbar_init();
@@ -232,314 +546,15 @@ __global__ void __launch_bounds__(NTHREADS, 1)
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
-    // The CTA is persistent: it takes items t = blockIdx.x, blockIdx.x + gridDim.x, ...; every
-    // role walks the same list, and every barrier's phase count runs on across items.
-
+    // The CTA is persistent: every role walks the same items and key tiles, and every
+    // barrier's phase count runs on across items.
     if (warp < 4) {
-        asm volatile("setmaxnreg.dec.sync.aligned.u32 56;" ::: "memory");
-        if (warp == 0 && lane == 0) {
-            // ---- producer: per item, query tile 0, the first key / value tile, query tile 1,
-            // the other key / value tiles (two stages).  A query slot is loaded again once the
-            // previous item's output tile has left it.
-            tma_prefetch_desc(&tq);
-            tma_prefetch_desc(&tk);
-            tma_prefetch_desc(&tv);
-            tma_prefetch_desc(&to);
-            int g = 0, n = 0;      // key / value tiles and items issued
-            bool ok = true;
-            auto load_q = [&](const SwaItem& it, int w) {
-                if (n > 0 && !(ok = wait_abortable(sm, &sm.q_free[w], (n - 1) & 1))) return;
-                mbar_arrive_expect_tx(&sm.q_full[w], TILE);
-                for (int half = 0; half < 2; ++half)
-                    tma_load_4d(sm.q[w] + half * SLAB, &tq, &sm.q_full[w], half * 64, it.h,
-                                (int)(it.q0 + BM * w), it.b);
-            };
-            auto load_kv = [&](const SwaItem& it, int i) {
-                const int st = g & 1;
-                if (g >= 2 && !(ok = wait_abortable(sm, &sm.kv_empty[st], ((g >> 1) - 1) & 1)))
-                    return;
-                const int tok = (int)((it.kt_lo + i) * BM);
-                mbar_arrive_expect_tx(&sm.kv_full[st], 2 * TILE);
-                for (int half = 0; half < 2; ++half) {
-                    tma_load_4d(sm.k[st] + half * SLAB, &tk, &sm.kv_full[st], half * 64, it.h,
-                                tok, it.b);
-                    tma_load_4d(sm.v[st] + half * SLAB, &tv, &sm.kv_full[st], half * 64, it.h,
-                                tok, it.b);
-                }
-                ++g;
-            };
-            for (int64_t t = blockIdx.x; t < p.n_items && ok; t += gridDim.x) {
-                const SwaItem it = item_of(p, t);
-                load_q(it, 0);
-                for (int i = 0; i < it.ntiles && ok; ++i) {
-                    load_kv(it, i);
-                    if (i == 0 && ok) load_q(it, 1);
-                }
-                if (ok) ++n;
-            }
-            // no TMA write into this CTA's shared memory may be in flight at exit
-            for (int gg = (g >= 2 ? g - 2 : 0); gg < g; ++gg)
-                mbar_wait_drain_(&sm.kv_full[gg & 1], (gg >> 1) & 1, DRAIN_NS);
-            if (n > 0)
-                for (int w = 0; w < 2; ++w) mbar_wait_drain_(&sm.q_full[w], (n - 1) & 1, DRAIN_NS);
-        } else if (warp == 1 && lane == 0) {
-            // ---- MMA issuer.  Query tile 0 runs one step ahead of tile 1: Q_0 K_{i+1}^T is
-            // issued right after P_0 V_i, before P_1 V_i, so that tile 0's next softmax overlaps
-            // tile 1's products instead of both tiles' softmaxes running at the same time.
-            // Every item waits each tile's q_full phase once and (after the first item) each
-            // tile's o_free phase once, before the first use or at the item's end.
-            bool ok = true;
-            int cnt[2] = {0, 0};   // P V products issued per query tile (all items)
-            int g = 0, n = 0;      // key / value tiles and items consumed
-            for (int64_t t = blockIdx.x; t < p.n_items && ok; t += gridDim.x) {
-                const SwaItem it = item_of(p, t);
-                bool need_q[2] = {true, true}, need_o[2] = {n > 0, n > 0}, first[2] = {true, true};
-                auto part = [&](int w, int i) {
-                    return takes_part(it.q0, w, it.kt_lo + i, p.window, p.N);
-                };
-                auto qk = [&](int w, int i) {   // S_w = Q_w K_i^T, once P V has read the last P
-                    if (need_q[w]) {
-                        if (!(ok = wait_abortable(sm, &sm.q_full[w], n & 1))) return;
-                        need_q[w] = false;
-                    }
-                    if (cnt[w] > 0 && !(ok = wait_abortable(sm, &sm.pv_done[w], (cnt[w] - 1) & 1)))
-                        return;
-                    tc_fence_after();
-                    mma_qk(tmem + BM * w, smem_u32(sm.q[w]), smem_u32(sm.k[(g + i) & 1]));
-                    mma_commit(&sm.s_full[w]);
-                };
-                auto pv = [&](int w, int i) {   // O_w += P_w V_i, one half of the keys at a time
-                    if (need_o[w]) {   // the previous item's O_w has been read
-                        if (!(ok = wait_abortable(sm, &sm.o_free[w], (n - 1) & 1))) return;
-                        need_o[w] = false;
-                    }
-                    const uint32_t vb = smem_u32(sm.v[(g + i) & 1]);
-                    for (int kh = 0; kh < 2 && ok; ++kh) {
-                        if (!(ok = wait_abortable(sm, &sm.p_ready[w][kh], cnt[w] & 1))) return;
-                        tc_fence_after();
-                        mma_pv(tmem + 256 + BM * w, tmem + BM * w, kh, vb, !first[w] || kh > 0);
-                    }
-                    first[w] = false;
-                    mma_commit(&sm.pv_done[w]);
-                    ++cnt[w];
-                };
-                auto kv_wait = [&](int i) {
-                    const int gi = g + i;
-                    if ((ok = wait_abortable(sm, &sm.kv_full[gi & 1], (gi >> 1) & 1))) tc_fence_after();
-                };
-                if (it.ntiles > 0) {
-                    kv_wait(0);
-                    if (ok && part(0, 0)) qk(0, 0);
-                    if (ok && part(1, 0)) qk(1, 0);
-                }
-                for (int i = 0; i < it.ntiles && ok; ++i) {
-                    const bool nxt = i + 1 < it.ntiles;
-                    if (part(0, i)) pv(0, i);
-                    if (ok && nxt) {
-                        kv_wait(i + 1);
-                        if (ok && part(0, i + 1)) qk(0, i + 1);
-                    }
-                    if (ok && part(1, i)) pv(1, i);
-                    if (!ok) break;
-                    // this stage: its K was read by Q K^T of both tiles and its V by both P V
-                    mma_commit(&sm.kv_empty[(g + i) & 1]);
-                    if (nxt && part(1, i + 1)) qk(1, i + 1);
-                }
-                // the phases this item did not need
-                for (int w = 0; w < 2 && ok; ++w) {
-                    if (need_q[w]) ok = wait_abortable(sm, &sm.q_full[w], n & 1);
-                    if (ok && need_o[w]) ok = wait_abortable(sm, &sm.o_free[w], (n - 1) & 1);
-                }
-                g += it.ntiles;
-                ++n;
-            }
-            mma_commit(&sm.drain);
-            mbar_wait_drain_(&sm.drain, 0, DRAIN_NS);
-        }
+        asm volatile("setmaxnreg.dec.sync.aligned.u32 80;" ::: "memory");
+        if (warp == 0 && lane == 0) producer(sm, p, &tq, &tk, &tv);
+        else if (warp == 1) mma_issuer(sm, p, tmem);
     } else {
-        asm volatile("setmaxnreg.inc.sync.aligned.u32 104;" ::: "memory");
-        // ---- softmax warpgroup (w, hf): query row r of query tile w, keys [64 hf, 64 hf + 64)
-        // of each key tile.  The two halves of a row share its running maximum (exchanged through
-        // shared memory each tile) and add their sums at the end.
-        const int wg = (warp - 4) >> 2;
-        const int w = wg >> 1, hf = wg & 1;
-        const int q = warp & 3, r = q * 32 + lane;
-        const uint32_t lane_base = ((uint32_t)(q * 32)) << 16;
-        const uint32_t s_addr = tmem + lane_base + BM * w + 64 * hf;        // this half of S / P
-        const uint32_t o_addr = tmem + lane_base + 256 + BM * w + 64 * hf;  // this half of O
-        int cnt = 0, flip = 0;   // key tiles taken part in (all items): the barriers' phases
-        bool ok = true;
-        for (int64_t t = blockIdx.x; t < p.n_items && ok; t += gridDim.x) {
-        // token positions fit in 32 bits (the host checks N)
-        int q0, kt_lo, ntiles;
-        {
-            const SwaItem it = item_of(p, t);
-            q0 = (int)it.q0;
-            kt_lo = (int)it.kt_lo;
-            ntiles = it.ntiles;
-        }
-        const int qi = q0 + BM * w + r;          // this thread's query position
-        float m_ref = -INFINITY, l = 0.f;
-        int cnt_item = 0;
-        for (int i = 0; i < ntiles && ok; ++i) {
-            const int kt = kt_lo + i;
-            if (!takes_part(q0, w, kt, p.window, p.N)) continue;
-            // pair-uniform outcome: no warp may split around the warp-wide TMEM accesses, and
-            // neither half may leave while the other waits at the pair's barrier
-            ok = pair_wait(sm, &sm.s_full[w], cnt & 1, w, hf, r, flip);
-            if (!ok) break;
-            tc_fence_after();
-            // visible keys of this row in this half: columns [c_lo, c_hi] of the half
-            const int c_lo64 = qi - p.window + 1 - BM * kt - 64 * hf, c_hi64 = qi - BM * kt - 64 * hf;
-            const int c_lo = c_lo64 < 0 ? 0 : (c_lo64 > 64 ? 64 : c_lo64);
-            const int c_hi = c_hi64 > 63 ? 63 : (c_hi64 < -1 ? -1 : c_hi64);
-            // scores in log2 units are c s; the half's maximum of c s over its visible keys is
-            // c max(s) for c >= 0 and c min(s) otherwise (eight independent partial extrema),
-            // 32 columns at a time.  Halves wholly inside every row's window skip the per-key
-            // mask.
-            const float c = p.scale_log2;
-            const bool full = __all_sync(0xffffffffu, c_lo == 0 && c_hi == 63);
-            const bool up = c >= 0.f;
-            float e8[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) e8[u] = up ? -INFINITY : INFINITY;
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                float sg[32];
-                tmem_ld32(s_addr + 32 * g, sg);
-                tmem_ld_wait();
-                if (full) {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        e8[e & 7] = up ? fmaxf(e8[e & 7], sg[e]) : fminf(e8[e & 7], sg[e]);
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 32; ++e)
-                        if (32 * g + e >= c_lo && 32 * g + e <= c_hi)
-                            e8[e & 7] = up ? fmaxf(e8[e & 7], sg[e]) : fminf(e8[e & 7], sg[e]);
-                }
-            }
-#pragma unroll
-            for (int u = 4; u > 0; u >>= 1)
-#pragma unroll
-                for (int v = 0; v < u; ++v)
-                    e8[v] = up ? fmaxf(e8[v], e8[v + u]) : fminf(e8[v], e8[v + u]);
-            const float ext = e8[0];
-            const float mx_half = (c_lo <= c_hi) ? c * ext : -INFINITY;
-            // the row's maximum over both halves
-            sm.xmax[cnt & 1][w][hf][r] = mx_half;
-            pair_sync(w);
-            const float mx = fmaxf(mx_half, sm.xmax[cnt & 1][w][hf ^ 1][r]);
-            // move the reference when the tile's maximum passes it by the margin: O and l scale
-            // by 2^(m_ref - mx) (both halves take the same decision from the same maximum; each
-            // scales its own columns of O and its own partial sum).  The tensor-memory accesses
-            // are warp-wide instructions, so the whole warp takes the branch when any of its
-            // rows needs it (factor 1 for the others).
-            const bool move = mx > m_ref + RESCALE_LOG2;
-            const bool rescale = move && m_ref > -INFINITY;
-            if (__any_sync(0xffffffffu, rescale)) {
-                const float f = rescale ? ex2f(m_ref - mx) : 1.f;
-                l *= f;
-#pragma unroll 1
-                for (int jc = 0; jc < 2; ++jc) {
-                    float t32[32];
-                    tmem_ld32(o_addr + jc * 32, t32);
-                    tmem_ld_wait();
-                    uint32_t u[32];
-#pragma unroll
-                    for (int e = 0; e < 32; ++e) u[e] = __float_as_uint(t32[e] * f);
-                    tmem_st32(o_addr + jc * 32, u);
-                }
-            }
-            if (move) m_ref = mx;
-            const float nm = -m_ref;   // finite whenever a key of the row is visible
-            float l4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
-            // P, one 32-key group at a time, the group's scores read again from tensor memory
-            // (so that the 64 scores of the maximum pass are not held through this one) and
-            // replaced in place by the group's P: 16 columns of high halves, then 16 of low
-            // halves, over the 32 columns the group's scores occupied.
-#pragma unroll
-            for (int g = 0; g < 2; ++g) {
-                float sg[32];
-                tmem_ld32(s_addr + 32 * g, sg);
-                tmem_ld_wait();
-                // eight key pairs at a time: their high halves to columns 32 g + 8 sub, their
-                // low halves to 32 g + 16 + 8 sub (the group's scores are all in sg already)
-#pragma unroll
-                for (int sub = 0; sub < 2; ++sub) {
-                    uint32_t hi8[8], lo8[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int k2 = 8 * sub + e;            // key pair within the group
-                        const int c0 = g * 32 + 2 * k2;
-                        float p0 = ex2f(fmaf(sg[2 * k2], c, nm));
-                        float p1 = ex2f(fmaf(sg[2 * k2 + 1], c, nm));
-                        if (!full) {
-                            p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
-                            p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
-                        }
-                        l4[e & 3] += p0 + p1;
-                        split2_trunc(p0, p1, hi8[e], lo8[e]);
-                    }
-                    tmem_st8(s_addr + 32 * g + 8 * sub, hi8);
-                    tmem_st8(s_addr + 32 * g + 16 + 8 * sub, lo8);
-                }
-            }
-            l += (l4[0] + l4[1]) + (l4[2] + l4[3]);
-            tmem_st_wait();
-            tc_fence_before();
-            mbar_arrive(&sm.p_ready[w][hf]);   // P V over this half's keys may run
-            ++cnt;
-            ++cnt_item;
-        }
-        // ---- epilogue: O / l in bf16 through this tile's query slot (each half its 64
-        // columns), then one TMA store.  O_w is released (o_free) once read, the query slot
-        // (q_free) once the store has read it; both once per item, also for a tile that took
-        // no part.
-        if (cnt_item > 0) {
-            if (ok) ok = pair_wait(sm, &sm.pv_done[w], (cnt - 1) & 1, w, hf, r, flip);
-            tc_fence_after();
-            sm.xl[w][hf][r] = l;
-            pair_sync(w);
-            const float lt = l + sm.xl[w][hf ^ 1][r];
-            const float inv = ok && lt > 0.f ? 1.f / lt : __int_as_float(0x7fc00000);
-            unsigned char* row = sm.q[w] + hf * SLAB + r * 128;
-#pragma unroll 1
-            for (int jc = 0; jc < 2; ++jc) {
-                float t32[32];
-                tmem_ld32(o_addr + jc * 32, t32);
-                tmem_ld_wait();
-                if (jc == 1) {
-                    tc_fence_before();
-                    mbar_arrive(&sm.o_free[w]);
-                }
-#pragma unroll
-                for (int v4 = 0; v4 < 4; ++v4) {
-                    uint4 u;
-                    u.x = pack_bf16x2(t32[8 * v4 + 0] * inv, t32[8 * v4 + 1] * inv);
-                    u.y = pack_bf16x2(t32[8 * v4 + 2] * inv, t32[8 * v4 + 3] * inv);
-                    u.z = pack_bf16x2(t32[8 * v4 + 4] * inv, t32[8 * v4 + 5] * inv);
-                    u.w = pack_bf16x2(t32[8 * v4 + 6] * inv, t32[8 * v4 + 7] * inv);
-                    const int cc = 4 * jc + v4;   // 16-byte chunk of the half-row
-                    *reinterpret_cast<uint4*>(row + ((cc ^ (r & 7)) << 4)) = u;
-                }
-            }
-            fence_proxy_async_smem();
-            pair_sync(w);   // both halves of the tile are written
-            if (hf == 0 && r == 0) {
-                const SwaItem it = item_of(p, t);
-                for (int half = 0; half < 2; ++half)
-                    tma_store_4d(&to, sm.q[w] + half * SLAB, half * 64, it.h, q0 + BM * w, it.b);
-                bulk_commit_group();
-                bulk_wait_group_read0();
-                mbar_arrive(&sm.q_free[w]);
-            }
-        } else {
-            mbar_arrive(&sm.o_free[w]);
-            if (hf == 0 && r == 0) mbar_arrive(&sm.q_free[w]);
-        }
-        }   // items
-        if (hf == 0 && r == 0) bulk_wait_group0();   // the last stores have completed
+        asm volatile("setmaxnreg.inc.sync.aligned.u32 144;" ::: "memory");
+        softmax_group(sm, p, tmem, (warp - 4) >> 2, warp, lane);
     }
     tc_fence_before();
     __syncthreads();
@@ -557,20 +572,20 @@ cudaError_t launch_swa(const SwaArgs& a, cudaStream_t stream) {
     const uint64_t strides[3] = {(uint64_t)D * 2, (uint64_t)a.H * D * 2,
                                  (uint64_t)a.N * a.H * D * 2};
     const uint32_t box[4] = {64, 1, BM, 1};
-    CUtensorMap tq, tk, tv, to;
+    CUtensorMap tq, tk, tv;
     if (!make_bf16_map(&tq, a.q, 4, dims, strides, box) ||
         !make_bf16_map(&tk, a.k, 4, dims, strides, box) ||
-        !make_bf16_map(&tv, a.v, 4, dims, strides, box) ||
-        !make_bf16_map(&to, a.o, 4, dims, strides, box))
+        !make_bf16_map(&tv, a.v, 4, dims, strides, box))
         return cudaErrorInvalidValue;
     if (a.N > (int64_t)0x7FFFFE00) return cudaErrorInvalidValue;   // 32-bit token coordinates
     SwaParams p;
+    p.o = a.o;
     p.scale_log2 = a.scale * 1.4426950408889634f;
     p.window = a.window;
     p.N = a.N;
     p.H = a.H;
-    p.n_qpairs = (int)((a.N + 2 * BM - 1) / (2 * BM));
-    p.n_items = (int64_t)a.B * a.H * p.n_qpairs;
+    p.n_qt = (int)((a.N + BM - 1) / BM);
+    p.n_items = (int64_t)a.B * a.H * p.n_qt;
     // persistent: one CTA per SM (at most one per item)
     int dev = 0, n_sm = 0;
     if (cudaGetDevice(&dev) != cudaSuccess ||
@@ -591,7 +606,7 @@ cudaError_t launch_swa(const SwaArgs& a, cudaStream_t stream) {
     }
     // the in-kernel register split (setmaxnreg) assumes exactly LAUNCH_REGS per thread
     if (regs != LAUNCH_REGS) return cudaErrorInvalidValue;
-    swa_tc_kernel<<<(unsigned)grid, NTHREADS, smem, stream>>>(tq, tk, tv, to, p);
+    swa_tc_kernel<<<(unsigned)grid, NTHREADS, smem, stream>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 

@@ -32,6 +32,8 @@ def inputs(B, N, H, seed):
     (1, 1000, 2, 300),     # several tiles per window
     (1, 700, 2, 1024),     # window longer than the sequence: causal attention
     (2, 2100, 2, 1024),    # the page's window, 17 tiles per query block
+    (1, 2000, 48, 100),    # 768 one- and two-key-tile items: several per CTA, back to back
+    (1, 1500, 40, 300),    # items of one to four key tiles, several per CTA
 ])
 def test_swa_matches_oracle(B, N, H, W):
     G = lib()
