@@ -291,6 +291,22 @@ __global__ void __launch_bounds__(NT, 1)
     if (tid == 0) load_kv(sm, 0, &tk, &tv, (c1 - 1) * C, h, b);
     float2 gcur[16], gnext[16];
     load_gate16x2(grow, gstride, (int64_t)(c1 - 1) * C + 16 * seg, p.N, gcur);
+    // per-token log2-decays of both channels over this thread's 16 tokens of chunk cc, in place,
+    // and their sum into the chunk's segment totals
+    auto decays = [&](int cc) {
+        const int Lc = (int)min64(C, p.N - (int64_t)cc * C);
+        float2 sum = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const bool in = 16 * seg + u < Lc;
+            gcur[u].x = in ? logsigmoid_fast(gcur[u].x) * p.inv_tau_log2e : 0.f;
+            gcur[u].y = in ? logsigmoid_fast(gcur[u].y) * p.inv_tau_log2e : 0.f;
+            sum.x += gcur[u].x;
+            sum.y += gcur[u].y;
+        }
+        *reinterpret_cast<float2*>(&sm.tot[seg][ch]) = sum;
+    };
+    decays(c1 - 1);
     float2 R = make_float2(0.f, 0.f);   // log2-decay after the current chunk, to the range end
     int issued = 1, consumed = 0;
     uint32_t n_mma = 0;
@@ -298,7 +314,6 @@ __global__ void __launch_bounds__(NT, 1)
 #pragma unroll 1
     for (int n = 0; n < n_ch; ++n) {
         const int c = c1 - 1 - n, st = n & 1;
-        const int L = (int)min64(C, p.N - (int64_t)c * C);
         // the previous chunk's MMAs are done: its stage and the low-half tile are free
         if (n > 0 && !(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
         if (n + 1 < n_ch) {
@@ -306,17 +321,8 @@ __global__ void __launch_bounds__(NT, 1)
             ++issued;
             load_gate16x2(grow, gstride, (int64_t)(c - 1) * C + 16 * seg, p.N, gnext);
         }
-        // per-token log2-decays of both channels over this thread's 16 tokens
-        float2 sum = make_float2(0.f, 0.f);
-#pragma unroll
-        for (int u = 0; u < 16; ++u) {
-            const bool in = 16 * seg + u < L;
-            gcur[u].x = in ? logsigmoid_fast(gcur[u].x) * p.inv_tau_log2e : 0.f;
-            gcur[u].y = in ? logsigmoid_fast(gcur[u].y) * p.inv_tau_log2e : 0.f;
-            sum.x += gcur[u].x;
-            sum.y += gcur[u].y;
-        }
-        *reinterpret_cast<float2*>(&sm.tot[seg][ch]) = sum;
+        // this chunk's segment totals (written at the end of the previous iteration, or before
+        // the loop) are visible to every thread
         __syncthreads();
         float2 after = make_float2(0.f, 0.f), total = make_float2(0.f, 0.f);
 #pragma unroll
@@ -366,8 +372,13 @@ __global__ void __launch_bounds__(NT, 1)
             mma_commit(&sm.mma_done);
         }
         ++n_mma;
+        // the next chunk's decays while this chunk's MMAs run (its gate logits have arrived
+        // in gnext meanwhile; the segment totals were last read before the barrier above)
+        if (n + 1 < n_ch) {
 #pragma unroll
-        for (int u = 0; u < 16; ++u) gcur[u] = gnext[u];
+            for (int u = 0; u < 16; ++u) gcur[u] = gnext[u];
+            decays(c - 1);
+        }
     }
     if (seg == 0) *reinterpret_cast<float2*>(&sm.rs[ch]) = R;   // read after the next barrier
     if (ok) ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err);
@@ -534,38 +545,42 @@ __global__ void __launch_bounds__(NT, 1)
         }
     }
     uint32_t n_g = 1, n_ld = 1, n_mma = 0;   // gate and q/k/v loads issued, MMA groups committed
-    bool ok = true;
-    for (int c = c0; c < c1; ++c) {
+    // per-channel passes: thread (cp, seg) takes channels 2 cp, 2 cp + 1 over tokens
+    // [16 seg, 16 seg + 16), with paired shared-memory accesses (float2, bf16x2)
+    const int cp = tid & 63, seg = tid >> 6, ch = 2 * cp;
+    // cumulative log2-decay of both channels over the segment of chunk cc's gate tile, in place
+    // (every load first); returns the segment's total
+    auto decays = [&](int cc) {
+        const int Lc = (int)min64(C, p.N - (int64_t)cc * C);
+        float2 x[16], cum = make_float2(0.f, 0.f);
+#pragma unroll
+        for (int u = 0; u < 16; ++u)
+            x[u] = *reinterpret_cast<const float2*>(&sm.g[(16 * seg + u) * D + ch]);
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            const bool in = 16 * seg + u < Lc;
+            x[u].x = in ? logsigmoid_fast(x[u].x) * p.inv_tau_log2e : 0.f;
+            x[u].y = in ? logsigmoid_fast(x[u].y) * p.inv_tau_log2e : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+            cum.x += x[u].x;
+            cum.y += x[u].y;
+            *reinterpret_cast<float2*>(&sm.g[(16 * seg + u) * D + ch]) = cum;
+        }
+        return cum;
+    };
+    bool ok = block_wait(&sm.g_full, 0, p.err);
+    float2 cum = ok ? decays(c0) : make_float2(0.f, 0.f);
+    for (int c = c0; c < c1 && ok; ++c) {
         const int L = (int)min64(C, p.N - (int64_t)c * C);
         const bool last = c == c1 - 1;
         if (c > c0) {   // the previous output tile has left x
             if (tid == 0) bulk_wait_group_read0();
             __syncthreads();
         }
-        if (!(ok = block_wait(&sm.g_full, (n_g - 1) & 1, p.err))) break;
-        // per-channel passes: thread (cp, seg) takes channels 2 cp, 2 cp + 1 over tokens
-        // [16 seg, 16 seg + 16), with paired shared-memory accesses (float2, bf16x2)
-        const int cp = tid & 63, seg = tid >> 6, ch = 2 * cp;
-        // cumulative log2-decay of both channels over the segment, in place (every load first)
-        float2 cum = make_float2(0.f, 0.f);
-        {
-            float2 x[16];
-#pragma unroll
-            for (int u = 0; u < 16; ++u)
-                x[u] = *reinterpret_cast<const float2*>(&sm.g[(16 * seg + u) * D + ch]);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                const bool in = 16 * seg + u < L;
-                x[u].x = in ? logsigmoid_fast(x[u].x) * p.inv_tau_log2e : 0.f;
-                x[u].y = in ? logsigmoid_fast(x[u].y) * p.inv_tau_log2e : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < 16; ++u) {
-                cum.x += x[u].x;
-                cum.y += x[u].y;
-                *reinterpret_cast<float2*>(&sm.g[(16 * seg + u) * D + ch]) = cum;
-            }
-        }
+        // this chunk's decays are in the gate tile already (computed while the previous chunk's
+        // output MMAs ran, or before the loop)
         float* tot = reinterpret_cast<float*>(sm.y);   // [8][D] segment totals; y is idle here
         *reinterpret_cast<float2*>(&tot[seg * D + ch]) = cum;
         __syncthreads();
@@ -701,6 +716,11 @@ __global__ void __launch_bounds__(NT, 1)
             mma_commit(&sm.mma_done);
         }
         ++n_mma;
+        // while they run: the next chunk's decays, in its gate tile (loaded after pass 2)
+        if (!last) {
+            if (!(ok = block_wait(&sm.g_full, (n_g - 1) & 1, p.err))) break;
+            cum = decays(c + 1);
+        }
         if (!(ok = block_wait(&sm.mma_done, (n_mma - 1) & 1, p.err))) break;
         tc_fence_after();
         if (!last) {   // q, k, v are free: the next chunk's tiles go now
