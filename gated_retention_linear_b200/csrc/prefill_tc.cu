@@ -70,6 +70,7 @@
 #include <stdlib.h>
 
 #include <algorithm>
+#include <cmath>
 
 #include "sm100.cuh"
 #include "tma_host.cuh"
@@ -1078,9 +1079,13 @@ bool make_map(CUtensorMap* map, const void* base, int64_t st, int64_t sh, int64_
 // fixed overhead of about 1.5 (its look-back and the switches between passes), and the
 // look-backs of one chain run one after another at about half a chunk-time each.  G minimises
 // the larger of the two over [2, 128]: at 32K x 24 heads it picks 43 (144 spans, one wave; the
-// fastest span size of a measured sweep), at 512K x 24 heads 111.
+// fastest span size of a measured sweep), at 512K x 24 heads 111.  With packed sequences of
+// unequal lengths (`ragged`, where the host knows only their mean, chunks_per_unit) each
+// sequence's last span is on average half empty, so a chain has chunks / G + 1/2 spans: on
+// the eight sequences of 1024 to 65536 tokens x 24 heads that picks 28 (2.73 ms) where the
+// mean alone picked 82 (2.88 ms; a measured sweep was flat at 2.68-2.74 ms over G = 12..32).
 // GRET_SPAN_CHUNKS overrides the choice.
-int span_chunks(int64_t chunks_per_unit, int64_t chains, int grid) {
+int span_chunks(double chunks_per_unit, int64_t chains, int grid, bool ragged) {
     static int forced = -2;
     if (forced == -2) {
         const char* e = getenv("GRET_SPAN_CHUNKS");
@@ -1091,14 +1096,15 @@ int span_chunks(int64_t chunks_per_unit, int64_t chains, int grid) {
     int best = 2;
     double best_cost = -1.0;
     for (int g = 2; g <= 128; ++g) {
-        const int64_t spans = std::max<int64_t>(1, (chunks_per_unit + g - 1) / g);
-        const int64_t waves = (chains * spans + grid - 1) / grid;
-        const double cost = std::max((double)waves * (g + 1.5), 0.5 * (double)spans + g);
+        const double whole = std::max(1.0, std::ceil(chunks_per_unit / g));
+        const double spans = ragged ? chunks_per_unit / g + 0.5 : whole;
+        const double waves = std::ceil(std::ceil((double)chains * spans) / grid);
+        const double cost = std::max(waves * (g + 1.5), 0.5 * spans + g);
         if (best_cost < 0.0 || cost < best_cost) {
             best = g;
             best_cost = cost;
         }
-        if (spans == 1) break;   // larger spans change nothing
+        if (!ragged && whole == 1.0) break;   // larger spans change nothing
     }
     return best;
 }
@@ -1112,9 +1118,12 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
     const int units = a.n_seqs;
     const WsLayout L = ws_layout(units, a.H);
     unsigned char* ws = (unsigned char*)a.workspace;
-    const int64_t chunks_per_unit =
-        units > 0 ? ((varlen ? a.N / units : a.N) + C - 1) / C : 0;   // varlen: the mean
-    const int G = span_chunks(chunks_per_unit, (int64_t)units * a.H, sm_count());
+    // chunks per sequence (varlen: their mean)
+    const double chunks_per_unit =
+        units <= 0 ? 0.0
+        : varlen   ? (double)a.N / units / C
+                   : (double)((a.N + C - 1) / C);
+    const int G = span_chunks(chunks_per_unit, (int64_t)units * a.H, sm_count(), varlen);
 
     TcParams p;
     p.g = a.g;
