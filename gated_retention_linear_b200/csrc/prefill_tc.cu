@@ -1079,11 +1079,12 @@ bool make_map(CUtensorMap* map, const void* base, int64_t st, int64_t sh, int64_
 // fixed overhead of about 1.5 (its look-back and the switches between passes), and the
 // look-backs of one chain run one after another at about half a chunk-time each.  G minimises
 // the larger of the two over [2, 128]: at 32K x 24 heads it picks 43 (144 spans, one wave; the
-// fastest span size of a measured sweep), at 512K x 24 heads 111.  With packed sequences of
-// unequal lengths (`ragged`, where the host knows only their mean, chunks_per_unit) each
-// sequence's last span is on average half empty, so a chain has chunks / G + 1/2 spans: on
-// the eight sequences of 1024 to 65536 tokens x 24 heads that picks 28 (2.73 ms) where the
-// mean alone picked 82 (2.88 ms; a measured sweep was flat at 2.68-2.74 ms over G = 12..32).
+// fastest span size of a measured sweep), at 512K x 24 heads 111.  With several packed
+// sequences of unequal lengths (`ragged`, where the host knows only their mean,
+// chunks_per_unit) each sequence's last span is on average half empty, so a chain has
+// chunks / G + 1/2 spans: on the eight sequences of 1024 to 65536 tokens x 24 heads that
+// picks 28 (2.71 ms) where the mean alone picked 82 (2.88 ms; a measured sweep was flat at
+// 2.68-2.74 ms over G = 12..32).
 // GRET_SPAN_CHUNKS overrides the choice.
 int span_chunks(double chunks_per_unit, int64_t chains, int grid, bool ragged) {
     static int forced = -2;
@@ -1123,7 +1124,9 @@ gret_status_t launch_prefill_tc(const PrefillArgs& a) {
         units <= 0 ? 0.0
         : varlen   ? (double)a.N / units / C
                    : (double)((a.N + C - 1) / C);
-    const int G = span_chunks(chunks_per_unit, (int64_t)units * a.H, sm_count(), varlen);
+    // packed sequences of unequal length: more than one (with one, the mean is its length)
+    const int G = span_chunks(chunks_per_unit, (int64_t)units * a.H, sm_count(),
+                              varlen && units > 1);
 
     TcParams p;
     p.g = a.g;
