@@ -236,8 +236,9 @@ __device__ __forceinline__ void mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_
 
 // Warp-wide forms of the two MMAs and of the commit: every lane of a converged warp makes the
 // call with the same operands, which can then live in uniform registers, and one lane chosen
-// by elect.sync issues the instruction.  Issued from a single lane of a diverged warp instead,
-// each instruction first has to move its operands into uniform registers.
+// by elect.sync issues the instruction.  Where each step's descriptor is formed just before
+// its MMA, this keeps the issue at the MMA rate; from one lane of a diverged warp the
+// sliding-window kernel's issue fell behind it.
 __device__ __forceinline__ void mma_ss_w(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
                                          uint32_t idesc, uint32_t accumulate) {
     asm volatile(

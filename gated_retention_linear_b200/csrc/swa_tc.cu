@@ -194,9 +194,9 @@ __device__ __forceinline__ bool group_any(bool x, int gid) {
 }
 
 // The MMA issue loops are fully unrolled over constant descriptor offsets, and the whole of
-// warp 1 runs them (one elected lane issues each instruction), so that the operands stay in
-// uniform registers: per-step descriptor arithmetic, or operands moved into uniform registers
-// per instruction, takes longer than a 128x128x16 MMA takes to execute.  The empty asm
+// warp 1 runs them (one elected lane issues each instruction), so that the operands can stay
+// in uniform registers: issued from one lane of a diverged warp, with each step's descriptor
+// formed just before its MMA, the issue took longer than a 128x128x16 MMA takes to execute.  The empty asm
 // statements pin each call's descriptor bases where they are made, so that the compiler does
 // not hoist every unrolled descriptor of every stage out of the key-tile loop.
 
