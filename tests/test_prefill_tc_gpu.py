@@ -69,6 +69,14 @@ def test_varlen_ragged_with_empty_sequences():
     run_varlen([0, 1, 127, 128, 129, 700, 0, 2000], 3, 128, 128, BF, seed=35, state=True)
 
 
+def test_varlen_more_than_1024_sequences():
+    """1100 packed sequences of 0 to 64 tokens: the span plan's prefix runs over two blocks of
+    1024 sequences, and the span size is the one chosen for many short, unequal sequences."""
+    rng = np.random.default_rng(37)
+    lens = [int(x) for x in rng.integers(0, 65, size=1100)]
+    run_varlen(lens, 1, 128, 128, BF, seed=37, state=True)
+
+
 def test_varlen_state_aliasing():
     run_varlen([1500, 0, 37, 600], 2, 128, 128, BF, seed=36, state=True, alias_state=True)
 
