@@ -150,6 +150,15 @@ __device__ __forceinline__ void split2_trunc(float x0, float x1, uint32_t& hi, u
     lo = __byte_perm(__float_as_uint(l0), __float_as_uint(l1), 0x7632);
 }
 
+// The same split as split2_trunc with the two remainders taken by one packed subtraction.
+__device__ __forceinline__ void split2_trunc_x2(float2 x, uint32_t& hi, uint32_t& lo) {
+    const uint32_t b0 = __float_as_uint(x.x), b1 = __float_as_uint(x.y);
+    const float2 h = make_float2(__uint_as_float(b0 & 0xFFFF0000u), __uint_as_float(b1 & 0xFFFF0000u));
+    const float2 l = add2(x, make_float2(-h.x, -h.y));
+    hi = __byte_perm(b0, b1, 0x7632);
+    lo = __byte_perm(__float_as_uint(l.x), __float_as_uint(l.y), 0x7632);
+}
+
 // Exit-time wait for this CTA's own asynchronous work; bounded, and not cut short by an abort.
 __device__ __forceinline__ void mbar_wait_drain_(uint64_t* bar, uint32_t parity, uint64_t limit_ns) {
     uint32_t never = 0;
@@ -406,7 +415,9 @@ __device__ void softmax_group(SwaSmem& sm, const SwaParams& p, uint32_t tmem, in
         // replaced in place by the group's P: 16 columns of high halves, then 16 of low halves.
         // P V over the first 64 keys may start once their P is written (unless O is rescaled).
         const float nm = -m;   // finite whenever a key of the row is visible
-        float l4[4] = {0.f, 0.f, 0.f, 0.f};   // independent partial sums
+        const float2 c2 = make_float2(c, c), nm2 = make_float2(nm, nm);
+        float2 l4[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                        make_float2(0.f, 0.f)};   // independent partial sums, two lanes each
 #pragma unroll 1
         for (int g = 0; g < 4; ++g) {
             float sg[32];
@@ -419,14 +430,14 @@ __device__ void softmax_group(SwaSmem& sm, const SwaParams& p, uint32_t tmem, in
                 for (int e = 0; e < 8; ++e) {
                     const int k2 = 8 * sub + e;            // key pair within the group
                     const int c0 = g * 32 + 2 * k2;
-                    float p0 = ex2f(fmaf(sg[2 * k2], c, nm));
-                    float p1 = ex2f(fmaf(sg[2 * k2 + 1], c, nm));
+                    const float2 arg = fma2(make_float2(sg[2 * k2], sg[2 * k2 + 1]), c2, nm2);
+                    float2 pp = make_float2(ex2f(arg.x), ex2f(arg.y));
                     if (!full) {
-                        p0 = (c0 >= c_lo && c0 <= c_hi) ? p0 : 0.f;
-                        p1 = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? p1 : 0.f;
+                        pp.x = (c0 >= c_lo && c0 <= c_hi) ? pp.x : 0.f;
+                        pp.y = (c0 + 1 >= c_lo && c0 + 1 <= c_hi) ? pp.y : 0.f;
                     }
-                    l4[e & 3] += p0 + p1;
-                    split2_trunc(p0, p1, hi8[e], lo8[e]);
+                    l4[e & 3] = add2(l4[e & 3], pp);
+                    split2_trunc_x2(pp, hi8[e], lo8[e]);
                 }
                 tmem_st8(s_addr + 32 * g + 8 * sub, hi8);
                 tmem_st8(s_addr + 32 * g + 16 + 8 * sub, lo8);
@@ -472,8 +483,8 @@ __device__ void softmax_group(SwaSmem& sm, const SwaParams& p, uint32_t tmem, in
                 break;
             if (i > 0) l_prev = sm.lsum[(j - 1) & 1][r];
         }
-        const float l = (rescale ? l_prev * ex2f(m_prev - m) : l_prev) +
-                        ((l4[0] + l4[1]) + (l4[2] + l4[3]));
+        const float2 l2 = add2(add2(l4[0], l4[1]), add2(l4[2], l4[3]));
+        const float l = (rescale ? l_prev * ex2f(m_prev - m) : l_prev) + (l2.x + l2.y);
         sm.lsum[j & 1][r] = l;
         mbar_arrive(&sm.l_full[j & 1]);
         if (i + 1 < wk.it.ntiles) continue;
