@@ -556,7 +556,8 @@ __device__ void mma_issuer(Smem& sm, const TcParams& p, uint32_t tmem) {
 __device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
     const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
     const float2 hf = __bfloat1622float2(h);
-    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    const float2 r = fma2(hf, make_float2(-1.f, -1.f), make_float2(x0, x1));   // x - hi
+    const __nv_bfloat162 l = __floats2bfloat162_rn(r.x, r.y);
     hi = *reinterpret_cast<const uint32_t*>(&h);
     lo = *reinterpret_cast<const uint32_t*>(&l);
 }
@@ -611,8 +612,8 @@ __device__ __forceinline__ void convert_wkt(const Smem& sm, int st, int r, uint3
                 kt + m0 * 128 + ((cch ^ (m0 & 7)) << 4)));
             const float k1 = __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(
                 kt + (m0 + 1) * 128 + ((cch ^ ((m0 + 1) & 7)) << 4)));
-            const float2 w = w2[m0 >> 1];
-            split2(k0 * w.x, k1 * w.y, ph[i], ph[16 + i]);
+            const float2 kw = mul2(make_float2(k0, k1), w2[m0 >> 1]);
+            split2(kw.x, kw.y, ph[i], ph[16 + i]);
         }
         tmem_st32(taddr + jc * 32, ph);
     }
@@ -683,12 +684,12 @@ __device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint
 #pragma unroll
                     for (int i2 = 0; i2 < 16; ++i2) {
                         const int m0 = jc * 32 + 2 * i2;
-                        const float p0 =
-                            (m0 <= r) ? ex2f(cr - sm.gc[st][m0]) * p.k_scale * a[2 * i2] : 0.f;
-                        const float p1 = (m0 + 1 <= r)
-                                             ? ex2f(cr - sm.gc[st][m0 + 1]) * p.k_scale * a[2 * i2 + 1]
-                                             : 0.f;
-                        split2(p0, p1, ph[i2], ph[16 + i2]);
+                        const float2 g2 = *reinterpret_cast<const float2*>(&sm.gc[st][m0]);
+                        const float2 arg = fma2(g2, make_float2(-1.f, -1.f), make_float2(cr, cr));
+                        const float2 pv = mul2(mul2(make_float2(ex2f(arg.x), ex2f(arg.y)),
+                                                    make_float2(p.k_scale, p.k_scale)),
+                                               make_float2(a[2 * i2], a[2 * i2 + 1]));
+                        split2(m0 <= r ? pv.x : 0.f, m0 + 1 <= r ? pv.y : 0.f, ph[i2], ph[16 + i2]);
                     }
                 } else {
 #pragma unroll
@@ -723,14 +724,16 @@ __device__ void p_group(Smem& sm, const TcParams& p, const CUtensorMap* to, uint
 #pragma unroll
                 for (int v4 = 0; v4 < 4; ++v4) {
                     uint4 u;
-                    u.x = pack_bf16x2(fmaf(ec, ox[8 * v4 + 0], o[8 * v4 + 0]),
-                                      fmaf(ec, ox[8 * v4 + 1], o[8 * v4 + 1]));
-                    u.y = pack_bf16x2(fmaf(ec, ox[8 * v4 + 2], o[8 * v4 + 2]),
-                                      fmaf(ec, ox[8 * v4 + 3], o[8 * v4 + 3]));
-                    u.z = pack_bf16x2(fmaf(ec, ox[8 * v4 + 4], o[8 * v4 + 4]),
-                                      fmaf(ec, ox[8 * v4 + 5], o[8 * v4 + 5]));
-                    u.w = pack_bf16x2(fmaf(ec, ox[8 * v4 + 6], o[8 * v4 + 6]),
-                                      fmaf(ec, ox[8 * v4 + 7], o[8 * v4 + 7]));
+                    const float2 ec2 = make_float2(ec, ec);
+                    float2 y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        y[e] = fma2(ec2, make_float2(ox[8 * v4 + 2 * e], ox[8 * v4 + 2 * e + 1]),
+                                    make_float2(o[8 * v4 + 2 * e], o[8 * v4 + 2 * e + 1]));
+                    u.x = pack_bf16x2(y[0].x, y[0].y);
+                    u.y = pack_bf16x2(y[1].x, y[1].y);
+                    u.z = pack_bf16x2(y[2].x, y[2].y);
+                    u.w = pack_bf16x2(y[3].x, y[3].y);
                     // columns 32 jc + 8 v4 .. + 7: 16-byte chunk cc = 4 jc + v4 of the row
                     const int cc = 4 * jc + v4;
                     if (full)
