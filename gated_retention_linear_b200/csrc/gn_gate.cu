@@ -284,11 +284,14 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
                     ow[4 * i + 3] = u.w;
                 }
                 uint32_t out[16];
+                // (o - mean) * inv as one packed fma per pair: o * inv + (-mean * inv)
+                const float2 inv2 = make_float2(inv, inv), nmi2 = make_float2(-mean * inv, -mean * inv);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int c = jc * 32 + 2 * i;
                     const float2 f = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&ow[i]));
-                    float n0 = (f.x - mean) * inv, n1 = (f.y - mean) * inv;
+                    const float2 nn = fma2(f, inv2, nmi2);
+                    float n0 = nn.x, n1 = nn.y;
                     if (p.gn_w) {
                         n0 *= __ldg(p.gn_w + col0 + c);
                         n1 *= __ldg(p.gn_w + col0 + c + 1);
@@ -298,7 +301,10 @@ __device__ void epilogue(GSmem& sm, const GParams& p, uint32_t tmem, int warp, i
                         n1 += __ldg(p.gn_b + col0 + c + 1);
                     }
                     const float z0 = z[2 * i], z1 = z[2 * i + 1];
-                    const float s0 = z0 / (1.f + __expf(-z0)), s1 = z1 / (1.f + __expf(-z1));
+                    // swish(z) = z sigmoid(z); the fast division (a few ulp) is far below the
+                    // bf16 rounding of the output
+                    const float s0 = __fdividef(z0, 1.f + __expf(-z0));
+                    const float s1 = __fdividef(z1, 1.f + __expf(-z1));
                     out[i] = pack_bf16x2(n0 * s0, n1 * s1);
                 }
                 uint4* d4 = reinterpret_cast<uint4*>(dst + jc * 32);
